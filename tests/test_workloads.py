@@ -1,0 +1,48 @@
+"""The seeded generator: deterministic, valid page tables, stated shapes."""
+import numpy as np
+import torch
+
+from sparse_indexed_attention_b200.workloads import CONFIGS, make_workload
+
+SMALL = {
+    "prefill": CONFIGS["tiny_prefill_1k"].scaled(ctx=(300, 300), topk=64),
+    "decode": CONFIGS["decode_b64_8k_32k"].scaled(batch=5, ctx=(100, 700), topk=128, planted=8),
+    "chunked": CONFIGS["chunked_prefill_16"].scaled(batch=3, prefix=(0, 500), chunk=(10, 90), topk=64),
+    "pool": CONFIGS["decode_b8_128k"].scaled(batch=2, ctx=(1000, 1000), pool_tokens=64 * 100, topk=128),
+}
+
+
+def test_deterministic_and_valid():
+    for name, spec in SMALL.items():
+        a, b = make_workload(spec), make_workload(spec)
+        for f in ("qI", "w", "kI", "q", "kv"):
+            assert torch.equal(getattr(a, f), getattr(b, f)), (name, f)
+        assert np.array_equal(a.page_table, b.page_table)
+        B = spec.batch
+        assert a.ctx_len.shape == (B,) and a.q_seq_start.shape == (B + 1,)
+        used = a.page_table[a.page_table >= 0]
+        assert used.size == np.unique(used).size                   # no page shared
+        assert used.max() < a.num_phys_pages
+        for bb in range(B):
+            need = (a.ctx_len[bb] + 63) // 64
+            assert np.all(a.page_table[bb, :need] >= 0) and np.all(a.page_table[bb, need:] < 0)
+        T = a.T
+        assert a.qI.shape == (T, 64, 128) and a.qI.dtype == torch.bfloat16
+        assert a.q.shape == (T, spec.heads, 576) and a.kv.shape == (a.num_phys_pages * 64, 576)
+        if spec.ki_fp8:
+            assert a.kI.dtype == torch.uint8 and a.kI_scale.shape == (a.num_phys_pages * 64,)
+            assert not torch.any((a.kI & 0x7F) == 0x7F)            # no NaN codes
+        pos = a.token_pos()
+        for bb in range(B):
+            seg = pos[a.q_seq_start[bb]:a.q_seq_start[bb + 1]]
+            assert seg[-1] == a.ctx_len[bb] - 1 and np.all(np.diff(seg) == 1) and seg[0] >= 0
+
+
+def test_modes():
+    d = make_workload(SMALL["decode"])
+    assert np.all(d.q_len == 1)
+    assert all(p.size == 8 for p in d.planted)
+    c = make_workload(SMALL["chunked"])
+    assert np.all(c.q_len <= c.ctx_len) and np.all(c.q_len >= 10)
+    p = make_workload(SMALL["pool"])
+    assert p.num_phys_pages == 100
