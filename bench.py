@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""DSA decode throughput at 128K context on B200: prints ONE JSON line.
+
+A step is one dsa_index_topk_attn call (indexer -> Top-K -> sparse MLA) over
+one batch of the long-context decode workload (8 sequences x 131072 cached
+tokens, one query token each, K = 2048, 128 heads, FP8 paged index cache in a
+2 Mi-token pool).  Inputs are synthetic and seeded (workloads.py).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank serves its own batch (weak scaling, no
+collective on the data path; a MAX all-reduce of the timings only).
+--impl reference times the fp64 CPU oracle on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_indexed_attention_b200.workloads import CONFIGS, make_workload  # noqa: E402
+
+METRIC = "DSA decode tokens/s at 128K ctx"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="decode_b8_128k", choices=list(CONFIGS))
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage-reps", type=int, default=20)
+    return ap.parse_args()
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.cmd = ["nvidia-smi", f"--id={gid}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                        "-lms", "100"]
+        except Exception:
+            self.cmd = None
+
+    def __enter__(self):
+        if self.cmd:
+            try:
+                self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.thread = threading.Thread(target=self._read, daemon=True)
+                self.thread.start()
+                time.sleep(0.3)
+            except Exception:
+                self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(wl, n_tokens: int):
+    """The fp64 oracle on a bounded sample (the first n_tokens query tokens)."""
+    from oracle import dsa_oracle as O
+    from sparse_indexed_attention_b200.workloads import bits16
+    seqs = O.Seqs(ctx_len=wl.ctx_len.astype(np.int64), q_seq_start=wl.q_seq_start.astype(np.int64),
+                  page_table=wl.page_table, page_size=wl.spec.page_size)
+    if wl.kI_scale is None:
+        kI, sc = bits16(wl.kI), None
+    else:
+        kI, sc = wl.kI.numpy(), wl.kI_scale.numpy()
+    qI, w, q, kv = bits16(wl.qI), wl.w.numpy(), bits16(wl.q), bits16(wl.kv)
+    toks = list(range(n_tokens))
+    t0 = time.perf_counter()
+    O.index_topk_attn(seqs, qI, w, kI, sc, q, kv, wl.spec.topk, wl.scale, tokens=toks)
+    dt = time.perf_counter() - t0
+    return dt, toks
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    spec = CONFIGS[args.config]
+    wl = make_workload(spec)
+    n_tok = wl.T                                   # one step = the whole batch, as in our arm
+    for _ in range(args.warmup):
+        cpu_baseline(wl, n_tok)
+    times = []
+    for _ in range(args.steps):
+        dt, _ = cpu_baseline(wl, n_tok)
+        times.append(dt)
+    step_s = sum(times) / len(times)
+    value = n_tok / step_s
+    sample = (f"fp64 oracle, whole path for {n_tok} query token(s) of {spec.name} "
+              f"(ctx {int(wl.ctx_len[0])}) per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": spec.name, "batch": spec.batch, "ctx": int(wl.ctx_len[0]), "topk": spec.topk,
+                       "heads": spec.heads, "index_cache": "fp8_e4m3" if spec.ki_fp8 else "bf16"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+
+def time_device(fn, steps, warmup, stream, flush):
+    """Mean device time (ms) of fn over `steps` runs, L2 flushed before each."""
+    for _ in range(warmup):
+        fn()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def run_ours(args, world, rank, local):
+    import sparse_indexed_attention_b200 as dsa
+    from sparse_indexed_attention_b200.workloads import to_device
+
+    spec = CONFIGS[args.config]
+    spec = spec.scaled(seed=spec.seed + 1000 * rank)     # each rank serves its own batch
+    wl = make_workload(spec)
+    d = to_device(wl)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    T, H, K = wl.T, spec.heads, spec.topk
+    out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, H), dtype=torch.float32, device=dev)
+    ws = torch.zeros(dsa.dsa_workspace_size(dsa.DSA_OP_INDEX_TOPK_ATTN, d.seqs, K, H), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse, ws=ws)
+
+    step()
+    launches_per_step = dsa.dsa_launches_in_last_call()
+    torch.cuda.synchronize()
+    if dsa.dsa_check_error(ws) != dsa.DSA_OK:
+        raise RuntimeError("device error flag set by the bench workload")
+
+    graph = None
+    run = step
+    if not args.no_graph:
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        run = graph.replay
+
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        times = time_device(run, args.steps, 0, stream, flush)
+        barrier(world)
+        torch.cuda.synchronize()
+    ms_local = sum(times) / len(times)
+    ms = reduce_max(ms_local, world)
+    tokens_total = T * world
+    value = tokens_total / (ms / 1e3)
+
+    # ---- per-stage device times (same kernels, same launch shapes) ----
+    scores = torch.empty((T, (wl.max_ctx + 3) // 4 * 4), dtype=torch.float32, device=dev)
+    ws_i = torch.zeros(dsa.dsa_workspace_size(dsa.DSA_OP_INDEX_SCORES, d.seqs, K, H), dtype=torch.uint8, device=dev)
+    ws_t = torch.zeros(dsa.dsa_workspace_size(dsa.DSA_OP_TOPK, None, K, rows=T, ld=scores.shape[1]),
+                       dtype=torch.uint8, device=dev)
+    ws_a = torch.zeros(dsa.dsa_workspace_size(dsa.DSA_OP_SPARSE_MLA, d.seqs, K, H), dtype=torch.uint8, device=dev)
+    row_len = torch.from_numpy((wl.token_pos() + 1).astype(np.int32)).to(dev)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    dsa.dsa_index_scores(d.seqs, d.qI, d.w, d.kI, d.kI_scale, scores=scores, ws=ws_i)
+    dsa.dsa_topk(scores, row_len, K, idx=idx, ws=ws_t)
+    reps = args.stage_reps
+    t_idx = time_device(lambda: dsa.dsa_index_scores(d.seqs, d.qI, d.w, d.kI, d.kI_scale, scores=scores, ws=ws_i),
+                        reps, 3, stream, flush)
+    t_topk = time_device(lambda: dsa.dsa_topk(scores, row_len, K, idx=idx, ws=ws_t), reps, 3, stream, flush)
+    t_attn = time_device(lambda: dsa.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out=out, lse=lse, ws=ws_a),
+                         reps, 3, stream, flush)
+    n_keys = int((wl.token_pos() + 1).sum())
+    n_sel = int(np.minimum(wl.token_pos() + 1, K).sum())
+    idx_bytes = n_keys * (132 if spec.ki_fp8 else 256)          # index-cache bytes read
+    attn_bytes = n_sel * 1152                                    # gathered latent rows
+    peak, peak_kind = hbm_peak()
+    ms_idx = statistics.mean(t_idx)
+    achieved = idx_bytes / (ms_idx / 1e3) / 1e9
+
+    # ---- end to end through the C ABI with host buffers ----
+    pin = lambda x: x.pin_memory()  # noqa: E731
+    h_qI, h_w, h_q = pin(wl.qI), pin(wl.w), pin(wl.q)
+    h_meta = [pin(torch.from_numpy(a.astype(np.int32))) for a in (wl.q_seq_start, wl.ctx_len, wl.page_table)]
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    d_meta = [d.seqs.q_seq_start, d.seqs.ctx_len, d.seqs.page_table]
+
+    def e2e_step():
+        d.qI.copy_(h_qI, non_blocking=True)
+        d.w.copy_(h_w, non_blocking=True)
+        d.q.copy_(h_q, non_blocking=True)
+        for dm, hm in zip(d_meta, h_meta):
+            dm.copy_(hm, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+
+    e2e_times = time_device(e2e_step, max(5, args.steps // 2), 2, stream, flush)
+    e2e_ms = reduce_max(sum(e2e_times) / len(e2e_times), world)
+    h2d = sum(x.numel() * x.element_size() for x in [h_qI, h_w, h_q, *h_meta])
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        spent, reps = 0.0, 0
+        while spent < 10.0:                      # whole batches until ~10 s of host work
+            dt, _ = cpu_baseline(wl, T)
+            spent += dt
+            reps += 1
+        cpu = {"value": reps * T / spent, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"fp64 oracle, whole path for all {T} query tokens (ctx {int(wl.ctx_len[0])}), "
+                         f"{reps} batch(es), {spent:.1f} s"}
+
+    if graph is not None:
+        del graph
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 index / bf16 attention / fp32 accum",
+            "data": "synthetic (seeded, 64 planted keys per sequence)",
+            "config": {"workload": spec.name, "batch_per_gpu": spec.batch, "global_batch": T * world,
+                       "ctx": int(wl.ctx_len[0]), "topk": K, "heads": H, "index_heads": 64, "index_dim": 128,
+                       "page_size": 64, "pool_tokens": wl.num_phys_pages * 64, "parallelism": f"dp{world}",
+                       "l2": "256 MiB buffer written before every timed step",
+                       "launch": "cuda graph replay" if graph is not None else "eager"},
+            "stages_us": {"index_scores": ms_idx * 1e3, "topk": statistics.mean(t_topk) * 1e3,
+                          "sparse_mla": statistics.mean(t_attn) * 1e3},
+            "roofline": {"kernel": "index_scores (quantize + score)", "bound": "hbm", "achieved": achieved,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_kind,
+                         "algorithmic_bytes": idx_bytes, "traffic": None},
+            "attention_roofline": {"bound": "hbm", "achieved": attn_bytes / (statistics.mean(t_attn) / 1e3) / 1e9,
+                                   "peak": peak, "unit": "GB/s",
+                                   "frac": attn_bytes / (statistics.mean(t_attn) / 1e3) / 1e9 / peak,
+                                   "algorithmic_bytes": attn_bytes},
+            "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "launches_per_step": launches_per_step,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

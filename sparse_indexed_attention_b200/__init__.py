@@ -1,0 +1,226 @@
+"""Python binding of libdsa (include/dsa.h): index-selected sparse attention on B200.
+
+Argument marshalling only.  Every step of the path runs in libdsa's CUDA
+kernels; torch provides device memory and the current stream.  There is no
+fallback: if libdsa.so is missing and cannot be built, importing this package
+raises.
+
+Functions carry the C names (``dsa_index_scores`` ...).  Outputs not passed in
+are allocated with torch on the inputs' device; workspaces are allocated
+zeroed and cached per (device, op, size), unless one is passed in.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+from . import build as _build
+
+# ---------------------------------------------------------------------------
+# Library loading
+# ---------------------------------------------------------------------------
+
+if _build.is_stale():
+    _build.build_library()
+_lib = ctypes.CDLL(_build.LIB)
+LIB_PATH = _build.LIB
+
+DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_BAD_INDEX, \
+    DSA_ERR_TIMEOUT = range(7)
+DSA_KI_BF16, DSA_KI_FP8_E4M3 = 0, 1
+DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_INDEX_TOPK_ATTN = range(5)
+
+# Names the C header declares (checked against include/dsa.h by the tests).
+EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_index_scores", "dsa_topk",
+           "dsa_sparse_mla_fwd", "dsa_index_topk_attn", "dsa_check_error", "dsa_launches_in_last_call", "dsa_status_string")
+
+
+class DsaSeqsC(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_tokens", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("max_pages", ctypes.c_int32), ("num_phys_pages", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
+                ("q_seq_start", ctypes.c_void_p), ("ctx_len", ctypes.c_void_p), ("page_table", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_I32, _I64, _SZ, _F = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+_SEQ = ctypes.POINTER(DsaSeqsC)
+_sig = {
+    "dsa_workspace_size": (_SZ, [ctypes.c_int, _SEQ, ctypes.c_int, ctypes.c_int]),
+    "dsa_quantize_index_query": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, _P]),
+    "dsa_index_scores": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _I64, _P, _SZ, _P]),
+    "dsa_topk": (ctypes.c_int, [_P, _I64, ctypes.c_int, _P, ctypes.c_int, _P, _P, _SZ, _P]),
+    "dsa_sparse_mla_fwd": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, ctypes.c_int, _F, _P, _P, _P, _SZ, _P]),
+    "dsa_index_topk_attn": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
+                                           _F, _P, _P, _P, _P, _SZ, _P]),
+    "dsa_check_error": (ctypes.c_int, [_P, _P]),
+    "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "dsa_launches_in_last_call": (ctypes.c_int, []),
+}
+for _name, (_res, _args) in _sig.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype, _fn.argtypes = _res, _args
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.dsa_status_string(status).decode()}")
+
+
+def _check(status: int, where: str):
+    if status != DSA_OK:
+        raise DsaError(status, where)
+
+
+def status_string(status: int) -> str:
+    return _lib.dsa_status_string(status).decode()
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+# ---------------------------------------------------------------------------
+# Batch geometry
+# ---------------------------------------------------------------------------
+
+
+@dataclass
+class Seqs:
+    """Batch geometry on the device (see dsa_seqs_t in include/dsa.h)."""
+    q_seq_start: torch.Tensor   # int32 [B+1]
+    ctx_len: torch.Tensor       # int32 [B]
+    page_table: torch.Tensor    # int32 [B, max_pages]
+    num_phys_pages: int
+    max_ctx: int
+    num_q_tokens: int
+
+    @staticmethod
+    def from_host(q_seq_start, ctx_len, page_table, num_phys_pages: int, device="cuda") -> "Seqs":
+        qs = torch.as_tensor(q_seq_start, dtype=torch.int32)
+        cl = torch.as_tensor(ctx_len, dtype=torch.int32)
+        pt = torch.as_tensor(page_table, dtype=torch.int32)
+        return Seqs(qs.to(device), cl.to(device), pt.contiguous().to(device), int(num_phys_pages),
+                    int(cl.max()), int(qs[-1]))
+
+    @property
+    def batch(self) -> int:
+        return self.ctx_len.shape[0]
+
+    def c(self) -> DsaSeqsC:
+        return DsaSeqsC(self.batch, self.num_q_tokens, 64, self.page_table.shape[1], self.num_phys_pages,
+                        self.max_ctx, self.q_seq_start.data_ptr(), self.ctx_len.data_ptr(),
+                        self.page_table.data_ptr())
+
+
+def dsa_workspace_size(op: int, seqs: Seqs | None = None, K: int = 1, H: int = 16, *, rows: int = 0,
+                       ld: int = 0) -> int:
+    c = seqs.c() if seqs is not None else DsaSeqsC(1, rows, 64, 1, 1, ld, None, None, None)
+    return int(_lib.dsa_workspace_size(op, ctypes.byref(c), K, H))
+
+
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device, key=None) -> torch.Tensor:
+    """A zeroed device workspace of at least nbytes (cached by key)."""
+    device = torch.device(device)
+    if device.type == "cuda" and device.index is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    k = (device, key)
+    ws = _ws_cache.get(k)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws_cache[k] = ws
+    return ws
+
+
+# ---------------------------------------------------------------------------
+# Entry points
+# ---------------------------------------------------------------------------
+
+
+def dsa_quantize_index_query(qI: torch.Tensor, w: torch.Tensor, codes=None, w_scaled=None):
+    T = qI.shape[0]
+    codes = codes if codes is not None else torch.empty((T, 64, 128), dtype=torch.uint8, device=qI.device)
+    w_scaled = w_scaled if w_scaled is not None else torch.empty((T, 64), dtype=torch.float32, device=qI.device)
+    _check(_lib.dsa_quantize_index_query(_ptr(qI), _ptr(w), T, _ptr(codes), _ptr(w_scaled), _stream(qI.device)),
+           "dsa_quantize_index_query")
+    return codes, w_scaled
+
+
+def dsa_index_scores(seqs: Seqs, qI, w, kI, kI_scale=None, scores=None, ld=None, ws=None):
+    T = seqs.num_q_tokens
+    ld = ld or (seqs.max_ctx + 3) // 4 * 4
+    if scores is None:
+        scores = torch.zeros((T, ld), dtype=torch.float32, device=qI.device)
+    ki_dtype = DSA_KI_FP8_E4M3 if kI_scale is not None else DSA_KI_BF16
+    c = seqs.c()
+    need = _lib.dsa_workspace_size(DSA_OP_INDEX_SCORES, ctypes.byref(c), 1, 16)
+    ws = ws if ws is not None else workspace(need, qI.device, "index_scores")
+    _check(_lib.dsa_index_scores(ctypes.byref(c), _ptr(qI), _ptr(w), _ptr(kI), _ptr(kI_scale), ki_dtype, _ptr(scores),
+                                 ld, _ptr(ws), ws.numel(), _stream(qI.device)), "dsa_index_scores")
+    return scores
+
+
+def dsa_topk(scores: torch.Tensor, row_len: torch.Tensor, K: int, idx=None, ws=None):
+    T, ld = scores.shape
+    idx = idx if idx is not None else torch.empty((T, K), dtype=torch.int32, device=scores.device)
+    c = DsaSeqsC(1, T, 64, 1, 1, ld, None, None, None)
+    need = _lib.dsa_workspace_size(DSA_OP_TOPK, ctypes.byref(c), K, 16)
+    ws = ws if ws is not None else workspace(need, scores.device, "topk")
+    _check(_lib.dsa_topk(_ptr(scores), ld, T, _ptr(row_len), K, _ptr(idx), _ptr(ws), ws.numel(),
+                         _stream(scores.device)), "dsa_topk")
+    return idx
+
+
+def dsa_sparse_mla_fwd(seqs: Seqs, q, kv, idx, scale: float, out=None, lse=None, want_lse=True, ws=None):
+    T, H, _ = q.shape
+    K = idx.shape[1]
+    out = out if out is not None else torch.empty((T, H, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    c = seqs.c()
+    need = _lib.dsa_workspace_size(DSA_OP_SPARSE_MLA, ctypes.byref(c), K, H)
+    ws = ws if ws is not None else workspace(need, q.device, "sparse_mla")
+    _check(_lib.dsa_sparse_mla_fwd(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(idx), K, H, scale, _ptr(out), _ptr(lse),
+                                   _ptr(ws), ws.numel(), _stream(q.device)), "dsa_sparse_mla_fwd")
+    return out, lse
+
+
+def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: float, out=None, lse=None,
+                        idx_out=None, want_lse=True, ws=None):
+    T, H, _ = q.shape
+    out = out if out is not None else torch.empty((T, H, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    ki_dtype = DSA_KI_FP8_E4M3 if kI_scale is not None else DSA_KI_BF16
+    c = seqs.c()
+    need = _lib.dsa_workspace_size(DSA_OP_INDEX_TOPK_ATTN, ctypes.byref(c), K, H)
+    ws = ws if ws is not None else workspace(need, q.device, "index_topk_attn")
+    _check(_lib.dsa_index_topk_attn(ctypes.byref(c), _ptr(qI), _ptr(w), _ptr(kI), _ptr(kI_scale), ki_dtype, _ptr(q),
+                                    _ptr(kv), K, H, scale, _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(ws), ws.numel(),
+                                    _stream(q.device)), "dsa_index_topk_attn")
+    return out, lse
+
+
+def dsa_check_error(ws: torch.Tensor) -> int:
+    """Synchronise the current stream and return (and clear) the device error status."""
+    return int(_lib.dsa_check_error(_ptr(ws), _stream(ws.device)))
+
+
+def dsa_launches_in_last_call() -> int:
+    """Kernels launched by this thread's most recent entry-point call."""
+    return int(_lib.dsa_launches_in_last_call())
+
+
+def raw():
+    """The ctypes handle of libdsa (for tests that call the C ABI directly)."""
+    return _lib

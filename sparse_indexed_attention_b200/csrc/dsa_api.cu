@@ -1,0 +1,266 @@
+// Host side of the C ABI declared in include/dsa.h: argument validation,
+// workspace layout and the launch sequence of each entry point.  Nothing here
+// allocates, synchronises (except dsa_check_error) or reads device memory.
+#include <cmath>
+
+#include "dsa_internal.cuh"
+
+using namespace dsa;
+
+namespace dsa {
+thread_local int g_launches = 0;
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Workspace carve-up.  Offsets are 256-byte aligned; the first 256 bytes hold
+// the sticky error word.
+struct Layout {
+  size_t tok_seq = 0, tok_pos = 0, q_codes = 0, w_scaled = 0, scores = 0, idx = 0, partials = 0;
+  size_t total = 0;
+  int64_t ld = 0;
+};
+
+Layout make_layout(dsa_op_t op, int T, int max_ctx, int K, int H) {
+  Layout L;
+  size_t off = kAlign;  // header
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  const bool seq_ops = op == DSA_OP_INDEX_SCORES || op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN;
+  if (seq_ops) {
+    L.tok_seq = take((size_t)T * sizeof(int32_t));
+    L.tok_pos = take((size_t)T * sizeof(int32_t));
+  }
+  if (op == DSA_OP_INDEX_SCORES || op == DSA_OP_INDEX_TOPK_ATTN) {
+    L.q_codes = take((size_t)T * kHI * kDI);
+    L.w_scaled = take((size_t)T * kHI * sizeof(float));
+  }
+  if (op == DSA_OP_INDEX_TOPK_ATTN) {
+    L.ld = ((int64_t)max_ctx + 3) / 4 * 4;
+    L.scores = take((size_t)T * (size_t)L.ld * sizeof(float));
+    L.idx = take((size_t)T * K * sizeof(int32_t));
+  }
+  if (op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN) L.partials = take(sparse_mla_partials_bytes(T, K, H));
+  L.total = off;
+  return L;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<char*>(ws) + off);
+}
+
+bool valid_H(int H) { return H == 16 || H == 32 || H == 64 || H == 128; }
+
+dsa_status_t check_seqs(const dsa_seqs_t* s) {
+  if (!s || !s->q_seq_start || !s->ctx_len || !s->page_table) return DSA_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->num_q_tokens < 1 || s->max_ctx < 1 || s->num_phys_pages < 1 || s->max_pages < 1)
+    return DSA_ERR_INVALID_ARG;
+  if (s->page_size != kPage) return DSA_ERR_UNSUPPORTED;
+  if ((int64_t)s->max_pages * kPage < (int64_t)s->max_ctx) return DSA_ERR_INVALID_ARG;
+  if ((int64_t)s->num_phys_pages * kPage > (int64_t)INT32_MAX * kPage) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status_t check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < need) return DSA_ERR_WORKSPACE;
+  return DSA_OK;
+}
+
+SeqsDev to_dev(const dsa_seqs_t* s) {
+  SeqsDev d;
+  d.batch = s->batch;
+  d.num_tokens = s->num_q_tokens;
+  d.max_pages = s->max_pages;
+  d.num_phys_pages = s->num_phys_pages;
+  d.max_ctx = s->max_ctx;
+  d.q_seq_start = s->q_seq_start;
+  d.ctx_len = s->ctx_len;
+  d.page_table = s->page_table;
+  return d;
+}
+
+dsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+#define DSA_TRY(x)                       \
+  do {                                   \
+    dsa_status_t _st = (x);              \
+    if (_st != DSA_OK) return _st;       \
+  } while (0)
+#define DSA_CUDA(x) DSA_TRY(cuda_status(x))
+
+dsa_status_t check_indexer_args(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
+                                const float* kI_scale, dsa_ki_dtype_t ki_dtype) {
+  DSA_TRY(check_seqs(seqs));
+  if (!qI || !w || !kI) return DSA_ERR_INVALID_ARG;
+  if (ki_dtype != DSA_KI_BF16 && ki_dtype != DSA_KI_FP8_E4M3) return DSA_ERR_UNSUPPORTED;
+  if ((ki_dtype == DSA_KI_FP8_E4M3) != (kI_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(qI, 16) || !aligned(w, 16) || !aligned(kI, 128) || (kI_scale && !aligned(kI_scale, 16)))
+    return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+dsa_status_t check_attn_args(const dsa_seqs_t* seqs, const void* q, const void* kv, int K, int H, float scale,
+                             const void* out, const float* lse) {
+  DSA_TRY(check_seqs(seqs));
+  if (!q || !kv || !out) return DSA_ERR_INVALID_ARG;
+  if (K < 1 || K > kMaxK || !valid_H(H)) return DSA_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kv, 128) || !aligned(out, 16) || (lse && !aligned(lse, 4)))
+    return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+// indexer launch sequence shared by dsa_index_scores and the fused call
+dsa_status_t run_indexer(const dsa_seqs_t* seqs, const SeqsDev& sd, TokenMap tm, const void* qI, const float* w,
+                         const void* kI, const float* kI_scale, dsa_ki_dtype_t ki_dtype, float* scores,
+                         int64_t ld, void* ws, const Layout& L, uint32_t* err, cudaStream_t st) {
+  const bool fp8 = ki_dtype == DSA_KI_FP8_E4M3;
+  const void* q_operand = qI;
+  const float* w_operand = w;
+  if (fp8) {
+    uint8_t* codes = at<uint8_t>(ws, L.q_codes);
+    float* w_scaled = at<float>(ws, L.w_scaled);
+    DSA_CUDA(launch_quantize_index_query(reinterpret_cast<const __nv_bfloat16*>(qI), w, seqs->num_q_tokens, codes,
+                                         w_scaled, st));
+    q_operand = codes;
+    w_operand = w_scaled;
+  }
+  DSA_CUDA(launch_index_scores(sd, tm, q_operand, w_operand, kI, kI_scale, fp8, scores, ld, err, st));
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dsa_workspace_size(dsa_op_t op, const dsa_seqs_t* seqs, int K, int H) {
+  if (!seqs || seqs->num_q_tokens < 1 || seqs->max_ctx < 1) return 0;
+  if (op == DSA_OP_QUANTIZE_INDEX_QUERY) return 0;
+  if (op == DSA_OP_TOPK) return make_layout(op, seqs->num_q_tokens, seqs->max_ctx, K, 16).total;
+  if (op < 0 || op > DSA_OP_INDEX_TOPK_ATTN) return 0;
+  if ((op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN) && (K < 1 || K > kMaxK || !valid_H(H))) return 0;
+  return make_layout(op, seqs->num_q_tokens, seqs->max_ctx, K, H).total;
+}
+
+dsa_status_t dsa_quantize_index_query(const void* qI, const float* w, int T, uint8_t* codes, float* w_scaled,
+                                      dsa_stream_t stream) {
+  g_launches = 0;
+  if (!qI || !w || !codes || !w_scaled || T < 1) return DSA_ERR_INVALID_ARG;
+  if (!aligned(qI, 16) || !aligned(codes, 16) || !aligned(w, 4) || !aligned(w_scaled, 4))
+    return DSA_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_index_query(reinterpret_cast<const __nv_bfloat16*>(qI), w, T, codes, w_scaled,
+                                                 (cudaStream_t)stream));
+}
+
+dsa_status_t dsa_index_scores(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
+                              const float* kI_scale, dsa_ki_dtype_t ki_dtype, float* scores, int64_t ld, void* ws,
+                              size_t ws_bytes, dsa_stream_t stream) {
+  g_launches = 0;
+  DSA_TRY(check_indexer_args(seqs, qI, w, kI, kI_scale, ki_dtype));
+  if (!scores || ld < seqs->max_ctx || !aligned(scores, 16)) return DSA_ERR_INVALID_ARG;
+  const Layout L = make_layout(DSA_OP_INDEX_SCORES, seqs->num_q_tokens, seqs->max_ctx, 1, 16);
+  DSA_TRY(check_ws(ws, ws_bytes, L.total));
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t* err = at<uint32_t>(ws, 0);
+  const SeqsDev sd = to_dev(seqs);
+  TokenMap tm{at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos)};
+  DSA_CUDA(launch_token_map(sd, at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos), err, st));
+  return run_indexer(seqs, sd, tm, qI, w, kI, kI_scale, ki_dtype, scores, ld, ws, L, err, st);
+}
+
+dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, int K, int32_t* idx, void* ws,
+                      size_t ws_bytes, dsa_stream_t stream) {
+  g_launches = 0;
+  if (!scores || !row_len || !idx || T < 1 || ld < 1) return DSA_ERR_INVALID_ARG;
+  if (K < 1 || K > kMaxK) return DSA_ERR_UNSUPPORTED;
+  if (ld > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (!aligned(scores, 16) || !aligned(row_len, 4) || !aligned(idx, 16)) return DSA_ERR_INVALID_ARG;
+  const Layout L = make_layout(DSA_OP_TOPK, T, (int)ld, K, 16);
+  DSA_TRY(check_ws(ws, ws_bytes, L.total));
+  return cuda_status(launch_topk(scores, ld, T, row_len, nullptr, K, idx, at<uint32_t>(ws, 0), (cudaStream_t)stream));
+}
+
+dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const void* kv, const int32_t* idx, int K,
+                                int H, float scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                                dsa_stream_t stream) {
+  g_launches = 0;
+  DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, lse));
+  if (!idx || !aligned(idx, 16)) return DSA_ERR_INVALID_ARG;
+  const Layout L = make_layout(DSA_OP_SPARSE_MLA, seqs->num_q_tokens, seqs->max_ctx, K, H);
+  DSA_TRY(check_ws(ws, ws_bytes, L.total));
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t* err = at<uint32_t>(ws, 0);
+  const SeqsDev sd = to_dev(seqs);
+  TokenMap tm{at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos)};
+  DSA_CUDA(launch_token_map(sd, at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos), err, st));
+  DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
+                             reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
+                             reinterpret_cast<__nv_bfloat16*>(out), lse, at<void>(ws, L.partials), err, st));
+  return DSA_OK;
+}
+
+dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
+                                 const float* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
+                                 int H, float scale, void* out, float* lse, int32_t* idx_out, void* ws,
+                                 size_t ws_bytes, dsa_stream_t stream) {
+  g_launches = 0;
+  DSA_TRY(check_indexer_args(seqs, qI, w, kI, kI_scale, ki_dtype));
+  DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, lse));
+  if (idx_out && !aligned(idx_out, 16)) return DSA_ERR_INVALID_ARG;
+  const Layout L = make_layout(DSA_OP_INDEX_TOPK_ATTN, seqs->num_q_tokens, seqs->max_ctx, K, H);
+  DSA_TRY(check_ws(ws, ws_bytes, L.total));
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t* err = at<uint32_t>(ws, 0);
+  const SeqsDev sd = to_dev(seqs);
+  TokenMap tm{at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos)};
+  float* scores = at<float>(ws, L.scores);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+  DSA_CUDA(launch_token_map(sd, at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos), err, st));
+  DSA_TRY(run_indexer(seqs, sd, tm, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, err, st));
+  DSA_CUDA(launch_topk(scores, L.ld, seqs->num_q_tokens, nullptr, tm.pos, K, idx, err, st));
+  DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
+                             reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
+                             reinterpret_cast<__nv_bfloat16*>(out), lse, at<void>(ws, L.partials), err, st));
+  return DSA_OK;
+}
+
+dsa_status_t dsa_check_error(void* ws, dsa_stream_t stream) {
+  if (!ws) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  uint32_t flag = 0;
+  if (cudaMemcpy(&flag, ws, sizeof(flag), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (flag) {
+    if (cudaMemsetAsync(ws, 0, sizeof(flag), st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  if (flag & kErrTimeout) return DSA_ERR_TIMEOUT;
+  if (flag & kErrBadIndex) return DSA_ERR_BAD_INDEX;
+  return DSA_OK;
+}
+
+int dsa_launches_in_last_call(void) { return g_launches; }
+
+const char* dsa_status_string(dsa_status_t s) {
+  switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_BAD_INDEX: return "DSA_ERR_BAD_INDEX";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+  }
+  return "DSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

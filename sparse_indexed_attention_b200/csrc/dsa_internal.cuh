@@ -1,0 +1,78 @@
+// Internal declarations shared by the libdsa translation units (not part of
+// the public ABI, which is include/dsa.h).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/dsa.h"
+
+namespace dsa {
+
+// Fixed sizes of the path (see include/dsa.h).
+constexpr int kPage = 64;        // tokens per page
+constexpr int kHI = 64;          // index heads
+constexpr int kDI = 128;         // index dim
+constexpr int kDQK = 576;        // latent key dims (512 latent + 64 rope)
+constexpr int kDV = 512;         // latent value dims
+constexpr int kMaxK = 2048;
+
+// Bits of the sticky device error word (first word of the workspace).
+constexpr uint32_t kErrBadIndex = 1u;
+constexpr uint32_t kErrTimeout = 2u;
+
+__device__ __forceinline__ void raise_error(uint32_t* err, uint32_t bit) {
+  if ((*(volatile uint32_t*)err & bit) == 0) atomicOr(err, bit);
+}
+
+// Per query token: its sequence and absolute position (-1 = invalid token).
+struct TokenMap {
+  const int32_t* seq;
+  const int32_t* pos;
+};
+
+// Physical pool row of logical position s of sequence b, or -1 (and the error
+// bit) when the page id is outside the pool.
+__device__ __forceinline__ int64_t phys_row(const int32_t* __restrict__ page_table, int max_pages,
+                                            int num_phys_pages, int b, int s, uint32_t* err) {
+  int page = __ldg(page_table + (int64_t)b * max_pages + (s >> 6));
+  if (page < 0 || page >= num_phys_pages) {
+    raise_error(err, kErrBadIndex);
+    return -1;
+  }
+  return (int64_t)page * kPage + (s & (kPage - 1));
+}
+
+// Device-side batch geometry passed by value to kernels.
+struct SeqsDev {
+  int batch, num_tokens, max_pages, num_phys_pages, max_ctx;
+  const int32_t* q_seq_start;
+  const int32_t* ctx_len;
+  const int32_t* page_table;
+};
+
+// Kernels launched by the current host thread since its last entry-point call
+// began (reported by dsa_launches_in_last_call).
+extern thread_local int g_launches;
+__host__ inline cudaError_t counted(cudaError_t e) {
+  if (e == cudaSuccess) ++g_launches;
+  return e;
+}
+
+// ---- launchers (each returns cudaGetLastError() of its launch) ----
+cudaError_t launch_token_map(const SeqsDev& s, int32_t* tok_seq, int32_t* tok_pos, uint32_t* err,
+                             cudaStream_t st);
+cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w, int T, uint8_t* codes,
+                                        float* w_scaled, cudaStream_t st);
+// FP8 cache: codes/w_scaled from the quantizer; bf16 cache: qI/w directly.
+cudaError_t launch_index_scores(const SeqsDev& s, TokenMap tm, const void* q_operand, const float* w_operand,
+                                const void* kI, const float* kI_scale, bool fp8, float* scores, int64_t ld,
+                                uint32_t* err, cudaStream_t st);
+cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, const int32_t* tok_pos,
+                        int K, int32_t* idx, uint32_t* err, cudaStream_t st);
+size_t sparse_mla_partials_bytes(int T, int K, int H);
+cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16* q, const __nv_bfloat16* kv,
+                              const int32_t* idx, int K, int H, float scale, __nv_bfloat16* out, float* lse,
+                              void* partials, uint32_t* err, cudaStream_t st);
+
+}  // namespace dsa

@@ -240,3 +240,36 @@ def make_workload(spec: Spec) -> Workload:
 def bits16(x: torch.Tensor) -> np.ndarray:
     """Raw 16-bit patterns of a bf16 CPU tensor (for the fp64 oracle)."""
     return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@dataclass
+class DeviceWorkload:
+    """A workload's tensors resident on one GPU, ready for the binding."""
+    wl: Workload
+    seqs: object                 # sparse_indexed_attention_b200.Seqs
+    qI: torch.Tensor
+    w: torch.Tensor
+    kI: torch.Tensor
+    kI_scale: torch.Tensor | None
+    q: torch.Tensor
+    kv: torch.Tensor
+
+    @property
+    def K(self) -> int:
+        return self.wl.spec.topk
+
+    @property
+    def scale(self) -> float:
+        return self.wl.scale
+
+    def h2d_bytes(self) -> int:
+        """Bytes of the per-step inputs (queries and batch metadata)."""
+        t = [self.qI, self.w, self.q, self.seqs.q_seq_start, self.seqs.ctx_len, self.seqs.page_table]
+        return sum(x.numel() * x.element_size() for x in t)
+
+
+def to_device(wl: Workload, device="cuda") -> DeviceWorkload:
+    from . import Seqs
+    seqs = Seqs.from_host(wl.q_seq_start, wl.ctx_len, wl.page_table, wl.num_phys_pages, device=device)
+    dev = lambda x: None if x is None else x.contiguous().to(device)  # noqa: E731
+    return DeviceWorkload(wl, seqs, dev(wl.qI), dev(wl.w), dev(wl.kI), dev(wl.kI_scale), dev(wl.q), dev(wl.kv))

@@ -1,0 +1,103 @@
+"""The C-ABI library without a GPU: it loads, exports every function that
+include/dsa.h declares, and its host-side validation answers before any
+launch.  No call here reaches a CUDA kernel."""
+import ctypes
+import os
+import re
+import subprocess
+
+import sparse_indexed_attention_b200 as dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"^[A-Za-z_][\w \*]*?\b(dsa_\w+)\s*\(", src, flags=re.M))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared()
+    assert {"dsa_index_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_index_topk_attn"} <= declared
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (dsa_\w+)", out))
+    assert declared <= exported, declared - exported
+    assert set(dsa.EXPORTS) == declared
+    lib = dsa.raw()
+    for name in declared:
+        assert getattr(lib, name) is not None
+
+
+def test_status_strings():
+    for code, name in enumerate(["DSA_OK", "DSA_ERR_INVALID_ARG", "DSA_ERR_UNSUPPORTED", "DSA_ERR_WORKSPACE",
+                                 "DSA_ERR_CUDA", "DSA_ERR_BAD_INDEX", "DSA_ERR_TIMEOUT"]):
+        assert dsa.status_string(code) == name
+    assert dsa.status_string(99) == "DSA_ERR_UNKNOWN"
+
+
+def _fake_seqs(T=4, B=1, max_ctx=100, page_size=64, max_pages=2, phys=8):
+    # host struct with non-null but never-dereferenced device pointers
+    fake = 0x10000
+    return dsa.DsaSeqsC(B, T, page_size, max_pages, phys, max_ctx, fake, fake, fake)
+
+
+def test_workspace_sizes():
+    lib = dsa.raw()
+    s = _fake_seqs(T=8, max_ctx=131072, max_pages=2048)
+    sz = {op: lib.dsa_workspace_size(op, ctypes.byref(s), 2048, 128) for op in range(5)}
+    assert sz[dsa.DSA_OP_QUANTIZE_INDEX_QUERY] == 0
+    assert sz[dsa.DSA_OP_INDEX_TOPK_ATTN] >= 8 * 131072 * 4 + 8 * 2048 * 4
+    assert all(v % 256 == 0 for v in sz.values())
+    assert lib.dsa_workspace_size(dsa.DSA_OP_SPARSE_MLA, ctypes.byref(s), 4096, 128) == 0     # K too large
+    assert lib.dsa_workspace_size(dsa.DSA_OP_SPARSE_MLA, ctypes.byref(s), 2048, 100) == 0     # bad H
+    assert lib.dsa_workspace_size(dsa.DSA_OP_TOPK, None, 16, 16) == 0
+
+
+def test_host_validation_rejects_before_launch():
+    lib = dsa.raw()
+    P = ctypes.c_void_p
+    good = P(0x10000)   # 256-aligned fake pointer, never dereferenced on these paths
+    s = _fake_seqs()
+    # dsa_topk
+    assert lib.dsa_topk(None, 128, 4, good, 16, good, good, 1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk(good, 128, 4, good, 0, good, good, 1 << 20, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_topk(good, 128, 4, good, 4096, good, good, 1 << 20, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_topk(good, 128, 4, good, 16, good, None, 1 << 20, None) == dsa.DSA_ERR_WORKSPACE
+    assert lib.dsa_topk(good, 128, 4, good, 16, good, P(0x10010), 1 << 20, None) == dsa.DSA_ERR_WORKSPACE
+    assert lib.dsa_topk(P(0x10004), 128, 4, good, 16, good, good, 1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
+    # dsa_sparse_mla_fwd
+    f = ctypes.c_float(0.04)
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 100, f, good, None, good, 1 << 20,
+                                  None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 128, ctypes.c_float(float("nan")), good,
+                                  None, good, 1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 128, f, good, None, good, 16,
+                                  None) == dsa.DSA_ERR_WORKSPACE
+    bad_ps = _fake_seqs(page_size=32)
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(bad_ps), good, good, good, 16, 128, f, good, None, good, 1 << 20,
+                                  None) == dsa.DSA_ERR_UNSUPPORTED
+    small_pt = _fake_seqs(max_ctx=200, max_pages=2)
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(small_pt), good, good, good, 16, 128, f, good, None, good, 1 << 20,
+                                  None) == dsa.DSA_ERR_INVALID_ARG
+    # dsa_index_scores: FP8 cache needs scales, bf16 cache must not have them
+    assert lib.dsa_index_scores(ctypes.byref(s), good, good, good, None, dsa.DSA_KI_FP8_E4M3, good, 128, good,
+                                1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_index_scores(ctypes.byref(s), good, good, good, good, dsa.DSA_KI_BF16, good, 128, good,
+                                1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_index_scores(ctypes.byref(s), good, good, good, None, dsa.DSA_KI_BF16, good, 64, good,
+                                1 << 20, None) == dsa.DSA_ERR_INVALID_ARG      # ld < max_ctx
+    assert lib.dsa_index_scores(ctypes.byref(s), good, good, P(0x10040), None, dsa.DSA_KI_BF16, good, 128, good,
+                                1 << 20, None) == dsa.DSA_ERR_INVALID_ARG      # pool not 128-B aligned
+    assert lib.dsa_index_scores(None, good, good, good, None, dsa.DSA_KI_BF16, good, 128, good, 1 << 20,
+                                None) == dsa.DSA_ERR_INVALID_ARG
+    # fused entry point
+    assert lib.dsa_index_topk_attn(ctypes.byref(s), good, good, good, None, dsa.DSA_KI_BF16, good, good, 0, 128, f,
+                                   good, None, None, good, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
+    # quantizer
+    assert lib.dsa_quantize_index_query(good, good, 0, good, good, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_check_error(None, None) == dsa.DSA_ERR_WORKSPACE

@@ -1,0 +1,52 @@
+"""dsa_index_topk_attn end to end: the selection criterion against the oracle's
+scores, and attention parity on every row whose index set equals the
+oracle's (the oracle never consumes a GPU result)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_oracle as O
+from sparse_indexed_attention_b200.workloads import bits16, to_device
+from tests import parity as P
+from tests.specs import FULL, SMALL, workload as make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _fused_check(lib, wl, tokens, min_agree=0.9):
+    d = to_device(wl)
+    K = wl.spec.topk
+    idx_out = torch.empty((wl.T, K), dtype=torch.int32, device="cuda")
+    out, lse = lib.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale,
+                                       idx_out=idx_out)
+    assert lib.dsa_check_error(lib.workspace(0, "cuda", "index_topk_attn")) == lib.DSA_OK
+    gidx = idx_out.cpu().numpy()
+    ref_rows = P.oracle_scores(wl, tokens)
+    agree = []
+    for t, r in zip(tokens, ref_rows):
+        bad = P.selection_violations(gidx[t], r, K)
+        assert not bad, f"token {t}: selection differs beyond near-ties: {bad[:8]}"
+        valid = gidx[t][gidx[t] >= 0]
+        assert np.all(np.diff(valid) > 0)                       # ascending, no duplicates
+        if np.array_equal(gidx[t], O.topk_select(r, K)):
+            agree.append(t)
+    assert len(agree) >= min_agree * len(tokens), f"{len(agree)}/{len(tokens)} rows with identical sets"
+    ref_idx = P.topk_idx_for(wl, [ref_rows[list(tokens).index(t)] for t in agree], agree)
+    ref_out, ref_lse = O.sparse_mla(P.oracle_seqs(wl), bits16(wl.q), bits16(wl.kv), ref_idx, wl.scale,
+                                    tokens=agree)
+    sel = torch.from_numpy(np.asarray(agree)).cuda()
+    P.assert_attention_close(out[sel], lse[sel], ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_fused_small(lib, name):
+    wl = make_workload(SMALL[name])
+    tokens = np.arange(wl.T) if wl.T <= 1100 else P.sample_tokens(wl, 64)
+    _fused_check(lib, wl, tokens)
+
+
+@pytest.mark.parametrize("name", ["decode_b8_128k", "decode_b64_8k_32k", "chunked_prefill_16", "long_prefill_32k"])
+def test_fused_full_size(lib, name):
+    wl = make_workload(FULL[name])
+    tokens = np.arange(wl.T) if wl.T <= 8 else P.sample_tokens(wl, 24)
+    _fused_check(lib, wl, tokens)

@@ -1,0 +1,71 @@
+"""dsa_topk against the oracle on identical fp32 scores: bit-exact index arrays."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(lib, scores_np, row_len_np, K):
+    scores = torch.from_numpy(scores_np).cuda()
+    row_len = torch.from_numpy(row_len_np.astype(np.int32)).cuda()
+    idx = lib.dsa_topk(scores, row_len, K).cpu().numpy()
+    for t in range(scores_np.shape[0]):
+        ref = O.topk_select(scores_np[t, : row_len_np[t]], K)
+        assert np.array_equal(idx[t], ref), (t, int(row_len_np[t]), K,
+                                              np.nonzero(idx[t] != ref)[0][:8])
+
+
+def test_random_rows_all_lengths(lib):
+    rng = np.random.default_rng(0)
+    T, ld = 24, 5004
+    s = rng.standard_normal((T, ld)).astype(np.float32)
+    lens = rng.integers(1, ld + 1, T)
+    lens[:4] = [1, 255, 256, 257]
+    for K in (1, 7, 256, 2048):
+        _run(lib, s, lens, K)
+
+
+def test_ties_and_signed_zero(lib):
+    rng = np.random.default_rng(1)
+    T, ld = 16, 3000
+    s = rng.integers(-2, 3, (T, ld)).astype(np.float32)
+    s[s == 0] = np.where(rng.random(np.count_nonzero(s == 0)) < 0.5, -0.0, 0.0).astype(np.float32)
+    s[3] = 1.5                                    # one value everywhere
+    s[4] = -0.0
+    s[5, ::2] = 0.0
+    s[5, 1::2] = -0.0
+    lens = np.full(T, ld)
+    lens[6] = 2047
+    lens[7] = 2048
+    lens[8] = 2049
+    for K in (1, 100, 2048):
+        _run(lib, s, lens, K)
+
+
+def test_index_like_distributions(lib):
+    rng = np.random.default_rng(2)
+    # ReLU-sum-like rows: a spike of exact zeros, a positive tail, a few planted
+    T, ld = 8, 131072
+    s = np.maximum(rng.standard_normal((T, ld)), 0).astype(np.float32) * rng.random((T, ld)).astype(np.float32)
+    s[:, rng.choice(ld, 64, replace=False)] += 50.0
+    s[2] = np.abs(s[2])
+    s[3, :100000] = 0.0
+    _run(lib, s, np.full(T, ld), 2048)
+    # causal prefill rows of a long sequence
+    T, ld = 48, 32768
+    s = (rng.standard_normal((T, ld)) * 3).astype(np.float32)
+    lens = np.sort(rng.integers(1, ld + 1, T))
+    _run(lib, s, lens, 2048)
+
+
+def test_denormals_and_extremes(lib):
+    rng = np.random.default_rng(3)
+    T, ld = 6, 4096
+    s = (rng.standard_normal((T, ld)) * 1e-40).astype(np.float32)   # subnormals
+    s[1] = rng.choice(np.array([np.float32(3.0e38), np.float32(-3.0e38), np.float32(1e-45)]), ld)
+    s[2] = np.float32(np.inf)
+    s[2, ::3] = -np.inf
+    _run(lib, s, np.full(T, ld), 1000)
