@@ -44,7 +44,8 @@
  *   64, 128}.  1 <= K <= 2048.  Anything else returns DSA_ERR_UNSUPPORTED.
  * Layouts.  Row-major, densely packed unless a leading dimension is given:
  *   qI [T,64,128] bf16, w [T,64] fp32, q [T,H,576] bf16, out [T,H,512] bf16,
- *   lse [T,H] fp32, idx [T,K] int32, scores [T,ld] fp32.
+ *   lse [T,H] fp32, idx [T,K] int32, scores [T,ld] fp32; out is bf16 or fp32
+ *   (dsa_out_dtype_t).
  * Memory.  Every pointer argument is DEVICE memory owned by the caller; the
  *   library allocates nothing, keeps no state between calls and never
  *   synchronises the stream except inside dsa_check_error.  Device pointers
@@ -91,6 +92,11 @@ typedef enum {
   DSA_KI_BF16 = 0,     /* kI pool is bf16 [R,128]; kI_scale must be NULL         */
   DSA_KI_FP8_E4M3 = 1  /* kI pool is OCP E4M3 codes [R,128] + fp32 kI_scale [R] */
 } dsa_ki_dtype_t;
+
+typedef enum {
+  DSA_OUT_BF16 = 0,    /* attention output stored as bf16 (rounded to nearest even) */
+  DSA_OUT_F32 = 1      /* attention output stored as fp32 (no output rounding)      */
+} dsa_out_dtype_t;
 
 typedef enum {
   DSA_OP_QUANTIZE_INDEX_QUERY = 0,
@@ -178,10 +184,12 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld, int T,
  * idx [T,K] holds logical positions 0..pos(t) of token t's sequence, -1 =
  * unused slot, any order, no duplicates; at least one valid entry per row.
  * An entry outside -1..pos(t) sets DSA_ERR_BAD_INDEX and is skipped.
- *   q bf16 [T,H,576]; kv bf16 pool [R,576]; out bf16 [T,H,512] (out). */
+ *   q bf16 [T,H,576]; kv bf16 pool [R,576]; out [T,H,512] (out) of
+ *   out_dtype (bf16 or fp32; the arithmetic is the same, fp32 accumulation). */
 dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t *seqs, const void *q,
                                 const void *kv, const int32_t *idx, int K,
-                                int H, float scale, void *out, float *lse,
+                                int H, float scale, void *out,
+                                dsa_out_dtype_t out_dtype, float *lse,
                                 void *ws, size_t ws_bytes, dsa_stream_t stream);
 
 /* The whole path in one call ([P1] Layer 1, "Sparse attention": scoring,
@@ -193,7 +201,8 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t *seqs, const void *qI,
                                  const float *w, const void *kI,
                                  const float *kI_scale, dsa_ki_dtype_t ki_dtype,
                                  const void *q, const void *kv, int K, int H,
-                                 float scale, void *out, float *lse,
+                                 float scale, void *out,
+                                 dsa_out_dtype_t out_dtype, float *lse,
                                  int32_t *idx_out, void *ws, size_t ws_bytes,
                                  dsa_stream_t stream);
 

@@ -31,6 +31,7 @@ LIB_PATH = _build.LIB
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_BAD_INDEX, \
     DSA_ERR_TIMEOUT = range(7)
 DSA_KI_BF16, DSA_KI_FP8_E4M3 = 0, 1
+DSA_OUT_BF16, DSA_OUT_F32 = 0, 1
 DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_INDEX_TOPK_ATTN = range(5)
 
 # Names the C header declares (checked against include/dsa.h by the tests).
@@ -52,9 +53,10 @@ _sig = {
     "dsa_quantize_index_query": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, _P]),
     "dsa_index_scores": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _I64, _P, _SZ, _P]),
     "dsa_topk": (ctypes.c_int, [_P, _I64, ctypes.c_int, _P, ctypes.c_int, _P, _P, _SZ, _P]),
-    "dsa_sparse_mla_fwd": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, ctypes.c_int, _F, _P, _P, _P, _SZ, _P]),
+    "dsa_sparse_mla_fwd": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, ctypes.c_int, _F, _P, ctypes.c_int, _P, _P,
+                                          _SZ, _P]),
     "dsa_index_topk_attn": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
-                                           _F, _P, _P, _P, _P, _SZ, _P]),
+                                           _F, _P, ctypes.c_int, _P, _P, _P, _SZ, _P]),
     "dsa_check_error": (ctypes.c_int, [_P, _P]),
     "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dsa_launches_in_last_call": (ctypes.c_int, []),
@@ -181,24 +183,34 @@ def dsa_topk(scores: torch.Tensor, row_len: torch.Tensor, K: int, idx=None, ws=N
     return idx
 
 
-def dsa_sparse_mla_fwd(seqs: Seqs, q, kv, idx, scale: float, out=None, lse=None, want_lse=True, ws=None):
+def _out_dtype(out: torch.Tensor) -> int:
+    if out.dtype == torch.bfloat16:
+        return DSA_OUT_BF16
+    if out.dtype == torch.float32:
+        return DSA_OUT_F32
+    raise TypeError("out must be bfloat16 or float32")
+
+
+def dsa_sparse_mla_fwd(seqs: Seqs, q, kv, idx, scale: float, out=None, lse=None, want_lse=True, ws=None,
+                       out_dtype=torch.bfloat16):
     T, H, _ = q.shape
     K = idx.shape[1]
-    out = out if out is not None else torch.empty((T, H, 512), dtype=torch.bfloat16, device=q.device)
+    out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
     c = seqs.c()
     need = _lib.dsa_workspace_size(DSA_OP_SPARSE_MLA, ctypes.byref(c), K, H)
     ws = ws if ws is not None else workspace(need, q.device, "sparse_mla")
-    _check(_lib.dsa_sparse_mla_fwd(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(idx), K, H, scale, _ptr(out), _ptr(lse),
-                                   _ptr(ws), ws.numel(), _stream(q.device)), "dsa_sparse_mla_fwd")
+    _check(_lib.dsa_sparse_mla_fwd(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(idx), K, H, scale, _ptr(out),
+                                   _out_dtype(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)),
+           "dsa_sparse_mla_fwd")
     return out, lse
 
 
 def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: float, out=None, lse=None,
-                        idx_out=None, want_lse=True, ws=None):
+                        idx_out=None, want_lse=True, ws=None, out_dtype=torch.bfloat16):
     T, H, _ = q.shape
-    out = out if out is not None else torch.empty((T, H, 512), dtype=torch.bfloat16, device=q.device)
+    out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
     ki_dtype = DSA_KI_FP8_E4M3 if kI_scale is not None else DSA_KI_BF16
@@ -206,8 +218,8 @@ def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: f
     need = _lib.dsa_workspace_size(DSA_OP_INDEX_TOPK_ATTN, ctypes.byref(c), K, H)
     ws = ws if ws is not None else workspace(need, q.device, "index_topk_attn")
     _check(_lib.dsa_index_topk_attn(ctypes.byref(c), _ptr(qI), _ptr(w), _ptr(kI), _ptr(kI_scale), ki_dtype, _ptr(q),
-                                    _ptr(kv), K, H, scale, _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(ws), ws.numel(),
-                                    _stream(q.device)), "dsa_index_topk_attn")
+                                    _ptr(kv), K, H, scale, _ptr(out), _out_dtype(out), _ptr(lse), _ptr(idx_out),
+                                    _ptr(ws), ws.numel(), _stream(q.device)), "dsa_index_topk_attn")
     return out, lse
 
 

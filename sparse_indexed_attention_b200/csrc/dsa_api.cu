@@ -109,8 +109,9 @@ dsa_status_t check_indexer_args(const dsa_seqs_t* seqs, const void* qI, const fl
 }
 
 dsa_status_t check_attn_args(const dsa_seqs_t* seqs, const void* q, const void* kv, int K, int H, float scale,
-                             const void* out, const float* lse) {
+                             const void* out, dsa_out_dtype_t out_dtype, const float* lse) {
   DSA_TRY(check_seqs(seqs));
+  if (out_dtype != DSA_OUT_BF16 && out_dtype != DSA_OUT_F32) return DSA_ERR_UNSUPPORTED;
   if (!q || !kv || !out) return DSA_ERR_INVALID_ARG;
   if (K < 1 || K > kMaxK || !valid_H(H)) return DSA_ERR_UNSUPPORTED;
   if (!std::isfinite(scale)) return DSA_ERR_INVALID_ARG;
@@ -190,10 +191,10 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row
 }
 
 dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const void* kv, const int32_t* idx, int K,
-                                int H, float scale, void* out, float* lse, void* ws, size_t ws_bytes,
-                                dsa_stream_t stream) {
+                                int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse, void* ws,
+                                size_t ws_bytes, dsa_stream_t stream) {
   g_launches = 0;
-  DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, lse));
+  DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, out_dtype, lse));
   if (!idx || !aligned(idx, 16)) return DSA_ERR_INVALID_ARG;
   const Layout L = make_layout(DSA_OP_SPARSE_MLA, seqs->num_q_tokens, seqs->max_ctx, K, H);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
@@ -204,17 +205,17 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const voi
   DSA_CUDA(launch_token_map(sd, at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos), err, st));
   DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
-                             reinterpret_cast<__nv_bfloat16*>(out), lse, at<void>(ws, L.partials), err, st));
+                             out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
   return DSA_OK;
 }
 
 dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
                                  const float* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
-                                 int H, float scale, void* out, float* lse, int32_t* idx_out, void* ws,
-                                 size_t ws_bytes, dsa_stream_t stream) {
+                                 int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse,
+                                 int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
   g_launches = 0;
   DSA_TRY(check_indexer_args(seqs, qI, w, kI, kI_scale, ki_dtype));
-  DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, lse));
+  DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, out_dtype, lse));
   if (idx_out && !aligned(idx_out, 16)) return DSA_ERR_INVALID_ARG;
   const Layout L = make_layout(DSA_OP_INDEX_TOPK_ATTN, seqs->num_q_tokens, seqs->max_ctx, K, H);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
@@ -229,7 +230,7 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const f
   DSA_CUDA(launch_topk(scores, L.ld, seqs->num_q_tokens, nullptr, tm.pos, K, idx, err, st));
   DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
-                             reinterpret_cast<__nv_bfloat16*>(out), lse, at<void>(ws, L.partials), err, st));
+                             out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
   return DSA_OK;
 }
 

@@ -72,7 +72,7 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* r
                         int K, int32_t* idx, uint32_t* err, cudaStream_t st);
 size_t sparse_mla_partials_bytes(int T, int K, int H);
 cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16* q, const __nv_bfloat16* kv,
-                              const int32_t* idx, int K, int H, float scale, __nv_bfloat16* out, float* lse,
-                              void* partials, uint32_t* err, cudaStream_t st);
+                              const int32_t* idx, int K, int H, float scale, void* out, bool out_f32,
+                              float* lse, void* partials, uint32_t* err, cudaStream_t st);
 
 }  // namespace dsa

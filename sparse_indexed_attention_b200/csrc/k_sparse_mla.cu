@@ -33,6 +33,13 @@ struct SmemLayout {
   int64_t row[kChunk];
 };
 
+__device__ __forceinline__ void store_out(void* out, bool f32, int64_t i, float v) {
+  if (f32)
+    reinterpret_cast<float*>(out)[i] = v;
+  else
+    reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16(v);
+}
+
 int attn_splits(int T, int H, int K) {
   int ctas = T * (H / kHG);
   int splits = 1;
@@ -52,7 +59,7 @@ int keys_per_split(int K, int splits) {
 __global__ void __launch_bounds__(kThreads)
 k_sparse_mla_simple(SeqsDev s, TokenMap tm, const __nv_bfloat16* __restrict__ q,
                     const __nv_bfloat16* __restrict__ kv, const int32_t* __restrict__ idx, int K, int H,
-                    float scale, int ks, int splits, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                    float scale, int ks, int splits, void* __restrict__ out, bool out_f32, float* __restrict__ lse,
                     float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SmemLayout& sm = *reinterpret_cast<SmemLayout*>(smem_raw);
@@ -167,8 +174,8 @@ k_sparse_mla_simple(SeqsDev s, TokenMap tm, const __nv_bfloat16* __restrict__ q,
       const float l = sm.l[h];
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int64_t o = ((int64_t)t * H + hg * kHG + h) * kDV;
-      out[o + tid] = __float2bfloat16(acc[h][0] * inv);
-      out[o + tid + 256] = __float2bfloat16(acc[h][1] * inv);
+      store_out(out, out_f32, o + tid, acc[h][0] * inv);
+      store_out(out, out_f32, o + tid + 256, acc[h][1] * inv);
     }
     if (lse && tid < kHG) lse[(int64_t)t * H + hg * kHG + tid] = sm.m[tid] + logf(sm.l[tid]);
   } else {
@@ -185,7 +192,7 @@ k_sparse_mla_simple(SeqsDev s, TokenMap tm, const __nv_bfloat16* __restrict__ q,
 // Merge the split partials of one (token, head): rescale to the common max.
 __global__ void __launch_bounds__(128)
 k_combine(int H, int splits, const float* __restrict__ part_o, const float2* __restrict__ part_ml,
-          const int32_t* __restrict__ tok_pos, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+          const int32_t* __restrict__ tok_pos, void* __restrict__ out, bool out_f32, float* __restrict__ lse) {
   const int t = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   if (tok_pos[t] < 0) return;
   float M = -INFINITY;
@@ -203,11 +210,9 @@ k_combine(int H, int splits, const float* __restrict__ part_o, const float2* __r
     o[3] += v.w * f;
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
-  __nv_bfloat16* dst = out + ((int64_t)t * H + h) * kDV + tid * 4;
-  dst[0] = __float2bfloat16(o[0] * inv);
-  dst[1] = __float2bfloat16(o[1] * inv);
-  dst[2] = __float2bfloat16(o[2] * inv);
-  dst[3] = __float2bfloat16(o[3] * inv);
+  const int64_t base = ((int64_t)t * H + h) * kDV + tid * 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) store_out(out, out_f32, base + i, o[i] * inv);
   if (lse && tid == 0) lse[(int64_t)t * H + h] = M + logf(L);
 }
 
@@ -220,8 +225,8 @@ size_t sparse_mla_partials_bytes(int T, int K, int H) {
 }
 
 cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16* q, const __nv_bfloat16* kv,
-                              const int32_t* idx, int K, int H, float scale, __nv_bfloat16* out, float* lse,
-                              void* partials, uint32_t* err, cudaStream_t st) {
+                              const int32_t* idx, int K, int H, float scale, void* out, bool out_f32,
+                              float* lse, void* partials, uint32_t* err, cudaStream_t st) {
   const int T = s.num_tokens;
   int splits = attn_splits(T, H, K);
   const int ks = keys_per_split(K, splits);
@@ -239,11 +244,11 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16
     attr_set_for = dev;
   }
   dim3 grid(T, H / kHG, splits);
-  k_sparse_mla_simple<<<grid, kThreads, smem, st>>>(s, tm, q, kv, idx, K, H, scale, ks, splits, out, lse, part_o,
+  k_sparse_mla_simple<<<grid, kThreads, smem, st>>>(s, tm, q, kv, idx, K, H, scale, ks, splits, out, out_f32, lse, part_o,
                                                      part_ml, err);
   e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
-  k_combine<<<dim3(T, H), 128, 0, st>>>(H, splits, part_o, part_ml, tm.pos, out, lse);
+  k_combine<<<dim3(T, H), 128, 0, st>>>(H, splits, part_o, part_ml, tm.pos, out, out_f32, lse);
   return counted(cudaGetLastError());
 }
 

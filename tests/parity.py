@@ -8,7 +8,10 @@ Tolerances (written here once, used by every GPU test):
   * end-to-end selection: every position in the symmetric difference of the
     GPU and oracle index sets has |ref_score - tau| <= 1e-3 * |tau|, tau = the
     oracle's K-th largest score of the row; rows with n <= K must match exactly;
-  * attention output: max |gpu - ref| <= 1e-2 * rms(ref) over the whole output;
+  * attention output: max |gpu - ref| <= 1e-2 * rms(ref) over the whole output
+    for fp32 output; a bf16 output may in addition differ by the half ulp of
+    bf16 at |ref| that storing in bf16 costs (that rounding belongs to the
+    output format: with max|out| above ~2.5 rms it alone exceeds 1e-2 rms);
     lse: |gpu - ref| <= 1e-3 * max(1, |ref|).
 """
 from __future__ import annotations
@@ -77,12 +80,24 @@ def selection_violations(gpu_idx_row, ref_row, K):
     return bad
 
 
+def bf16_half_ulp(x):
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.exp2(e - 8)
+
+
 def assert_attention_close(gpu_out, gpu_lse, ref_out, ref_lse):
     ref_out = np.asarray(ref_out)
     g = gpu_out.float().cpu().numpy().astype(np.float64)
     rms = float(np.sqrt(np.mean(ref_out * ref_out)))
-    err = float(np.max(np.abs(g - ref_out)))
-    assert err <= OUT_TOL * rms, f"attention max err {err:.3e} vs rms {rms:.3e}"
+    diff = np.abs(g - ref_out)
+    if gpu_out.dtype == torch.float32:
+        err = float(diff.max())
+        assert err <= OUT_TOL * rms, f"attention (fp32 out) max err {err:.3e} vs rms {rms:.3e}"
+    else:
+        excess = diff - bf16_half_ulp(ref_out)
+        err = float(excess.max())
+        assert err <= OUT_TOL * rms, f"attention (bf16 out) max err beyond half-ulp {err:.3e} vs rms {rms:.3e}"
     if gpu_lse is not None:
         gl = gpu_lse.cpu().numpy().astype(np.float64)
         lerr = np.abs(gl - ref_lse) / np.maximum(1.0, np.abs(ref_lse))

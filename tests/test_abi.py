@@ -72,18 +72,21 @@ def test_host_validation_rejects_before_launch():
     assert lib.dsa_topk(P(0x10004), 128, 4, good, 16, good, good, 1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
     # dsa_sparse_mla_fwd
     f = ctypes.c_float(0.04)
-    assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 100, f, good, None, good, 1 << 20,
+    B16 = dsa.DSA_OUT_BF16
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 100, f, good, B16, None, good, 1 << 20,
                                   None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 128, f, good, 7, None, good, 1 << 20,
+                                  None) == dsa.DSA_ERR_UNSUPPORTED                  # unknown output dtype
     assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 128, ctypes.c_float(float("nan")), good,
-                                  None, good, 1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
-    assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 128, f, good, None, good, 16,
+                                  B16, None, good, 1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(s), good, good, good, 16, 128, f, good, B16, None, good, 16,
                                   None) == dsa.DSA_ERR_WORKSPACE
     bad_ps = _fake_seqs(page_size=32)
-    assert lib.dsa_sparse_mla_fwd(ctypes.byref(bad_ps), good, good, good, 16, 128, f, good, None, good, 1 << 20,
-                                  None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(bad_ps), good, good, good, 16, 128, f, good, B16, None, good,
+                                  1 << 20, None) == dsa.DSA_ERR_UNSUPPORTED
     small_pt = _fake_seqs(max_ctx=200, max_pages=2)
-    assert lib.dsa_sparse_mla_fwd(ctypes.byref(small_pt), good, good, good, 16, 128, f, good, None, good, 1 << 20,
-                                  None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_sparse_mla_fwd(ctypes.byref(small_pt), good, good, good, 16, 128, f, good, B16, None, good,
+                                  1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
     # dsa_index_scores: FP8 cache needs scales, bf16 cache must not have them
     assert lib.dsa_index_scores(ctypes.byref(s), good, good, good, None, dsa.DSA_KI_FP8_E4M3, good, 128, good,
                                 1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
@@ -97,7 +100,7 @@ def test_host_validation_rejects_before_launch():
                                 None) == dsa.DSA_ERR_INVALID_ARG
     # fused entry point
     assert lib.dsa_index_topk_attn(ctypes.byref(s), good, good, good, None, dsa.DSA_KI_BF16, good, good, 0, 128, f,
-                                   good, None, None, good, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
+                                   good, B16, None, None, good, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
     # quantizer
     assert lib.dsa_quantize_index_query(good, good, 0, good, good, None) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_check_error(None, None) == dsa.DSA_ERR_WORKSPACE

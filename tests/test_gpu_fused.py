@@ -13,12 +13,12 @@ from tests.specs import FULL, SMALL, workload as make_workload
 pytestmark = pytest.mark.gpu
 
 
-def _fused_check(lib, wl, tokens, min_agree=0.9):
+def _fused_check(lib, wl, tokens, min_agree=0.9, out_dtype=torch.bfloat16):
     d = to_device(wl)
     K = wl.spec.topk
     idx_out = torch.empty((wl.T, K), dtype=torch.int32, device="cuda")
     out, lse = lib.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale,
-                                       idx_out=idx_out)
+                                       idx_out=idx_out, out_dtype=out_dtype)
     assert lib.dsa_check_error(lib.workspace(0, "cuda", "index_topk_attn")) == lib.DSA_OK
     gidx = idx_out.cpu().numpy()
     ref_rows = P.oracle_scores(wl, tokens)
@@ -42,7 +42,8 @@ def _fused_check(lib, wl, tokens, min_agree=0.9):
 def test_fused_small(lib, name):
     wl = make_workload(SMALL[name])
     tokens = np.arange(wl.T) if wl.T <= 1100 else P.sample_tokens(wl, 64)
-    _fused_check(lib, wl, tokens)
+    _fused_check(lib, wl, tokens, out_dtype=torch.float32)
+    _fused_check(lib, wl, tokens, out_dtype=torch.bfloat16)
 
 
 @pytest.mark.parametrize("name", ["decode_b8_128k", "decode_b64_8k_32k", "chunked_prefill_16", "long_prefill_32k"])
