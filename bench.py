@@ -347,6 +347,7 @@ def run_ours(args, world, rank, local):
                "sample": f"fp64 oracle, whole path for all {T} query tokens (ctx {int(wl.ctx_len[0])}), "
                          f"{reps} batch(es), {spent:.1f} s"}
 
+    launch_mode = "cuda graph replay" if graph is not None else "eager"
     if graph is not None:
         del graph
     if rank == 0:
@@ -359,7 +360,7 @@ def run_ours(args, world, rank, local):
                        "ctx": int(wl.ctx_len[0]), "topk": K, "heads": H, "index_heads": 64, "index_dim": 128,
                        "page_size": 64, "pool_tokens": wl.num_phys_pages * 64, "parallelism": f"dp{world}",
                        "l2": "256 MiB buffer written before every timed step",
-                       "launch": "cuda graph replay" if graph is not None else "eager"},
+                       "launch": launch_mode},
             "stages_us": {"index_scores": ms_idx * 1e3, "topk": statistics.mean(t_topk) * 1e3,
                           "sparse_mla": statistics.mean(t_attn) * 1e3},
             "roofline": {"kernel": "index_scores (quantize + score)", "bound": "hbm", "achieved": achieved,

@@ -21,25 +21,36 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // Workspace carve-up.  Offsets are 256-byte aligned; the first 256 bytes hold
 // the sticky error word.
 struct Layout {
-  size_t tok_seq = 0, tok_pos = 0, q_codes = 0, w_scaled = 0, scores = 0, idx = 0, partials = 0;
+  size_t tok_seq = 0, tok_pos = 0, seq_gstart = 0, groups = 0, items = 0, counts = 0;
+  size_t q_codes = 0, w_scaled = 0, scores = 0, idx = 0, partials = 0;
   size_t total = 0;
   int64_t ld = 0;
 };
 
-Layout make_layout(dsa_op_t op, int T, int max_ctx, int K, int H) {
+// The indexer's work-list capacity must hold for either index-cache dtype, so
+// it is sized for the smaller group (more groups, more items).
+int sizing_group_tokens(int T, int B) { return T == B ? 1 : 2; }
+
+Layout make_layout(dsa_op_t op, int T, int B, int max_ctx, int K, int H) {
   Layout L;
-  size_t off = kAlign;  // header
+  size_t off = kAlign;  // header: the sticky error word
   auto take = [&](size_t bytes) {
     size_t o = off;
     off = align_up(off + bytes);
     return o;
   };
   const bool seq_ops = op == DSA_OP_INDEX_SCORES || op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN;
+  const bool indexer = op == DSA_OP_INDEX_SCORES || op == DSA_OP_INDEX_TOPK_ATTN;
   if (seq_ops) {
     L.tok_seq = take((size_t)T * sizeof(int32_t));
     L.tok_pos = take((size_t)T * sizeof(int32_t));
+    L.seq_gstart = take((size_t)(B + 1) * sizeof(int32_t));
+    L.counts = take(4 * sizeof(int32_t));
   }
-  if (op == DSA_OP_INDEX_SCORES || op == DSA_OP_INDEX_TOPK_ATTN) {
+  if (indexer) {
+    const int tg = sizing_group_tokens(T, B);
+    L.groups = take((size_t)plan_max_groups(T, B, tg) * sizeof(int4));
+    L.items = take((size_t)plan_max_items(T, B, max_ctx, tg) * sizeof(int4));
     L.q_codes = take((size_t)T * kHI * kDI);
     L.w_scaled = take((size_t)T * kHI * sizeof(float));
   }
@@ -120,10 +131,22 @@ dsa_status_t check_attn_args(const dsa_seqs_t* seqs, const void* q, const void* 
   return DSA_OK;
 }
 
+PlanBufs plan_bufs(void* ws, const Layout& L) {
+  PlanBufs p;
+  p.tok_seq = at<int32_t>(ws, L.tok_seq);
+  p.tok_pos = at<int32_t>(ws, L.tok_pos);
+  p.seq_gstart = at<int32_t>(ws, L.seq_gstart);
+  p.groups = L.groups ? at<int4>(ws, L.groups) : nullptr;
+  p.items = L.items ? at<int4>(ws, L.items) : nullptr;
+  p.counts = at<int32_t>(ws, L.counts);
+  return p;
+}
+
 // indexer launch sequence shared by dsa_index_scores and the fused call
-dsa_status_t run_indexer(const dsa_seqs_t* seqs, const SeqsDev& sd, TokenMap tm, const void* qI, const float* w,
-                         const void* kI, const float* kI_scale, dsa_ki_dtype_t ki_dtype, float* scores,
-                         int64_t ld, void* ws, const Layout& L, uint32_t* err, cudaStream_t st) {
+// (the plan has already been launched)
+dsa_status_t run_indexer(const dsa_seqs_t* seqs, const SeqsDev& sd, const PlanBufs& plan, int tg, const void* qI,
+                         const float* w, const void* kI, const float* kI_scale, dsa_ki_dtype_t ki_dtype,
+                         float* scores, int64_t ld, void* ws, const Layout& L, uint32_t* err, cudaStream_t st) {
   const bool fp8 = ki_dtype == DSA_KI_FP8_E4M3;
   const void* q_operand = qI;
   const float* w_operand = w;
@@ -135,7 +158,7 @@ dsa_status_t run_indexer(const dsa_seqs_t* seqs, const SeqsDev& sd, TokenMap tm,
     q_operand = codes;
     w_operand = w_scaled;
   }
-  DSA_CUDA(launch_index_scores(sd, tm, q_operand, w_operand, kI, kI_scale, fp8, scores, ld, err, st));
+  DSA_CUDA(launch_index_scores(sd, plan, tg, q_operand, w_operand, kI, kI_scale, fp8, scores, ld, err, st));
   return DSA_OK;
 }
 
@@ -146,10 +169,11 @@ extern "C" {
 size_t dsa_workspace_size(dsa_op_t op, const dsa_seqs_t* seqs, int K, int H) {
   if (!seqs || seqs->num_q_tokens < 1 || seqs->max_ctx < 1) return 0;
   if (op == DSA_OP_QUANTIZE_INDEX_QUERY) return 0;
-  if (op == DSA_OP_TOPK) return make_layout(op, seqs->num_q_tokens, seqs->max_ctx, K, 16).total;
+  if (op == DSA_OP_TOPK) return make_layout(op, seqs->num_q_tokens, 1, seqs->max_ctx, K, 16).total;
   if (op < 0 || op > DSA_OP_INDEX_TOPK_ATTN) return 0;
+  if (seqs->batch < 1) return 0;
   if ((op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN) && (K < 1 || K > kMaxK || !valid_H(H))) return 0;
-  return make_layout(op, seqs->num_q_tokens, seqs->max_ctx, K, H).total;
+  return make_layout(op, seqs->num_q_tokens, seqs->batch, seqs->max_ctx, K, H).total;
 }
 
 dsa_status_t dsa_quantize_index_query(const void* qI, const float* w, int T, uint8_t* codes, float* w_scaled,
@@ -168,14 +192,15 @@ dsa_status_t dsa_index_scores(const dsa_seqs_t* seqs, const void* qI, const floa
   g_launches = 0;
   DSA_TRY(check_indexer_args(seqs, qI, w, kI, kI_scale, ki_dtype));
   if (!scores || ld < seqs->max_ctx || !aligned(scores, 16)) return DSA_ERR_INVALID_ARG;
-  const Layout L = make_layout(DSA_OP_INDEX_SCORES, seqs->num_q_tokens, seqs->max_ctx, 1, 16);
+  const Layout L = make_layout(DSA_OP_INDEX_SCORES, seqs->num_q_tokens, seqs->batch, seqs->max_ctx, 1, 16);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = (cudaStream_t)stream;
   uint32_t* err = at<uint32_t>(ws, 0);
   const SeqsDev sd = to_dev(seqs);
-  TokenMap tm{at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos)};
-  DSA_CUDA(launch_token_map(sd, at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos), err, st));
-  return run_indexer(seqs, sd, tm, qI, w, kI, kI_scale, ki_dtype, scores, ld, ws, L, err, st);
+  const PlanBufs plan = plan_bufs(ws, L);
+  const int tg = indexer_group_tokens(seqs->num_q_tokens, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
+  DSA_CUDA(launch_plan(sd, tg, indexer_item_tiles(tg), plan, err, st));
+  return run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, ld, ws, L, err, st);
 }
 
 dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, int K, int32_t* idx, void* ws,
@@ -185,7 +210,7 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row
   if (K < 1 || K > kMaxK) return DSA_ERR_UNSUPPORTED;
   if (ld > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   if (!aligned(scores, 16) || !aligned(row_len, 4) || !aligned(idx, 16)) return DSA_ERR_INVALID_ARG;
-  const Layout L = make_layout(DSA_OP_TOPK, T, (int)ld, K, 16);
+  const Layout L = make_layout(DSA_OP_TOPK, T, 1, (int)ld, K, 16);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
   return cuda_status(launch_topk(scores, ld, T, row_len, nullptr, K, idx, at<uint32_t>(ws, 0), (cudaStream_t)stream));
 }
@@ -196,13 +221,14 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const voi
   g_launches = 0;
   DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, out_dtype, lse));
   if (!idx || !aligned(idx, 16)) return DSA_ERR_INVALID_ARG;
-  const Layout L = make_layout(DSA_OP_SPARSE_MLA, seqs->num_q_tokens, seqs->max_ctx, K, H);
+  const Layout L = make_layout(DSA_OP_SPARSE_MLA, seqs->num_q_tokens, seqs->batch, seqs->max_ctx, K, H);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = (cudaStream_t)stream;
   uint32_t* err = at<uint32_t>(ws, 0);
   const SeqsDev sd = to_dev(seqs);
-  TokenMap tm{at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos)};
-  DSA_CUDA(launch_token_map(sd, at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos), err, st));
+  const PlanBufs plan = plan_bufs(ws, L);
+  TokenMap tm{plan.tok_seq, plan.tok_pos};
+  DSA_CUDA(launch_plan(sd, 1, 0, plan, err, st));  // token geometry only
   DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
                              out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
@@ -217,16 +243,18 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const f
   DSA_TRY(check_indexer_args(seqs, qI, w, kI, kI_scale, ki_dtype));
   DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, out_dtype, lse));
   if (idx_out && !aligned(idx_out, 16)) return DSA_ERR_INVALID_ARG;
-  const Layout L = make_layout(DSA_OP_INDEX_TOPK_ATTN, seqs->num_q_tokens, seqs->max_ctx, K, H);
+  const Layout L = make_layout(DSA_OP_INDEX_TOPK_ATTN, seqs->num_q_tokens, seqs->batch, seqs->max_ctx, K, H);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = (cudaStream_t)stream;
   uint32_t* err = at<uint32_t>(ws, 0);
   const SeqsDev sd = to_dev(seqs);
-  TokenMap tm{at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos)};
+  const PlanBufs plan = plan_bufs(ws, L);
+  TokenMap tm{plan.tok_seq, plan.tok_pos};
   float* scores = at<float>(ws, L.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
-  DSA_CUDA(launch_token_map(sd, at<int32_t>(ws, L.tok_seq), at<int32_t>(ws, L.tok_pos), err, st));
-  DSA_TRY(run_indexer(seqs, sd, tm, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, err, st));
+  const int tg = indexer_group_tokens(seqs->num_q_tokens, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
+  DSA_CUDA(launch_plan(sd, tg, indexer_item_tiles(tg), plan, err, st));
+  DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, err, st));
   DSA_CUDA(launch_topk(scores, L.ld, seqs->num_q_tokens, nullptr, tm.pos, K, idx, err, st));
   DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,

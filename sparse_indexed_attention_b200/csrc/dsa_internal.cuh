@@ -59,15 +59,38 @@ __host__ inline cudaError_t counted(cudaError_t e) {
   return e;
 }
 
+// Work plan written by k_plan (see k_prep.cu).
+struct PlanBufs {
+  int32_t* tok_seq;     // [T]
+  int32_t* tok_pos;     // [T]
+  int32_t* seq_gstart;  // [B+1]
+  int4* groups;         // [max groups]  {b, t0, cnt, pos0}
+  int4* items;          // [max items]   {g, tile_begin, tile_end, 0}
+  int32_t* counts;      // {groups, items}
+};
+
+// Tokens per indexer group and key tiles per work item for a geometry.
+inline int indexer_group_tokens(int T, int B, bool fp8) { return T == B ? 1 : (fp8 ? 4 : 2); }
+inline int indexer_item_tiles(int tg) { return tg == 1 ? 4 : 16; }
+inline int64_t plan_max_groups(int T, int B, int tg) {
+  const int64_t g = (int64_t)T / tg + B;
+  return g < T ? g : T;
+}
+inline int64_t plan_max_items(int T, int B, int max_ctx, int tg) {
+  const int64_t G = plan_max_groups(T, B, tg);
+  const int64_t tiles = ((int64_t)max_ctx + 127) / 128;
+  const int ch = indexer_item_tiles(tg);
+  return G + (G * tiles + ch - 1) / ch;
+}
+
 // ---- launchers (each returns cudaGetLastError() of its launch) ----
-cudaError_t launch_token_map(const SeqsDev& s, int32_t* tok_seq, int32_t* tok_pos, uint32_t* err,
-                             cudaStream_t st);
+cudaError_t launch_plan(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err, cudaStream_t st);
 cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w, int T, uint8_t* codes,
                                         float* w_scaled, cudaStream_t st);
 // FP8 cache: codes/w_scaled from the quantizer; bf16 cache: qI/w directly.
-cudaError_t launch_index_scores(const SeqsDev& s, TokenMap tm, const void* q_operand, const float* w_operand,
-                                const void* kI, const float* kI_scale, bool fp8, float* scores, int64_t ld,
-                                uint32_t* err, cudaStream_t st);
+cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
+                                const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
+                                float* scores, int64_t ld, uint32_t* err, cudaStream_t st);
 cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, const int32_t* tok_pos,
                         int K, int32_t* idx, uint32_t* err, cudaStream_t st);
 size_t sparse_mla_partials_bytes(int T, int K, int H);

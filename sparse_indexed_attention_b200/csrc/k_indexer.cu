@@ -1,103 +1,361 @@
-// Lightweight-indexer scores ([P2] "Hybrid Attention LLM Inference
-// Acceleration...", section 2 item 2 and section 4(1); [P4] "Optimizing
-// Inference for Hybrid-Architecture Large Language Models...", section 3.1):
-//   score[t,s] = kI_scale[s] * sum_h w'[t,h] * ReLU(q^[t,h,:] . k^[s,:])
-// read straight from the paged index cache; the head reduction happens in
-// registers, so no [T, H_I, N] tensor is ever written.
+// Lightweight-indexer scores on the 5th-generation tensor cores
+// ([P2] "Hybrid Attention LLM Inference Acceleration...", section 2 item 2 and
+// section 4(1): scoring + head weighting read the paged K cache directly;
+// [P4] "Optimizing Inference for Hybrid-Architecture Large Language
+// Models...", section 3.1):
 //
-// Simple CUDA-core form: one thread per candidate key, the token's 64 x 128
-// query held in shared memory as fp32.
-#include <cuda_fp8.h>
+//   score[t,s] = kI_scale[s] * sum_h w'[t,h] * ReLU(q^[t,h,:] . k^[s,:])
+//
+// As a GEMM per (token group, key tile): D[s, (t,h)] = sum_d K[s,d] Q[(t,h),d]
+// with M = 128 keys (two 64-row pages), N = 64 heads x TG tokens, K = 128.
+//  * warp 0, one lane: TMA producer.  Each key tile is two TMA loads of one
+//    8 KB page each, straight from the paged pool (the page table is read
+//    here), plus a 256-byte bulk copy of each page's row scales.  The group's
+//    quantized query rows and head weights are loaded once per group.
+//  * warp 1, one lane: issues tcgen05.mma (kind::f8f6f4 E4M3, or kind::f16
+//    bf16) into a ring of TMEM accumulators; tcgen05.commit frees the stage
+//    and publishes the accumulator.
+//  * warp 2: allocates and frees TMEM.
+//  * warps 4-7: epilogue.  Thread r owns TMEM lane r = key row r, so the
+//    ReLU, the head weighting and the reduction over heads stay inside one
+//    thread; no [T, H_I, N] value ever leaves the SM.
+// The CTA grid is persistent (one CTA per SM) over the work items of k_plan.
+#include <cudaTypedefs.h>
 
-#include "dsa_internal.cuh"
+#include "sm100.cuh"
 
 namespace dsa {
 
 namespace {
 
-constexpr int kKeysPerBlock = 128;
+using namespace sm100;
 
-template <bool kFp8>
-__global__ void __launch_bounds__(kKeysPerBlock)
-k_index_scores_simple(SeqsDev s, TokenMap tm, const void* __restrict__ q_operand,
-                      const float* __restrict__ w_operand, const void* __restrict__ kI,
-                      const float* __restrict__ kI_scale, float* __restrict__ scores, int64_t ld,
-                      uint32_t* err) {
-  const int t = blockIdx.x;
-  const int pos = tm.pos[t];
-  const int s0 = blockIdx.y * kKeysPerBlock;
-  if (pos < 0 || s0 > pos) return;
-  const int b = tm.seq[t];
+template <bool kBf16, int TG>
+struct IdxCfg {
+  static constexpr int N = 64 * TG;                        // MMA N: heads x tokens of a group
+  static constexpr int A_BYTES = kBf16 ? 32768 : 16384;    // 128 keys x d_I
+  static constexpr int B_BYTES = kBf16 ? N * 256 : N * 128;
+  static constexpr int KSTEPS = kBf16 ? 8 : 4;             // 32-byte K steps per tile
+  static constexpr int NS = kBf16 ? (TG == 1 ? 4 : 3) : (TG == 1 ? 8 : 6);
+  static constexpr int NACC = (512 / N) < 4 ? (512 / N) : 4;
+  static constexpr int TMEM_COLS = (NACC * N) <= 256 ? 256 : 512;
+  // shared-memory layout (offsets from a 1024-aligned base)
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + NS * A_BYTES;
+  static constexpr int OFF_SC = OFF_B + 2 * B_BYTES;       // NS x 128 fp32 row scales
+  static constexpr int OFF_W = OFF_SC + NS * 512;          // 2 x TG x 64 fp32 head weights
+  static constexpr int OFF_BAR = OFF_W + 2 * TG * 256;
+  static constexpr int NBARS = 2 * NS + 4 + 2 * NACC;
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM = BYTES + 1024;                // slack for 1024-byte alignment
+  static constexpr uint32_t IDESC = make_idesc(kBf16, 128, N);
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(NACC * N <= TMEM_COLS, "TMEM");
+};
 
-  __shared__ float qs[kHI][kDI];
-  __shared__ float ws[kHI];
-  for (int i = threadIdx.x; i < kHI * kDI; i += blockDim.x) {
-    float v;
-    if constexpr (kFp8) {
-      __nv_fp8_e4m3 c;
-      c.__x = reinterpret_cast<const uint8_t*>(q_operand)[(int64_t)t * kHI * kDI + i];
-      v = float(c);
-    } else {
-      v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q_operand)[(int64_t)t * kHI * kDI + i]);
+struct IdxArgs {
+  SeqsDev s;
+  PlanBufs plan;
+  const float* w_operand;  // [T, 64] head weights (scaled by 2^e for FP8)
+  const float* kI_scale;   // [R] (FP8) or null
+  float* scores;
+  int64_t ld;
+  uint32_t* err;
+};
+
+template <bool kBf16, int TG>
+__global__ void __launch_bounds__(256, 1)
+k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                  const IdxArgs a) {
+  using C = IdxCfg<kBf16, TG>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full = bars;                      // [NS]  stage loaded
+  uint64_t* empty = bars + C::NS;             // [NS]  stage consumed (MMA + epilogue)
+  uint64_t* b_full = bars + 2 * C::NS;        // [2]   group operands loaded
+  uint64_t* b_empty = b_full + 2;             // [2]   group operands released
+  uint64_t* acc_full = b_empty + 2;           // [NACC]
+  uint64_t* acc_empty = acc_full + C::NACC;   // [NACC]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  const float* sc_smem = reinterpret_cast<const float*>(smem + C::OFF_SC);
+  const float* w_smem = reinterpret_cast<const float*>(smem + C::OFF_W);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1 + 4);
     }
-    qs[i / kDI][i % kDI] = v;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1 + 4);
+    }
+    for (int i = 0; i < C::NACC; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  if (threadIdx.x < kHI) ws[threadIdx.x] = w_operand[(int64_t)t * kHI + threadIdx.x];
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  const int sidx = s0 + threadIdx.x;
-  if (sidx > pos) return;
-  const int64_t row = phys_row(s.page_table, s.max_pages, s.num_phys_pages, b, sidx, err);
-  if (row < 0) return;
+  // this CTA's contiguous share of the work items
+  const int n_items = a.plan.counts[1];
+  const int it_lo = (int)(((int64_t)n_items * blockIdx.x) / gridDim.x);
+  const int it_hi = (int)(((int64_t)n_items * (blockIdx.x + 1)) / gridDim.x);
 
-  float k[kDI];
-  if constexpr (kFp8) {
-    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(kI) + row * kDI);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_q);
+      int stage = 0, sphase = 0, prev_g = -1, gcount = 0;
+      for (int it = it_lo; it < it_hi && !*abort_flag; ++it) {
+        const int4 item = a.plan.items[it];
+        const int4 grp = a.plan.groups[item.x];  // {b, t0, cnt, pos0}
+        if (item.x != prev_g) {
+          const int slot = gcount & 1, use = gcount >> 1;
+          if (!mbar_wait(&b_empty[slot], (use & 1) ^ 1, a.err)) { *abort_flag = 1; break; }
+          const uint32_t wbytes = (uint32_t)grp.z * 256u;
+          mbar_arrive_expect_tx(&b_full[slot], (uint32_t)C::B_BYTES + wbytes);
+          uint8_t* bdst = smem + C::OFF_B + slot * C::B_BYTES;
+          if constexpr (kBf16) {
+            tma_load_2d(bdst, &tmap_q, &b_full[slot], 0, grp.y * 64);
+            tma_load_2d(bdst + C::N * 128, &tmap_q, &b_full[slot], 64, grp.y * 64);
+          } else {
+            tma_load_2d(bdst, &tmap_q, &b_full[slot], 0, grp.y * 64);
+          }
+          bulk_load(smem + C::OFF_W + slot * TG * 256, a.w_operand + (int64_t)grp.y * 64, wbytes, &b_full[slot]);
+          prev_g = item.x;
+          ++gcount;
+        }
+        const int last = grp.w + grp.z - 1;  // last position of the group
+        for (int tile = item.y; tile < item.z; ++tile) {
+          if (!mbar_wait(&empty[stage], sphase ^ 1, a.err)) { *abort_flag = 1; break; }
+          int rows[2];
+          uint32_t bytes = 0;
 #pragma unroll
-    for (int c = 0; c < kDI / 16; ++c) {
-      uint4 v = __ldg(src + c);
-      const uint8_t* bytes = reinterpret_cast<const uint8_t*>(&v);
+          for (int h = 0; h < 2; ++h) {
+            rows[h] = -1;
+            const int lp = tile * 2 + h;
+            if (lp * kPage <= last) {
+              const int page = __ldg(a.s.page_table + (int64_t)grp.x * a.s.max_pages + lp);
+              if (page >= 0 && page < a.s.num_phys_pages) {
+                rows[h] = page * kPage;
+                bytes += (uint32_t)(C::A_BYTES / 2) + (kBf16 ? 0u : 256u);
+              } else {
+                raise_error(a.err, kErrBadIndex);
+              }
+            }
+          }
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          uint8_t* adst = smem + C::OFF_A + stage * C::A_BYTES;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        __nv_fp8_e4m3 e;
-        e.__x = bytes[j];
-        k[c * 16 + j] = float(e);
+          for (int h = 0; h < 2; ++h) {
+            if (rows[h] < 0) continue;
+            if constexpr (kBf16) {
+              tma_load_2d(adst + h * 8192, &tmap_k, &full[stage], 0, rows[h]);
+              tma_load_2d(adst + 16384 + h * 8192, &tmap_k, &full[stage], 64, rows[h]);
+            } else {
+              tma_load_2d(adst + h * 8192, &tmap_k, &full[stage], 0, rows[h]);
+              bulk_load(smem + C::OFF_SC + stage * 512 + h * 256, a.kI_scale + rows[h], 256, &full[stage]);
+            }
+          }
+          if (++stage == C::NS) { stage = 0; sphase ^= 1; }
+        }
+      }
+      // drain: every issued stage has been consumed before the CTA exits
+      for (int i = 0; i < C::NS && !*abort_flag; ++i) {
+        if (!mbar_wait(&empty[stage], sphase ^ 1, a.err)) break;
+        if (++stage == C::NS) { stage = 0; sphase ^= 1; }
       }
     }
-  } else {
-    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(kI) + row * kDI);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      int stage = 0, sphase = 0, acc = 0, aphase = 0, prev_g = -1, gcount = 0, slot = 0;
+      for (int it = it_lo; it < it_hi && !*abort_flag; ++it) {
+        const int4 item = a.plan.items[it];
+        if (item.x != prev_g) {
+          if (prev_g >= 0) mma_commit(&b_empty[slot]);  // previous group's operands free once its MMAs finish
+          slot = gcount & 1;
+          if (!mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err)) { *abort_flag = 1; break; }
+          prev_g = item.x;
+          ++gcount;
+        }
+        const uint32_t b_base = smem_u32(smem + C::OFF_B + slot * C::B_BYTES);
+        for (int tile = item.y; tile < item.z; ++tile) {
+          if (!mbar_wait(&full[stage], sphase, a.err)) { *abort_flag = 1; break; }
+          if (!mbar_wait(&acc_empty[acc], aphase ^ 1, a.err)) { *abort_flag = 1; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
 #pragma unroll
-    for (int c = 0; c < kDI / 8; ++c) {
-      uint4 v = __ldg(src + c);
-      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) k[c * 8 + j] = __bfloat162float(h[j]);
+          for (int k = 0; k < C::KSTEPS; ++k) {
+            // K step k: 32 bytes inside a 128-byte swizzle row; bf16 rows span two 128-byte blocks
+            const uint32_t a_off = kBf16 ? (k >> 2) * 16384 + (k & 3) * 32 : k * 32;
+            const uint32_t b_off = kBf16 ? (k >> 2) * (C::N * 128) + (k & 3) * 32 : k * 32;
+            mma_ss<kBf16>(tmem + acc * C::N, sw128_kmajor_desc(a_base + a_off), sw128_kmajor_desc(b_base + b_off),
+                          C::IDESC, k > 0);
+          }
+          mma_commit(&empty[stage]);
+          mma_commit(&acc_full[acc]);
+          if (++stage == C::NS) { stage = 0; sphase ^= 1; }
+          if (++acc == C::NACC) { acc = 0; aphase ^= 1; }
+        }
+      }
     }
-  }
-  float acc = 0.f;
-  for (int h = 0; h < kHI; ++h) {
-    float d = 0.f;
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp - 4;            // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;       // key row of the tile
+    const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+    int stage = 0, sphase = 0, acc = 0, aphase = 0, prev_g = -1, gcount = 0, slot = 0;
+    float wreg[64];
+    for (int it = it_lo; it < it_hi && !*abort_flag; ++it) {
+      const int4 item = a.plan.items[it];
+      const int4 grp = a.plan.groups[item.x];
+      if (item.x != prev_g) {
+        if (prev_g >= 0) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_empty[slot]);
+        }
+        slot = gcount & 1;
+        if (!mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err)) { *abort_flag = 1; break; }
+        if constexpr (TG == 1) {
 #pragma unroll
-    for (int i = 0; i < kDI; ++i) d = fmaf(qs[h][i], k[i], d);
-    acc = fmaf(ws[h], fmaxf(d, 0.f), acc);
+          for (int h = 0; h < 64; ++h) wreg[h] = w_smem[slot * TG * 64 + h];
+        }
+        prev_g = item.x;
+        ++gcount;
+      }
+      for (int tile = item.y; tile < item.z; ++tile) {
+        if (!mbar_wait(&acc_full[acc], aphase, a.err)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        // the row scales arrived with the stage's TMA; observe that completion here too
+        if (!kBf16 && !mbar_wait(&full[stage], sphase, a.err)) { *abort_flag = 1; break; }
+        const float sk = kBf16 ? 1.f : sc_smem[stage * 128 + r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        const int s = tile * 128 + r;
+#pragma unroll 1
+        for (int k = 0; k < TG; ++k) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(t_lane + acc * C::N + k * 64, v0);
+          tmem_ld32(t_lane + acc * C::N + k * 64 + 32, v1);
+          tmem_ld_wait();
+          if (k == TG - 1) {  // every TMEM read of this accumulator is complete
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          }
+          const float* wk = w_smem + slot * TG * 64 + k * 64;
+          float sum = 0.f;
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            const float w0 = TG == 1 ? wreg[h] : wk[h];
+            const float w1 = TG == 1 ? wreg[h + 32] : wk[h + 32];
+            sum = fmaf(w0, fmaxf(__uint_as_float(v0[h]), 0.f), sum);
+            sum = fmaf(w1, fmaxf(__uint_as_float(v1[h]), 0.f), sum);
+          }
+          if (k < grp.z && s <= grp.w + k) a.scores[(int64_t)(grp.y + k) * a.ld + s] = sum * sk;
+        }
+        if (++stage == C::NS) { stage = 0; sphase ^= 1; }
+        if (++acc == C::NACC) { acc = 0; aphase ^= 1; }
+      }
+    }
+    __syncwarp();
   }
-  if constexpr (kFp8) acc *= __ldg(kI_scale + row);
-  scores[(int64_t)t * ld + sidx] = acc;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major 2-D map: rows of `row_elems` elements, box of box_x x box_y, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t row_elems, uint64_t rows, uint32_t box_x,
+              uint32_t box_y) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {row_elems, rows};
+  const cuuint64_t strides[1] = {row_elems * (bf16 ? 2 : 1)};
+  const cuuint32_t box[2] = {box_x, box_y};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <bool kBf16, int TG>
+cudaError_t launch_tc(const CUtensorMap& mk, const CUtensorMap& mq, const IdxArgs& a, cudaStream_t st) {
+  using C = IdxCfg<kBf16, TG>;
+  static thread_local int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(k_index_scores_tc<kBf16, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_dev = dev;
+  }
+  k_index_scores_tc<kBf16, TG><<<sm_count(), 256, C::SMEM, st>>>(mk, mq, a);
+  return counted(cudaGetLastError());
 }
 
 }  // namespace
 
-cudaError_t launch_index_scores(const SeqsDev& s, TokenMap tm, const void* q_operand, const float* w_operand,
-                                const void* kI, const float* kI_scale, bool fp8, float* scores, int64_t ld,
-                                uint32_t* err, cudaStream_t st) {
-  dim3 grid(s.num_tokens, (s.max_ctx + kKeysPerBlock - 1) / kKeysPerBlock);
-  if (fp8)
-    k_index_scores_simple<true><<<grid, kKeysPerBlock, 0, st>>>(s, tm, q_operand, w_operand, kI, kI_scale,
-                                                                 scores, ld, err);
-  else
-    k_index_scores_simple<false><<<grid, kKeysPerBlock, 0, st>>>(s, tm, q_operand, w_operand, kI, kI_scale,
-                                                                  scores, ld, err);
-  return counted(cudaGetLastError());
+cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
+                                const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
+                                float* scores, int64_t ld, uint32_t* err, cudaStream_t st) {
+  const bool bf16 = !fp8;
+  const uint64_t R = (uint64_t)s.num_phys_pages * kPage;
+  const uint64_t qrows = (uint64_t)s.num_tokens * kHI;
+  CUtensorMap mk, mq;
+  if (!make_map(&mk, kI, bf16, kDI, R, bf16 ? 64 : 128, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&mq, q_operand, bf16, kDI, qrows, bf16 ? 64 : 128, 64 * tg)) return cudaErrorInvalidValue;
+  IdxArgs a{s, plan, w_operand, kI_scale, scores, ld, err};
+  if (fp8) {
+    if (tg == 1) return launch_tc<false, 1>(mk, mq, a, st);
+    if (tg == 4) return launch_tc<false, 4>(mk, mq, a, st);
+  } else {
+    if (tg == 1) return launch_tc<true, 1>(mk, mq, a, st);
+    if (tg == 2) return launch_tc<true, 2>(mk, mq, a, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace dsa

@@ -1,9 +1,9 @@
 // Per-token geometry and index-query quantization.
 //
-// token_map: the sequence and absolute position of every query token
-//   (pos = ctx_len[b] - q_len[b] + j), validated once so that later kernels can
-//   trust it; a token of an invalid sequence gets pos = -1 and sets the error
-//   bit.
+// plan: the sequence and absolute position of every query token (pos =
+//   ctx_len[b] - q_len[b] + j), validated once so that later kernels can trust
+//   it, plus the indexer's work list (token groups x runs of key tiles), built
+//   on the device so the host never needs the device-side lengths.
 // quantize_index_query: the "Q quantization" input-preparation step of the
 //   indexer ([P2] "Hybrid Attention LLM Inference Acceleration...", section
 //   4(2); [P3] "Inference Acceleration for a New Domestic LLM Architecture...",
@@ -15,36 +15,130 @@
 
 namespace dsa {
 
-__global__ void k_token_map(SeqsDev s, int32_t* __restrict__ tok_seq, int32_t* __restrict__ tok_pos,
-                            uint32_t* err) {
-  int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= s.num_tokens) return;
-  // sequence b with q_seq_start[b] <= t < q_seq_start[b+1] (binary search)
-  int lo = 0, hi = s.batch - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (__ldg(s.q_seq_start + mid) <= t) lo = mid; else hi = mid - 1;
+namespace {
+
+// Exclusive prefix sum over a 1024-thread block; returns the thread's prefix
+// and writes the block total to *total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_buf, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
   }
-  int b = lo;
-  int start = __ldg(s.q_seq_start + b), end = __ldg(s.q_seq_start + b + 1);
-  int ctx = __ldg(s.ctx_len + b);
-  int q_len = end - start;
-  int pos = ctx - q_len + (t - start);
-  bool ok = (__ldg(s.q_seq_start) == 0) && t >= start && t < end && ctx >= 1 && ctx <= s.max_ctx &&
-            q_len <= ctx && ((ctx + kPage - 1) / kPage) <= s.max_pages && pos >= 0;
-  if (!ok) {
-    raise_error(err, kErrBadIndex);
-    pos = -1;
+  if (lane == 31) warp_buf[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = warp_buf[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    warp_buf[lane] = wi - w;
+    if (lane == 31) warp_buf[32] = wi;
   }
-  tok_seq[t] = b;
-  tok_pos[t] = pos;
+  __syncthreads();
+  const int r = warp_buf[warp] + incl - v;
+  *total = warp_buf[32];
+  __syncthreads();
+  return r;
 }
 
-cudaError_t launch_token_map(const SeqsDev& s, int32_t* tok_seq, int32_t* tok_pos, uint32_t* err,
-                             cudaStream_t st) {
-  int threads = 256;
-  int blocks = (s.num_tokens + threads - 1) / threads;
-  k_token_map<<<blocks, threads, 0, st>>>(s, tok_seq, tok_pos, err);
+__device__ __forceinline__ bool seq_ok(const SeqsDev& s, int b, int* q_len_out, int* ctx_out) {
+  const int q_len = __ldg(s.q_seq_start + b + 1) - __ldg(s.q_seq_start + b);
+  const int ctx = __ldg(s.ctx_len + b);
+  *q_len_out = q_len;
+  *ctx_out = ctx;
+  return q_len >= 0 && ctx >= 1 && ctx <= s.max_ctx && q_len <= ctx && (ctx + kPage - 1) / kPage <= s.max_pages;
+}
+
+}  // namespace
+
+// One CTA of 1024 threads.  Writes
+//   tok_seq/tok_pos [T]   sequence and absolute position of every query token
+//                         (pos = -1 and the error bit for an invalid one);
+//   groups [G]            {b, t0, cnt, pos0}: up to `tg` consecutive query tokens
+//                         of one sequence (their positions are pos0 .. pos0+cnt-1);
+//   items [I]             {g, tile_begin, tile_end}: a run of <= `ch` key tiles of
+//                         128 positions of group g (tiles cover 0 .. last pos);
+//   counts                {G, I}.
+__global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBufs p, uint32_t* err) {
+  __shared__ int warp_buf[33];
+  const int tid = threadIdx.x;
+  for (int t = tid; t < s.num_tokens; t += blockDim.x) {
+    int lo = 0, hi = s.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(s.q_seq_start + mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int start = __ldg(s.q_seq_start + b), end = __ldg(s.q_seq_start + b + 1);
+    int q_len, ctx;
+    const bool ok = seq_ok(s, b, &q_len, &ctx) && __ldg(s.q_seq_start) == 0 && t >= start && t < end;
+    int pos = ctx - q_len + (t - start);
+    if (!ok || pos < 0) {
+      raise_error(err, kErrBadIndex);
+      pos = -1;
+    }
+    p.tok_seq[t] = b;
+    p.tok_pos[t] = pos;
+  }
+  if (ch <= 0) return;  // token geometry only
+  // groups per sequence -> start offsets (an invalid sequence gets none)
+  int running = 0;
+  for (int base = 0; base < s.batch; base += blockDim.x) {
+    const int b = base + tid;
+    int cnt = 0;
+    if (b < s.batch) {
+      int q_len, ctx;
+      if (seq_ok(s, b, &q_len, &ctx))
+        cnt = (q_len + tg - 1) / tg;
+      else
+        raise_error(err, kErrBadIndex);
+    }
+    int total;
+    const int excl = block_exclusive_scan(cnt, warp_buf, &total);
+    if (b < s.batch) p.seq_gstart[b] = running + excl;
+    running += total;
+  }
+  if (tid == 0) p.seq_gstart[s.batch] = running;
+  __syncthreads();
+  const int G = running;
+  int irun = 0;
+  for (int gbase = 0; gbase < G; gbase += blockDim.x) {
+    const int g = gbase + tid;
+    int nitems = 0, tiles = 0;
+    if (g < G) {
+      int lo = 0, hi = s.batch - 1;  // largest b with seq_gstart[b] <= g
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.seq_gstart[mid] <= g) lo = mid; else hi = mid - 1;
+      }
+      const int b = lo;
+      const int q_len = __ldg(s.q_seq_start + b + 1) - __ldg(s.q_seq_start + b);
+      const int j0 = (g - p.seq_gstart[b]) * tg;
+      const int cnt = min(tg, q_len - j0);
+      const int pos0 = __ldg(s.ctx_len + b) - q_len + j0;
+      tiles = (pos0 + cnt - 1) / 128 + 1;
+      nitems = (tiles + ch - 1) / ch;
+      p.groups[g] = make_int4(b, __ldg(s.q_seq_start + b) + j0, cnt, pos0);
+    }
+    int total;
+    const int istart = irun + block_exclusive_scan(nitems, warp_buf, &total);
+    for (int j = 0; j < nitems; ++j) p.items[istart + j] = make_int4(g, j * ch, min(tiles, (j + 1) * ch), 0);
+    irun += total;
+  }
+  if (tid == 0) {
+    p.counts[0] = G;
+    p.counts[1] = irun;
+  }
+}
+
+cudaError_t launch_plan(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err, cudaStream_t st) {
+  k_plan<<<1, 1024, 0, st>>>(s, tg, ch, p, err);
   return counted(cudaGetLastError());
 }
 
