@@ -192,6 +192,37 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t *seqs, const void *q,
                                 dsa_out_dtype_t out_dtype, float *lse,
                                 void *ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* Size of the scratch array dsa_sparse_mla_fwd_noalloc uses (32 MiB). */
+#define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* dsa_sparse_mla_fwd for callers that cannot allocate device memory.  The
+ * pages have no counterpart to this entry point: it serves code that only ever
+ * receives input and output buffers -- a plugin inside a host framework that
+ * owns every device allocation, or a caller running where cudaMalloc is not
+ * permitted -- and so has nothing to pass as `ws`.
+ * Inputs, outputs and results are those of dsa_sparse_mla_fwd.  The scratch is
+ * a fixed array of DSA_NOALLOC_SCRATCH_BYTES in the library's device image:
+ *   - every GPU that loads the library holds that memory until the process exits;
+ *   - a geometry whose scratch (dsa_workspace_size(DSA_OP_SPARSE_MLA, ...))
+ *     exceeds it returns DSA_ERR_WORKSPACE before any CUDA call (decode batches
+ *     below 74 tokens need at most ~20 MiB; larger batches need only 8 bytes per
+ *     token plus 4 per sequence);
+ *   - the first call on each device, with that device current, looks up the
+ *     array's device address; make that first call before any stream capture;
+ *   - nothing is allocated or freed (no cudaMalloc, cudaFree or allocating
+ *     library routine); the array's error word is cleared at the start of each
+ *     call with an asynchronous memset;
+ *   - all calls share the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other host threads) race
+ *     and corrupt each other's results, so serialise them;
+ *   - bad device-side indices or page ids are skipped as in dsa_sparse_mla_fwd,
+ *     but cannot be reported: the error word lives in the shared array. */
+dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_seqs_t *seqs, const void *q,
+                                        const void *kv, const int32_t *idx,
+                                        int K, int H, float scale, void *out,
+                                        dsa_out_dtype_t out_dtype, float *lse,
+                                        dsa_stream_t stream);
+
 /* The whole path in one call ([P1] Layer 1, "Sparse attention": scoring,
  * selection, gathering and attention integrated; [P3] section 3 pseudocode):
  * dsa_index_scores -> dsa_topk -> dsa_sparse_mla_fwd on the caller's stream,

@@ -32,11 +32,12 @@ DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUD
     DSA_ERR_TIMEOUT = range(7)
 DSA_KI_BF16, DSA_KI_FP8_E4M3 = 0, 1
 DSA_OUT_BF16, DSA_OUT_F32 = 0, 1
+DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_INDEX_TOPK_ATTN = range(5)
 
 # Names the C header declares (checked against include/dsa.h by the tests).
 EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_index_scores", "dsa_topk",
-           "dsa_sparse_mla_fwd", "dsa_index_topk_attn", "dsa_check_error", "dsa_launches_in_last_call", "dsa_status_string")
+           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_noalloc", "dsa_index_topk_attn", "dsa_check_error", "dsa_launches_in_last_call", "dsa_status_string")
 
 
 class DsaSeqsC(ctypes.Structure):
@@ -55,6 +56,8 @@ _sig = {
     "dsa_topk": (ctypes.c_int, [_P, _I64, ctypes.c_int, _P, ctypes.c_int, _P, _P, _SZ, _P]),
     "dsa_sparse_mla_fwd": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, ctypes.c_int, _F, _P, ctypes.c_int, _P, _P,
                                           _SZ, _P]),
+    "dsa_sparse_mla_fwd_noalloc": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, ctypes.c_int, _F, _P, ctypes.c_int,
+                                                  _P, _P]),
     "dsa_index_topk_attn": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
                                            _F, _P, ctypes.c_int, _P, _P, _P, _SZ, _P]),
     "dsa_check_error": (ctypes.c_int, [_P, _P]),
@@ -204,6 +207,23 @@ def dsa_sparse_mla_fwd(seqs: Seqs, q, kv, idx, scale: float, out=None, lse=None,
     _check(_lib.dsa_sparse_mla_fwd(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(idx), K, H, scale, _ptr(out),
                                    _out_dtype(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)),
            "dsa_sparse_mla_fwd")
+    return out, lse
+
+
+def dsa_sparse_mla_fwd_noalloc(seqs: Seqs, q, kv, idx, scale: float, out=None, lse=None, want_lse=True,
+                               out_dtype=torch.bfloat16):
+    """dsa_sparse_mla_fwd without a workspace: the library's built-in scratch
+    array is used (for callers that cannot allocate device memory; see
+    include/dsa.h).  Outputs not passed in are allocated here for convenience."""
+    T, H, _ = q.shape
+    K = idx.shape[1]
+    out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    c = seqs.c()
+    _check(_lib.dsa_sparse_mla_fwd_noalloc(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(idx), K, H, scale, _ptr(out),
+                                           _out_dtype(out), _ptr(lse), _stream(q.device)),
+           "dsa_sparse_mla_fwd_noalloc")
     return out, lse
 
 
