@@ -22,7 +22,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // the sticky error word.
 struct Layout {
   size_t tok_seq = 0, tok_pos = 0, seq_gstart = 0, groups = 0, items = 0, counts = 0;
-  size_t q_codes = 0, w_scaled = 0, scores = 0, idx = 0, partials = 0;
+  size_t q_codes = 0, w_scaled = 0, scores = 0, idx = 0, topk = 0, partials = 0;
   size_t total = 0;
   int64_t ld = 0;
 };
@@ -50,7 +50,7 @@ Layout make_layout(dsa_op_t op, int T, int B, int max_ctx, int K, int H) {
   if (indexer) {
     const int tg = sizing_group_tokens(T, B);
     L.groups = take((size_t)plan_max_groups(T, B, tg) * sizeof(int4));
-    L.items = take((size_t)plan_max_items(T, B, max_ctx, tg) * sizeof(int4));
+    L.items = take((size_t)plan_max_items(T, B, max_ctx, tg) * 2 * sizeof(int4));
     L.q_codes = take((size_t)T * kHI * kDI);
     L.w_scaled = take((size_t)T * kHI * sizeof(float));
   }
@@ -58,7 +58,9 @@ Layout make_layout(dsa_op_t op, int T, int B, int max_ctx, int K, int H) {
     L.ld = ((int64_t)max_ctx + 3) / 4 * 4;
     L.scores = take((size_t)T * (size_t)L.ld * sizeof(float));
     L.idx = take((size_t)T * K * sizeof(int32_t));
+    L.topk = take(topk_scratch_bytes(T, L.ld, K));
   }
+  if (op == DSA_OP_TOPK) L.topk = take(topk_scratch_bytes(T, max_ctx, K));
   if (op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN) L.partials = take(sparse_mla_partials_bytes(T, K, H));
   L.total = off;
   return L;
@@ -212,7 +214,8 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row
   if (!aligned(scores, 16) || !aligned(row_len, 4) || !aligned(idx, 16)) return DSA_ERR_INVALID_ARG;
   const Layout L = make_layout(DSA_OP_TOPK, T, 1, (int)ld, K, 16);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
-  return cuda_status(launch_topk(scores, ld, T, row_len, nullptr, K, idx, at<uint32_t>(ws, 0), (cudaStream_t)stream));
+  return cuda_status(
+      launch_topk(scores, ld, T, row_len, nullptr, K, idx, at<void>(ws, L.topk), at<uint32_t>(ws, 0), (cudaStream_t)stream));
 }
 
 dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const void* kv, const int32_t* idx, int K,
@@ -255,7 +258,7 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const f
   const int tg = indexer_group_tokens(seqs->num_q_tokens, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
   DSA_CUDA(launch_plan(sd, tg, indexer_item_tiles(tg), plan, err, st));
   DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, err, st));
-  DSA_CUDA(launch_topk(scores, L.ld, seqs->num_q_tokens, nullptr, tm.pos, K, idx, err, st));
+  DSA_CUDA(launch_topk(scores, L.ld, seqs->num_q_tokens, nullptr, tm.pos, K, idx, at<void>(ws, L.topk), err, st));
   DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
                              out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));

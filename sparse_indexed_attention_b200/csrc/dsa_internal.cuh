@@ -65,7 +65,7 @@ struct PlanBufs {
   int32_t* tok_pos;     // [T]
   int32_t* seq_gstart;  // [B+1]
   int4* groups;         // [max groups]  {b, t0, cnt, pos0}
-  int4* items;          // [max items]   {g, tile_begin, tile_end, 0}
+  int4* items;          // [2 x max items] {b, t0, cnt, pos0}, {tile_begin, tile_end, g, 0}
   int32_t* counts;      // {groups, items}
 };
 
@@ -91,8 +91,9 @@ cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w,
 cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
                                 const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
                                 float* scores, int64_t ld, uint32_t* err, cudaStream_t st);
+size_t topk_scratch_bytes(int T, int64_t ld, int K);
 cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, const int32_t* tok_pos,
-                        int K, int32_t* idx, uint32_t* err, cudaStream_t st);
+                        int K, int32_t* idx, void* scratch, uint32_t* err, cudaStream_t st);
 size_t sparse_mla_partials_bytes(int T, int K, int H);
 cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16* q, const __nv_bfloat16* kv,
                               const int32_t* idx, int K, int H, float scale, void* out, bool out_f32,

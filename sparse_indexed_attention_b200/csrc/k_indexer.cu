@@ -114,67 +114,101 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
   const int it_lo = (int)(((int64_t)n_items * blockIdx.x) / gridDim.x);
   const int it_hi = (int)(((int64_t)n_items * (blockIdx.x + 1)) / gridDim.x);
 
+  const int4* recs = a.plan.items;  // item i: recs[2i] = {b, t0, cnt, pos0}, recs[2i+1] = {tile_begin, tile_end, g, 0}
+
   if (warp == 0) {
+    // ------------------------------------------------------------ producer (whole warp)
+    // Item records are fetched two ahead and each item's page ids (one lane
+    // per page, <= 32 pages per item) one ahead, so the page-table reads
+    // overlap the TMA issue of the current item.
     if (lane == 0) {
-      // ------------------------------------------------------------ producer
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_q);
-      int stage = 0, sphase = 0, prev_g = -1, gcount = 0;
-      for (int it = it_lo; it < it_hi && !*abort_flag; ++it) {
-        const int4 item = a.plan.items[it];
-        const int4 grp = a.plan.groups[item.x];  // {b, t0, cnt, pos0}
-        if (item.x != prev_g) {
+    }
+    auto load_pages = [&](const int4& ga, const int4& gb) -> int {
+      const int lp = 2 * gb.x + lane;
+      const int last = ga.w + ga.z - 1;
+      if (lane < 2 * (gb.y - gb.x) && lp * kPage <= last) return __ldg(a.s.page_table + (int64_t)ga.x * a.s.max_pages + lp);
+      return -1;
+    };
+    int4 ca = make_int4(0, 0, 0, 0), cb = ca, na = ca, nb = ca, fa = ca, fb = ca;
+    if (it_lo < it_hi) { ca = recs[2 * it_lo]; cb = recs[2 * it_lo + 1]; }
+    if (it_lo + 1 < it_hi) { na = recs[2 * it_lo + 2]; nb = recs[2 * it_lo + 3]; }
+    int pages = it_lo < it_hi ? load_pages(ca, cb) : -1;
+    int stage = 0, sphase = 0, prev_g = -1, gcount = 0;
+    bool ok = true;
+    for (int it = it_lo; it < it_hi && ok; ++it) {
+      if (it + 2 < it_hi) { fa = recs[2 * it + 4]; fb = recs[2 * it + 5]; }
+      const int next_pages = (it + 1 < it_hi) ? load_pages(na, nb) : -1;
+      const int4 grp = ca;  // {b, t0, cnt, pos0}
+      if (cb.z != prev_g) {
+        if (lane == 0) {
           const int slot = gcount & 1, use = gcount >> 1;
-          if (!mbar_wait(&b_empty[slot], (use & 1) ^ 1, a.err)) { *abort_flag = 1; break; }
-          const uint32_t wbytes = (uint32_t)grp.z * 256u;
-          mbar_arrive_expect_tx(&b_full[slot], (uint32_t)C::B_BYTES + wbytes);
-          uint8_t* bdst = smem + C::OFF_B + slot * C::B_BYTES;
-          if constexpr (kBf16) {
-            tma_load_2d(bdst, &tmap_q, &b_full[slot], 0, grp.y * 64);
-            tma_load_2d(bdst + C::N * 128, &tmap_q, &b_full[slot], 64, grp.y * 64);
+          if (!mbar_wait(&b_empty[slot], (use & 1) ^ 1, a.err)) {
+            *abort_flag = 1;
           } else {
-            tma_load_2d(bdst, &tmap_q, &b_full[slot], 0, grp.y * 64);
+            const uint32_t wbytes = (uint32_t)grp.z * 256u;
+            mbar_arrive_expect_tx(&b_full[slot], (uint32_t)C::B_BYTES + wbytes);
+            uint8_t* bdst = smem + C::OFF_B + slot * C::B_BYTES;
+            if constexpr (kBf16) {
+              tma_load_2d(bdst, &tmap_q, &b_full[slot], 0, grp.y * 64);
+              tma_load_2d(bdst + C::N * 128, &tmap_q, &b_full[slot], 64, grp.y * 64);
+            } else {
+              tma_load_2d(bdst, &tmap_q, &b_full[slot], 0, grp.y * 64);
+            }
+            bulk_load(smem + C::OFF_W + slot * TG * 256, a.w_operand + (int64_t)grp.y * 64, wbytes, &b_full[slot]);
           }
-          bulk_load(smem + C::OFF_W + slot * TG * 256, a.w_operand + (int64_t)grp.y * 64, wbytes, &b_full[slot]);
-          prev_g = item.x;
-          ++gcount;
         }
-        const int last = grp.w + grp.z - 1;  // last position of the group
-        for (int tile = item.y; tile < item.z; ++tile) {
-          if (!mbar_wait(&empty[stage], sphase ^ 1, a.err)) { *abort_flag = 1; break; }
-          int rows[2];
-          uint32_t bytes = 0;
+        prev_g = cb.z;
+        ++gcount;
+      }
+      for (int tile = cb.x; tile < cb.y; ++tile) {
+        const int j = tile - cb.x;
+        const int pg0 = __shfl_sync(0xffffffffu, pages, 2 * j);
+        const int pg1 = __shfl_sync(0xffffffffu, pages, 2 * j + 1);
+        if (lane == 0 && !*abort_flag) {
+          if (!mbar_wait(&empty[stage], sphase ^ 1, a.err)) {
+            *abort_flag = 1;
+          } else {
+            const int last = grp.w + grp.z - 1;
+            int rows[2];
+            const int pg[2] = {pg0, pg1};
+            uint32_t bytes = 0;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            rows[h] = -1;
-            const int lp = tile * 2 + h;
-            if (lp * kPage <= last) {
-              const int page = __ldg(a.s.page_table + (int64_t)grp.x * a.s.max_pages + lp);
-              if (page >= 0 && page < a.s.num_phys_pages) {
-                rows[h] = page * kPage;
-                bytes += (uint32_t)(C::A_BYTES / 2) + (kBf16 ? 0u : 256u);
+            for (int h = 0; h < 2; ++h) {
+              rows[h] = -1;
+              if ((tile * 2 + h) * kPage <= last) {
+                if (pg[h] >= 0 && pg[h] < a.s.num_phys_pages) {
+                  rows[h] = pg[h] * kPage;
+                  bytes += (uint32_t)(C::A_BYTES / 2) + (kBf16 ? 0u : 256u);
+                } else {
+                  raise_error(a.err, kErrBadIndex);
+                }
+              }
+            }
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            uint8_t* adst = smem + C::OFF_A + stage * C::A_BYTES;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (rows[h] < 0) continue;
+              if constexpr (kBf16) {
+                tma_load_2d(adst + h * 8192, &tmap_k, &full[stage], 0, rows[h]);
+                tma_load_2d(adst + 16384 + h * 8192, &tmap_k, &full[stage], 64, rows[h]);
               } else {
-                raise_error(a.err, kErrBadIndex);
+                tma_load_2d(adst + h * 8192, &tmap_k, &full[stage], 0, rows[h]);
+                bulk_load(smem + C::OFF_SC + stage * 512 + h * 256, a.kI_scale + rows[h], 256, &full[stage]);
               }
             }
           }
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          uint8_t* adst = smem + C::OFF_A + stage * C::A_BYTES;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (rows[h] < 0) continue;
-            if constexpr (kBf16) {
-              tma_load_2d(adst + h * 8192, &tmap_k, &full[stage], 0, rows[h]);
-              tma_load_2d(adst + 16384 + h * 8192, &tmap_k, &full[stage], 64, rows[h]);
-            } else {
-              tma_load_2d(adst + h * 8192, &tmap_k, &full[stage], 0, rows[h]);
-              bulk_load(smem + C::OFF_SC + stage * 512 + h * 256, a.kI_scale + rows[h], 256, &full[stage]);
-            }
-          }
-          if (++stage == C::NS) { stage = 0; sphase ^= 1; }
         }
+        if (++stage == C::NS) { stage = 0; sphase ^= 1; }
       }
-      // drain: every issued stage has been consumed before the CTA exits
+      ok = __shfl_sync(0xffffffffu, (int)(*abort_flag == 0), 0) != 0;  // lane 0's view, warp-uniform
+      ca = na; cb = nb; na = fa; nb = fb;
+      pages = next_pages;
+    }
+    // drain: every issued stage has been consumed before the CTA exits
+    if (lane == 0) {
       for (int i = 0; i < C::NS && !*abort_flag; ++i) {
         if (!mbar_wait(&empty[stage], sphase ^ 1, a.err)) break;
         if (++stage == C::NS) { stage = 0; sphase ^= 1; }
@@ -185,8 +219,10 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       int stage = 0, sphase = 0, acc = 0, aphase = 0, prev_g = -1, gcount = 0, slot = 0;
+      int4 nb = it_lo < it_hi ? recs[2 * it_lo + 1] : make_int4(0, 0, 0, 0);
       for (int it = it_lo; it < it_hi && !*abort_flag; ++it) {
-        const int4 item = a.plan.items[it];
+        const int4 item = make_int4(nb.z, nb.x, nb.y, 0);  // {g, tile_begin, tile_end}
+        if (it + 1 < it_hi) nb = recs[2 * it + 3];
         if (item.x != prev_g) {
           if (prev_g >= 0) mma_commit(&b_empty[slot]);  // previous group's operands free once its MMAs finish
           slot = gcount & 1;
@@ -223,16 +259,19 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     int stage = 0, sphase = 0, acc = 0, aphase = 0, prev_g = -1, gcount = 0, slot = 0;
     float wreg[64];
+    int4 na = make_int4(0, 0, 0, 0), nb = na;
+    if (it_lo < it_hi) { na = recs[2 * it_lo]; nb = recs[2 * it_lo + 1]; }
     for (int it = it_lo; it < it_hi && !*abort_flag; ++it) {
-      const int4 item = a.plan.items[it];
-      const int4 grp = a.plan.groups[item.x];
+      const int4 grp = na;                                // {b, t0, cnt, pos0}
+      const int4 item = make_int4(nb.z, nb.x, nb.y, 0);  // {g, tile_begin, tile_end}
+      if (it + 1 < it_hi) { na = recs[2 * it + 2]; nb = recs[2 * it + 3]; }
       if (item.x != prev_g) {
         if (prev_g >= 0) {
           __syncwarp();
           if (lane == 0) mbar_arrive(&b_empty[slot]);
         }
         slot = gcount & 1;
-        if (!mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err)) { *abort_flag = 1; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err))) { *abort_flag = 1; break; }
         if constexpr (TG == 1) {
 #pragma unroll
           for (int h = 0; h < 64; ++h) wreg[h] = w_smem[slot * TG * 64 + h];
@@ -241,10 +280,11 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
         ++gcount;
       }
       for (int tile = item.y; tile < item.z; ++tile) {
-        if (!mbar_wait(&acc_full[acc], aphase, a.err)) { *abort_flag = 1; break; }
-        tc_fence_after();
+        bool okw = mbar_wait(&acc_full[acc], aphase, a.err);
         // the row scales arrived with the stage's TMA; observe that completion here too
-        if (!kBf16 && !mbar_wait(&full[stage], sphase, a.err)) { *abort_flag = 1; break; }
+        if (!kBf16) okw = okw && mbar_wait(&full[stage], sphase, a.err);
+        if (!__all_sync(0xffffffffu, okw)) { *abort_flag = 1; break; }
+        tc_fence_after();
         const float sk = kBf16 ? 1.f : sc_smem[stage * 128 + r];
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);

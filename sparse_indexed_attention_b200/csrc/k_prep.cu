@@ -62,8 +62,9 @@ __device__ __forceinline__ bool seq_ok(const SeqsDev& s, int b, int* q_len_out, 
 //                         (pos = -1 and the error bit for an invalid one);
 //   groups [G]            {b, t0, cnt, pos0}: up to `tg` consecutive query tokens
 //                         of one sequence (their positions are pos0 .. pos0+cnt-1);
-//   items [I]             {g, tile_begin, tile_end}: a run of <= `ch` key tiles of
-//                         128 positions of group g (tiles cover 0 .. last pos);
+//   items [I]             two int4 per item: {b, t0, cnt, pos0} of its group and
+//                         {tile_begin, tile_end, g, 0}: a run of <= `ch` key tiles
+//                         of 128 positions (tiles cover 0 .. last pos);
 //   counts                {G, I}.
 __global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBufs p, uint32_t* err) {
   __shared__ int warp_buf[33];
@@ -107,10 +108,14 @@ __global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBu
   if (tid == 0) p.seq_gstart[s.batch] = running;
   __syncthreads();
   const int G = running;
+  __shared__ int s_istart[1025];
+  __shared__ int s_tiles[1024];
+  __shared__ int4 s_gd[1024];
   int irun = 0;
   for (int gbase = 0; gbase < G; gbase += blockDim.x) {
     const int g = gbase + tid;
     int nitems = 0, tiles = 0;
+    int4 gd = make_int4(0, 0, 0, 0);
     if (g < G) {
       int lo = 0, hi = s.batch - 1;  // largest b with seq_gstart[b] <= g
       while (lo < hi) {
@@ -124,12 +129,30 @@ __global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBu
       const int pos0 = __ldg(s.ctx_len + b) - q_len + j0;
       tiles = (pos0 + cnt - 1) / 128 + 1;
       nitems = (tiles + ch - 1) / ch;
-      p.groups[g] = make_int4(b, __ldg(s.q_seq_start + b) + j0, cnt, pos0);
+      gd = make_int4(b, __ldg(s.q_seq_start + b) + j0, cnt, pos0);
+      p.groups[g] = gd;
     }
     int total;
-    const int istart = irun + block_exclusive_scan(nitems, warp_buf, &total);
-    for (int j = 0; j < nitems; ++j) p.items[istart + j] = make_int4(g, j * ch, min(tiles, (j + 1) * ch), 0);
+    const int excl = block_exclusive_scan(nitems, warp_buf, &total);
+    s_istart[tid] = excl;
+    s_tiles[tid] = tiles;
+    s_gd[tid] = gd;
+    if (tid == 0) s_istart[blockDim.x] = total;
+    __syncthreads();
+    // write this chunk's items cooperatively: item i belongs to the last group j with s_istart[j] <= i
+    for (int i = tid; i < total; i += blockDim.x) {
+      int lo = 0, hi = blockDim.x - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_istart[mid] <= i) lo = mid; else hi = mid - 1;
+      }
+      const int j = i - s_istart[lo];
+      const int tl = s_tiles[lo];
+      p.items[2 * (irun + i)] = s_gd[lo];
+      p.items[2 * (irun + i) + 1] = make_int4(j * ch, min(tl, (j + 1) * ch), gbase + lo, 0);
+    }
     irun += total;
+    __syncthreads();
   }
   if (tid == 0) {
     p.counts[0] = G;
