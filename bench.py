@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage-reps", type=int, default=20)
+    ap.add_argument("--only", choices=["index_scores", "topk", "sparse_mla"], default=None,
+                    help="time one stage alone on the bench workload (profiling aid)")
     return ap.parse_args()
 
 
@@ -238,6 +240,28 @@ def time_device(fn, steps, warmup, stream, flush):
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
 
+def run_only(args, dsa, wl, d, dev, stream, flush, world):
+    """One stage alone, `--steps` timed launches after `--warmup` (profiling aid)."""
+    spec = wl.spec
+    T, H, K = wl.T, spec.heads, spec.topk
+    scores = torch.empty((T, (wl.max_ctx + 3) // 4 * 4), dtype=torch.float32, device=dev)
+    row_len = torch.from_numpy((wl.token_pos() + 1).astype(np.int32)).to(dev)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, H), dtype=torch.float32, device=dev)
+    dsa.dsa_index_scores(d.seqs, d.qI, d.w, d.kI, d.kI_scale, scores=scores)
+    dsa.dsa_topk(scores, row_len, K, idx=idx)
+    fns = {
+        "index_scores": lambda: dsa.dsa_index_scores(d.seqs, d.qI, d.w, d.kI, d.kI_scale, scores=scores),
+        "topk": lambda: dsa.dsa_topk(scores, row_len, K, idx=idx),
+        "sparse_mla": lambda: dsa.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out=out, lse=lse),
+    }
+    times = time_device(fns[args.only], args.steps, args.warmup, stream, flush)
+    if world == 1 or int(os.environ.get("RANK", "0")) == 0:
+        print(json.dumps({"stage": args.only, "workload": spec.name, "us_mean": 1e3 * sum(times) / len(times),
+                          "us_min": 1e3 * min(times), "launches": dsa.dsa_launches_in_last_call()}), flush=True)
+
+
 def run_ours(args, world, rank, local):
     import sparse_indexed_attention_b200 as dsa
     from sparse_indexed_attention_b200.workloads import to_device
@@ -257,6 +281,10 @@ def run_ours(args, world, rank, local):
 
     def step():
         dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse, ws=ws)
+
+    if args.only:
+        run_only(args, dsa, wl, d, dev, stream, flush, world)
+        return
 
     step()
     launches_per_step = dsa.dsa_launches_in_last_call()
