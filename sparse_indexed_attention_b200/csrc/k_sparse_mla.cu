@@ -1,37 +1,67 @@
-// Sparse MLA attention over the selected latent rows ([P1] "Day 0 Inference
-// Adaptation and Performance Optimization for Hybrid Attention LLMs",
-// Understanding the New Architecture item 2; [P2] "Hybrid Attention LLM
-// Inference Acceleration...", section 2 item 2 "Sparse attention computation";
-// [P5] "Day-0 Inference Adaptation for Large Language Models...", Operator
-// Fusion and Memory Access Optimization, bullet 1: the Top-K indices go
-// straight into the compute kernel, which gathers the rows itself).
+// Sparse MLA attention over the selected latent rows, on the 5th-generation
+// tensor cores ([P1] "Day 0 Inference Adaptation and Performance Optimization
+// for Hybrid Attention LLMs", Understanding the New Architecture item 2;
+// [P2] "Hybrid Attention LLM Inference Acceleration...", section 2 item 2
+// "Sparse attention computation"; [P5] "Day-0 Inference Adaptation for Large
+// Language Models...", Operator Fusion and Memory Access Optimization,
+// bullet 1: the Top-K indices go straight into the compute kernel, which
+// gathers the rows itself -- no gathered KV copy exists):
 //
 //   out[t,h,:] = sum_{s in idx[t]} p_s KV[s,0:512],
 //   p = softmax_s(scale * q[t,h,:] . KV[s,0:576]),   lse = ln sum exp(...)
 //
-// Simple CUDA-core form: a CTA owns (token, 16 heads, a slice of the index
-// list), gathers 64 selected rows at a time into shared memory, and keeps an
-// online softmax; slices of one token are merged by k_combine.
-#include "dsa_internal.cuh"
+// The fp32 accumulator of 128 heads x 512 value dims fills all of TMEM, so
+// the work of one (token, slice of the index list) goes to a CLUSTER OF TWO
+// CTAs.  CTA r owns value dims [256r, 256r+256) and the key dims
+// {256r..256r+255} u {512+32r..512+32r+31}; it gathers only those 576 bytes of
+// each selected row (TMA tile::gather4 through the page table, 128-byte /
+// 64-byte swizzle).  Per block of 64 selected rows:
+//   * S_r = Q_r K_r^T (M = 128 heads, N = 64 rows, K = 288 dims) into TMEM;
+//   * the two partial S are exchanged through distributed shared memory and
+//     summed (a + b = b + a, so both CTAs hold bit-identical logits and take
+//     identical softmax decisions);
+//   * online softmax in registers (one head row per thread, base-2 exponent,
+//     the running maximum is only moved -- and O rescaled in TMEM -- when it
+//     grows by more than 2^8, which is exact because O and l share it);
+//   * P goes to shared memory as two bf16 terms, P = P_hi + P_lo (together
+//     within 2^-17 of the fp32 value; one bf16 term alone would leave a
+//     relative error of 2^-9 on rows dominated by a few selected keys), and
+//     O_r += P_hi V_r + P_lo V_r (M = 128, N = 256, K = 64) accumulates in
+//     TMEM, V_r being the same gathered bytes read as an MN-major operand.
+// Slices of one token are merged by k_combine (log-sum-exp weights).
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
 
 namespace dsa {
 
 namespace {
 
-constexpr int kHG = 16;          // heads per CTA
-constexpr int kChunk = 64;       // selected rows per shared-memory chunk
-constexpr int kThreads = 256;
-constexpr int kRowPad = kDQK + 8;  // bf16 elements per staged row (bank spread)
+using namespace sm100;
 
-struct SmemLayout {
-  float q[kHG][kDQK];
-  __nv_bfloat16 kv[kChunk][kRowPad];
-  float p[kHG][kChunk];
-  float alpha[kHG];
-  float m[kHG];
-  float l[kHG];
-  int64_t row[kChunk];
-};
+constexpr int kBK = 64;                      // selected rows per block
+constexpr int kQLatBytes = 128 * 128;        // one 64-dim swizzle atom of 128 head rows
+constexpr int kQBytes = 4 * kQLatBytes + 128 * 64;
+constexpr int kKVStage = 4 * kBK * 128 + kBK * 64;  // 36864: 4 latent atoms + rope quarter
+constexpr int kPBytes = 128 * kBK * 2;       // 16 KB per bf16 term
+constexpr int kXPitch = 68;                  // floats per exchanged row (64 + pad)
+constexpr int OFF_Q = 0;
+constexpr int OFF_KV = OFF_Q + kQBytes;                 // 73728
+constexpr int OFF_P = OFF_KV + 2 * kKVStage;            // 147456
+constexpr int OFF_X = OFF_P + 2 * kPBytes;              // 180224 (P_hi, P_lo)
+constexpr int OFF_META = OFF_X + 128 * kXPitch * 4;     // 215040
+constexpr int OFF_BAR = OFF_META + 16;
+constexpr int kNBars = 13;
+constexpr int OFF_MISC = OFF_BAR + kNBars * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(OFF_KV % 1024 == 0 && kKVStage % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms need 1024-B alignment");
+
+constexpr uint32_t IDESC_QK = make_idesc_major(true, 128, kBK, 0, 0);  // S = Q K^T, both K-major
+constexpr uint32_t IDESC_PV = make_idesc_major(true, 128, 256, 0, 1);  // O += P V, V MN-major
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
 __device__ __forceinline__ void store_out(void* out, bool f32, int64_t i, float v) {
   if (f32)
@@ -40,152 +70,371 @@ __device__ __forceinline__ void store_out(void* out, bool f32, int64_t i, float 
     reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16(v);
 }
 
-int attn_splits(int T, int H, int K) {
-  int ctas = T * (H / kHG);
-  int splits = 1;
-  if (ctas < 2 * 148) {
-    int want = (2 * 148 + ctas - 1) / ctas;
-    int most = (K + kChunk - 1) / kChunk;
-    splits = want < most ? want : most;
-  }
-  return splits;
-}
+struct AttnArgs {
+  SeqsDev s;
+  TokenMap tm;
+  const int32_t* idx;
+  int K, H, ks, splits;
+  float scale_log2;  // scale * log2(e)
+  void* out;
+  bool out_f32;
+  float* lse;
+  float* part_o;
+  float2* part_ml;
+  uint32_t* err;
+};
 
-int keys_per_split(int K, int splits) {
-  int ks = (K + splits - 1) / splits;
-  return (ks + kChunk - 1) / kChunk * kChunk;
-}
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constant__ CUtensorMap tq_rope,
+                const __grid_constant__ CUtensorMap tkv_lat, const __grid_constant__ CUtensorMap tkv_rope,
+                const AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;    // [2]
+  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* s_empty = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* o_done = bars + 10;
+  uint64_t* x_full = bars + 11;    // the peer's partial S has landed in my X
+  uint64_t* x_free = bars + 12;    // the peer has consumed what I wrote into its X
+  uint64_t* meta_mask = reinterpret_cast<uint64_t*>(smem + OFF_META);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
-__global__ void __launch_bounds__(kThreads)
-k_sparse_mla_simple(SeqsDev s, TokenMap tm, const __nv_bfloat16* __restrict__ q,
-                    const __nv_bfloat16* __restrict__ kv, const int32_t* __restrict__ idx, int K, int H,
-                    float scale, int ks, int splits, void* __restrict__ out, bool out_f32, float* __restrict__ lse,
-                    float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* err) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  SmemLayout& sm = *reinterpret_cast<SmemLayout*>(smem_raw);
-  const int t = blockIdx.x, hg = blockIdx.y, sp = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int pos = tm.pos[t];
-  if (pos < 0) return;
-  const int b = tm.seq[t];
-  const int k_begin = sp * ks;
-  const int k_end = min(K, k_begin + ks);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const int cluster = blockIdx.x >> 1;
+  const int t = cluster / a.splits, sp = cluster % a.splits;
+  const int pos = a.tm.pos[t];
+  const int b = a.tm.seq[t];
+  const int kbeg = sp * a.ks;
+  const int kend = min(a.K, kbeg + a.ks);
+  const int nblk = (pos >= 0 && kend > kbeg) ? (kend - kbeg + kBK - 1) / kBK : 0;
 
-  for (int i = tid; i < kHG * kDQK; i += kThreads)
-    sm.q[i / kDQK][i % kDQK] =
-        __bfloat162float(q[((int64_t)t * H + hg * kHG + i / kDQK) * kDQK + i % kDQK]);
-  if (tid < kHG) {
-    sm.m[tid] = -INFINITY;
-    sm.l[tid] = 0.f;
-  }
-  float acc[kHG][2];
-#pragma unroll
-  for (int h = 0; h < kHG; ++h) acc[h][0] = acc[h][1] = 0.f;
-
-  for (int c0 = k_begin; c0 < k_end; c0 += kChunk) {
-    __syncthreads();
-    if (tid < kChunk) {
-      int64_t r = -1;
-      if (c0 + tid < k_end) {
-        const int sidx = idx[(int64_t)t * K + c0 + tid];
-        if (sidx >= 0 && sidx <= pos)
-          r = phys_row(s.page_table, s.max_pages, s.num_phys_pages, b, sidx, err);
-        else if (sidx != -1)
-          raise_error(err, kErrBadIndex);
-      }
-      sm.row[tid] = r;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
     }
-    __syncthreads();
-    for (int i = tid; i < kChunk * (kDQK / 8); i += kThreads) {
-      const int j = i / (kDQK / 8), c = i % (kDQK / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (sm.row[j] >= 0) v = __ldg(reinterpret_cast<const uint4*>(kv + sm.row[j] * kDQK) + c);
-      *reinterpret_cast<uint4*>(&sm.kv[j][c * 8]) = v;
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(x_full, 128);
+    mbar_init(x_free, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;  // O at columns [0,256), S buffers at [256,320), [320,384)
+
+  if (warp == 0 && nblk > 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&tkv_lat);
+      prefetch_tmap(&tkv_rope);
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      for (int at = 0; at < 4; ++at)
+        tma_load_2d(smem + OFF_Q + at * kQLatBytes, &tq_lat, q_full, 256 * rank + 64 * at, t * a.H);
+      tma_load_2d(smem + OFF_Q + 4 * kQLatBytes, &tq_rope, q_full, 512 + 32 * rank, t * a.H);
     }
-    __syncthreads();
-    {  // logits: thread -> key j, heads 4*(tid/64) .. +3
-      const int j = tid % kChunk, h0 = (tid / kChunk) * 4;
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int c = 0; c < kDQK; c += 8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(&sm.kv[j][c]);
-        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v);
+    for (int j = 0; j < nblk; ++j) {
+      const int stage = j & 1;
+      int rows[2];
+      bool valid[2];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float kvv = __bfloat162float(e[u]);
-#pragma unroll
-          for (int hh = 0; hh < 4; ++hh) d[hh] = fmaf(sm.q[h0 + hh][c + u], kvv, d[hh]);
+      for (int u = 0; u < 2; ++u) {
+        const int kk = kbeg + j * kBK + 2 * lane + u;
+        rows[u] = 0;
+        valid[u] = false;
+        if (kk < kend) {
+          const int sidx = __ldg(a.idx + (int64_t)t * a.K + kk);
+          if (sidx >= 0 && sidx <= pos) {
+            const int64_t r = phys_row(a.s.page_table, a.s.max_pages, a.s.num_phys_pages, b, sidx, a.err);
+            if (r >= 0) {
+              rows[u] = (int)r;
+              valid[u] = true;
+            }
+          } else if (sidx != -1) {
+            raise_error(a.err, kErrBadIndex);
+          }
         }
       }
-      const bool valid = sm.row[j] >= 0;
-#pragma unroll
-      for (int hh = 0; hh < 4; ++hh) sm.p[h0 + hh][j] = valid ? d[hh] * scale : -INFINITY;
-    }
-    __syncthreads();
-    // online softmax: warp w updates heads 2w, 2w+1
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int h = warp * 2 + r;
-      const float v0 = sm.p[h][lane], v1 = sm.p[h][lane + 32];
-      float cm = fmaxf(v0, v1);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
-      const float m_old = sm.m[h];
-      const float m_new = fmaxf(m_old, cm);
-      float p0 = 0.f, p1 = 0.f, alpha = 1.f;
-      if (m_new != -INFINITY) {
-        p0 = __expf(v0 - m_new);
-        p1 = __expf(v1 - m_new);
-        alpha = __expf(m_old - m_new);
+      const uint32_t m0 = __ballot_sync(0xffffffffu, valid[0]);  // bit l: row 2l
+      const uint32_t m1 = __ballot_sync(0xffffffffu, valid[1]);  // bit l: row 2l+1
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&kv_empty[stage], ((j >> 1) & 1) ^ 1, a.err);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        *abort_flag = 1;
+        break;
       }
-      float ps = p0 + p1;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-      __syncwarp();
-      sm.p[h][lane] = p0;
-      sm.p[h][lane + 32] = p1;
       if (lane == 0) {
-        sm.alpha[h] = alpha;
-        sm.m[h] = m_new;
-        sm.l[h] = sm.l[h] * alpha + ps;
+        uint64_t mask = 0;
+        for (int i = 0; i < 32; ++i)
+          mask |= ((uint64_t)((m0 >> i) & 1u) << (2 * i)) | ((uint64_t)((m1 >> i) & 1u) << (2 * i + 1));
+        meta_mask[stage] = mask;
+        mbar_arrive_expect_tx(&kv_full[stage], kKVStage);
+      }
+      __syncwarp();
+      // lane g < 16 gathers rows 4g .. 4g+3 (held by lanes 2g and 2g+1)
+      const int g = lane & 15;
+      const int r0 = __shfl_sync(0xffffffffu, rows[0], 2 * g);
+      const int r1 = __shfl_sync(0xffffffffu, rows[1], 2 * g);
+      const int r2 = __shfl_sync(0xffffffffu, rows[0], 2 * g + 1);
+      const int r3 = __shfl_sync(0xffffffffu, rows[1], 2 * g + 1);
+      if (lane < 16) {
+        uint8_t* st = smem + OFF_KV + stage * kKVStage;
+#pragma unroll
+        for (int at = 0; at < 4; ++at)
+          tma_gather4(st + at * (kBK * 128) + g * 4 * 128, &tkv_lat, &kv_full[stage], 256 * rank + 64 * at, r0, r1,
+                      r2, r3);
+        tma_gather4(st + 4 * (kBK * 128) + g * 4 * 64, &tkv_rope, &kv_full[stage], 512 + 32 * rank, r0, r1, r2, r3);
       }
     }
-    __syncthreads();
-    // O += p V : thread owns value dims tid and tid + 256 for all 16 heads
-#pragma unroll
-    for (int h = 0; h < kHG; ++h) {
-      acc[h][0] *= sm.alpha[h];
-      acc[h][1] *= sm.alpha[h];
+    // drain: every gather has landed and every MMA commit has arrived
+    if (lane == 0 && !*abort_flag) {
+      for (int j = nblk; j < nblk + 2; ++j)
+        if (!mbar_wait(&kv_empty[j & 1], ((j >> 1) & 1) ^ 1, a.err)) break;
     }
-    for (int j = 0; j < kChunk; ++j) {
-      const float v0 = __bfloat162float(sm.kv[j][tid]);
-      const float v1 = __bfloat162float(sm.kv[j][tid + 256]);
+    __syncwarp();
+  } else if (warp == 1 && nblk > 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(smem + OFF_Q);
+      const uint32_t kv_base = smem_u32(smem + OFF_KV);
+      const uint32_t p_base = smem_u32(smem + OFF_P);
+      bool ok = mbar_wait(q_full, 0, a.err);
+      auto pv = [&](int i) -> bool {
+        if (!mbar_wait(p_full, i & 1, a.err)) return false;
+        tc_fence_after();
+        const uint32_t vb = kv_base + (i & 1) * kKVStage;
 #pragma unroll
-      for (int h = 0; h < kHG; ++h) {
-        const float p = sm.p[h][j];
-        acc[h][0] = fmaf(p, v0, acc[h][0]);
-        acc[h][1] = fmaf(p, v1, acc[h][1]);
+        for (int term = 0; term < 2; ++term)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss<true>(tmem, smem_desc(p_base + term * kPBytes + kk * 32, 16, 1024, 2),
+                         smem_desc(vb + kk * 2048, 8192, 1024, 2), IDESC_PV, i > 0 || term > 0 || kk > 0);
+        mma_commit(&kv_empty[i & 1]);
+        mma_commit(o_done);
+        return true;
+      };
+      for (int j = 0; j < nblk && ok && !*abort_flag; ++j) {
+        const int sb = j & 1;
+        if (!mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err) ||
+            !mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + 256 + kBK * sb;
+        const uint32_t kb = kv_base + (j & 1) * kKVStage;
+#pragma unroll
+        for (int at = 0; at < 4; ++at)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss<true>(d, smem_desc(q_base + at * kQLatBytes + kk * 32, 16, 1024, 2),
+                         smem_desc(kb + at * (kBK * 128) + kk * 32, 16, 1024, 2), IDESC_QK, (at | kk) != 0);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_ss<true>(d, smem_desc(q_base + 4 * kQLatBytes + kk * 32, 16, 512, 4),
+                       smem_desc(kb + 4 * (kBK * 128) + kk * 32, 16, 512, 4), IDESC_QK, true);
+        mma_commit(&s_full[sb]);
+        if (j >= 1 && !pv(j - 1)) {
+          ok = false;
+          break;
+        }
       }
+      if (ok && !*abort_flag) ok = pv(nblk - 1);
+      if (!ok) *abort_flag = 1;
     }
+    __syncwarp();
+  } else if (warp >= 4 && nblk > 0) {
+    // ---------------------------------------------------------------- softmax / exchange / epilogue
+    const int qw = warp - 4;
+    const int h = qw * 32 + lane;  // head row = TMEM lane
+    const uint32_t t_lane = tmem + ((uint32_t)(qw * 32) << 16);
+    float* xrow = reinterpret_cast<float*>(smem + OFF_X) + h * kXPitch;
+    const uint32_t x_peer = map_peer(smem_u32(xrow), peer);
+    const uint32_t x_full_peer = map_peer(smem_u32(x_full), peer);
+    const uint32_t x_free_peer = map_peer(smem_u32(x_free), peer);
+    uint8_t* p_row0 = smem + OFF_P + (h >> 3) * 1024 + (h & 7) * 128;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk && ok; ++j) {
+      const int sb = j & 1;
+      ok = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&s_full[sb], (j >> 1) & 1, a.err));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld32(t_lane + 256 + kBK * sb, v0);
+      tmem_ld32(t_lane + 256 + kBK * sb + 32, v1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      // exchange partial logits with the peer
+      ok = __all_sync(0xffffffffu, mbar_wait_cluster(x_free, (j & 1) ^ 1, a.err));
+      if (!ok) break;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        st_cluster_v4(x_peer + c * 16, __uint_as_float(v0[4 * c]), __uint_as_float(v0[4 * c + 1]),
+                      __uint_as_float(v0[4 * c + 2]), __uint_as_float(v0[4 * c + 3]));
+        st_cluster_v4(x_peer + 128 + c * 16, __uint_as_float(v1[4 * c]), __uint_as_float(v1[4 * c + 1]),
+                      __uint_as_float(v1[4 * c + 2]), __uint_as_float(v1[4 * c + 3]));
+      }
+      mbar_arrive_remote(x_full_peer);
+      ok = __all_sync(0xffffffffu, mbar_wait_cluster(x_full, j & 1, a.err));
+      if (!ok) break;
+      float s[64];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float4 pv4 = reinterpret_cast<const float4*>(xrow)[c];
+        const uint32_t* mine = c < 8 ? &v0[4 * c] : &v1[4 * (c - 8)];
+        s[4 * c + 0] = __uint_as_float(mine[0]) + pv4.x;
+        s[4 * c + 1] = __uint_as_float(mine[1]) + pv4.y;
+        s[4 * c + 2] = __uint_as_float(mine[2]) + pv4.z;
+        s[4 * c + 3] = __uint_as_float(mine[3]) + pv4.w;
+      }
+      mbar_arrive_remote(x_free_peer);
+      // validity of the block's rows (written before the stage's TMA was armed)
+      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err));
+      if (!ok) break;
+      const uint64_t mask = meta_mask[j & 1];
+      float mblk = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        s[i] = ((mask >> i) & 1ull) ? s[i] * a.scale_log2 : -INFINITY;
+        mblk = fmaxf(mblk, s[i]);
+      }
+      const bool move = mblk > m_ref + kRescaleThreshold;
+      const float m_new = move ? mblk : m_ref;
+      const float alpha = move ? exp2f(m_ref - m_new) : 1.f;  // exp2(-inf) = 0 on the first block
+      uint32_t pk[32], pl[32];
+      float psum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float e0 = m_new == -INFINITY ? 0.f : exp2f(s[2 * i] - m_new);
+        const float e1 = m_new == -INFINITY ? 0.f : exp2f(s[2 * i + 1] - m_new);
+        psum += e0 + e1;
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(e0, e1);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(e0 - __low2float(hi), e1 - __high2float(hi));
+        pk[i] = *reinterpret_cast<const uint32_t*>(&hi);
+        pl[i] = *reinterpret_cast<const uint32_t*>(&lo);
+      }
+      // PV of the previous block must be complete before O is touched or P's buffer reused
+      if (j >= 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, a.err));
+        if (!ok) break;
+        tc_fence_after();
+        // TMEM loads/stores are warp-wide: if any head of the warp moved its
+        // maximum, the whole warp rescales (alpha = 1 leaves a row exact).
+        if (__any_sync(0xffffffffu, move && m_ref != -INFINITY)) {
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_lane + 32 * c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_lane + 32 * c, o);
+          }
+          tmem_st_wait();
+        }
+      }
+      l = l * alpha + psum;
+      m_ref = m_new;
+      // P's buffer is free: PV of the previous block has completed (o_done above)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        *reinterpret_cast<uint4*>(p_row0 + ((c ^ (h & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(p_row0 + kPBytes + ((c ^ (h & 7)) << 4)) =
+            make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // epilogue: O / l for this CTA's 256 value dims.  tcgen05.ld is warp-wide,
+    // so a warp with any valid head loads; only the stores test h < H.
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(o_done, (nblk - 1) & 1, a.err));
+    if (ok) {
+      tc_fence_after();
+      const bool store = h < a.H;
+      if (qw * 32 < a.H) {
+        const float m_nat = m_ref * kLn2;
+        if (a.splits == 1) {
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          const int64_t base = ((int64_t)t * a.H + h) * kDV + 256 * rank;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_lane + 32 * c, o);
+            tmem_ld_wait();
+            if (!store) continue;
+            if (a.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                     __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint32_t w[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(o[8 * i + 2 * k]) * inv,
+                                                                  __uint_as_float(o[8 * i + 2 * k + 1]) * inv);
+                  w[k] = *reinterpret_cast<const uint32_t*>(&v2);
+                }
+                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+          }
+          if (store && rank == 0 && a.lse) a.lse[(int64_t)t * a.H + h] = m_nat + logf(l);
+        } else {
+          const int64_t prow = ((int64_t)t * a.splits + sp) * a.H + h;
+          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * kDV + 256 * rank);
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_lane + 32 * c, o);
+            tmem_ld_wait();
+            if (!store) continue;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[8 * c + i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                           __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+          }
+          if (store && rank == 0) a.part_ml[prow] = make_float2(m_nat, l);
+        }
+      }
+    } else {
+      *abort_flag = 1;
+    }
+    __syncwarp();
   }
+  tc_fence_before();
   __syncthreads();
-  if (splits == 1) {
-#pragma unroll
-    for (int h = 0; h < kHG; ++h) {
-      const float l = sm.l[h];
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int64_t o = ((int64_t)t * H + hg * kHG + h) * kDV;
-      store_out(out, out_f32, o + tid, acc[h][0] * inv);
-      store_out(out, out_f32, o + tid + 256, acc[h][1] * inv);
-    }
-    if (lse && tid < kHG) lse[(int64_t)t * H + hg * kHG + tid] = sm.m[tid] + logf(sm.l[tid]);
-  } else {
-#pragma unroll
-    for (int h = 0; h < kHG; ++h) {
-      const int64_t o = (((int64_t)t * splits + sp) * H + hg * kHG + h) * kDV;
-      part_o[o + tid] = acc[h][0];
-      part_o[o + tid + 256] = acc[h][1];
-    }
-    if (tid < kHG) part_ml[((int64_t)t * splits + sp) * H + hg * kHG + tid] = make_float2(sm.m[tid], sm.l[tid]);
+  cluster_sync();  // no peer still writes into this CTA's shared memory
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -216,10 +465,49 @@ k_combine(int H, int splits, const float* __restrict__ part_o, const float2* __r
   if (lse && tid == 0) lse[(int64_t)t * H + h] = M + logf(L);
 }
 
+int attn_splits(int T, int K) {
+  const int clusters = 74;  // 148 SMs / 2
+  if (T >= clusters) return 1;
+  const int want = clusters / T;
+  const int most = (K + kBK - 1) / kBK;
+  return want < 1 ? 1 : (want < most ? want : most);
+}
+
+int keys_per_split(int K, int splits) {
+  const int ks = (K + splits - 1) / splits;
+  return (ks + kBK - 1) / kBK * kBK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 [rows, 576] map with a box of box_x x box_y and the given swizzle.
+bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_x, uint32_t box_y,
+                  CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kDQK, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kDQK * 2};
+  const cuuint32_t box[2] = {box_x, box_y};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 size_t sparse_mla_partials_bytes(int T, int K, int H) {
-  const int splits = attn_splits(T, H, K);
+  const int splits = attn_splits(T, K);
   if (splits == 1) return 0;
   return (size_t)T * splits * H * (kDV * sizeof(float) + sizeof(float2));
 }
@@ -228,25 +516,29 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16
                               const int32_t* idx, int K, int H, float scale, void* out, bool out_f32,
                               float* lse, void* partials, uint32_t* err, cudaStream_t st) {
   const int T = s.num_tokens;
-  int splits = attn_splits(T, H, K);
+  int splits = attn_splits(T, K);
   const int ks = keys_per_split(K, splits);
   splits = (K + ks - 1) / ks;
   float* part_o = reinterpret_cast<float*>(partials);
   float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)T * splits * H * kDV);
-  const size_t smem = sizeof(SmemLayout);
-  cudaError_t e = cudaSuccess;
-  static thread_local int attr_set_for = -1;  // set once per device and thread, outside any capture
+  const uint64_t R = (uint64_t)s.num_phys_pages * kPage;
+  CUtensorMap tq_lat, tq_rope, tkv_lat, tkv_rope;
+  if (!make_map_576(&tq_lat, q, (uint64_t)T * H, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_576(&tq_rope, q, (uint64_t)T * H, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_576(&tkv_lat, kv, R, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_576(&tkv_rope, kv, R, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  static thread_local int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (attr_set_for != dev) {
-    e = cudaFuncSetAttribute(k_sparse_mla_simple, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (attr_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(k_sparse_mla_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set_for = dev;
+    attr_dev = dev;
   }
-  dim3 grid(T, H / kHG, splits);
-  k_sparse_mla_simple<<<grid, kThreads, smem, st>>>(s, tm, q, kv, idx, K, H, scale, ks, splits, out, out_f32, lse, part_o,
-                                                     part_ml, err);
-  e = counted(cudaGetLastError());
+  AttnArgs a{s, tm, idx, K, H, ks, splits, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
+  k_sparse_mla_tc<<<2 * T * splits, 256, SMEM_BYTES, st>>>(tq_lat, tq_rope, tkv_lat, tkv_rope, a);
+  cudaError_t e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
   k_combine<<<dim3(T, H), 128, 0, st>>>(H, splits, part_o, part_ml, tm.pos, out, out_f32, lse);
   return counted(cudaGetLastError());
