@@ -144,23 +144,26 @@ PlanBufs plan_bufs(void* ws, const Layout& L) {
   return p;
 }
 
-// indexer launch sequence shared by dsa_index_scores and the fused call
-// (the plan has already been launched)
+// Indexer launch sequence shared by dsa_index_scores and the fused call: one
+// prep launch (plan, FP8 query quantization, zeroing of `zero`) and the
+// indexer, which also accumulates Top-K's first-digit histogram into `hist`
+// when that is given (one token per group).
 dsa_status_t run_indexer(const dsa_seqs_t* seqs, const SeqsDev& sd, const PlanBufs& plan, int tg, const void* qI,
                          const float* w, const void* kI, const float* kI_scale, dsa_ki_dtype_t ki_dtype,
-                         float* scores, int64_t ld, void* ws, const Layout& L, uint32_t* err, cudaStream_t st) {
+                         float* scores, int64_t ld, void* ws, const Layout& L, uint32_t* hist, uint32_t* zero,
+                         int64_t zero_words, uint32_t* err, cudaStream_t st) {
   const bool fp8 = ki_dtype == DSA_KI_FP8_E4M3;
   const void* q_operand = qI;
   const float* w_operand = w;
+  uint8_t* codes = fp8 ? at<uint8_t>(ws, L.q_codes) : nullptr;
+  float* w_scaled = fp8 ? at<float>(ws, L.w_scaled) : nullptr;
+  DSA_CUDA(launch_prep(sd, tg, indexer_item_tiles(tg), plan, fp8 ? reinterpret_cast<const __nv_bfloat16*>(qI) : nullptr,
+                       w, codes, w_scaled, zero, zero_words, err, st));
   if (fp8) {
-    uint8_t* codes = at<uint8_t>(ws, L.q_codes);
-    float* w_scaled = at<float>(ws, L.w_scaled);
-    DSA_CUDA(launch_quantize_index_query(reinterpret_cast<const __nv_bfloat16*>(qI), w, seqs->num_q_tokens, codes,
-                                         w_scaled, st));
     q_operand = codes;
     w_operand = w_scaled;
   }
-  DSA_CUDA(launch_index_scores(sd, plan, tg, q_operand, w_operand, kI, kI_scale, fp8, scores, ld, err, st));
+  DSA_CUDA(launch_index_scores(sd, plan, tg, q_operand, w_operand, kI, kI_scale, fp8, scores, ld, hist, err, st));
   return DSA_OK;
 }
 
@@ -201,8 +204,8 @@ dsa_status_t dsa_index_scores(const dsa_seqs_t* seqs, const void* qI, const floa
   const SeqsDev sd = to_dev(seqs);
   const PlanBufs plan = plan_bufs(ws, L);
   const int tg = indexer_group_tokens(seqs->num_q_tokens, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
-  DSA_CUDA(launch_plan(sd, tg, indexer_item_tiles(tg), plan, err, st));
-  return run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, ld, ws, L, err, st);
+  return run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, ld, ws, L, nullptr, nullptr, 0, err,
+                     st);
 }
 
 dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, int K, int32_t* idx, void* ws,
@@ -215,7 +218,8 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row
   const Layout L = make_layout(DSA_OP_TOPK, T, 1, (int)ld, K, 16);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
   return cuda_status(
-      launch_topk(scores, ld, T, row_len, nullptr, K, idx, at<void>(ws, L.topk), at<uint32_t>(ws, 0), (cudaStream_t)stream));
+      launch_topk(scores, ld, T, row_len, nullptr, K, idx, at<void>(ws, L.topk), false, at<uint32_t>(ws, 0),
+                  (cudaStream_t)stream));
 }
 
 dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const void* kv, const int32_t* idx, int K,
@@ -255,10 +259,15 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const f
   TokenMap tm{plan.tok_seq, plan.tok_pos};
   float* scores = at<float>(ws, L.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
-  const int tg = indexer_group_tokens(seqs->num_q_tokens, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
-  DSA_CUDA(launch_plan(sd, tg, indexer_item_tiles(tg), plan, err, st));
-  DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, err, st));
-  DSA_CUDA(launch_topk(scores, L.ld, seqs->num_q_tokens, nullptr, tm.pos, K, idx, at<void>(ws, L.topk), err, st));
+  const int T = seqs->num_q_tokens;
+  const int tg = indexer_group_tokens(T, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
+  // one token per group: the indexer also builds Top-K's first-digit histogram
+  const bool fuse_hist = tg == 1 && topk_uses_hist(T, L.ld);
+  uint32_t* hist = fuse_hist ? topk_hist_in_scratch(at<void>(ws, L.topk), T) : nullptr;
+  uint32_t* zero = fuse_hist ? at<uint32_t>(ws, L.topk) : nullptr;  // Top-K's counters + histogram
+  DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, hist, zero,
+                      fuse_hist ? topk_zero_words(T) : 0, err, st));
+  DSA_CUDA(launch_topk(scores, L.ld, T, nullptr, tm.pos, K, idx, at<void>(ws, L.topk), hist != nullptr, err, st));
   DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
                              out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));

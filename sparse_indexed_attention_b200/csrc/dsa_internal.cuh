@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/dsa.h"
 
 namespace dsa {
@@ -23,6 +25,28 @@ constexpr uint32_t kErrTimeout = 2u;
 
 __device__ __forceinline__ void raise_error(uint32_t* err, uint32_t bit) {
   if ((*(volatile uint32_t*)err & bit) == 0) atomicOr(err, bit);
+}
+
+// Order-preserving 32-bit key of a score: larger score <=> larger key;
+// -0.0 ranks equal to +0.0.  Shared by Top-K and the indexer epilogue (which
+// builds Top-K's first-digit histogram while it writes the scores).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-K's first digit: the top 11 key bits.
+constexpr int kTopkHistBins = 2048;
+constexpr int kTopkLowBits = 21;
+
+// Adds one to hist[bin]; lanes of the warp holding the same bin add once.
+// Every lane of the warp must call it (active or not).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  const uint32_t act = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const uint32_t peers = __match_any_sync(act, bin);
+  if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
 }
 
 // Per query token: its sequence and absolute position (-1 = invalid token).
@@ -50,6 +74,31 @@ struct SeqsDev {
   const int32_t* ctx_len;
   const int32_t* page_table;
 };
+
+// Programmatic dependent launch: every kernel of the path is launched with
+// programmatic stream serialization, so its launch and its set-up (barrier
+// init, TMEM allocation, tensor-map prefetch) overlap the previous kernel's
+// tail.  A kernel touches global memory only after pdl_wait(), which returns
+// once the previous grid has completed and its writes are visible, and lets
+// the next kernel launch (pdl_trigger) right after.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Kernels launched by the current host thread since its last entry-point call
 // began (reported by dsa_launches_in_last_call).
@@ -85,15 +134,26 @@ inline int64_t plan_max_items(int T, int B, int max_ctx, int tg) {
 
 // ---- launchers (each returns cudaGetLastError() of its launch) ----
 cudaError_t launch_plan(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err, cudaStream_t st);
+// Plan + (FP8 cache: qI quantization) + zeroing of `zero_words` words, one launch.
+cudaError_t launch_prep(const SeqsDev& s, int tg, int ch, const PlanBufs& plan, const __nv_bfloat16* qI,
+                        const float* w, uint8_t* codes, float* w_scaled, uint32_t* zero, int64_t zero_words,
+                        uint32_t* err, cudaStream_t st);
 cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w, int T, uint8_t* codes,
                                         float* w_scaled, cudaStream_t st);
 // FP8 cache: codes/w_scaled from the quantizer; bf16 cache: qI/w directly.
+// hist (may be null; used for one token per group): Top-K first-digit histogram to accumulate into.
 cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
                                 const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
-                                float* scores, int64_t ld, uint32_t* err, cudaStream_t st);
+                                float* scores, int64_t ld, uint32_t* hist, uint32_t* err, cudaStream_t st);
 size_t topk_scratch_bytes(int T, int64_t ld, int K);
+// Several CTAs per row use a region at the head of the scratch that must be
+// zero when they start (row counters + first-digit histogram, topk_zero_words
+// words); `hist_ready` says the caller has zeroed it and filled the histogram.
+bool topk_uses_hist(int T, int64_t ld);
+int64_t topk_zero_words(int T);
+uint32_t* topk_hist_in_scratch(void* scratch, int T);
 cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, const int32_t* tok_pos,
-                        int K, int32_t* idx, void* scratch, uint32_t* err, cudaStream_t st);
+                        int K, int32_t* idx, void* scratch, bool hist_ready, uint32_t* err, cudaStream_t st);
 size_t sparse_mla_partials_bytes(int T, int K, int H);
 cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16* q, const __nv_bfloat16* kv,
                               const int32_t* idx, int K, int H, float scale, void* out, bool out_f32,

@@ -16,9 +16,10 @@
 //    bf16) into a ring of TMEM accumulators; tcgen05.commit frees the stage
 //    and publishes the accumulator.
 //  * warp 2: allocates and frees TMEM.
-//  * warps 4-7: epilogue.  Thread r owns TMEM lane r = key row r, so the
-//    ReLU, the head weighting and the reduction over heads stay inside one
-//    thread; no [T, H_I, N] value ever leaves the SM.
+//  * warps 4-11: epilogue, two warpgroups taking alternate tiles.  Thread r
+//    of a warpgroup owns TMEM lane r = key row r, so the ReLU, the head
+//    weighting and the reduction over heads stay inside one thread; no
+//    [T, H_I, N] value ever leaves the SM.
 // The CTA grid is persistent (one CTA per SM) over the work items of k_plan.
 #include <cudaTypedefs.h>
 
@@ -30,13 +31,16 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kEpiWarps = 8;                 // two epilogue warpgroups (warps 4-11)
+constexpr int kIdxThreads = (4 + kEpiWarps) * 32;
+
 template <bool kBf16, int TG>
 struct IdxCfg {
   static constexpr int N = 64 * TG;                        // MMA N: heads x tokens of a group
   static constexpr int A_BYTES = kBf16 ? 32768 : 16384;    // 128 keys x d_I
   static constexpr int B_BYTES = kBf16 ? N * 256 : N * 128;
   static constexpr int KSTEPS = kBf16 ? 8 : 4;             // 32-byte K steps per tile
-  static constexpr int NS = kBf16 ? (TG == 1 ? 4 : 3) : (TG == 1 ? 8 : 6);
+  static constexpr int NS = kBf16 ? 3 : (TG == 1 ? 8 : 6);
   static constexpr int NACC = (512 / N) < 4 ? (512 / N) : 4;
   static constexpr int TMEM_COLS = (NACC * N) <= 256 ? 256 : 512;
   // shared-memory layout (offsets from a 1024-aligned base)
@@ -44,7 +48,8 @@ struct IdxCfg {
   static constexpr int OFF_B = OFF_A + NS * A_BYTES;
   static constexpr int OFF_SC = OFF_B + 2 * B_BYTES;       // NS x 128 fp32 row scales
   static constexpr int OFF_W = OFF_SC + NS * 512;          // 2 x TG x 64 fp32 head weights
-  static constexpr int OFF_BAR = OFF_W + 2 * TG * 256;
+  static constexpr int OFF_HIST = OFF_W + 2 * TG * 256;   // TG == 1: per-epilogue-warp Top-K histograms
+  static constexpr int OFF_BAR = OFF_HIST + (TG == 1 ? kEpiWarps * kTopkHistBins * 4 : 0);
   static constexpr int NBARS = 2 * NS + 4 + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
@@ -61,11 +66,26 @@ struct IdxArgs {
   const float* kI_scale;   // [R] (FP8) or null
   float* scores;
   int64_t ld;
+  uint32_t* hist;          // TG == 1 only, may be null: Top-K first-digit histogram [T][2048]
   uint32_t* err;
 };
 
+// Adds one epilogue warp's histogram of the current token to the global one
+// and clears it (warp-private, so only the warp synchronises).
+__device__ __forceinline__ void flush_hist(uint32_t* sh, uint32_t* gh, int t, int lane) {
+  __syncwarp();
+  for (int i = lane; i < kTopkHistBins; i += 32) {
+    const uint32_t v = sh[i];
+    if (v) {
+      atomicAdd(gh + (int64_t)t * kTopkHistBins + i, v);
+      sh[i] = 0u;
+    }
+  }
+  __syncwarp();
+}
+
 template <bool kBf16, int TG>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kIdxThreads, 1)
 k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                   const IdxArgs a) {
   using C = IdxCfg<kBf16, TG>;
@@ -91,7 +111,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b_full[i], 1);
-      mbar_init(&b_empty[i], 1 + 4);
+      mbar_init(&b_empty[i], 1 + kEpiWarps);
     }
     for (int i = 0; i < C::NACC; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -108,6 +128,8 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the plan and the quantized query come from the previous kernel
+  pdl_trigger();
 
   // this CTA's contiguous share of the work items
   const int n_items = a.plan.counts[1];
@@ -254,11 +276,20 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp - 4;            // TMEM lane quarter of this warp
+    // Two warpgroups take alternate tiles (tile i -> warpgroup i & 1, which
+    // therefore owns every other TMEM accumulator); both follow every group.
+    const int q = (warp - 4) & 3;      // TMEM lane quarter of this warp
+    const int wg = (warp - 4) >> 2;    // epilogue warpgroup
     const int r = q * 32 + lane;       // key row of the tile
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
-    int stage = 0, sphase = 0, acc = 0, aphase = 0, prev_g = -1, gcount = 0, slot = 0;
+    int stage = 0, sphase = 0, acc = 0, aphase = 0, prev_g = -1, gcount = 0, slot = 0, prev_t = -1, ti = 0;
     float wreg[64];
+    uint32_t* sh_hist = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST) + (warp - 4) * kTopkHistBins;
+    const bool do_hist = TG == 1 && a.hist != nullptr;
+    if (do_hist) {
+      for (int i = lane; i < kTopkHistBins; i += 32) sh_hist[i] = 0u;
+      __syncwarp();
+    }
     int4 na = make_int4(0, 0, 0, 0), nb = na;
     if (it_lo < it_hi) { na = recs[2 * it_lo]; nb = recs[2 * it_lo + 1]; }
     for (int it = it_lo; it < it_hi && !*abort_flag; ++it) {
@@ -270,6 +301,8 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
           __syncwarp();
           if (lane == 0) mbar_arrive(&b_empty[slot]);
         }
+        if (do_hist && prev_t >= 0 && prev_t != grp.y) flush_hist(sh_hist, a.hist, prev_t, lane);
+        prev_t = grp.y;
         slot = gcount & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err))) { *abort_flag = 1; break; }
         if constexpr (TG == 1) {
@@ -279,42 +312,52 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
         prev_g = item.x;
         ++gcount;
       }
-      for (int tile = item.y; tile < item.z; ++tile) {
-        bool okw = mbar_wait(&acc_full[acc], aphase, a.err);
-        // the row scales arrived with the stage's TMA; observe that completion here too
-        if (!kBf16) okw = okw && mbar_wait(&full[stage], sphase, a.err);
-        if (!__all_sync(0xffffffffu, okw)) { *abort_flag = 1; break; }
-        tc_fence_after();
-        const float sk = kBf16 ? 1.f : sc_smem[stage * 128 + r];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
-        const int s = tile * 128 + r;
+      for (int tile = item.y; tile < item.z; ++tile, ++ti) {
+        if ((ti & 1) == wg) {
+          bool okw = mbar_wait(&acc_full[acc], aphase, a.err);
+          // the row scales arrived with the stage's TMA; observe that completion here too
+          if (!kBf16) okw = okw && mbar_wait(&full[stage], sphase, a.err);
+          if (!__all_sync(0xffffffffu, okw)) { *abort_flag = 1; break; }
+          tc_fence_after();
+          const float sk = kBf16 ? 1.f : sc_smem[stage * 128 + r];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[stage]);
+          const int s = tile * 128 + r;
 #pragma unroll 1
-        for (int k = 0; k < TG; ++k) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(t_lane + acc * C::N + k * 64, v0);
-          tmem_ld32(t_lane + acc * C::N + k * 64 + 32, v1);
-          tmem_ld_wait();
-          if (k == TG - 1) {  // every TMEM read of this accumulator is complete
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
-          }
-          const float* wk = w_smem + slot * TG * 64 + k * 64;
-          float sum = 0.f;
+          for (int k = 0; k < TG; ++k) {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(t_lane + acc * C::N + k * 64, v0);
+            tmem_ld32(t_lane + acc * C::N + k * 64 + 32, v1);
+            tmem_ld_wait();
+            if (k == TG - 1) {  // every TMEM read of this accumulator is complete
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            }
+            const float* wk = w_smem + slot * TG * 64 + k * 64;
+            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;  // four chains instead of one
 #pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            const float w0 = TG == 1 ? wreg[h] : wk[h];
-            const float w1 = TG == 1 ? wreg[h + 32] : wk[h + 32];
-            sum = fmaf(w0, fmaxf(__uint_as_float(v0[h]), 0.f), sum);
-            sum = fmaf(w1, fmaxf(__uint_as_float(v1[h]), 0.f), sum);
+            for (int h = 0; h < 32; h += 2) {
+              const float w0 = TG == 1 ? wreg[h] : wk[h];
+              const float w1 = TG == 1 ? wreg[h + 1] : wk[h + 1];
+              const float w2 = TG == 1 ? wreg[h + 32] : wk[h + 32];
+              const float w3 = TG == 1 ? wreg[h + 33] : wk[h + 33];
+              p0 = fmaf(w0, fmaxf(__uint_as_float(v0[h]), 0.f), p0);
+              p1 = fmaf(w1, fmaxf(__uint_as_float(v0[h + 1]), 0.f), p1);
+              p2 = fmaf(w2, fmaxf(__uint_as_float(v1[h]), 0.f), p2);
+              p3 = fmaf(w3, fmaxf(__uint_as_float(v1[h + 1]), 0.f), p3);
+            }
+            const float score = ((p0 + p1) + (p2 + p3)) * sk;
+            const bool valid = k < grp.z && s <= grp.w + k;
+            if (valid) a.scores[(int64_t)(grp.y + k) * a.ld + s] = score;
+            if (do_hist) hist_add(sh_hist, order_key(score) >> kTopkLowBits, valid);
           }
-          if (k < grp.z && s <= grp.w + k) a.scores[(int64_t)(grp.y + k) * a.ld + s] = sum * sk;
         }
         if (++stage == C::NS) { stage = 0; sphase ^= 1; }
         if (++acc == C::NACC) { acc = 0; aphase ^= 1; }
       }
     }
+    if (do_hist && prev_t >= 0) flush_hist(sh_hist, a.hist, prev_t, lane);
     __syncwarp();
   }
   tc_fence_before();
@@ -372,7 +415,9 @@ cudaError_t launch_tc(const CUtensorMap& mk, const CUtensorMap& mq, const IdxArg
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  k_index_scores_tc<kBf16, TG><<<sm_count(), 256, C::SMEM, st>>>(mk, mq, a);
+  cudaError_t e = launch_pdl(k_index_scores_tc<kBf16, TG>, dim3(sm_count()), dim3(kIdxThreads), (size_t)C::SMEM, st, mk,
+                             mq, a);
+  if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }
 
@@ -380,14 +425,14 @@ cudaError_t launch_tc(const CUtensorMap& mk, const CUtensorMap& mq, const IdxArg
 
 cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
                                 const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
-                                float* scores, int64_t ld, uint32_t* err, cudaStream_t st) {
+                                float* scores, int64_t ld, uint32_t* hist, uint32_t* err, cudaStream_t st) {
   const bool bf16 = !fp8;
   const uint64_t R = (uint64_t)s.num_phys_pages * kPage;
   const uint64_t qrows = (uint64_t)s.num_tokens * kHI;
   CUtensorMap mk, mq;
   if (!make_map(&mk, kI, bf16, kDI, R, bf16 ? 64 : 128, 64)) return cudaErrorInvalidValue;
   if (!make_map(&mq, q_operand, bf16, kDI, qrows, bf16 ? 64 : 128, 64 * tg)) return cudaErrorInvalidValue;
-  IdxArgs a{s, plan, w_operand, kI_scale, scores, ld, err};
+  IdxArgs a{s, plan, w_operand, kI_scale, scores, ld, tg == 1 ? hist : nullptr, err};
   if (fp8) {
     if (tg == 1) return launch_tc<false, 1>(mk, mq, a, st);
     if (tg == 4) return launch_tc<false, 4>(mk, mq, a, st);

@@ -66,7 +66,7 @@ __device__ __forceinline__ bool seq_ok(const SeqsDev& s, int b, int* q_len_out, 
 //                         {tile_begin, tile_end, g, 0}: a run of <= `ch` key tiles
 //                         of 128 positions (tiles cover 0 .. last pos);
 //   counts                {G, I}.
-__global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBufs p, uint32_t* err) {
+__device__ __forceinline__ void plan_body(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err) {
   __shared__ int warp_buf[33];
   const int tid = threadIdx.x;
   for (int t = tid; t < s.num_tokens; t += blockDim.x) {
@@ -160,18 +160,23 @@ __global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBu
   }
 }
 
+__global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBufs p, uint32_t* err) {
+  pdl_wait();
+  pdl_trigger();
+  plan_body(s, tg, ch, p, err);
+}
+
 cudaError_t launch_plan(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err, cudaStream_t st) {
-  k_plan<<<1, 1024, 0, st>>>(s, tg, ch, p, err);
+  cudaError_t e = launch_pdl(k_plan, dim3(1), dim3(1024), 0, st, s, tg, ch, p, err);
+  if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }
 
-// One warp per (token, head) row of 128 bf16: lane l holds elements 4l..4l+3.
-__global__ void k_quantize_index_query(const __nv_bfloat16* __restrict__ qI, const float* __restrict__ w,
-                                       int rows, uint8_t* __restrict__ codes, float* __restrict__ w_scaled) {
-  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
-  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qI + (int64_t)warp * kDI) + lane);
+// One warp quantizes one (token, head) row of 128 bf16: lane l holds elements 4l..4l+3.
+__device__ __forceinline__ void quant_row(const __nv_bfloat16* __restrict__ qI, const float* __restrict__ w, int row,
+                                          uint8_t* __restrict__ codes, float* __restrict__ w_scaled) {
+  const int lane = threadIdx.x & 31;
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qI + (int64_t)row * kDI) + lane);
   __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
   __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
   float x[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
@@ -194,9 +199,65 @@ __global__ void k_quantize_index_query(const __nv_bfloat16* __restrict__ qI, con
   for (int i = 0; i < 4; ++i) y[i] = (float)ldexp((double)x[i], -e);
   __nv_fp8x2_storage_t c01 = __nv_cvt_float2_to_fp8x2(make_float2(y[0], y[1]), __NV_SATFINITE, __NV_E4M3);
   __nv_fp8x2_storage_t c23 = __nv_cvt_float2_to_fp8x2(make_float2(y[2], y[3]), __NV_SATFINITE, __NV_E4M3);
-  uint32_t packed = (uint32_t)c01 | ((uint32_t)c23 << 16);
-  reinterpret_cast<uint32_t*>(codes + (int64_t)warp * kDI)[lane] = packed;
-  if (lane == 0) w_scaled[warp] = (float)ldexp((double)__ldg(w + warp), e);
+  const uint32_t packed = (uint32_t)c01 | ((uint32_t)c23 << 16);
+  reinterpret_cast<uint32_t*>(codes + (int64_t)row * kDI)[lane] = packed;
+  if (lane == 0) w_scaled[row] = (float)ldexp((double)__ldg(w + row), e);
+}
+
+__global__ void k_quantize_index_query(const __nv_bfloat16* __restrict__ qI, const float* __restrict__ w,
+                                       int rows, uint8_t* __restrict__ codes, float* __restrict__ w_scaled) {
+  pdl_wait();
+  pdl_trigger();
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (row < rows) quant_row(qI, w, row, codes, w_scaled);
+}
+
+// Everything the indexer needs before it starts, in one launch: block 0 builds
+// the plan; the other blocks quantize the index query (32 rows per block, FP8
+// cache only) and zero a scratch range (Top-K's first-digit histogram).
+struct PrepArgs {
+  SeqsDev s;
+  int tg, ch;
+  PlanBufs plan;
+  uint32_t* err;
+  const __nv_bfloat16* qI;
+  const float* w;
+  uint8_t* codes;
+  float* w_scaled;
+  int quant_rows;
+  uint32_t* zero;
+  int64_t zero_words;
+};
+
+__global__ void __launch_bounds__(1024) k_prep(const PrepArgs a) {
+  pdl_wait();  // the previous call may still read the plan and the scratch this kernel rewrites
+  pdl_trigger();
+  if (blockIdx.x == 0) {
+    plan_body(a.s, a.tg, a.ch, a.plan, a.err);
+    return;
+  }
+  const int b = blockIdx.x - 1, nb = gridDim.x - 1;
+  if (a.qI) {
+    const int row = b * 32 + (threadIdx.x >> 5);
+    if (row < a.quant_rows) quant_row(a.qI, a.w, row, a.codes, a.w_scaled);
+  }
+  if (a.zero) {
+    const int64_t per = (a.zero_words + nb - 1) / nb;
+    const int64_t z0 = (int64_t)b * per, z1 = min(a.zero_words, z0 + per);
+    for (int64_t i = z0 + threadIdx.x; i < z1; i += blockDim.x) a.zero[i] = 0u;
+  }
+}
+
+cudaError_t launch_prep(const SeqsDev& s, int tg, int ch, const PlanBufs& plan, const __nv_bfloat16* qI,
+                        const float* w, uint8_t* codes, float* w_scaled, uint32_t* zero, int64_t zero_words,
+                        uint32_t* err, cudaStream_t st) {
+  PrepArgs a{s, tg, ch, plan, err, qI, w, codes, w_scaled, qI ? s.num_tokens * kHI : 0, zero, zero ? zero_words : 0};
+  const int64_t nq = qI ? ((int64_t)s.num_tokens * kHI + 31) / 32 : 0;
+  const int64_t nz = zero ? (zero_words + 4095) / 4096 : 0;
+  const int64_t extra = nq > nz ? nq : nz;
+  cudaError_t e = launch_pdl(k_prep, dim3((unsigned)(1 + extra)), dim3(1024), 0, st, a);
+  if (e != cudaSuccess) return e;
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w, int T, uint8_t* codes,
@@ -204,7 +265,8 @@ cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w,
   int rows = T * kHI;
   int threads = 256;
   int blocks = (rows * 32 + threads - 1) / threads;
-  k_quantize_index_query<<<blocks, threads, 0, st>>>(qI, w, rows, codes, w_scaled);
+  cudaError_t e = launch_pdl(k_quantize_index_query, dim3(blocks), dim3(threads), 0, st, qI, w, rows, codes, w_scaled);
+  if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }
 

@@ -109,11 +109,8 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   const uint32_t peer = rank ^ 1u;
   const int cluster = blockIdx.x >> 1;
   const int t = cluster / a.splits, sp = cluster % a.splits;
-  const int pos = a.tm.pos[t];
-  const int b = a.tm.seq[t];
   const int kbeg = sp * a.ks;
   const int kend = min(a.K, kbeg + a.ks);
-  const int nblk = (pos >= 0 && kend > kbeg) ? (kend - kbeg + kBK - 1) / kBK : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -123,10 +120,10 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
     }
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 4);   // one arrival per softmax warp
     mbar_init(o_done, 1);
-    mbar_init(x_full, 128);
-    mbar_init(x_free, 128);
+    mbar_init(x_full, 4);   // one arrival per peer softmax warp
+    mbar_init(x_free, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -139,6 +136,11 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   cluster_sync();  // the peer's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;  // O at columns [0,256), S buffers at [256,320), [320,384)
+  pdl_wait();  // the token map and the index lists come from earlier kernels
+  pdl_trigger();
+  const int pos = a.tm.pos[t];
+  const int b = a.tm.seq[t];
+  const int nblk = (pos >= 0 && kend > kbeg) ? (kend - kbeg + kBK - 1) / kBK : 0;
 
   if (warp == 0 && nblk > 0) {
     // ---------------------------------------------------------------- producer
@@ -295,7 +297,9 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         st_cluster_v4(x_peer + 128 + c * 16, __uint_as_float(v1[4 * c]), __uint_as_float(v1[4 * c + 1]),
                       __uint_as_float(v1[4 * c + 2]), __uint_as_float(v1[4 * c + 3]));
       }
-      mbar_arrive_remote(x_full_peer);
+      // the warp barrier orders every lane's stores before lane 0's cluster-scope release
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(x_full_peer);
       ok = __all_sync(0xffffffffu, mbar_wait_cluster(x_full, j & 1, a.err));
       if (!ok) break;
       float s[64];
@@ -308,7 +312,8 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         s[4 * c + 2] = __uint_as_float(mine[2]) + pv4.z;
         s[4 * c + 3] = __uint_as_float(mine[3]) + pv4.w;
       }
-      mbar_arrive_remote(x_free_peer);
+      __syncwarp();  // every lane has read its row of X
+      if (lane == 0) mbar_arrive_remote(x_free_peer);
       // validity of the block's rows (written before the stage's TMA was armed)
       ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err));
       if (!ok) break;
@@ -364,9 +369,10 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         *reinterpret_cast<uint4*>(p_row0 + kPBytes + ((c ^ (h & 7)) << 4)) =
             make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
       }
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();  // this thread's P stores -> visible to the tensor core
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
     }
     // epilogue: O / l for this CTA's 256 value dims.  tcgen05.ld is warp-wide,
     // so a warp with any valid head loads; only the stores test h < H.
@@ -443,6 +449,8 @@ __global__ void __launch_bounds__(128)
 k_combine(int H, int splits, const float* __restrict__ part_o, const float2* __restrict__ part_ml,
           const int32_t* __restrict__ tok_pos, void* __restrict__ out, bool out_f32, float* __restrict__ lse) {
   const int t = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (tok_pos[t] < 0) return;
   float M = -INFINITY;
   for (int i = 0; i < splits; ++i) M = fmaxf(M, part_ml[((int64_t)t * splits + i) * H + h].x);
@@ -537,10 +545,13 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16
     attr_dev = dev;
   }
   AttnArgs a{s, tm, idx, K, H, ks, splits, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
-  k_sparse_mla_tc<<<2 * T * splits, 256, SMEM_BYTES, st>>>(tq_lat, tq_rope, tkv_lat, tkv_rope, a);
-  cudaError_t e = counted(cudaGetLastError());
+  cudaError_t e = launch_pdl(k_sparse_mla_tc, dim3(2 * T * splits), dim3(256), (size_t)SMEM_BYTES, st, tq_lat, tq_rope,
+                             tkv_lat, tkv_rope, a);
+  if (e == cudaSuccess) e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
-  k_combine<<<dim3(T, H), 128, 0, st>>>(H, splits, part_o, part_ml, tm.pos, out, out_f32, lse);
+  e = launch_pdl(k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o, (const float2*)part_ml,
+                 tm.pos, out, out_f32, lse);
+  if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }
 

@@ -26,25 +26,11 @@ namespace dsa {
 
 namespace {
 
-constexpr int kHistBins = 2048;      // top 11 key bits
-constexpr int kLowBits = 21;
+constexpr int kHistBins = kTopkHistBins;  // top 11 key bits
+constexpr int kLowBits = kTopkLowBits;
 constexpr int kRowThreads = 1024;
 constexpr int kCandCap = 12288;      // candidates kept in shared memory by the one-CTA path
 constexpr int kChunkThreads = 512;
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;  // -0.0 ranks equal to +0.0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Adds one to hist[bin]; lanes of the warp holding the same bin add once.
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
-  const uint32_t act = __ballot_sync(0xffffffffu, active);
-  if (!active) return;
-  const uint32_t peers = __match_any_sync(act, bin);
-  if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-}
 
 // Exclusive block-wide prefix sum of v (blockDim.x a multiple of 32, <= 1024);
 // *total receives the sum.  Uses the 33-word scratch `buf`.
@@ -272,6 +258,8 @@ k_topk_row(const float* __restrict__ scores, int64_t ld, const int32_t* __restri
            const int32_t* __restrict__ tok_pos, int K, int32_t* __restrict__ idx, uint32_t* err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RowSmem& sm = *reinterpret_cast<RowSmem*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const float* __restrict__ row = scores + (int64_t)t * ld;
   int32_t* __restrict__ out = idx + (int64_t)t * K;
@@ -349,6 +337,8 @@ __global__ void __launch_bounds__(kChunkThreads)
 k_topk_hist(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
             const int32_t* __restrict__ tok_pos, int K, int chunk, uint32_t* __restrict__ ghist, uint32_t* err) {
   __shared__ uint32_t hist[kHistBins];
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.y, c = blockIdx.x;
   const int n = row_length(row_len, tok_pos, t, ld, err);
   const int b0 = c * chunk, b1 = min(n, b0 + chunk);
@@ -367,21 +357,129 @@ k_topk_hist(const float* __restrict__ scores, int64_t ld, const int32_t* __restr
     if (hist[i]) atomicAdd(&ghist[(int64_t)t * kHistBins + i], hist[i]);
 }
 
+constexpr int kMaxChunks = 64;
+constexpr int kSelCap = 4096;  // candidates staged in shared memory by the select step
+
+struct SelSmem {
+  uint32_t hist[kHistBins];
+  uint32_t hist128[128];
+  uint32_t buf[33];
+  uint32_t bin, above;
+  int sure_off[kMaxChunks + 1], cand_off[kMaxChunks + 1];
+  int32_t sure[kMaxK];
+  int32_t sel[kMaxK];
+  int32_t cpos[kSelCap];
+  uint32_t ckey[kSelCap];
+  int last;
+};
+
+// Index of the last offset <= i in off[0..C-1] (off ascending).
+__device__ __forceinline__ int chunk_of(const int* off, int C, int i) {
+  int lo = 0, hi = C - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Exact selection for row t once every chunk of it has been filtered.  The
+// lists were written by other CTAs of this grid: read through L2 (__ldcg).
+// Every global read is issued in parallel (no chains over chunks).
+__device__ void select_row(int t, const float* __restrict__ row, int K, int chunk, int C,
+                           const uint32_t* __restrict__ ghist, const int2* __restrict__ counts,
+                           const int32_t* __restrict__ sure, const int32_t* __restrict__ cand,
+                           int32_t* __restrict__ out, SelSmem& sm) {
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sm.hist[i] = __ldcg(ghist + (int64_t)t * kHistBins + i);
+  if (threadIdx.x < 64) {  // chunk counts -> offsets: two lanes' worth per thread of warps 0-1, scanned by warp 0
+    const int2 v = threadIdx.x < C ? __ldcg(counts + (int64_t)t * C + threadIdx.x) : make_int2(0, 0);
+    sm.sure_off[threadIdx.x + 1] = v.x;
+    sm.cand_off[threadIdx.x + 1] = v.y;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int a0 = sm.sure_off[2 * lane + 1], a1 = sm.sure_off[2 * lane + 2];
+    int c0 = sm.cand_off[2 * lane + 1], c1 = sm.cand_off[2 * lane + 2];
+    int sa = a0 + a1, sc = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ua = __shfl_up_sync(0xffffffffu, sa, o), uc = __shfl_up_sync(0xffffffffu, sc, o);
+      if (lane >= o) { sa += ua; sc += uc; }
+    }
+    // sa / sc are inclusive sums through element 2*lane+1
+    sm.sure_off[2 * lane + 2] = sa;
+    sm.sure_off[2 * lane + 1] = sa - a1;
+    sm.cand_off[2 * lane + 2] = sc;
+    sm.cand_off[2 * lane + 1] = sc - c1;
+    if (lane == 0) {
+      sm.sure_off[0] = 0;
+      sm.cand_off[0] = 0;
+    }
+  }
+  __syncthreads();
+  find_bin(sm.hist, kHistBins, (uint32_t)K, &sm.bin, &sm.above);
+  const uint32_t bstar = sm.bin, above = sm.above;
+  const uint32_t need = (uint32_t)K - above;
+  const int m = sm.cand_off[C];
+  const int A = min(sm.sure_off[C], kMaxK);
+  // the sure list, concatenated in chunk order (already ascending)
+  for (int i = threadIdx.x; i < A; i += blockDim.x) {
+    const int c = chunk_of(sm.sure_off, C, i);
+    sm.sure[i] = __ldcg(sure + ((int64_t)t * C + c) * K + (i - sm.sure_off[c]));
+  }
+  // candidate i of the row-wide list lives in chunk c at offset i - cand_off[c]
+  auto cand_pos = [&](int i) -> int32_t {
+    const int c = chunk_of(sm.cand_off, C, i);
+    return __ldcg(cand + ((int64_t)t * C + c) * chunk + (i - sm.cand_off[c]));
+  };
+  uint32_t tau, r;
+  if (m <= kSelCap) {
+    for (int i = threadIdx.x; i < m; i += blockDim.x) {
+      const int32_t pos = cand_pos(i);
+      sm.cpos[i] = pos;
+      sm.ckey[i] = order_key(row[pos]);
+    }
+    __syncthreads();
+    select_among(
+        m, need, bstar, [&](int i) { return sm.ckey[i]; }, sm.hist128, &sm.bin, &sm.above, &tau, &r);
+    emit_selected(
+        m, tau, r, need, [&](int i) { return sm.cpos[i]; }, [&](int i) { return sm.ckey[i]; }, sm.sel, sm.buf);
+  } else {
+    __syncthreads();
+    select_among(
+        m, need, bstar, [&](int i) { return order_key(row[cand_pos(i)]); }, sm.hist128, &sm.bin, &sm.above, &tau,
+        &r);
+    emit_selected(
+        m, tau, r, need, cand_pos, [&](int i) { return order_key(row[cand_pos(i)]); }, sm.sel, sm.buf);
+  }
+  merge_lists(sm.sure, (int)above, sm.sel, (int)need, out);
+}
+
+// Filters chunk c of row t into its sure and candidate lists; the CTA that
+// finishes a row's last chunk then selects that row.
 __global__ void __launch_bounds__(kChunkThreads)
-k_topk_filter(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
-              const int32_t* __restrict__ tok_pos, int K, int chunk, int C, const uint32_t* __restrict__ ghist,
-              int2* __restrict__ counts, int32_t* __restrict__ sure, int32_t* __restrict__ cand) {
-  __shared__ uint32_t hist[kHistBins];
-  __shared__ uint32_t buf[33];
-  __shared__ uint32_t s_bin, s_above;
+k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
+                     const int32_t* __restrict__ tok_pos, int K, int chunk, int C, const uint32_t* __restrict__ ghist,
+                     int2* __restrict__ counts, int32_t* __restrict__ sure, int32_t* __restrict__ cand,
+                     int* __restrict__ row_done, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.y, c = blockIdx.x;
   const int n = row_length(row_len, tok_pos, t, ld, nullptr);
-  if (n <= K) return;
+  int32_t* __restrict__ out = idx + (int64_t)t * K;
+  if (n <= K) {  // every candidate is selected
+    if (c == 0)
+      for (int i = threadIdx.x; i < K; i += blockDim.x) out[i] = i < n ? i : -1;
+    return;
+  }
   const int b0 = c * chunk, b1 = min(n, b0 + chunk);
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = ghist[(int64_t)t * kHistBins + i];
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sm.hist[i] = __ldcg(ghist + (int64_t)t * kHistBins + i);
   __syncthreads();
-  find_bin(hist, kHistBins, (uint32_t)K, &s_bin, &s_above);
-  const uint32_t bstar = s_bin;
+  find_bin(sm.hist, kHistBins, (uint32_t)K, &sm.bin, &sm.above);
+  const uint32_t bstar = sm.bin;
   const float* __restrict__ row = scores + (int64_t)t * ld;
   int32_t* my_sure = sure + ((int64_t)t * C + c) * K;
   int32_t* my_cand = cand + ((int64_t)t * C + c) * chunk;
@@ -396,7 +494,7 @@ k_topk_filter(const float* __restrict__ scores, int64_t ld, const int32_t* __res
         sa |= (uint32_t)(bin > bstar) << j;
         cb |= (uint32_t)(bin == bstar) << j;
       }
-    const TwoLists L = scan_two(sa, cb, run_s, run_c, buf);
+    const TwoLists L = scan_two(sa, cb, run_s, run_c, sm.buf);
     uint32_t ps = L.pa, pc = L.pb;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -410,75 +508,16 @@ k_topk_filter(const float* __restrict__ scores, int64_t ld, const int32_t* __res
     run_s += L.ta;
     run_c += L.tb;
   }
-  if (threadIdx.x == 0) counts[(int64_t)t * C + c] = make_int2((int)run_s, (int)run_c);
-}
-
-constexpr int kMaxChunks = 64;
-
-struct SelSmem {
-  uint32_t hist[kHistBins];
-  uint32_t hist128[128];
-  uint32_t buf[33];
-  uint32_t bin, above;
-  int sure_off[kMaxChunks + 1], cand_off[kMaxChunks + 1];
-  int32_t sure[kMaxK];
-  int32_t sel[kMaxK];
-};
-
-__global__ void __launch_bounds__(kRowThreads)
-k_topk_select(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
-              const int32_t* __restrict__ tok_pos, int K, int chunk, int C, const uint32_t* __restrict__ ghist,
-              const int2* __restrict__ counts, const int32_t* __restrict__ sure, const int32_t* __restrict__ cand,
-              int32_t* __restrict__ idx) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw);
-  const int t = blockIdx.x;
-  const int n = row_length(row_len, tok_pos, t, ld, nullptr);
-  int32_t* __restrict__ out = idx + (int64_t)t * K;
-  if (n <= K) {
-    for (int i = threadIdx.x; i < K; i += blockDim.x) out[i] = i < n ? i : -1;
-    return;
-  }
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sm.hist[i] = ghist[(int64_t)t * kHistBins + i];
+  __syncthreads();  // every list write of this CTA precedes the count
   if (threadIdx.x == 0) {
-    int so = 0, co = 0;
-    for (int c = 0; c < C; ++c) {
-      sm.sure_off[c] = so;
-      sm.cand_off[c] = co;
-      const int2 v = counts[(int64_t)t * C + c];
-      so += v.x;
-      co += v.y;
-    }
-    sm.sure_off[C] = so;
-    sm.cand_off[C] = co;
+    counts[(int64_t)t * C + c] = make_int2((int)run_s, (int)run_c);
+    __threadfence();
+    sm.last = atomicAdd(&row_done[t], 1) == C - 1;
   }
   __syncthreads();
-  find_bin(sm.hist, kHistBins, (uint32_t)K, &sm.bin, &sm.above);
-  const uint32_t bstar = sm.bin, above = sm.above;
-  const uint32_t need = (uint32_t)K - above;
-  const int m = sm.cand_off[C];
-  const float* __restrict__ row = scores + (int64_t)t * ld;
-  // candidate i of the row-wide list lives in chunk c at offset i - cand_off[c]
-  auto cand_pos = [&](int i) -> int32_t {
-    int lo = 0, hi = C - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (sm.cand_off[mid] <= i) lo = mid; else hi = mid - 1;
-    }
-    return cand[((int64_t)t * C + lo) * chunk + (i - sm.cand_off[lo])];
-  };
-  // the sure list, concatenated in chunk order (already ascending)
-  for (int c = 0; c < C; ++c) {
-    const int cnt = sm.sure_off[c + 1] - sm.sure_off[c];
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x)
-      if (sm.sure_off[c] + i < kMaxK) sm.sure[sm.sure_off[c] + i] = sure[((int64_t)t * C + c) * K + i];
-  }
-  uint32_t tau, r;
-  select_among(
-      m, need, bstar, [&](int i) { return order_key(row[cand_pos(i)]); }, sm.hist128, &sm.bin, &sm.above, &tau, &r);
-  emit_selected(
-      m, tau, r, need, cand_pos, [&](int i) { return order_key(row[cand_pos(i)]); }, sm.sel, sm.buf);
-  merge_lists(sm.sure, (int)above, sm.sel, (int)need, out);
+  if (!sm.last) return;
+  __threadfence();  // the other chunks' lists are visible from here on
+  select_row(t, row, K, chunk, C, ghist, counts, sure, cand, out, sm);
 }
 
 // Chunking of a row: several CTAs per row only when there are few rows.
@@ -509,46 +548,62 @@ cudaError_t set_smem_once(F* kernel, int bytes, int* dev_set) {
 
 }  // namespace
 
+// Scratch layout (several CTAs per row): a region zeroed on every call --
+// row_done [T] (padded to 16 words) then the first-digit histogram [T][2048]
+// -- followed by counts [T][C], sure lists [T][C][K] and candidates [T][C][chunk].
+int64_t topk_zero_words(int T) { return (int64_t)(T + 15) / 16 * 16 + (int64_t)T * kHistBins; }
+
 size_t topk_scratch_bytes(int T, int64_t ld, int K) {
   int C, chunk;
   topk_chunks(T, ld, &C, &chunk);
   if (C == 1) return 0;
-  return (size_t)T * kHistBins * 4 + (size_t)T * C * sizeof(int2) + (size_t)T * C * K * 4 +
+  return (size_t)topk_zero_words(T) * 4 + (size_t)T * C * sizeof(int2) + (size_t)T * C * K * 4 +
          (size_t)T * C * chunk * 4;
 }
 
+uint32_t* topk_hist_in_scratch(void* scratch, int T) {
+  return reinterpret_cast<uint32_t*>(scratch) + (T + 15) / 16 * 16;
+}
+
+bool topk_uses_hist(int T, int64_t ld) {
+  int C, chunk;
+  topk_chunks(T, ld, &C, &chunk);
+  return C > 1;
+}
+
 cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, const int32_t* tok_pos,
-                        int K, int32_t* idx, void* scratch, uint32_t* err, cudaStream_t st) {
+                        int K, int32_t* idx, void* scratch, bool hist_ready, uint32_t* err, cudaStream_t st) {
   int C, chunk;
   topk_chunks(T, ld, &C, &chunk);
   if (C == 1) {
     static thread_local int dev_row = -1;
     cudaError_t e = set_smem_once(k_topk_row, (int)sizeof(RowSmem), &dev_row);
     if (e != cudaSuccess) return e;
-    k_topk_row<<<T, kRowThreads, sizeof(RowSmem), st>>>(scores, ld, row_len, tok_pos, K, idx, err);
+    e = launch_pdl(k_topk_row, dim3(T), dim3(kRowThreads), sizeof(RowSmem), st, scores, ld, row_len, tok_pos, K, idx,
+                   err);
+    if (e != cudaSuccess) return e;
     return counted(cudaGetLastError());
   }
-  char* p = reinterpret_cast<char*>(scratch);
-  uint32_t* ghist = reinterpret_cast<uint32_t*>(p);
-  p += (size_t)T * kHistBins * 4;
+  int* row_done = reinterpret_cast<int*>(scratch);
+  uint32_t* ghist = topk_hist_in_scratch(scratch, T);
+  char* p = reinterpret_cast<char*>(scratch) + topk_zero_words(T) * 4;
   int2* counts = reinterpret_cast<int2*>(p);
   p += (size_t)T * C * sizeof(int2);
   int32_t* sure = reinterpret_cast<int32_t*>(p);
   p += (size_t)T * C * K * 4;
   int32_t* cand = reinterpret_cast<int32_t*>(p);
-  cudaError_t e = cudaMemsetAsync(ghist, 0, (size_t)T * kHistBins * 4, st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   const dim3 grid(C, T);
-  k_topk_hist<<<grid, kChunkThreads, 0, st>>>(scores, ld, row_len, tok_pos, K, chunk, ghist, err);
-  if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
-  k_topk_filter<<<grid, kChunkThreads, 0, st>>>(scores, ld, row_len, tok_pos, K, chunk, C, ghist, counts, sure,
-                                                 cand);
-  if ((e = counted(cudaGetLastError())) != cudaSuccess) return e;
-  static thread_local int dev_sel = -1;
-  e = set_smem_once(k_topk_select, (int)sizeof(SelSmem), &dev_sel);
+  if (!hist_ready) {  // otherwise the caller has zeroed the region and filled the histogram
+    if ((e = cudaMemsetAsync(scratch, 0, (size_t)topk_zero_words(T) * 4, st)) != cudaSuccess) return e;
+    e = launch_pdl(k_topk_hist, grid, dim3(kChunkThreads), 0, st, scores, ld, row_len, tok_pos, K, chunk, ghist, err);
+    if (e != cudaSuccess || (e = counted(cudaGetLastError())) != cudaSuccess) return e;
+  }
+  static thread_local int dev_fs = -1;
+  if ((e = set_smem_once(k_topk_filter_select, (int)sizeof(SelSmem), &dev_fs)) != cudaSuccess) return e;
+  e = launch_pdl(k_topk_filter_select, grid, dim3(kChunkThreads), sizeof(SelSmem), st, scores, ld, row_len, tok_pos, K,
+                 chunk, C, (const uint32_t*)ghist, counts, sure, cand, row_done, idx);
   if (e != cudaSuccess) return e;
-  k_topk_select<<<T, kRowThreads, sizeof(SelSmem), st>>>(scores, ld, row_len, tok_pos, K, chunk, C, ghist, counts,
-                                                          sure, cand, idx);
   return counted(cudaGetLastError());
 }
 

@@ -51,3 +51,25 @@ def test_fused_full_size(lib, name):
     wl = make_workload(FULL[name])
     tokens = np.arange(wl.T) if wl.T <= 8 else P.sample_tokens(wl, 24)
     _fused_check(lib, wl, tokens)
+
+
+def test_fused_workspace_reused_across_geometries(lib):
+    """One workspace, sized for the largest call, serves calls of different
+    shapes back to back; state a call leaves behind must not leak into the next."""
+    specs = [SMALL["pool_b2_128k"], SMALL["decode_b4_8k_32k"], SMALL["decode_small"], SMALL["pool_b2_128k"]]
+    wls = [make_workload(s) for s in specs]
+    devs = [to_device(w) for w in wls]
+    need = max(lib.dsa_workspace_size(lib.DSA_OP_INDEX_TOPK_ATTN, d.seqs, w.spec.topk, w.spec.heads)
+               for w, d in zip(wls, devs))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ws[256:].fill_(0xA5)  # everything but the error word starts dirty
+    for wl, d in zip(wls, devs):
+        K = wl.spec.topk
+        idx_out = torch.empty((wl.T, K), dtype=torch.int32, device="cuda")
+        lib.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, idx_out=idx_out,
+                                ws=ws)
+        assert lib.dsa_check_error(ws) == lib.DSA_OK
+        gidx = idx_out.cpu().numpy()
+        tokens = np.arange(wl.T)
+        for t, r in zip(tokens, P.oracle_scores(wl, tokens)):
+            assert not P.selection_violations(gidx[t], r, K)
