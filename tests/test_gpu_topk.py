@@ -69,3 +69,36 @@ def test_denormals_and_extremes(lib):
     s[2] = np.float32(np.inf)
     s[2, ::3] = -np.inf
     _run(lib, s, np.full(T, ld), 1000)
+
+
+def _low_bits_row(rng, n, distinct):
+    """Values that share their top 22 key bits and differ in the low 10 only."""
+    return (np.float32(1.0) + rng.integers(0, distinct, n).astype(np.float32) * np.float32(2.0 ** -23)).astype(
+        np.float32)
+
+
+def test_degenerate_threshold_bins(lib):
+    rng = np.random.default_rng(4)
+    # few rows (several CTAs per row): rows whose kept pairs overflow shared memory
+    T, ld = 8, 40000
+    s = rng.standard_normal((T, ld)).astype(np.float32)
+    s[0] = 2.0                                          # one value everywhere
+    s[1] = rng.integers(0, 3, ld).astype(np.float32)    # three values, ties at the threshold
+    s[2] = _low_bits_row(rng, ld, 1024)                 # digit 3 decides, with ties
+    s[3] = _low_bits_row(rng, ld, 7)
+    s[4, :] = 0.0
+    s[4, rng.choice(ld, 5000, replace=False)] = 1.0     # threshold inside the exact ones
+    s[5] = np.where(rng.random(ld) < 0.5, np.float32(1.0), np.float32(1.0 + 2.0 ** -22))
+    lens = np.full(T, ld)
+    lens[6] = 9000
+    for K in (2048, 1000):
+        _run(lib, s, lens, K)
+    # many rows (one CTA per row): kept pairs beyond the one-CTA stage
+    T, ld = 300, 16384
+    s = rng.standard_normal((T, ld)).astype(np.float32)
+    s[0] = 7.0
+    s[1] = rng.integers(0, 2, ld).astype(np.float32)
+    s[2] = _low_bits_row(rng, ld, 1024)
+    s[3] = _low_bits_row(rng, ld, 3)
+    s[4:8] = np.float32(1.0) + (rng.standard_normal((4, ld)) * 1e-3).astype(np.float32)
+    _run(lib, s, np.full(T, ld), 2048)
