@@ -32,6 +32,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kEpiWarps = 8;                 // two epilogue warpgroups (warps 4-11)
+constexpr int kRingSlots = 8;                // producer's look-ahead ring (items)
+constexpr int kRecAhead = 6;                 // item records are fetched this many items ahead
+constexpr int kPgAhead = 3;                  // page ids this many items ahead
 constexpr int kIdxThreads = (4 + kEpiWarps) * 32;
 
 template <bool kBf16, int TG>
@@ -49,7 +52,8 @@ struct IdxCfg {
   static constexpr int OFF_SC = OFF_B + 2 * B_BYTES;       // NS x 128 fp32 row scales
   static constexpr int OFF_W = OFF_SC + NS * 512;          // 2 x TG x 64 fp32 head weights
   static constexpr int OFF_HIST = OFF_W + 2 * TG * 256;   // TG == 1: per-epilogue-warp Top-K histograms
-  static constexpr int OFF_BAR = OFF_HIST + (TG == 1 ? kEpiWarps * kTopkHistBins * 4 : 0);
+  static constexpr int OFF_RING = OFF_HIST + (TG == 1 ? kEpiWarps * kTopkHistBins * 4 : 0);
+  static constexpr int OFF_BAR = OFF_RING + kRingSlots * (32 + 128);  // producer's item records + page ids
   static constexpr int NBARS = 2 * NS + 4 + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
@@ -140,28 +144,49 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp)
-    // Item records are fetched two ahead and each item's page ids (one lane
-    // per page, <= 32 pages per item) one ahead, so the page-table reads
-    // overlap the TMA issue of the current item.
+    // Item records are fetched kRecAhead items ahead and each item's page ids
+    // (one lane per page, <= 32 pages per item) kPgAhead items ahead, as
+    // asynchronous copies into a ring in shared memory: one commit group per
+    // item, so a page-table read has several items' worth of TMA issue to
+    // hide behind.
     if (lane == 0) {
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_q);
     }
-    auto load_pages = [&](const int4& ga, const int4& gb) -> int {
+    int4* ring_rec = reinterpret_cast<int4*>(smem + C::OFF_RING);                     // [slot][2]
+    int* ring_pg = reinterpret_cast<int*>(smem + C::OFF_RING + kRingSlots * 32);     // [slot][32]
+    auto issue_rec = [&](int it) {
+      if (it < it_hi && lane < 2) cp_async_16(&ring_rec[(it % kRingSlots) * 2 + lane], recs + 2 * it + lane);
+    };
+    auto issue_pages = [&](int it) {  // the item's record is already in the ring
+      if (it >= it_hi) return;
+      const int4 ga = ring_rec[(it % kRingSlots) * 2], gb = ring_rec[(it % kRingSlots) * 2 + 1];
       const int lp = 2 * gb.x + lane;
       const int last = ga.w + ga.z - 1;
-      if (lane < 2 * (gb.y - gb.x) && lp * kPage <= last) return __ldg(a.s.page_table + (int64_t)ga.x * a.s.max_pages + lp);
-      return -1;
+      if (lane < 2 * (gb.y - gb.x) && lp * kPage <= last)
+        cp_async_4(&ring_pg[(it % kRingSlots) * 32 + lane], a.s.page_table + (int64_t)ga.x * a.s.max_pages + lp);
     };
-    int4 ca = make_int4(0, 0, 0, 0), cb = ca, na = ca, nb = ca, fa = ca, fb = ca;
-    if (it_lo < it_hi) { ca = recs[2 * it_lo]; cb = recs[2 * it_lo + 1]; }
-    if (it_lo + 1 < it_hi) { na = recs[2 * it_lo + 2]; nb = recs[2 * it_lo + 3]; }
-    int pages = it_lo < it_hi ? load_pages(ca, cb) : -1;
+    for (int i = 0; i < kRecAhead; ++i) issue_rec(it_lo + i);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
+    for (int i = 0; i < kPgAhead; ++i) {
+      issue_pages(it_lo + i);
+      cp_async_commit();
+    }
     int stage = 0, sphase = 0, prev_g = -1, gcount = 0;
     bool ok = true;
     for (int it = it_lo; it < it_hi && ok; ++it) {
-      if (it + 2 < it_hi) { fa = recs[2 * it + 4]; fb = recs[2 * it + 5]; }
-      const int next_pages = (it + 1 < it_hi) ? load_pages(na, nb) : -1;
+      // groups so far: the page ids of it_lo .. it_lo+kPgAhead-1, then one
+      // group per earlier iteration; all but the newest kPgAhead-1 hold what
+      // this iteration reads (page ids of it, record of it+kPgAhead)
+      cp_async_wait<kPgAhead - 1>();
+      __syncwarp();
+      issue_rec(it + kRecAhead);
+      issue_pages(it + kPgAhead);
+      cp_async_commit();
+      const int4 ca = ring_rec[(it % kRingSlots) * 2], cb = ring_rec[(it % kRingSlots) * 2 + 1];
+      const int pages = ring_pg[(it % kRingSlots) * 32 + lane];  // lanes past the item's pages are unused
       const int4 grp = ca;  // {b, t0, cnt, pos0}
       if (cb.z != prev_g) {
         if (lane == 0) {
@@ -226,9 +251,8 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
         if (++stage == C::NS) { stage = 0; sphase ^= 1; }
       }
       ok = __shfl_sync(0xffffffffu, (int)(*abort_flag == 0), 0) != 0;  // lane 0's view, warp-uniform
-      ca = na; cb = nb; na = fa; nb = fb;
-      pages = next_pages;
     }
+    cp_async_wait<0>();  // no copy into the ring is still in flight at exit
     // drain: every issued stage has been consumed before the CTA exits
     if (lane == 0) {
       for (int i = 0; i < C::NS && !*abort_flag; ++i) {

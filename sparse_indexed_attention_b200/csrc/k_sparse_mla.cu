@@ -14,8 +14,11 @@
 // the work of one (token, slice of the index list) goes to a CLUSTER OF TWO
 // CTAs.  CTA r owns value dims [256r, 256r+256) and the key dims
 // {256r..256r+255} u {512+32r..512+32r+31}; it gathers only those 576 bytes of
-// each selected row (TMA tile::gather4 through the page table, 128-byte /
-// 64-byte swizzle).  Per block of 64 selected rows:
+// each selected row.  Three warps resolve the rows (index list -> page table)
+// two blocks ahead and copy them with 16-byte cp.async straight into the
+// 128-byte / 64-byte swizzled operand layouts -- many small copies in flight
+// from 96 threads instead of a queue of four-row TMA gathers.  Per block of 64
+// selected rows:
 //   * S_r = Q_r K_r^T (M = 128 heads, N = 64 rows, K = 288 dims) into TMEM;
 //   * the two partial S are exchanged through distributed shared memory and
 //     summed (a + b = b + a, so both CTAs hold bit-identical logits and take
@@ -44,13 +47,18 @@ constexpr int kQLatBytes = 128 * 128;        // one 64-dim swizzle atom of 128 h
 constexpr int kQBytes = 4 * kQLatBytes + 128 * 64;
 constexpr int kKVStage = 4 * kBK * 128 + kBK * 64;  // 36864: 4 latent atoms + rope quarter
 constexpr int kPBytes = 128 * kBK * 2;       // 16 KB per bf16 term
-constexpr int kXPitch = 68;                  // floats per exchanged row (64 + pad)
+constexpr int kXBytes = 128 * kBK * 4;       // one partial S: [16 column quads][128 heads][4] fp32
+constexpr int kLoaders = 96;                 // warps 0, 2, 3 copy the selected rows
+constexpr int kChunksPerRow = 36;            // 16-byte pieces of a CTA's 576 bytes of a row
+constexpr int kRingBlocks = 4;               // resolved row ids, blocks j .. j+2 live
+constexpr int kLoaderBarrier = 1;            // named barrier of the loader warps
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + kQBytes;                 // 73728
 constexpr int OFF_P = OFF_KV + 2 * kKVStage;            // 147456
 constexpr int OFF_X = OFF_P + 2 * kPBytes;              // 180224 (P_hi, P_lo)
-constexpr int OFF_META = OFF_X + 128 * kXPitch * 4;     // 215040
-constexpr int OFF_BAR = OFF_META + 16;
+constexpr int OFF_ROWS = OFF_X + kXBytes;               // 212992: [ring][64] pool rows (-1 = masked)
+constexpr int OFF_MASK = OFF_ROWS + kRingBlocks * kBK * 4;  // [ring] 64-bit validity masks
+constexpr int OFF_BAR = OFF_MASK + kRingBlocks * 8;
 constexpr int kNBars = 13;
 constexpr int OFF_MISC = OFF_BAR + kNBars * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -73,6 +81,7 @@ __device__ __forceinline__ void store_out(void* out, bool f32, int64_t i, float 
 struct AttnArgs {
   SeqsDev s;
   TokenMap tm;
+  const __nv_bfloat16* kv;  // latent pool [rows, 576]
   const int32_t* idx;
   int K, H, ks, splits;
   float scale_log2;  // scale * log2(e)
@@ -86,7 +95,6 @@ struct AttnArgs {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
 k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constant__ CUtensorMap tq_rope,
-                const __grid_constant__ CUtensorMap tkv_lat, const __grid_constant__ CUtensorMap tkv_rope,
                 const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -100,7 +108,8 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   uint64_t* o_done = bars + 10;
   uint64_t* x_full = bars + 11;    // the peer's partial S has landed in my X
   uint64_t* x_free = bars + 12;    // the peer has consumed what I wrote into its X
-  uint64_t* meta_mask = reinterpret_cast<uint64_t*>(smem + OFF_META);
+  int32_t* ring_rows = reinterpret_cast<int32_t*>(smem + OFF_ROWS);
+  uint64_t* ring_mask = reinterpret_cast<uint64_t*>(smem + OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -115,7 +124,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_full[i], kLoaders + 1);  // every loader's copies + the mask's publisher
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
@@ -142,72 +151,73 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   const int b = a.tm.seq[t];
   const int nblk = (pos >= 0 && kend > kbeg) ? (kend - kbeg + kBK - 1) / kBK : 0;
 
-  if (warp == 0 && nblk > 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      prefetch_tmap(&tkv_lat);
-      prefetch_tmap(&tkv_rope);
+  if ((warp == 0 || warp == 2 || warp == 3) && nblk > 0) {
+    // ---------------------------------------------------------------- loaders
+    const int li = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0 .. 95
+    if (li == 0) {
+      prefetch_tmap(&tq_lat);
       mbar_arrive_expect_tx(q_full, kQBytes);
       for (int at = 0; at < 4; ++at)
         tma_load_2d(smem + OFF_Q + at * kQLatBytes, &tq_lat, q_full, 256 * rank + 64 * at, t * a.H);
       tma_load_2d(smem + OFF_Q + 4 * kQLatBytes, &tq_rope, q_full, 512 + 32 * rank, t * a.H);
     }
-    for (int j = 0; j < nblk; ++j) {
-      const int stage = j & 1;
-      int rows[2];
-      bool valid[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int kk = kbeg + j * kBK + 2 * lane + u;
-        rows[u] = 0;
-        valid[u] = false;
-        if (kk < kend) {
-          const int sidx = __ldg(a.idx + (int64_t)t * a.K + kk);
-          if (sidx >= 0 && sidx <= pos) {
-            const int64_t r = phys_row(a.s.page_table, a.s.max_pages, a.s.num_phys_pages, b, sidx, a.err);
-            if (r >= 0) {
-              rows[u] = (int)r;
-              valid[u] = true;
-            }
-          } else if (sidx != -1) {
-            raise_error(a.err, kErrBadIndex);
-          }
+    // Pool rows of block j into ring slot j % kRingBlocks: warps 0 and 2 take
+    // one selected row each (index list -> page table -> row, -1 = masked).
+    auto resolve = [&](int j) {
+      if (j >= nblk || warp == 3) return;
+      const int r = (warp == 0 ? 0 : 32) + lane;
+      const int kk = kbeg + j * kBK + r;
+      int row = -1;
+      if (kk < kend) {
+        const int sidx = __ldg(a.idx + (int64_t)t * a.K + kk);
+        if (sidx >= 0 && sidx <= pos) {
+          const int64_t pr = phys_row(a.s.page_table, a.s.max_pages, a.s.num_phys_pages, b, sidx, a.err);
+          if (pr >= 0) row = (int)pr;
+        } else if (sidx != -1) {
+          raise_error(a.err, kErrBadIndex);
         }
       }
-      const uint32_t m0 = __ballot_sync(0xffffffffu, valid[0]);  // bit l: row 2l
-      const uint32_t m1 = __ballot_sync(0xffffffffu, valid[1]);  // bit l: row 2l+1
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(&kv_empty[stage], ((j >> 1) & 1) ^ 1, a.err);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        *abort_flag = 1;
-        break;
+      const int slot = j % kRingBlocks;
+      ring_rows[slot * kBK + r] = row;
+      const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
+      if (lane == 0) reinterpret_cast<uint32_t*>(&ring_mask[slot])[warp == 0 ? 0 : 1] = m;
+    };
+    const uint32_t kv_smem = smem_u32(smem + OFF_KV);
+    const __nv_bfloat16* kv_base = reinterpret_cast<const __nv_bfloat16*>(a.kv);
+    resolve(0);
+    resolve(1);
+    bool failed = bar_red_or(kLoaderBarrier, kLoaders, false);
+    for (int j = 0; j < nblk && !failed; ++j) {
+      const int stage = j & 1, slot = j % kRingBlocks;
+      bool ok = mbar_wait(&kv_empty[stage], ((j >> 1) & 1) ^ 1, a.err);
+      if (ok) {
+        const uint32_t dst0 = kv_smem + stage * kKVStage;
+        for (int c = li; c < kBK * kChunksPerRow; c += kLoaders) {
+          const int r = c / kChunksPerRow, k = c - r * kChunksPerRow;
+          const int row = ring_rows[slot * kBK + r];
+          uint32_t dst;
+          int64_t col;
+          if (k < 32) {  // latent dims 256*rank + 8k .. +7: 128-byte swizzle atom k/8
+            dst = dst0 + (k >> 3) * (kBK * 128) + r * 128 + ((((uint32_t)k & 7u) ^ ((uint32_t)r & 7u)) << 4);
+            col = 256 * rank + 8 * k;
+          } else {       // rope dims 512 + 32*rank + 8(k-32) .. +7: 64-byte swizzle
+            const uint32_t kr = (uint32_t)(k - 32);
+            dst = dst0 + 4 * (kBK * 128) + r * 64 + ((kr ^ (((uint32_t)r >> 1) & 3u)) << 4);
+            col = 512 + 32 * rank + 8 * kr;
+          }
+          const bool v = row >= 0;
+          cp_async_16_zfill(dst, kv_base + (v ? (int64_t)row * kDQK + col : 0), v ? 16u : 0u);
+        }
       }
-      if (lane == 0) {
-        uint64_t mask = 0;
-        for (int i = 0; i < 32; ++i)
-          mask |= ((uint64_t)((m0 >> i) & 1u) << (2 * i)) | ((uint64_t)((m1 >> i) & 1u) << (2 * i + 1));
-        meta_mask[stage] = mask;
-        mbar_arrive_expect_tx(&kv_full[stage], kKVStage);
-      }
-      __syncwarp();
-      // lane g < 16 gathers rows 4g .. 4g+3 (held by lanes 2g and 2g+1)
-      const int g = lane & 15;
-      const int r0 = __shfl_sync(0xffffffffu, rows[0], 2 * g);
-      const int r1 = __shfl_sync(0xffffffffu, rows[1], 2 * g);
-      const int r2 = __shfl_sync(0xffffffffu, rows[0], 2 * g + 1);
-      const int r3 = __shfl_sync(0xffffffffu, rows[1], 2 * g + 1);
-      if (lane < 16) {
-        uint8_t* st = smem + OFF_KV + stage * kKVStage;
-#pragma unroll
-        for (int at = 0; at < 4; ++at)
-          tma_gather4(st + at * (kBK * 128) + g * 4 * 128, &tkv_lat, &kv_full[stage], 256 * rank + 64 * at, r0, r1,
-                      r2, r3);
-        tma_gather4(st + 4 * (kBK * 128) + g * 4 * 64, &tkv_rope, &kv_full[stage], 512 + 32 * rank, r0, r1, r2, r3);
-      }
+      cp_async_mbar_arrive(&kv_full[stage]);  // counts once this thread's copies land
+      if (li == 0) mbar_arrive(&kv_full[stage]);  // releases the ring mask read by the softmax warps
+      resolve(j + 2);
+      failed = bar_red_or(kLoaderBarrier, kLoaders, !ok);
+      if (failed) *abort_flag = 1;
     }
-    // drain: every gather has landed and every MMA commit has arrived
-    if (lane == 0 && !*abort_flag) {
+    cp_async_wait_all();
+    // drain: every stage has been consumed by the MMA before the CTA exits
+    if (li == 0 && !*abort_flag) {
       for (int j = nblk; j < nblk + 2; ++j)
         if (!mbar_wait(&kv_empty[j & 1], ((j >> 1) & 1) ^ 1, a.err)) break;
     }
@@ -240,6 +250,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
           ok = false;
           break;
         }
+        fence_proxy_async_smem();  // the rows were written by cp.async (generic proxy)
         tc_fence_after();
         const uint32_t d = tmem + 256 + kBK * sb;
         const uint32_t kb = kv_base + (j & 1) * kKVStage;
@@ -268,8 +279,10 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     const int qw = warp - 4;
     const int h = qw * 32 + lane;  // head row = TMEM lane
     const uint32_t t_lane = tmem + ((uint32_t)(qw * 32) << 16);
-    float* xrow = reinterpret_cast<float*>(smem + OFF_X) + h * kXPitch;
-    const uint32_t x_peer = map_peer(smem_u32(xrow), peer);
+    // X[c][h] holds logits 4c .. 4c+3 of head h: a warp's stores of one c are
+    // 512 contiguous bytes
+    const float4* xcol = reinterpret_cast<const float4*>(smem + OFF_X) + h;
+    const uint32_t x_peer = map_peer(smem_u32(smem + OFF_X), peer) + (uint32_t)h * 16u;
     const uint32_t x_full_peer = map_peer(smem_u32(x_full), peer);
     const uint32_t x_free_peer = map_peer(smem_u32(x_free), peer);
     uint8_t* p_row0 = smem + OFF_P + (h >> 3) * 1024 + (h & 7) * 128;
@@ -292,9 +305,9 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       if (!ok) break;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        st_cluster_v4(x_peer + c * 16, __uint_as_float(v0[4 * c]), __uint_as_float(v0[4 * c + 1]),
+        st_cluster_v4(x_peer + c * 2048, __uint_as_float(v0[4 * c]), __uint_as_float(v0[4 * c + 1]),
                       __uint_as_float(v0[4 * c + 2]), __uint_as_float(v0[4 * c + 3]));
-        st_cluster_v4(x_peer + 128 + c * 16, __uint_as_float(v1[4 * c]), __uint_as_float(v1[4 * c + 1]),
+        st_cluster_v4(x_peer + (c + 8) * 2048, __uint_as_float(v1[4 * c]), __uint_as_float(v1[4 * c + 1]),
                       __uint_as_float(v1[4 * c + 2]), __uint_as_float(v1[4 * c + 3]));
       }
       // the warp barrier orders every lane's stores before lane 0's cluster-scope release
@@ -305,7 +318,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       float s[64];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float4 pv4 = reinterpret_cast<const float4*>(xrow)[c];
+        const float4 pv4 = xcol[c * 128];
         const uint32_t* mine = c < 8 ? &v0[4 * c] : &v1[4 * (c - 8)];
         s[4 * c + 0] = __uint_as_float(mine[0]) + pv4.x;
         s[4 * c + 1] = __uint_as_float(mine[1]) + pv4.y;
@@ -314,10 +327,10 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       }
       __syncwarp();  // every lane has read its row of X
       if (lane == 0) mbar_arrive_remote(x_free_peer);
-      // validity of the block's rows (written before the stage's TMA was armed)
+      // validity of the block's rows (published before the stage completed)
       ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err));
       if (!ok) break;
-      const uint64_t mask = meta_mask[j & 1];
+      const uint64_t mask = ring_mask[j % kRingBlocks];
       float mblk = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
@@ -529,12 +542,9 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16
   splits = (K + ks - 1) / ks;
   float* part_o = reinterpret_cast<float*>(partials);
   float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)T * splits * H * kDV);
-  const uint64_t R = (uint64_t)s.num_phys_pages * kPage;
-  CUtensorMap tq_lat, tq_rope, tkv_lat, tkv_rope;
+  CUtensorMap tq_lat, tq_rope;
   if (!make_map_576(&tq_lat, q, (uint64_t)T * H, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_576(&tq_rope, q, (uint64_t)T * H, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_576(&tkv_lat, kv, R, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_576(&tkv_rope, kv, R, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+      !make_map_576(&tq_rope, q, (uint64_t)T * H, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   static thread_local int attr_dev = -1;
   int dev = 0;
@@ -544,9 +554,9 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  AttnArgs a{s, tm, idx, K, H, ks, splits, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
+  AttnArgs a{s, tm, kv, idx, K, H, ks, splits, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
   cudaError_t e = launch_pdl(k_sparse_mla_tc, dim3(2 * T * splits), dim3(256), (size_t)SMEM_BYTES, st, tq_lat, tq_rope,
-                             tkv_lat, tkv_rope, a);
+                             a);
   if (e == cudaSuccess) e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
   e = launch_pdl(k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o, (const float2*)part_ml,
