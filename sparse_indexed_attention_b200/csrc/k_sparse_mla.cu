@@ -20,17 +20,21 @@
 // from 96 threads instead of a queue of four-row TMA gathers.  Per block of 64
 // selected rows:
 //   * S_r = Q_r K_r^T (M = 128 heads, N = 64 rows, K = 288 dims) into TMEM;
-//   * the two partial S are exchanged through distributed shared memory and
-//     summed (a + b = b + a, so both CTAs hold bit-identical logits and take
+//   * the two partial S are exchanged through distributed shared memory
+//     (st.async into the peer's double-buffered receive area, counted on the
+//     peer's mbarrier, so no cluster-scope fence sits on the path) and summed
+//     (a + b = b + a, so both CTAs hold bit-identical logits and take
 //     identical softmax decisions);
 //   * online softmax in registers (one head row per thread, base-2 exponent,
 //     the running maximum is only moved -- and O rescaled in TMEM -- when it
 //     grows by more than 2^8, which is exact because O and l share it);
-//   * P goes to shared memory as two bf16 terms, P = P_hi + P_lo (together
-//     within 2^-17 of the fp32 value; one bf16 term alone would leave a
-//     relative error of 2^-9 on rows dominated by a few selected keys), and
+//   * P goes to TMEM as two bf16 terms, P = P_hi + P_lo (together within
+//     2^-17 of the fp32 value; one bf16 term alone would leave a relative
+//     error of 2^-9 on rows dominated by a few selected keys), and
 //     O_r += P_hi V_r + P_lo V_r (M = 128, N = 256, K = 64) accumulates in
-//     TMEM, V_r being the same gathered bytes read as an MN-major operand.
+//     TMEM with P read from TMEM, V_r being the same gathered bytes read as an
+//     MN-major operand.  TMEM columns: O [0, 256), S [256, 384) (two
+//     buffers), P [384, 512) (two buffers of hi + lo).
 // Slices of one token are merged by k_combine (log-sum-exp weights).
 #include <cudaTypedefs.h>
 
@@ -46,7 +50,6 @@ constexpr int kBK = 64;                      // selected rows per block
 constexpr int kQLatBytes = 128 * 128;        // one 64-dim swizzle atom of 128 head rows
 constexpr int kQBytes = 4 * kQLatBytes + 128 * 64;
 constexpr int kKVStage = 4 * kBK * 128 + kBK * 64;  // 36864: 4 latent atoms + rope quarter
-constexpr int kPBytes = 128 * kBK * 2;       // 16 KB per bf16 term
 constexpr int kXBytes = 128 * kBK * 4;       // one partial S: [16 column quads][128 heads][4] fp32
 constexpr int kLoaders = 96;                 // warps 0, 2, 3 copy the selected rows
 constexpr int kChunksPerRow = 36;            // 16-byte pieces of a CTA's 576 bytes of a row
@@ -54,16 +57,16 @@ constexpr int kRingBlocks = 4;               // resolved row ids, blocks j .. j+
 constexpr int kLoaderBarrier = 1;            // named barrier of the loader warps
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + kQBytes;                 // 73728
-constexpr int OFF_P = OFF_KV + 2 * kKVStage;            // 147456
-constexpr int OFF_X = OFF_P + 2 * kPBytes;              // 180224 (P_hi, P_lo)
-constexpr int OFF_ROWS = OFF_X + kXBytes;               // 212992: [ring][64] pool rows (-1 = masked)
+constexpr int OFF_X = OFF_KV + 2 * kKVStage;            // 147456: two receive buffers
+constexpr int OFF_ROWS = OFF_X + 2 * kXBytes;           // 212992: [ring][64] pool rows (-1 = masked)
 constexpr int OFF_MASK = OFF_ROWS + kRingBlocks * kBK * 4;  // [ring] 64-bit validity masks
 constexpr int OFF_BAR = OFF_MASK + kRingBlocks * 8;
-constexpr int kNBars = 13;
+constexpr int kNBars = 14;
 constexpr int OFF_MISC = OFF_BAR + kNBars * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-static_assert(OFF_KV % 1024 == 0 && kKVStage % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms need 1024-B alignment");
+static_assert(OFF_KV % 1024 == 0 && kKVStage % 1024 == 0, "swizzle atoms need 1024-B alignment");
+constexpr uint32_t kTmemS = 256, kTmemP = 384;  // TMEM column bases (O at 0)
 
 constexpr uint32_t IDESC_QK = make_idesc_major(true, 128, kBK, 0, 0);  // S = Q K^T, both K-major
 constexpr uint32_t IDESC_PV = make_idesc_major(true, 128, 256, 0, 1);  // O += P V, V MN-major
@@ -105,9 +108,8 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   uint64_t* s_full = bars + 5;     // [2]
   uint64_t* s_empty = bars + 7;    // [2]
   uint64_t* p_full = bars + 9;
-  uint64_t* o_done = bars + 10;
-  uint64_t* x_full = bars + 11;    // the peer's partial S has landed in my X
-  uint64_t* x_free = bars + 12;    // the peer has consumed what I wrote into its X
+  uint64_t* o_done = bars + 10;    // [2] PV of block i (buffer i & 1) has completed
+  uint64_t* x_full = bars + 12;    // [2] the peer's partial S of a block has landed in my X[buffer]
   int32_t* ring_rows = reinterpret_cast<int32_t*>(smem + OFF_ROWS);
   uint64_t* ring_mask = reinterpret_cast<uint64_t*>(smem + OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
@@ -130,11 +132,16 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       mbar_init(&s_empty[i], 4);
     }
     mbar_init(p_full, 4);   // one arrival per softmax warp
-    mbar_init(o_done, 1);
-    mbar_init(x_full, 4);   // one arrival per peer softmax warp
-    mbar_init(x_free, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&o_done[i], 1);
+      mbar_init(&x_full[i], 1);  // armed by this CTA (expect_tx), filled by the peer's st.async
+    }
     *abort_flag = 0;
     fence_mbar_init();
+    // receive areas of blocks 0 and 1 armed before the cluster barrier below
+    // lets the peer store into them
+    mbar_arrive_expect_tx(&x_full[0], kXBytes);
+    mbar_arrive_expect_tx(&x_full[1], kXBytes);
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, 512);
@@ -144,7 +151,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   __syncthreads();
   cluster_sync();  // the peer's barriers exist before any remote arrive
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // O at columns [0,256), S buffers at [256,320), [320,384)
+  const uint32_t tmem = *tmem_slot;
   pdl_wait();  // the token map and the index lists come from earlier kernels
   pdl_trigger();
   const int pos = a.tm.pos[t];
@@ -227,20 +234,20 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     if (lane == 0) {
       const uint32_t q_base = smem_u32(smem + OFF_Q);
       const uint32_t kv_base = smem_u32(smem + OFF_KV);
-      const uint32_t p_base = smem_u32(smem + OFF_P);
       bool ok = mbar_wait(q_full, 0, a.err);
       auto pv = [&](int i) -> bool {
         if (!mbar_wait(p_full, i & 1, a.err)) return false;
         tc_fence_after();
         const uint32_t vb = kv_base + (i & 1) * kKVStage;
+        const uint32_t pb = tmem + kTmemP + 64 * (i & 1);  // P_hi at +0, P_lo at +32 (16 keys per 8 columns)
 #pragma unroll
         for (int term = 0; term < 2; ++term)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss<true>(tmem, smem_desc(p_base + term * kPBytes + kk * 32, 16, 1024, 2),
-                         smem_desc(vb + kk * 2048, 8192, 1024, 2), IDESC_PV, i > 0 || term > 0 || kk > 0);
+            mma_ts_bf16(tmem, pb + 32 * term + 8 * kk, smem_desc(vb + kk * 2048, 8192, 1024, 2), IDESC_PV,
+                        i > 0 || term > 0 || kk > 0);
         mma_commit(&kv_empty[i & 1]);
-        mma_commit(o_done);
+        mma_commit(&o_done[i & 1]);
         return true;
       };
       for (int j = 0; j < nblk && ok && !*abort_flag; ++j) {
@@ -252,7 +259,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         }
         fence_proxy_async_smem();  // the rows were written by cp.async (generic proxy)
         tc_fence_after();
-        const uint32_t d = tmem + 256 + kBK * sb;
+        const uint32_t d = tmem + kTmemS + kBK * sb;
         const uint32_t kb = kv_base + (j & 1) * kKVStage;
 #pragma unroll
         for (int at = 0; at < 4; ++at)
@@ -279,56 +286,53 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     const int qw = warp - 4;
     const int h = qw * 32 + lane;  // head row = TMEM lane
     const uint32_t t_lane = tmem + ((uint32_t)(qw * 32) << 16);
-    // X[c][h] holds logits 4c .. 4c+3 of head h: a warp's stores of one c are
-    // 512 contiguous bytes
+    // X[b][c][h] holds logits 4c .. 4c+3 of head h: a warp's stores of one c
+    // are 512 contiguous bytes
     const float4* xcol = reinterpret_cast<const float4*>(smem + OFF_X) + h;
     const uint32_t x_peer = map_peer(smem_u32(smem + OFF_X), peer) + (uint32_t)h * 16u;
     const uint32_t x_full_peer = map_peer(smem_u32(x_full), peer);
-    const uint32_t x_free_peer = map_peer(smem_u32(x_free), peer);
-    uint8_t* p_row0 = smem + OFF_P + (h >> 3) * 1024 + (h & 7) * 128;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nblk && ok; ++j) {
       const int sb = j & 1;
+      // s_full(j) also means PV(j-2) is complete (it was issued before QK(j)),
+      // so P's buffer sb is free
       ok = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&s_full[sb], (j >> 1) & 1, a.err));
       if (!ok) break;
       tc_fence_after();
       uint32_t v0[32], v1[32];
-      tmem_ld32(t_lane + 256 + kBK * sb, v0);
-      tmem_ld32(t_lane + 256 + kBK * sb + 32, v1);
+      tmem_ld32(t_lane + kTmemS + kBK * sb, v0);
+      tmem_ld32(t_lane + kTmemS + kBK * sb + 32, v1);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
-      // exchange partial logits with the peer
-      ok = __all_sync(0xffffffffu, mbar_wait_cluster(x_free, (j & 1) ^ 1, a.err));
-      if (!ok) break;
+      // my partial logits -> the peer's receive area sb
+      const uint32_t xp = x_peer + (uint32_t)sb * kXBytes;
+      const uint32_t xb = x_full_peer + (uint32_t)sb * 8u;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        st_cluster_v4(x_peer + c * 2048, __uint_as_float(v0[4 * c]), __uint_as_float(v0[4 * c + 1]),
-                      __uint_as_float(v0[4 * c + 2]), __uint_as_float(v0[4 * c + 3]));
-        st_cluster_v4(x_peer + (c + 8) * 2048, __uint_as_float(v1[4 * c]), __uint_as_float(v1[4 * c + 1]),
-                      __uint_as_float(v1[4 * c + 2]), __uint_as_float(v1[4 * c + 3]));
+        st_async_v4(xp + c * 2048, v0[4 * c], v0[4 * c + 1], v0[4 * c + 2], v0[4 * c + 3], xb);
+        st_async_v4(xp + (c + 8) * 2048, v1[4 * c], v1[4 * c + 1], v1[4 * c + 2], v1[4 * c + 3], xb);
       }
-      // the warp barrier orders every lane's stores before lane 0's cluster-scope release
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(x_full_peer);
-      ok = __all_sync(0xffffffffu, mbar_wait_cluster(x_full, j & 1, a.err));
+      ok = __all_sync(0xffffffffu, mbar_wait_cluster(&x_full[sb], (j >> 1) & 1, a.err));
       if (!ok) break;
       float s[64];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float4 pv4 = xcol[c * 128];
+        const float4 pv4 = xcol[sb * (kXBytes / 16) + c * 128];
         const uint32_t* mine = c < 8 ? &v0[4 * c] : &v1[4 * (c - 8)];
         s[4 * c + 0] = __uint_as_float(mine[0]) + pv4.x;
         s[4 * c + 1] = __uint_as_float(mine[1]) + pv4.y;
         s[4 * c + 2] = __uint_as_float(mine[2]) + pv4.z;
         s[4 * c + 3] = __uint_as_float(mine[3]) + pv4.w;
       }
-      __syncwarp();  // every lane has read its row of X
-      if (lane == 0) mbar_arrive_remote(x_free_peer);
+      // re-arm receive area sb for block j+2: the peer only stores into it
+      // after its block j+1 completed, which needs every warp's block j+1
+      // stores from here -- issued after this warp's reads above
+      if (qw == 0 && lane == 0 && j + 2 < nblk) mbar_arrive_expect_tx(&x_full[sb], kXBytes);
       // validity of the block's rows (published before the stage completed)
-      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[sb], (j >> 1) & 1, a.err));
       if (!ok) break;
       const uint64_t mask = ring_mask[j % kRingBlocks];
       float mblk = -INFINITY;
@@ -352,44 +356,35 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         pk[i] = *reinterpret_cast<const uint32_t*>(&hi);
         pl[i] = *reinterpret_cast<const uint32_t*>(&lo);
       }
-      // PV of the previous block must be complete before O is touched or P's buffer reused
-      if (j >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, a.err));
+      tmem_st32(t_lane + kTmemP + 64 * sb, pk);
+      tmem_st32(t_lane + kTmemP + 64 * sb + 32, pl);
+      // TMEM loads/stores are warp-wide: if any head of the warp moved its
+      // maximum, the whole warp rescales O (alpha = 1 leaves a row exact),
+      // once PV(j-1) -- the last writer of O -- has completed
+      if (j >= 1 && __any_sync(0xffffffffu, move && m_ref != -INFINITY)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err));
         if (!ok) break;
         tc_fence_after();
-        // TMEM loads/stores are warp-wide: if any head of the warp moved its
-        // maximum, the whole warp rescales (alpha = 1 leaves a row exact).
-        if (__any_sync(0xffffffffu, move && m_ref != -INFINITY)) {
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_lane + 32 * c, o);
-            tmem_ld_wait();
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_lane + 32 * c, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(t_lane + 32 * c, o);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(t_lane + 32 * c, o);
         }
       }
       l = l * alpha + psum;
       m_ref = m_new;
-      // P's buffer is free: PV of the previous block has completed (o_done above)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        *reinterpret_cast<uint4*>(p_row0 + ((c ^ (h & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(p_row0 + kPBytes + ((c ^ (h & 7)) << 4)) =
-            make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
-      }
-      fence_proxy_async_smem();  // this thread's P stores -> visible to the tensor core
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
     // epilogue: O / l for this CTA's 256 value dims.  tcgen05.ld is warp-wide,
     // so a warp with any valid head loads; only the stores test h < H.
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(o_done, (nblk - 1) & 1, a.err));
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(&o_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.err));
     if (ok) {
       tc_fence_after();
       const bool store = h < a.H;
