@@ -52,20 +52,28 @@ def parse():
     return ap.parse_args()
 
 
-def dist_setup(args):
+def dist_setup(args, backend=None):
+    """World size, rank and local rank from the torchrun environment; for N > 1
+    a process group (NCCL on GPUs, gloo without) with a short timeout."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
+
+
+def rank_spec(spec, rank: int):
+    """The workload rank `rank` serves: same shape, its own seed (weak scaling)."""
+    return spec.scaled(seed=spec.seed + 1000 * rank)
 
 
 def reduce_max(x: float, world: int) -> float:
@@ -240,6 +248,32 @@ def time_device(fn, steps, warmup, stream, flush):
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
 
+def kernel_times(dsa, step, steps, stream, flush):
+    """{kernel: [device ms per call]} over `steps` eager calls, L2 flushed before each."""
+    per = {}
+    dsa.dsa_launch_timing(True)
+    try:
+        for i in range(3 + steps):
+            flush.fill_(i & 0xFF)
+            step()
+            got = dsa.dsa_last_launch_times()
+            if i >= 3:
+                for name, ms in got:
+                    per.setdefault(name, []).append(ms)
+    finally:
+        dsa.dsa_launch_timing(False)
+    torch.cuda.synchronize()
+    return per
+
+
+def roofline_entry(name, per, algorithmic_bytes, peak, peak_kind):
+    ms = statistics.mean(per[name])
+    achieved = algorithmic_bytes / (ms / 1e3) / 1e9
+    return {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_source": peak_kind, "algorithmic_bytes": algorithmic_bytes,
+            "launch_us": ms * 1e3, "traffic": None}
+
+
 def run_only(args, dsa, wl, d, dev, stream, flush, world):
     """One stage alone, `--steps` timed launches after `--warmup` (profiling aid)."""
     spec = wl.spec
@@ -267,7 +301,7 @@ def run_ours(args, world, rank, local):
     from sparse_indexed_attention_b200.workloads import to_device
 
     spec = CONFIGS[args.config]
-    spec = spec.scaled(seed=spec.seed + 1000 * rank)     # each rank serves its own batch
+    spec = rank_spec(spec, rank)                         # each rank serves its own batch
     wl = make_workload(spec)
     d = to_device(wl)
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -317,6 +351,10 @@ def run_ours(args, world, rank, local):
     tokens_total = T * world
     value = tokens_total / (ms / 1e3)
 
+    # ---- per-kernel device times inside the same call (events around every
+    # launch; this pass serialises the kernels, so it is timed separately) ----
+    kern = kernel_times(dsa, step, args.steps, stream, flush)
+
     # ---- per-stage device times (same kernels, same launch shapes) ----
     scores = torch.empty((T, (wl.max_ctx + 3) // 4 * 4), dtype=torch.float32, device=dev)
     ws_i = torch.zeros(dsa.dsa_workspace_size(dsa.DSA_OP_INDEX_SCORES, d.seqs, K, H), dtype=torch.uint8, device=dev)
@@ -339,7 +377,13 @@ def run_ours(args, world, rank, local):
     attn_bytes = n_sel * 1152                                    # gathered latent rows
     peak, peak_kind = hbm_peak()
     ms_idx = statistics.mean(t_idx)
-    achieved = idx_bytes / (ms_idx / 1e3) / 1e9
+    score_bytes = n_keys * 4 + T * K * 4                          # Top-K: score rows read, indices written
+    roofs = {}
+    for name, nbytes in (("index_scores", idx_bytes), ("topk_filter_select", score_bytes),
+                         ("sparse_mla", attn_bytes)):
+        if name in kern:
+            roofs[name] = roofline_entry(name, kern, nbytes, peak, peak_kind)
+    dominant = max(roofs.values(), key=lambda r: r["launch_us"])
 
     # ---- end to end through the C ABI with host buffers ----
     pin = lambda x: x.pin_memory()  # noqa: E731
@@ -391,13 +435,9 @@ def run_ours(args, world, rank, local):
                        "launch": launch_mode},
             "stages_us": {"index_scores": ms_idx * 1e3, "topk": statistics.mean(t_topk) * 1e3,
                           "sparse_mla": statistics.mean(t_attn) * 1e3},
-            "roofline": {"kernel": "index_scores (quantize + score)", "bound": "hbm", "achieved": achieved,
-                         "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_kind,
-                         "algorithmic_bytes": idx_bytes, "traffic": None},
-            "attention_roofline": {"bound": "hbm", "achieved": attn_bytes / (statistics.mean(t_attn) / 1e3) / 1e9,
-                                   "peak": peak, "unit": "GB/s",
-                                   "frac": attn_bytes / (statistics.mean(t_attn) / 1e3) / 1e9 / peak,
-                                   "algorithmic_bytes": attn_bytes},
+            "roofline": dominant,
+            "kernel_rooflines": roofs,
+            "kernels_us": {k: 1e3 * statistics.mean(v) for k, v in kern.items()},
             "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,

@@ -246,6 +246,24 @@ dsa_status_t dsa_check_error(void *ws, dsa_stream_t stream);
  * (dsa_quantize_index_query .. dsa_index_topk_attn) launched.  Host only. */
 int dsa_launches_in_last_call(void);
 
+/* Per-launch device timing: a measurement aid with no counterpart in the
+ * method's description.  enable != 0: every later entry-point call made by the
+ * calling host thread records a CUDA event on its stream before its first
+ * kernel and one after each kernel it launches -- so each kernel then runs
+ * without overlapping its neighbours, and the call is slower than untimed.
+ * enable == 0 stops this and destroys the events.  The events belong to the
+ * device current at the enabling call (thread-local library state, the one
+ * exception to "no state between calls").  Returns DSA_OK or DSA_ERR_CUDA. */
+dsa_status_t dsa_launch_timing(int enable);
+
+/* For the calling thread's most recent entry-point call made with timing on:
+ * waits for its last event, then writes up to `cap` entries -- ms[i], the
+ * device milliseconds from the event before kernel i to the one after it, and
+ * names[i], a static string naming the kernel (either array may be NULL).
+ * Returns how many kernels that call launched (possibly more than cap; at
+ * most 16 are timed), 0 if timing was off for it, -1 on a CUDA error. */
+int dsa_last_launch_times(float *ms, const char **names, int cap);
+
 /* Static, human-readable name of a status. */
 const char *dsa_status_string(dsa_status_t status);
 

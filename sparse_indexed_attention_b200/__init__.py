@@ -37,7 +37,8 @@ DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA
 
 # Names the C header declares (checked against include/dsa.h by the tests).
 EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_index_scores", "dsa_topk",
-           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_noalloc", "dsa_index_topk_attn", "dsa_check_error", "dsa_launches_in_last_call", "dsa_status_string")
+           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_noalloc", "dsa_index_topk_attn", "dsa_check_error", "dsa_launches_in_last_call",
+           "dsa_launch_timing", "dsa_last_launch_times", "dsa_status_string")
 
 
 class DsaSeqsC(ctypes.Structure):
@@ -63,6 +64,9 @@ _sig = {
     "dsa_check_error": (ctypes.c_int, [_P, _P]),
     "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dsa_launches_in_last_call": (ctypes.c_int, []),
+    "dsa_launch_timing": (ctypes.c_int, [ctypes.c_int]),
+    "dsa_last_launch_times": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_char_p),
+                                             ctypes.c_int]),
 }
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)
@@ -251,6 +255,22 @@ def dsa_check_error(ws: torch.Tensor) -> int:
 def dsa_launches_in_last_call() -> int:
     """Kernels launched by this thread's most recent entry-point call."""
     return int(_lib.dsa_launches_in_last_call())
+
+
+def dsa_launch_timing(enable: bool) -> None:
+    """Record device events around every kernel of this thread's later calls."""
+    _check(_lib.dsa_launch_timing(1 if enable else 0), "dsa_launch_timing")
+
+
+def dsa_last_launch_times() -> list:
+    """[(kernel name, device ms)] of this thread's last call made with timing on."""
+    cap = 16
+    ms = (ctypes.c_float * cap)()
+    names = (ctypes.c_char_p * cap)()
+    n = int(_lib.dsa_last_launch_times(ms, names, cap))
+    if n < 0:
+        raise DsaError(DSA_ERR_CUDA, "dsa_last_launch_times")
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n, cap))]
 
 
 def raw():

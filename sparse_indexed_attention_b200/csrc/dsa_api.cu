@@ -9,6 +9,7 @@ using namespace dsa;
 
 namespace dsa {
 thread_local int g_launches = 0;
+thread_local LaunchTimer g_timer;
 }
 
 namespace {
@@ -187,6 +188,7 @@ dsa_status_t dsa_quantize_index_query(const void* qI, const float* w, int T, uin
   if (!qI || !w || !codes || !w_scaled || T < 1) return DSA_ERR_INVALID_ARG;
   if (!aligned(qI, 16) || !aligned(codes, 16) || !aligned(w, 4) || !aligned(w_scaled, 4))
     return DSA_ERR_INVALID_ARG;
+  timer_begin((cudaStream_t)stream);
   return cuda_status(launch_quantize_index_query(reinterpret_cast<const __nv_bfloat16*>(qI), w, T, codes, w_scaled,
                                                  (cudaStream_t)stream));
 }
@@ -204,6 +206,7 @@ dsa_status_t dsa_index_scores(const dsa_seqs_t* seqs, const void* qI, const floa
   const SeqsDev sd = to_dev(seqs);
   const PlanBufs plan = plan_bufs(ws, L);
   const int tg = indexer_group_tokens(seqs->num_q_tokens, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
+  timer_begin(st);
   return run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, ld, ws, L, nullptr, nullptr, 0, err,
                      st);
 }
@@ -217,6 +220,7 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row
   if (!aligned(scores, 16) || !aligned(row_len, 4) || !aligned(idx, 16)) return DSA_ERR_INVALID_ARG;
   const Layout L = make_layout(DSA_OP_TOPK, T, 1, (int)ld, K, 16);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
+  timer_begin((cudaStream_t)stream);
   return cuda_status(
       launch_topk(scores, ld, T, row_len, nullptr, K, idx, at<void>(ws, L.topk), false, at<uint32_t>(ws, 0),
                   (cudaStream_t)stream));
@@ -235,6 +239,7 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const voi
   const SeqsDev sd = to_dev(seqs);
   const PlanBufs plan = plan_bufs(ws, L);
   TokenMap tm{plan.tok_seq, plan.tok_pos};
+  timer_begin(st);
   DSA_CUDA(launch_plan(sd, 1, 0, plan, err, st));  // token geometry only
   DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
@@ -265,6 +270,7 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const f
   const bool fuse_hist = tg == 1 && topk_uses_hist(T, L.ld);
   uint32_t* hist = fuse_hist ? topk_hist_in_scratch(at<void>(ws, L.topk), T) : nullptr;
   uint32_t* zero = fuse_hist ? at<uint32_t>(ws, L.topk) : nullptr;  // Top-K's counters + histogram
+  timer_begin(st);
   DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, hist, zero,
                       fuse_hist ? topk_zero_words(T) : 0, err, st));
   DSA_CUDA(launch_topk(scores, L.ld, T, nullptr, tm.pos, K, idx, at<void>(ws, L.topk), hist != nullptr, err, st));
@@ -290,6 +296,41 @@ dsa_status_t dsa_check_error(void* ws, dsa_stream_t stream) {
 }
 
 int dsa_launches_in_last_call(void) { return g_launches; }
+
+dsa_status_t dsa_launch_timing(int enable) {
+  LaunchTimer& tm = g_timer;
+  if (tm.device >= 0) {  // tear down (also before re-enabling)
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != tm.device) cudaSetDevice(tm.device);
+    for (cudaEvent_t& e : tm.ev) {
+      if (e) cudaEventDestroy(e);
+      e = nullptr;
+    }
+    if (cur >= 0 && cur != tm.device) cudaSetDevice(cur);
+    tm.device = -1;
+  }
+  tm.armed = false;
+  tm.n = 0;
+  if (!enable) return DSA_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  for (cudaEvent_t& e : tm.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) return DSA_ERR_CUDA;
+  tm.device = dev;
+  return DSA_OK;
+}
+
+int dsa_last_launch_times(float* ms, const char** names, int cap) {
+  const LaunchTimer& tm = g_timer;
+  if (!tm.armed || tm.n == 0) return 0;
+  if (cudaEventSynchronize(tm.ev[tm.n]) != cudaSuccess) return -1;
+  for (int i = 0; i < tm.n && i < cap; ++i) {
+    if (ms && cudaEventElapsedTime(&ms[i], tm.ev[i], tm.ev[i + 1]) != cudaSuccess) return -1;
+    if (names) names[i] = tm.name[i];
+  }
+  return g_launches > tm.n ? g_launches : tm.n;
+}
 
 const char* dsa_status_string(dsa_status_t s) {
   switch (s) {

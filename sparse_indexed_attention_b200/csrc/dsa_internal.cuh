@@ -84,9 +84,34 @@ struct SeqsDev {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Optional per-launch timing (dsa_launch_timing): event 0 before a call's
+// first kernel, event i+1 after its kernel i.
+constexpr int kMaxTimedLaunches = 16;
+struct LaunchTimer {
+  int device = -1;     // the events exist, on this device, when >= 0
+  bool armed = false;  // the current call records events
+  int n = 0;           // kernels timed in the current / last timed call
+  cudaEvent_t ev[kMaxTimedLaunches + 1] = {};
+  const char* name[kMaxTimedLaunches] = {};
+};
+extern thread_local LaunchTimer g_timer;
+
+// Start of an entry point's launches on stream st.
+__host__ inline void timer_begin(cudaStream_t st) {
+  g_timer.armed = g_timer.device >= 0;
+  g_timer.n = 0;
+  if (g_timer.armed) cudaEventRecord(g_timer.ev[0], st);
+}
+
+__host__ inline void timer_mark(const char* name, cudaStream_t st) {
+  if (!g_timer.armed || g_timer.n >= kMaxTimedLaunches) return;
+  g_timer.name[g_timer.n] = name;
+  cudaEventRecord(g_timer.ev[++g_timer.n], st);
+}
+
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                              Args&&... args) {
+inline cudaError_t launch_pdl(const char* name, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -97,7 +122,9 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) timer_mark(name, st);
+  return e;
 }
 
 // Kernels launched by the current host thread since its last entry-point call
@@ -107,6 +134,7 @@ __host__ inline cudaError_t counted(cudaError_t e) {
   if (e == cudaSuccess) ++g_launches;
   return e;
 }
+
 
 // Work plan written by k_plan (see k_prep.cu).
 struct PlanBufs {

@@ -439,7 +439,7 @@ cudaError_t launch_tc(const CUtensorMap& mk, const CUtensorMap& mq, const IdxArg
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  cudaError_t e = launch_pdl(k_index_scores_tc<kBf16, TG>, dim3(sm_count()), dim3(kIdxThreads), (size_t)C::SMEM, st, mk,
+  cudaError_t e = launch_pdl("index_scores", k_index_scores_tc<kBf16, TG>, dim3(sm_count()), dim3(kIdxThreads), (size_t)C::SMEM, st, mk,
                              mq, a);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());

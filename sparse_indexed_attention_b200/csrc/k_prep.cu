@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBu
 }
 
 cudaError_t launch_plan(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err, cudaStream_t st) {
-  cudaError_t e = launch_pdl(k_plan, dim3(1), dim3(1024), 0, st, s, tg, ch, p, err);
+  cudaError_t e = launch_pdl("plan", k_plan, dim3(1), dim3(1024), 0, st, s, tg, ch, p, err);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }
@@ -255,7 +255,7 @@ cudaError_t launch_prep(const SeqsDev& s, int tg, int ch, const PlanBufs& plan, 
   const int64_t nq = qI ? ((int64_t)s.num_tokens * kHI + 31) / 32 : 0;
   const int64_t nz = zero ? (zero_words + 4095) / 4096 : 0;
   const int64_t extra = nq > nz ? nq : nz;
-  cudaError_t e = launch_pdl(k_prep, dim3((unsigned)(1 + extra)), dim3(1024), 0, st, a);
+  cudaError_t e = launch_pdl("prep", k_prep, dim3((unsigned)(1 + extra)), dim3(1024), 0, st, a);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }
@@ -265,7 +265,7 @@ cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w,
   int rows = T * kHI;
   int threads = 256;
   int blocks = (rows * 32 + threads - 1) / threads;
-  cudaError_t e = launch_pdl(k_quantize_index_query, dim3(blocks), dim3(threads), 0, st, qI, w, rows, codes, w_scaled);
+  cudaError_t e = launch_pdl("quantize_index_query", k_quantize_index_query, dim3(blocks), dim3(threads), 0, st, qI, w, rows, codes, w_scaled);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }

@@ -550,11 +550,11 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16
     attr_dev = dev;
   }
   AttnArgs a{s, tm, kv, idx, K, H, ks, splits, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
-  cudaError_t e = launch_pdl(k_sparse_mla_tc, dim3(2 * T * splits), dim3(256), (size_t)SMEM_BYTES, st, tq_lat, tq_rope,
+  cudaError_t e = launch_pdl("sparse_mla", k_sparse_mla_tc, dim3(2 * T * splits), dim3(256), (size_t)SMEM_BYTES, st, tq_lat, tq_rope,
                              a);
   if (e == cudaSuccess) e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
-  e = launch_pdl(k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o, (const float2*)part_ml,
+  e = launch_pdl("sparse_mla_combine", k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o, (const float2*)part_ml,
                  tm.pos, out, out_f32, lse);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());

@@ -514,7 +514,7 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* r
     static thread_local int dev_row = -1;
     cudaError_t e = set_smem_once(k_topk_row, (int)sizeof(RowSmem), &dev_row);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(k_topk_row, dim3(T), dim3(kRowThreads), sizeof(RowSmem), st, scores, ld, row_len, tok_pos, K, idx,
+    e = launch_pdl("topk_row", k_topk_row, dim3(T), dim3(kRowThreads), sizeof(RowSmem), st, scores, ld, row_len, tok_pos, K, idx,
                    err);
     if (e != cudaSuccess) return e;
     return counted(cudaGetLastError());
@@ -530,12 +530,12 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* r
   const dim3 grid(C, T);
   if (!hist_ready) {  // otherwise the caller has zeroed the region and filled the histogram
     if ((e = cudaMemsetAsync(scratch, 0, (size_t)topk_zero_words(T) * 4, st)) != cudaSuccess) return e;
-    e = launch_pdl(k_topk_hist, grid, dim3(kChunkThreads), 0, st, scores, ld, row_len, tok_pos, K, chunk, ghist, err);
+    e = launch_pdl("topk_hist", k_topk_hist, grid, dim3(kChunkThreads), 0, st, scores, ld, row_len, tok_pos, K, chunk, ghist, err);
     if (e != cudaSuccess || (e = counted(cudaGetLastError())) != cudaSuccess) return e;
   }
   static thread_local int dev_fs = -1;
   if ((e = set_smem_once(k_topk_filter_select, (int)sizeof(SelSmem), &dev_fs)) != cudaSuccess) return e;
-  e = launch_pdl(k_topk_filter_select, grid, dim3(kChunkThreads), sizeof(SelSmem), st, scores, ld, row_len, tok_pos, K,
+  e = launch_pdl("topk_filter_select", k_topk_filter_select, grid, dim3(kChunkThreads), sizeof(SelSmem), st, scores, ld, row_len, tok_pos, K,
                  chunk, C, (const uint32_t*)ghist, ghist2, counts, kept, row_done, idx);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
