@@ -47,8 +47,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage-reps", type=int, default=20)
-    ap.add_argument("--only", choices=["index_scores", "topk", "sparse_mla"], default=None,
-                    help="time one stage alone on the bench workload (profiling aid)")
+    ap.add_argument("--only", choices=["index_scores", "topk", "sparse_mla", "fused"], default=None,
+                    help="time one stage (or the fused call, eagerly) alone on the bench workload (profiling aid)")
     return ap.parse_args()
 
 
@@ -274,7 +274,7 @@ def roofline_entry(name, per, algorithmic_bytes, peak, peak_kind):
             "launch_us": ms * 1e3, "traffic": None}
 
 
-def run_only(args, dsa, wl, d, dev, stream, flush, world):
+def run_only(args, dsa, wl, d, dev, stream, flush, world, fused=None):
     """One stage alone, `--steps` timed launches after `--warmup` (profiling aid)."""
     spec = wl.spec
     T, H, K = wl.T, spec.heads, spec.topk
@@ -289,6 +289,7 @@ def run_only(args, dsa, wl, d, dev, stream, flush, world):
         "index_scores": lambda: dsa.dsa_index_scores(d.seqs, d.qI, d.w, d.kI, d.kI_scale, scores=scores),
         "topk": lambda: dsa.dsa_topk(scores, row_len, K, idx=idx),
         "sparse_mla": lambda: dsa.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out=out, lse=lse),
+        "fused": fused,
     }
     times = time_device(fns[args.only], args.steps, args.warmup, stream, flush)
     if world == 1 or int(os.environ.get("RANK", "0")) == 0:
@@ -317,7 +318,7 @@ def run_ours(args, world, rank, local):
         dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse, ws=ws)
 
     if args.only:
-        run_only(args, dsa, wl, d, dev, stream, flush, world)
+        run_only(args, dsa, wl, d, dev, stream, flush, world, fused=step)
         return
 
     step()

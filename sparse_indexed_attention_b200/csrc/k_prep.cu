@@ -47,9 +47,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_buf, int* t
   return r;
 }
 
-__device__ __forceinline__ bool seq_ok(const SeqsDev& s, int b, int* q_len_out, int* ctx_out) {
-  const int q_len = __ldg(s.q_seq_start + b + 1) - __ldg(s.q_seq_start + b);
-  const int ctx = __ldg(s.ctx_len + b);
+// Sequences whose q_seq_start / ctx_len the plan stages in shared memory
+// (larger batches are read from global memory).
+constexpr int kPlanSeqs = 1024;
+
+// qs / cl: q_seq_start and ctx_len, staged in shared memory or global.
+__device__ __forceinline__ bool seq_ok(const SeqsDev& s, const int* qs, const int* cl, int b, int* q_len_out,
+                                       int* ctx_out) {
+  const int q_len = qs[b + 1] - qs[b];
+  const int ctx = cl[b];
   *q_len_out = q_len;
   *ctx_out = ctx;
   return q_len >= 0 && ctx >= 1 && ctx <= s.max_ctx && q_len <= ctx && (ctx + kPage - 1) / kPage <= s.max_pages;
@@ -68,17 +74,30 @@ __device__ __forceinline__ bool seq_ok(const SeqsDev& s, int b, int* q_len_out, 
 //   counts                {G, I}.
 __device__ __forceinline__ void plan_body(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err) {
   __shared__ int warp_buf[33];
+  __shared__ int sh_qs[kPlanSeqs + 1], sh_cl[kPlanSeqs], sh_gs[kPlanSeqs + 1];
   const int tid = threadIdx.x;
+  // one round of coalesced loads instead of chains of dependent ones
+  const bool staged = s.batch <= kPlanSeqs;
+  if (staged) {
+    for (int b = tid; b <= s.batch; b += blockDim.x) {
+      sh_qs[b] = __ldg(s.q_seq_start + b);
+      if (b < s.batch) sh_cl[b] = __ldg(s.ctx_len + b);
+    }
+    __syncthreads();
+  }
+  const int* qs = staged ? sh_qs : s.q_seq_start;
+  const int* cl = staged ? sh_cl : s.ctx_len;
+  int* gs = staged ? sh_gs : p.seq_gstart;
   for (int t = tid; t < s.num_tokens; t += blockDim.x) {
     int lo = 0, hi = s.batch - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(s.q_seq_start + mid) <= t) lo = mid; else hi = mid - 1;
+      if (qs[mid] <= t) lo = mid; else hi = mid - 1;
     }
     const int b = lo;
-    const int start = __ldg(s.q_seq_start + b), end = __ldg(s.q_seq_start + b + 1);
+    const int start = qs[b], end = qs[b + 1];
     int q_len, ctx;
-    const bool ok = seq_ok(s, b, &q_len, &ctx) && __ldg(s.q_seq_start) == 0 && t >= start && t < end;
+    const bool ok = seq_ok(s, qs, cl, b, &q_len, &ctx) && qs[0] == 0 && t >= start && t < end;
     int pos = ctx - q_len + (t - start);
     if (!ok || pos < 0) {
       raise_error(err, kErrBadIndex);
@@ -95,17 +114,23 @@ __device__ __forceinline__ void plan_body(const SeqsDev& s, int tg, int ch, cons
     int cnt = 0;
     if (b < s.batch) {
       int q_len, ctx;
-      if (seq_ok(s, b, &q_len, &ctx))
+      if (seq_ok(s, qs, cl, b, &q_len, &ctx))
         cnt = (q_len + tg - 1) / tg;
       else
         raise_error(err, kErrBadIndex);
     }
     int total;
     const int excl = block_exclusive_scan(cnt, warp_buf, &total);
-    if (b < s.batch) p.seq_gstart[b] = running + excl;
+    if (b < s.batch) {
+      gs[b] = running + excl;
+      p.seq_gstart[b] = running + excl;
+    }
     running += total;
   }
-  if (tid == 0) p.seq_gstart[s.batch] = running;
+  if (tid == 0) {
+    gs[s.batch] = running;
+    p.seq_gstart[s.batch] = running;
+  }
   __syncthreads();
   const int G = running;
   __shared__ int s_istart[1025];
@@ -120,16 +145,16 @@ __device__ __forceinline__ void plan_body(const SeqsDev& s, int tg, int ch, cons
       int lo = 0, hi = s.batch - 1;  // largest b with seq_gstart[b] <= g
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (p.seq_gstart[mid] <= g) lo = mid; else hi = mid - 1;
+        if (gs[mid] <= g) lo = mid; else hi = mid - 1;
       }
       const int b = lo;
-      const int q_len = __ldg(s.q_seq_start + b + 1) - __ldg(s.q_seq_start + b);
-      const int j0 = (g - p.seq_gstart[b]) * tg;
+      const int q_len = qs[b + 1] - qs[b];
+      const int j0 = (g - gs[b]) * tg;
       const int cnt = min(tg, q_len - j0);
-      const int pos0 = __ldg(s.ctx_len + b) - q_len + j0;
+      const int pos0 = cl[b] - q_len + j0;
       tiles = (pos0 + cnt - 1) / 128 + 1;
       nitems = (tiles + ch - 1) / ch;
-      gd = make_int4(b, __ldg(s.q_seq_start + b) + j0, cnt, pos0);
+      gd = make_int4(b, qs[b] + j0, cnt, pos0);
       p.groups[g] = gd;
     }
     int total;
