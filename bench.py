@@ -36,6 +36,29 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
+# DRAM bytes (read + write) per launch from one ncu capture on this workload
+# (profiles/<kernel>_decode_b8_128k.md), valid only while the kernel's sources
+# hash to what was captured: any edit turns the figure back into null.
+NCU_TRAFFIC = {
+    "index_scores": (143.71e6, ("k_indexer.cu",), "032c38f69f0b5616"),
+    "topk_filter_select": (4.41e6, ("k_topk.cu",), "c122968935f163f0"),
+    "sparse_mla": (20.25e6, ("k_sparse_mla.cu",), "60cb7ea372510e1a"),
+}
+CSRC = os.path.join(ROOT, "sparse_indexed_attention_b200", "csrc")
+
+
+def ncu_traffic(kernel: str, config: str):
+    """Captured DRAM traffic of `kernel` per launch, or None if stale / not captured."""
+    if config != "decode_b8_128k" or kernel not in NCU_TRAFFIC:
+        return None
+    import hashlib
+    nbytes, files, digest = NCU_TRAFFIC[kernel]
+    m = hashlib.sha256()
+    for f in (*files, "dsa_internal.cuh", "sm100.cuh"):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            m.update(fh.read())
+    return nbytes if m.hexdigest()[:16] == digest else None
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -266,12 +289,12 @@ def kernel_times(dsa, step, steps, stream, flush):
     return per
 
 
-def roofline_entry(name, per, algorithmic_bytes, peak, peak_kind):
+def roofline_entry(name, per, algorithmic_bytes, peak, peak_kind, config):
     ms = statistics.mean(per[name])
     achieved = algorithmic_bytes / (ms / 1e3) / 1e9
     return {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": peak_kind, "algorithmic_bytes": algorithmic_bytes,
-            "launch_us": ms * 1e3, "traffic": None}
+            "launch_us": ms * 1e3, "traffic": ncu_traffic(name, config)}
 
 
 def run_only(args, dsa, wl, d, dev, stream, flush, world, fused=None):
@@ -383,7 +406,7 @@ def run_ours(args, world, rank, local):
     for name, nbytes in (("index_scores", idx_bytes), ("topk_filter_select", score_bytes),
                          ("sparse_mla", attn_bytes)):
         if name in kern:
-            roofs[name] = roofline_entry(name, kern, nbytes, peak, peak_kind)
+            roofs[name] = roofline_entry(name, kern, nbytes, peak, peak_kind, spec.name)
     dominant = max(roofs.values(), key=lambda r: r["launch_us"])
 
     # ---- end to end through the C ABI with host buffers ----
