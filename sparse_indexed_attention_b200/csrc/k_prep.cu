@@ -72,22 +72,34 @@ __device__ __forceinline__ bool seq_ok(const SeqsDev& s, const int* qs, const in
 //                         {tile_begin, tile_end, g, 0}: a run of <= `ch` key tiles
 //                         of 128 positions (tiles cover 0 .. last pos);
 //   counts                {G, I}.
-__device__ __forceinline__ void plan_body(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err) {
-  __shared__ int warp_buf[33];
-  __shared__ int sh_qs[kPlanSeqs + 1], sh_cl[kPlanSeqs], sh_gs[kPlanSeqs + 1];
+// The plan's shared memory (declared once, used by either instantiation).
+struct PlanSmem {
+  int warp_buf[33];
+  int qs[kPlanSeqs + 1], cl[kPlanSeqs], gs[kPlanSeqs + 1];  // staged sequence arrays
+  int istart[1025];
+  int tiles[1024];
+  int4 gd[1024];
+};
+
+template <bool kStaged>
+__device__ __forceinline__ void plan_impl(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err,
+                                          PlanSmem& sm) {
+  int* warp_buf = sm.warp_buf;
+  int* sh_qs = sm.qs;
+  int* sh_cl = sm.cl;
+  int* sh_gs = sm.gs;
   const int tid = threadIdx.x;
-  // one round of coalesced loads instead of chains of dependent ones
-  const bool staged = s.batch <= kPlanSeqs;
-  if (staged) {
+  // staged: one round of coalesced loads instead of chains of dependent ones
+  if constexpr (kStaged) {
     for (int b = tid; b <= s.batch; b += blockDim.x) {
       sh_qs[b] = __ldg(s.q_seq_start + b);
       if (b < s.batch) sh_cl[b] = __ldg(s.ctx_len + b);
     }
     __syncthreads();
   }
-  const int* qs = staged ? sh_qs : s.q_seq_start;
-  const int* cl = staged ? sh_cl : s.ctx_len;
-  int* gs = staged ? sh_gs : p.seq_gstart;
+  const int* qs = kStaged ? sh_qs : s.q_seq_start;
+  const int* cl = kStaged ? sh_cl : s.ctx_len;
+  int* gs = kStaged ? sh_gs : p.seq_gstart;
   for (int t = tid; t < s.num_tokens; t += blockDim.x) {
     int lo = 0, hi = s.batch - 1;
     while (lo < hi) {
@@ -133,9 +145,9 @@ __device__ __forceinline__ void plan_body(const SeqsDev& s, int tg, int ch, cons
   }
   __syncthreads();
   const int G = running;
-  __shared__ int s_istart[1025];
-  __shared__ int s_tiles[1024];
-  __shared__ int4 s_gd[1024];
+  int* s_istart = sm.istart;
+  int* s_tiles = sm.tiles;
+  int4* s_gd = sm.gd;
   int irun = 0;
   for (int gbase = 0; gbase < G; gbase += blockDim.x) {
     const int g = gbase + tid;
@@ -185,6 +197,14 @@ __device__ __forceinline__ void plan_body(const SeqsDev& s, int tg, int ch, cons
   }
 }
 
+__device__ __forceinline__ void plan_body(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err) {
+  __shared__ PlanSmem sm;
+  if (s.batch <= kPlanSeqs)
+    plan_impl<true>(s, tg, ch, p, err, sm);
+  else
+    plan_impl<false>(s, tg, ch, p, err, sm);
+}
+
 __global__ void __launch_bounds__(1024) k_plan(SeqsDev s, int tg, int ch, PlanBufs p, uint32_t* err) {
   pdl_wait();
   pdl_trigger();
@@ -218,15 +238,16 @@ __device__ __forceinline__ void quant_row(const __nv_bfloat16* __restrict__ qI, 
     while (amax > ldexpf(448.f, e)) ++e;
     while (amax <= ldexpf(448.f, e - 1)) --e;
   }
-  // x * 2^-e is exact in double; the result lies within [-448, 448].
+  // x * 2^-e, correctly rounded (exact unless the result is subnormal, where
+  // E4M3 rounds it to zero anyway); the result lies within [-448, 448].
   float y[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) y[i] = (float)ldexp((double)x[i], -e);
+  for (int i = 0; i < 4; ++i) y[i] = ldexpf(x[i], -e);
   __nv_fp8x2_storage_t c01 = __nv_cvt_float2_to_fp8x2(make_float2(y[0], y[1]), __NV_SATFINITE, __NV_E4M3);
   __nv_fp8x2_storage_t c23 = __nv_cvt_float2_to_fp8x2(make_float2(y[2], y[3]), __NV_SATFINITE, __NV_E4M3);
   const uint32_t packed = (uint32_t)c01 | ((uint32_t)c23 << 16);
   reinterpret_cast<uint32_t*>(codes + (int64_t)row * kDI)[lane] = packed;
-  if (lane == 0) w_scaled[row] = (float)ldexp((double)__ldg(w + row), e);
+  if (lane == 0) w_scaled[row] = ldexpf(__ldg(w + row), e);
 }
 
 __global__ void k_quantize_index_query(const __nv_bfloat16* __restrict__ qI, const float* __restrict__ w,

@@ -52,7 +52,6 @@ constexpr int kQBytes = 4 * kQLatBytes + 128 * 64;
 constexpr int kKVStage = 4 * kBK * 128 + kBK * 64;  // 36864: 4 latent atoms + rope quarter
 constexpr int kXBytes = 128 * kBK * 4;       // one partial S: [16 column quads][128 heads][4] fp32
 constexpr int kLoaders = 96;                 // warps 0, 2, 3 copy the selected rows
-constexpr int kChunksPerRow = 36;            // 16-byte pieces of a CTA's 576 bytes of a row
 constexpr int kRingBlocks = 4;               // resolved row ids, blocks j .. j+2 live
 constexpr int kLoaderBarrier = 1;            // named barrier of the loader warps
 constexpr int OFF_Q = 0;
@@ -73,6 +72,14 @@ constexpr uint32_t IDESC_PV = make_idesc_major(true, 128, 256, 0, 1);  // O += P
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
+
+// 2^x from the MUFU unit (approximate, subnormal results flushed to 0;
+// ex2(-inf) = +0).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ void store_out(void* out, bool f32, int64_t i, float v) {
   if (f32)
@@ -198,22 +205,24 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       const int stage = j & 1, slot = j % kRingBlocks;
       bool ok = mbar_wait(&kv_empty[stage], ((j >> 1) & 1) ^ 1, a.err);
       if (ok) {
+        // one warp per row: lane k copies latent piece k (16 B = 8 dims) of
+        // the CTA's 256 latent dims; rope pieces go 8 rows per instruction
         const uint32_t dst0 = kv_smem + stage * kKVStage;
-        for (int c = li; c < kBK * kChunksPerRow; c += kLoaders) {
-          const int r = c / kChunksPerRow, k = c - r * kChunksPerRow;
+        const int lw = warp == 0 ? 0 : warp - 1;  // loader warp 0 .. 2
+        for (int r = lw; r < kBK; r += 3) {
           const int row = ring_rows[slot * kBK + r];
-          uint32_t dst;
-          int64_t col;
-          if (k < 32) {  // latent dims 256*rank + 8k .. +7: 128-byte swizzle atom k/8
-            dst = dst0 + (k >> 3) * (kBK * 128) + r * 128 + ((((uint32_t)k & 7u) ^ ((uint32_t)r & 7u)) << 4);
-            col = 256 * rank + 8 * k;
-          } else {       // rope dims 512 + 32*rank + 8(k-32) .. +7: 64-byte swizzle
-            const uint32_t kr = (uint32_t)(k - 32);
-            dst = dst0 + 4 * (kBK * 128) + r * 64 + ((kr ^ (((uint32_t)r >> 1) & 3u)) << 4);
-            col = 512 + 32 * rank + 8 * kr;
-          }
           const bool v = row >= 0;
-          cp_async_16_zfill(dst, kv_base + (v ? (int64_t)row * kDQK + col : 0), v ? 16u : 0u);
+          const uint32_t dst = dst0 + (lane >> 3) * (kBK * 128) + r * 128 +
+                               ((((uint32_t)lane & 7u) ^ ((uint32_t)r & 7u)) << 4);
+          cp_async_16_zfill(dst, kv_base + (v ? (int64_t)row * kDQK + 256 * rank + 8 * lane : 0), v ? 16u : 0u);
+        }
+        for (int g8 = lw; g8 < kBK / 8; g8 += 3) {
+          const int r = 8 * g8 + (lane >> 2);
+          const uint32_t kr = (uint32_t)lane & 3u;
+          const int row = ring_rows[slot * kBK + r];
+          const bool v = row >= 0;
+          const uint32_t dst = dst0 + 4 * (kBK * 128) + r * 64 + ((kr ^ (((uint32_t)r >> 1) & 3u)) << 4);
+          cp_async_16_zfill(dst, kv_base + (v ? (int64_t)row * kDQK + 512 + 32 * rank + 8 * kr : 0), v ? 16u : 0u);
         }
       }
       cp_async_mbar_arrive(&kv_full[stage]);  // counts once this thread's copies land
@@ -335,25 +344,37 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[sb], (j >> 1) & 1, a.err));
       if (!ok) break;
       const uint64_t mask = ring_mask[j % kRingBlocks];
-      float mblk = -INFINITY;
+      // masked rows -> -inf; with scale > 0 the scaled maximum is the scaled
+      // raw maximum, and each probability is one FMA and one ex2
+      float mraw = -INFINITY, mneg = INFINITY;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        s[i] = ((mask >> i) & 1ull) ? s[i] * a.scale_log2 : -INFINITY;
-        mblk = fmaxf(mblk, s[i]);
+        const bool on = (mask >> i) & 1ull;
+        s[i] = on ? s[i] : -INFINITY;
+        mraw = fmaxf(mraw, s[i]);
+        mneg = fminf(mneg, on ? s[i] : INFINITY);
       }
+      const float sc = a.scale_log2;
+      // scale <= 0 (allowed, if odd): the largest scaled logit comes from the smallest raw one
+      const float mblk = mraw == -INFINITY ? -INFINITY : (sc > 0.f ? mraw * sc : mneg * sc);
       const bool move = mblk > m_ref + kRescaleThreshold;
       const float m_new = move ? mblk : m_ref;
       const float alpha = move ? exp2f(m_ref - m_new) : 1.f;  // exp2(-inf) = 0 on the first block
+      const float mu = m_new == -INFINITY ? 0.f : m_new;      // nothing unmasked yet: every term is 0
       uint32_t pk[32], pl[32];
       float psum = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float e0 = m_new == -INFINITY ? 0.f : exp2f(s[2 * i] - m_new);
-        const float e1 = m_new == -INFINITY ? 0.f : exp2f(s[2 * i + 1] - m_new);
+        // masked: s = -inf and sc > 0 give ex2(-inf) = 0; sc <= 0 takes the select
+        const float x0 = fmaf(s[2 * i], sc, -mu), x1 = fmaf(s[2 * i + 1], sc, -mu);
+        const float e0 = sc > 0.f ? ex2_ftz(x0) : (s[2 * i] == -INFINITY ? 0.f : ex2_ftz(x0));
+        const float e1 = sc > 0.f ? ex2_ftz(x1) : (s[2 * i + 1] == -INFINITY ? 0.f : ex2_ftz(x1));
         psum += e0 + e1;
         const __nv_bfloat162 hi = __floats2bfloat162_rn(e0, e1);
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(e0 - __low2float(hi), e1 - __high2float(hi));
-        pk[i] = *reinterpret_cast<const uint32_t*>(&hi);
+        const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hi);
+        const __nv_bfloat162 lo =
+            __floats2bfloat162_rn(e0 - __uint_as_float(hb << 16), e1 - __uint_as_float(hb & 0xFFFF0000u));
+        pk[i] = hb;
         pl[i] = *reinterpret_cast<const uint32_t*>(&lo);
       }
       tmem_st32(t_lane + kTmemP + 64 * sb, pk);
@@ -453,26 +474,52 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
 }
 
 // Merge the split partials of one (token, head): rescale to the common max.
+// The (max, sum) pairs go through shared memory; the partial rows are loaded
+// in batches of 8 slices, each batch's loads issued together, the first batch
+// alongside the pairs (one round trip for up to 8 slices).
+constexpr int kMaxSplits = 32;  // ceil(K / 64) for K <= 2048
+constexpr int kCombineBatch = 8;
+
 __global__ void __launch_bounds__(128)
 k_combine(int H, int splits, const float* __restrict__ part_o, const float2* __restrict__ part_ml,
           const int32_t* __restrict__ tok_pos, void* __restrict__ out, bool out_f32, float* __restrict__ lse) {
+  __shared__ float2 s_ml[kMaxSplits];
+  __shared__ int s_pos;
   const int t = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (tok_pos[t] < 0) return;
+  const int64_t row0 = (int64_t)t * splits * H + h;  // slice i: row0 + i * H
+  if (tid < splits) s_ml[tid] = __ldcg(part_ml + row0 + (int64_t)tid * H);
+  if (tid == 0) s_pos = tok_pos[t];
+  float4 v[kCombineBatch];
+#pragma unroll
+  for (int i = 0; i < kCombineBatch; ++i)
+    if (i < splits) v[i] = __ldcg(reinterpret_cast<const float4*>(part_o + (row0 + (int64_t)i * H) * kDV) + tid);
+  __syncthreads();
+  if (s_pos < 0) return;
   float M = -INFINITY;
-  for (int i = 0; i < splits; ++i) M = fmaxf(M, part_ml[((int64_t)t * splits + i) * H + h].x);
+  for (int i = 0; i < splits; ++i)
+    if (s_ml[i].y != 0.f) M = fmaxf(M, s_ml[i].x);
   float L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int i = 0; i < splits; ++i) {
-    const float2 ml = part_ml[((int64_t)t * splits + i) * H + h];
-    if (ml.y == 0.f) continue;
-    const float f = __expf(ml.x - M);
-    L += ml.y * f;
-    const float4 v = *reinterpret_cast<const float4*>(part_o + (((int64_t)t * splits + i) * H + h) * kDV + tid * 4);
-    o[0] += v.x * f;
-    o[1] += v.y * f;
-    o[2] += v.z * f;
-    o[3] += v.w * f;
+  for (int b0 = 0; b0 < splits; b0 += kCombineBatch) {
+    if (b0 > 0) {
+#pragma unroll
+      for (int i = 0; i < kCombineBatch; ++i)
+        if (b0 + i < splits)
+          v[i] = __ldcg(reinterpret_cast<const float4*>(part_o + (row0 + (int64_t)(b0 + i) * H) * kDV) + tid);
+    }
+#pragma unroll
+    for (int i = 0; i < kCombineBatch; ++i) {
+      const int k = b0 + i;
+      if (k < splits && s_ml[k].y != 0.f) {  // an empty slice wrote nothing usable
+        const float f = __expf(s_ml[k].x - M);
+        L += s_ml[k].y * f;
+        o[0] += v[i].x * f;
+        o[1] += v[i].y * f;
+        o[2] += v[i].z * f;
+        o[3] += v[i].w * f;
+      }
+    }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const int64_t base = ((int64_t)t * H + h) * kDV + tid * 4;

@@ -24,11 +24,15 @@
 // chunk does 3 and 4); otherwise one CTA does a row.  A degenerate row that
 // keeps more pairs than shared memory holds is resolved from global memory
 // (several CTAs per row) or by four 8-bit radix passes over the row (one CTA).
-#include "dsa_internal.cuh"
+#include "sm100.cuh"
 
 namespace dsa {
 
 namespace {
+
+using sm100::cp_async_8;
+using sm100::cp_async_16;
+using sm100::cp_async_wait_all;
 
 constexpr int kHistBins = kTopkHistBins;  // digit 1: key bits 31..21
 constexpr int kLowBits = kTopkLowBits;
@@ -39,6 +43,7 @@ constexpr int kRowStage = 12288;          // kept pairs in shared memory, one-CT
 constexpr int kChunkThreads = 512;
 constexpr int kMaxChunks = 64;
 constexpr int kSelStage = 8192;           // kept pairs in shared memory, selecting CTA
+constexpr int kPerThread = 8;             // consecutive scores per thread per pass
 
 __device__ __forceinline__ uint32_t digit2(uint32_t key) { return (key >> 10) & (kD2Bins - 1); }
 
@@ -126,6 +131,30 @@ __device__ __forceinline__ int row_length(const int32_t* row_len, const int32_t*
   const int64_t n64 = row_len ? (int64_t)row_len[t] : (int64_t)tok_pos[t] + 1;
   if (row_len && err && (n64 < 0 || n64 > ld)) raise_error(err, kErrBadIndex);
   return (int)(n64 < 0 ? 0 : (n64 > ld ? ld : n64));
+}
+
+// Keys of positions s0 .. s0+7 (those < end; others 0) and the bit mask of
+// the ones that exist.  s0 is a multiple of 8; `vec` says the row start is
+// 16-byte aligned, so two float4 loads serve a full run.
+__device__ __forceinline__ uint32_t load_keys8(const float* __restrict__ row, int s0, int end, bool vec,
+                                               uint32_t (&keys)[kPerThread]) {
+  if (vec && s0 + kPerThread <= end) {
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(row + s0));
+    const float4 b = __ldcg(reinterpret_cast<const float4*>(row + s0 + 4));
+    keys[0] = order_key(a.x); keys[1] = order_key(a.y); keys[2] = order_key(a.z); keys[3] = order_key(a.w);
+    keys[4] = order_key(b.x); keys[5] = order_key(b.y); keys[6] = order_key(b.z); keys[7] = order_key(b.w);
+    return 0xFFu;
+  }
+  uint32_t have = 0;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    keys[j] = 0;
+    if (s0 + j < end) {
+      keys[j] = order_key(__ldcg(row + s0 + j));
+      have |= 1u << j;
+    }
+  }
+  return have;
 }
 
 // Emits, in the order of the list, the position of every element whose key is
@@ -258,11 +287,12 @@ k_topk_row(const float* __restrict__ scores, int64_t ld, const int32_t* __restri
     return;
   }
   __syncthreads();
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int s = base + threadIdx.x;
-    const bool act = s < n;
-    const uint32_t key = act ? order_key(row[s]) : 0u;
-    hist_add(sm.hist, key >> kLowBits, act);
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  for (int base = 0; base < n; base += blockDim.x * kPerThread) {
+    uint32_t keys[kPerThread];
+    const uint32_t have = load_keys8(row, base + threadIdx.x * kPerThread, n, vec, keys);
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) hist_add(sm.hist, keys[j] >> kLowBits, (have >> j) & 1u);
   }
   __syncthreads();
   find_bin(sm.hist, kHistBins, (uint32_t)K, sm.buf, &sm.bin, &sm.above);
@@ -275,23 +305,20 @@ k_topk_row(const float* __restrict__ scores, int64_t ld, const int32_t* __restri
   }
   // keep (position, key) for digit 1 >= b1, in position order; digit 2 of b1's members
   uint32_t run = 0;
-  for (int base = 0; base < n; base += blockDim.x * 4) {
-    const int s0 = base + threadIdx.x * 4;
-    uint32_t keep = 0, keys[4];
+  for (int base = 0; base < n; base += blockDim.x * kPerThread) {
+    const int s0 = base + threadIdx.x * kPerThread;
+    uint32_t keys[kPerThread];
+    const uint32_t have = load_keys8(row, s0, n, vec, keys);
+    uint32_t keep = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      keys[j] = 0;
-      if (s0 + j < n) {
-        keys[j] = order_key(row[s0 + j]);
-        keep |= (uint32_t)((keys[j] >> kLowBits) >= b1) << j;
-      }
-    }
+    for (int j = 0; j < kPerThread; ++j) keep |= (uint32_t)(((have >> j) & 1u) && (keys[j] >> kLowBits) >= b1) << j;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) hist_add(sm.hist2, digit2(keys[j]), (keep >> j & 1u) && (keys[j] >> kLowBits) == b1);
+    for (int j = 0; j < kPerThread; ++j)
+      hist_add(sm.hist2, digit2(keys[j]), (keep >> j & 1u) && (keys[j] >> kLowBits) == b1);
     uint32_t total;
     uint32_t p = run + block_scan((uint32_t)__popc(keep), sm.buf, &total);
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < kPerThread; ++j)
       if (keep >> j & 1u) {
         if (p < (uint32_t)kRowStage) sm.kept[p] = make_int2(s0 + j, (int)keys[j]);
         ++p;
@@ -321,11 +348,12 @@ k_topk_hist(const float* __restrict__ scores, int64_t ld, const int32_t* __restr
   if (n <= K || b0 >= b1) return;
   __syncthreads();
   const float* __restrict__ row = scores + (int64_t)t * ld;
-  for (int base = b0; base < b1; base += blockDim.x) {
-    const int s = base + threadIdx.x;
-    const bool act = s < b1;
-    const uint32_t key = act ? order_key(row[s]) : 0u;
-    hist_add(hist, key >> kLowBits, act);
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  for (int base = b0; base < b1; base += blockDim.x * kPerThread) {
+    uint32_t keys[kPerThread];
+    const uint32_t have = load_keys8(row, base + threadIdx.x * kPerThread, b1, vec, keys);
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) hist_add(hist, keys[j] >> kLowBits, (have >> j) & 1u);
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
@@ -348,7 +376,9 @@ struct SelSmem {
 __device__ void select_row(int t, int K, int chunk, int C, uint32_t b1, uint32_t above,
                            const uint32_t* __restrict__ ghist2, const int* __restrict__ counts,
                            const int2* __restrict__ kept, int32_t* __restrict__ out, SelSmem& sm) {
-  for (int i = threadIdx.x; i < kD2Bins; i += blockDim.x) sm.hist2[i] = __ldcg(ghist2 + (int64_t)t * kD2Bins + i);
+  // asynchronous copies: the whole histogram is one round trip, not a chain
+  for (int i = 4 * threadIdx.x; i < kD2Bins; i += 4 * blockDim.x)
+    cp_async_16(&sm.hist2[i], ghist2 + (int64_t)t * kD2Bins + i);
   if (threadIdx.x < 32) {  // chunk counts -> offsets (two chunks per lane)
     const int lane = threadIdx.x;
     const int a0 = 2 * lane < C ? __ldcg(counts + (int64_t)t * C + 2 * lane) : 0;
@@ -367,16 +397,19 @@ __device__ void select_row(int t, int K, int chunk, int C, uint32_t b1, uint32_t
   const int L = sm.off[C];  // offsets past C hold the same total
   const int2* row_kept = kept + (int64_t)t * C * chunk;
   if (L <= kSelStage) {
-    // each warp copies whole chunks: contiguous, independent loads
+    // each warp copies whole chunks, every copy in flight at once
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int c = warp; c < C; c += nw) {
       const int o = sm.off[c], cnt = sm.off[c + 1] - o;
-      for (int i = lane; i < cnt; i += 32) sm.kept[o + i] = __ldcg(row_kept + (int64_t)c * chunk + i);
+      for (int i = lane; i < cnt; i += 32) cp_async_8(&sm.kept[o + i], row_kept + (int64_t)c * chunk + i);
     }
+    cp_async_wait_all();
     __syncthreads();
     resolve_row([&](int i) { return sm.kept[i]; }, L, b1, (uint32_t)K - above, K, sm.hist2, sm.buf, &sm.bin,
                 &sm.above, out);
   } else {  // degenerate row: read the pairs where the chunks left them
+    cp_async_wait_all();  // the histogram
+    __syncthreads();
     auto get = [&](int i) -> int2 {
       int lo = 0, hi = C - 1;  // last chunk whose offset <= i
       while (lo < hi) {
@@ -410,47 +443,49 @@ k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t
     return;
   }
   const int b0 = c * chunk, b1 = min(n, b0 + chunk);
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sm.hist[i] = __ldcg(ghist + (int64_t)t * kHistBins + i);
+  for (int i = 4 * threadIdx.x; i < kHistBins; i += 4 * blockDim.x)
+    cp_async_16(&sm.hist[i], ghist + (int64_t)t * kHistBins + i);
+  cp_async_wait_all();
   __syncthreads();
   find_bin(sm.hist, kHistBins, (uint32_t)K, sm.buf, &sm.bin, &sm.above);
   const uint32_t bstar = sm.bin, above = sm.above;
   const float* __restrict__ row = scores + (int64_t)t * ld;
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
   int2* my_kept = kept + ((int64_t)t * C + c) * chunk;
   uint32_t run = 0;
-  for (int base = b0; base < b1; base += blockDim.x * 4) {
-    const int s0 = base + threadIdx.x * 4;
-    uint32_t keep = 0, keys[4];
+  for (int base = b0; base < b1; base += blockDim.x * kPerThread) {
+    const int s0 = base + threadIdx.x * kPerThread;
+    uint32_t keys[kPerThread];
+    const uint32_t have = load_keys8(row, s0, b1, vec, keys);
+    uint32_t keep = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      keys[j] = 0;
-      if (s0 + j < b1) {
-        keys[j] = order_key(row[s0 + j]);
-        keep |= (uint32_t)((keys[j] >> kLowBits) >= bstar) << j;
-      }
-    }
+    for (int j = 0; j < kPerThread; ++j) keep |= (uint32_t)(((have >> j) & 1u) && (keys[j] >> kLowBits) >= bstar) << j;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < kPerThread; ++j)
       hist_add(sm.hist2, digit2(keys[j]), (keep >> j & 1u) && (keys[j] >> kLowBits) == bstar);
     uint32_t total;
     uint32_t p = run + block_scan((uint32_t)__popc(keep), sm.buf, &total);
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < kPerThread; ++j)
       if (keep >> j & 1u) my_kept[p++] = make_int2(s0 + j, (int)keys[j]);  // p < chunk: one pair per position
     run += total;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kD2Bins; i += blockDim.x)
     if (sm.hist2[i]) atomicAdd(&ghist2[(int64_t)t * kD2Bins + i], sm.hist2[i]);
-  __threadfence();  // this thread's pairs and histogram adds precede the count
+  // The barrier orders every thread's pairs and histogram adds before thread
+  // 0's device-scope fence and count; the row's last CTA fences after seeing
+  // the count, before its barrier -- a release / acquire pair through row_done.
   __syncthreads();
   if (threadIdx.x == 0) {
     counts[(int64_t)t * C + c] = (int)run;
     __threadfence();
-    sm.last = atomicAdd(&row_done[t], 1) == C - 1;
+    const bool last = atomicAdd(&row_done[t], 1) == C - 1;
+    if (last) __threadfence();
+    sm.last = last;
   }
   __syncthreads();
   if (!sm.last) return;
-  __threadfence();  // the other chunks' pairs are visible from here on
   select_row(t, K, chunk, C, bstar, above, ghist2, counts, kept, out, sm);
 }
 
