@@ -17,6 +17,16 @@ namespace dsa {
 
 namespace {
 
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
 // Exclusive prefix sum over a 1024-thread block; returns the thread's prefix
 // and writes the block total to *total.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_buf, int* total) {
@@ -120,9 +130,7 @@ __device__ __forceinline__ void plan_impl(const SeqsDev& s, int tg, int ch, cons
   }
   if (ch <= 0) return;  // token geometry only
   // groups per sequence -> start offsets (an invalid sequence gets none)
-  int running = 0;
-  for (int base = 0; base < s.batch; base += blockDim.x) {
-    const int b = base + tid;
+  auto groups_of = [&](int b) -> int {
     int cnt = 0;
     if (b < s.batch) {
       int q_len, ctx;
@@ -131,54 +139,67 @@ __device__ __forceinline__ void plan_impl(const SeqsDev& s, int tg, int ch, cons
       else
         raise_error(err, kErrBadIndex);
     }
-    int total;
-    const int excl = block_exclusive_scan(cnt, warp_buf, &total);
-    if (b < s.batch) {
-      gs[b] = running + excl;
-      p.seq_gstart[b] = running + excl;
+    return cnt;
+  };
+  int running = 0;
+  if (s.batch <= 32) {  // one warp, shuffles only
+    if (tid < 32) {
+      const int cnt = groups_of(tid);
+      const int incl = warp_inclusive_scan(cnt);
+      if (tid < s.batch) {
+        gs[tid] = incl - cnt;
+        p.seq_gstart[tid] = incl - cnt;
+      }
+      if (tid == 31) {  // lanes past the batch add nothing
+        gs[s.batch] = incl;
+        p.seq_gstart[s.batch] = incl;
+      }
     }
-    running += total;
+    __syncthreads();
+    running = gs[s.batch];
+  } else {
+    for (int base = 0; base < s.batch; base += blockDim.x) {
+      const int b = base + tid;
+      const int cnt = groups_of(b);
+      int total;
+      const int excl = block_exclusive_scan(cnt, warp_buf, &total);
+      if (b < s.batch) {
+        gs[b] = running + excl;
+        p.seq_gstart[b] = running + excl;
+      }
+      running += total;
+    }
+    if (tid == 0) {
+      gs[s.batch] = running;
+      p.seq_gstart[s.batch] = running;
+    }
+    __syncthreads();
   }
-  if (tid == 0) {
-    gs[s.batch] = running;
-    p.seq_gstart[s.batch] = running;
-  }
-  __syncthreads();
   const int G = running;
   int* s_istart = sm.istart;
   int* s_tiles = sm.tiles;
   int4* s_gd = sm.gd;
-  int irun = 0;
-  for (int gbase = 0; gbase < G; gbase += blockDim.x) {
-    const int g = gbase + tid;
-    int nitems = 0, tiles = 0;
-    int4 gd = make_int4(0, 0, 0, 0);
-    if (g < G) {
-      int lo = 0, hi = s.batch - 1;  // largest b with seq_gstart[b] <= g
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (gs[mid] <= g) lo = mid; else hi = mid - 1;
-      }
-      const int b = lo;
-      const int q_len = qs[b + 1] - qs[b];
-      const int j0 = (g - gs[b]) * tg;
-      const int cnt = min(tg, q_len - j0);
-      const int pos0 = cl[b] - q_len + j0;
-      tiles = (pos0 + cnt - 1) / 128 + 1;
-      nitems = (tiles + ch - 1) / ch;
-      gd = make_int4(b, qs[b] + j0, cnt, pos0);
-      p.groups[g] = gd;
+  // group g: its descriptor, key tiles and work items
+  auto describe = [&](int g, int* tiles, int* nitems) -> int4 {
+    int lo = 0, hi = s.batch - 1;  // largest b with seq_gstart[b] <= g
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (gs[mid] <= g) lo = mid; else hi = mid - 1;
     }
-    int total;
-    const int excl = block_exclusive_scan(nitems, warp_buf, &total);
-    s_istart[tid] = excl;
-    s_tiles[tid] = tiles;
-    s_gd[tid] = gd;
-    if (tid == 0) s_istart[blockDim.x] = total;
-    __syncthreads();
-    // write this chunk's items cooperatively: item i belongs to the last group j with s_istart[j] <= i
+    const int b = lo;
+    const int q_len = qs[b + 1] - qs[b];
+    const int j0 = (g - gs[b]) * tg;
+    const int cnt = min(tg, q_len - j0);
+    const int pos0 = cl[b] - q_len + j0;
+    *tiles = (pos0 + cnt - 1) / 128 + 1;
+    *nitems = (*tiles + ch - 1) / ch;
+    return make_int4(b, qs[b] + j0, cnt, pos0);
+  };
+  // items [irun, irun + total) of groups gbase .. gbase + ng - 1, whose
+  // prefixes / tiles / descriptors sit in s_istart / s_tiles / s_gd
+  auto write_items = [&](int irun, int total, int gbase, int ng) {
     for (int i = tid; i < total; i += blockDim.x) {
-      int lo = 0, hi = blockDim.x - 1;
+      int lo = 0, hi = ng - 1;  // last local group with s_istart <= i
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (s_istart[mid] <= i) lo = mid; else hi = mid - 1;
@@ -188,8 +209,45 @@ __device__ __forceinline__ void plan_impl(const SeqsDev& s, int tg, int ch, cons
       p.items[2 * (irun + i)] = s_gd[lo];
       p.items[2 * (irun + i) + 1] = make_int4(j * ch, min(tl, (j + 1) * ch), gbase + lo, 0);
     }
-    irun += total;
+  };
+  int irun = 0;
+  if (G <= 32) {  // one warp, shuffles only
+    if (tid < 32) {
+      int nitems = 0, tiles = 0;
+      int4 gd = make_int4(0, 0, 0, 0);
+      if (tid < G) {
+        gd = describe(tid, &tiles, &nitems);
+        p.groups[tid] = gd;
+      }
+      const int incl = warp_inclusive_scan(nitems);
+      s_istart[tid] = incl - nitems;
+      s_tiles[tid] = tiles;
+      s_gd[tid] = gd;
+      if (tid == 31) s_istart[32] = incl;
+    }
     __syncthreads();
+    irun = s_istart[32];
+    write_items(0, irun, 0, G);
+  } else {
+    for (int gbase = 0; gbase < G; gbase += blockDim.x) {
+      const int g = gbase + tid;
+      int nitems = 0, tiles = 0;
+      int4 gd = make_int4(0, 0, 0, 0);
+      if (g < G) {
+        gd = describe(g, &tiles, &nitems);
+        p.groups[g] = gd;
+      }
+      int total;
+      const int excl = block_exclusive_scan(nitems, warp_buf, &total);
+      s_istart[tid] = excl;
+      s_tiles[tid] = tiles;
+      s_gd[tid] = gd;
+      if (tid == 0) s_istart[blockDim.x] = total;
+      __syncthreads();
+      write_items(irun, total, gbase, min((int)blockDim.x, G - gbase));
+      irun += total;
+      __syncthreads();
+    }
   }
   if (tid == 0) {
     p.counts[0] = G;

@@ -48,7 +48,9 @@ constexpr int kPerThread = 8;             // consecutive scores per thread per p
 __device__ __forceinline__ uint32_t digit2(uint32_t key) { return (key >> 10) & (kD2Bins - 1); }
 
 // Exclusive block-wide prefix sum of v (blockDim.x a multiple of 32, <= 1024);
-// *total receives the sum.  Uses the 33-word scratch `buf`.
+// *total receives the sum.  Each warp scans its own values; the warp totals
+// go through `buf` (32 words) and every warp reduces them itself -- two
+// barriers and no second serial scan.
 __device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* buf, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   uint32_t incl = v;
@@ -59,55 +61,73 @@ __device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* buf, uint32
   }
   if (lane == 31) buf[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    const uint32_t w = lane < nw ? buf[lane] : 0u;
-    uint32_t wi = w;
+  const uint32_t x = lane < nw ? buf[lane] : 0u;
+  uint32_t below = lane < warp ? x : 0u, all = x;  // totals of the earlier warps / of every warp
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t u = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += u;
-    }
-    buf[lane] = wi - w;
-    if (lane == 31) buf[32] = wi;
+  for (int o = 16; o > 0; o >>= 1) {
+    below += __shfl_xor_sync(0xffffffffu, below, o);
+    all += __shfl_xor_sync(0xffffffffu, all, o);
   }
-  __syncthreads();
-  const uint32_t r = buf[warp] + incl - v;
-  *total = buf[32];
-  __syncthreads();
-  return r;
+  *total = all;
+  __syncthreads();  // buf is free for the next scan
+  return below + incl - v;
 }
 
-// In a histogram of `bins` bins (a power of two, >= 32), find d such that the
-// keys above d number `above` < need <= above + hist[d].  The whole block
-// takes part: thread i sums a run of bins counted from the top, one block scan
-// gives every run the count above it, and the thread whose run holds the
-// crossing writes the result.  If no bin qualifies (need 0 or above the total)
-// the result is bin 0 with nothing above it.  Ends with a barrier.
+// In a histogram of `bins` bins (a power of two, 256 .. 2048), find d such
+// that the keys above d number `above` < need <= above + hist[d].  Warp 0
+// alone: lane l sums the bins [l*per, l*per + per) (rotated reads, no bank
+// conflicts), a suffix scan over the lanes finds the lane holding the
+// crossing, and a second pass splits that lane's bins over the warp.  If no
+// bin qualifies (need 0 or above the total) the result is bin 0 with nothing
+// above it.  Ends with a barrier; `buf` is unused.
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int bins, uint32_t need, uint32_t* buf,
                                          uint32_t* out_bin, uint32_t* out_above) {
-  const int per = bins > (int)blockDim.x ? bins / (int)blockDim.x : 1;
-  const int runs = bins / per;
-  const int i = threadIdx.x;
-  const int top = bins - 1 - i * per;  // this thread's run: top, top-1, ..., top-per+1
-  uint32_t sum = 0;
-  if (i < runs)
-    for (int j = 0; j < per; ++j) sum += hist[top - j];
-  if (i == 0) {
-    *out_bin = 0u;
-    *out_above = 0u;
-  }
-  uint32_t total;
-  const uint32_t excl = block_scan(sum, buf, &total);  // barriers order the defaults first
-  if (i < runs && sum != 0 && excl < need && need <= excl + sum) {
-    uint32_t above = excl;
-    for (int j = 0; j < per; ++j) {
-      const uint32_t c = hist[top - j];
-      if (above + c >= need) {
-        *out_bin = (uint32_t)(top - j);
-        *out_above = above;
-        break;
+  (void)buf;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = bins >> 5;
+    uint32_t sum = 0;
+    for (int j = 0; j < per; ++j) sum += hist[lane * per + ((j + lane) & (per - 1))];
+    uint32_t incl = sum;  // keys in this lane's bins and every higher lane's
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += u;
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, incl - sum < need && need <= incl);
+    if (who == 0) {
+      if (lane == 0) {
+        *out_bin = 0u;
+        *out_above = 0u;
       }
-      above += c;
+    } else {
+      const int L = __ffs(who) - 1;
+      const uint32_t above_l = __shfl_sync(0xffffffffu, incl - sum, L);
+      const int q = per >= 32 ? per >> 5 : 1;    // bins per lane in the second pass
+      const int top = L * per + per - 1 - lane * q;  // this lane's bins: top, top-1, ..., top-q+1
+      const bool mine = lane * q < per;
+      uint32_t s2 = 0;
+      if (mine)
+        for (int j = 0; j < q; ++j) s2 += hist[top - j];
+      uint32_t inc2 = s2;  // from the top of L's range down to this lane's bins
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xffffffffu, inc2, o);
+        if (lane >= o) inc2 += u;
+      }
+      const uint32_t ex = above_l + inc2 - s2;
+      if (mine && s2 != 0 && ex < need && need <= ex + s2) {
+        uint32_t above = ex;
+        for (int j = 0; j < q; ++j) {
+          const uint32_t c = hist[top - j];
+          if (above + c >= need) {
+            *out_bin = (uint32_t)(top - j);
+            *out_above = above;
+            break;
+          }
+          above += c;
+        }
+      }
     }
   }
   __syncthreads();
@@ -445,18 +465,20 @@ k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t
   const int b0 = c * chunk, b1 = min(n, b0 + chunk);
   for (int i = 4 * threadIdx.x; i < kHistBins; i += 4 * blockDim.x)
     cp_async_16(&sm.hist[i], ghist + (int64_t)t * kHistBins + i);
+  // the first pass's scores are in flight together with the histogram
+  const float* __restrict__ row = scores + (int64_t)t * ld;
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  uint32_t keys[kPerThread];
+  uint32_t have = load_keys8(row, b0 + threadIdx.x * kPerThread, b1, vec, keys);
   cp_async_wait_all();
   __syncthreads();
   find_bin(sm.hist, kHistBins, (uint32_t)K, sm.buf, &sm.bin, &sm.above);
   const uint32_t bstar = sm.bin, above = sm.above;
-  const float* __restrict__ row = scores + (int64_t)t * ld;
-  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
   int2* my_kept = kept + ((int64_t)t * C + c) * chunk;
   uint32_t run = 0;
   for (int base = b0; base < b1; base += blockDim.x * kPerThread) {
     const int s0 = base + threadIdx.x * kPerThread;
-    uint32_t keys[kPerThread];
-    const uint32_t have = load_keys8(row, s0, b1, vec, keys);
+    if (base != b0) have = load_keys8(row, s0, b1, vec, keys);
     uint32_t keep = 0;
 #pragma unroll
     for (int j = 0; j < kPerThread; ++j) keep |= (uint32_t)(((have >> j) & 1u) && (keys[j] >> kLowBits) >= bstar) << j;
