@@ -61,8 +61,11 @@ constexpr int OFF_ROWS = OFF_X + 2 * kXBytes;           // 212992: [ring][64] po
 constexpr int OFF_MASK = OFF_ROWS + kRingBlocks * kBK * 4;  // [ring] 64-bit validity masks
 constexpr int OFF_BAR = OFF_MASK + kRingBlocks * 8;
 constexpr int kNBars = 14;
-constexpr int OFF_MISC = OFF_BAR + kNBars * 8;
+constexpr int OFF_PAIR = OFF_BAR + kNBars * 8;          // [2 parity][2 half][128 heads] float2
+constexpr int OFF_MISC = OFF_PAIR + 2 * 2 * 128 * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+constexpr int kThreads = 384;                // warps 0, 2, 3 load; 1 issues MMAs; 4-11 softmax
+constexpr int kPairBarrier = 2;              // named barriers 2..5: softmax warps w and w+4
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 static_assert(OFF_KV % 1024 == 0 && kKVStage % 1024 == 0, "swizzle atoms need 1024-B alignment");
 constexpr uint32_t kTmemS = 256, kTmemP = 384;  // TMEM column bases (O at 0)
@@ -103,7 +106,7 @@ struct AttnArgs {
   uint32_t* err;
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constant__ CUtensorMap tq_rope,
                 const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -136,9 +139,9 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       mbar_init(&kv_full[i], kLoaders + 1);  // every loader's copies + the mask's publisher
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
+      mbar_init(&s_empty[i], 8);
     }
-    mbar_init(p_full, 4);   // one arrival per softmax warp
+    mbar_init(p_full, 8);   // one arrival per softmax warp
     for (int i = 0; i < 2; ++i) {
       mbar_init(&o_done[i], 1);
       mbar_init(&x_full[i], 1);  // armed by this CTA (expect_tx), filled by the peer's st.async
@@ -292,79 +295,93 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     __syncwarp();
   } else if (warp >= 4 && nblk > 0) {
     // ---------------------------------------------------------------- softmax / exchange / epilogue
-    const int qw = warp - 4;
+    // Eight warps: warp 4+q and warp 8+q share TMEM lane quarter q (heads
+    // 32q .. 32q+31); half g = 0 / 1 takes logits 32g .. 32g+31 of every
+    // block and value dims 128g .. 128g+127 of O.  The two halves of a head
+    // combine their maxima (and at the end their sums) through shared memory
+    // at a 64-thread named barrier, which also carries any failure, so both
+    // warps of a pair always leave together.
+    const int sw = warp - 4, half = sw >> 2, qw = sw & 3;
     const int h = qw * 32 + lane;  // head row = TMEM lane
+    const int cb = 32 * half;      // this half's first logit of a block
     const uint32_t t_lane = tmem + ((uint32_t)(qw * 32) << 16);
+    const int pair_bar = kPairBarrier + qw;
+    float2* pair = reinterpret_cast<float2*>(smem + OFF_PAIR);  // [parity][half][head]
     // X[b][c][h] holds logits 4c .. 4c+3 of head h: a warp's stores of one c
     // are 512 contiguous bytes
     const float4* xcol = reinterpret_cast<const float4*>(smem + OFF_X) + h;
     const uint32_t x_peer = map_peer(smem_u32(smem + OFF_X), peer) + (uint32_t)h * 16u;
     const uint32_t x_full_peer = map_peer(smem_u32(x_full), peer);
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nblk && ok; ++j) {
+    const float sc = a.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;  // l: this half's share of the sum
+    bool good = true;
+    for (int j = 0; j < nblk; ++j) {
       const int sb = j & 1;
       // s_full(j) also means PV(j-2) is complete (it was issued before QK(j)),
       // so P's buffer sb is free
-      ok = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&s_full[sb], (j >> 1) & 1, a.err));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(t_lane + kTmemS + kBK * sb, v0);
-      tmem_ld32(t_lane + kTmemS + kBK * sb + 32, v1);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
-      // my partial logits -> the peer's receive area sb
-      const uint32_t xp = x_peer + (uint32_t)sb * kXBytes;
-      const uint32_t xb = x_full_peer + (uint32_t)sb * 8u;
+      good = good && __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&s_full[sb], (j >> 1) & 1, a.err));
+      uint32_t v[32];
+      if (good) {
+        tc_fence_after();
+        tmem_ld32(t_lane + kTmemS + kBK * sb + cb, v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[sb]);
+        // my partial logits -> the peer's receive area sb
+        const uint32_t xp = x_peer + (uint32_t)sb * kXBytes;
+        const uint32_t xb = x_full_peer + (uint32_t)sb * 8u;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        st_async_v4(xp + c * 2048, v0[4 * c], v0[4 * c + 1], v0[4 * c + 2], v0[4 * c + 3], xb);
-        st_async_v4(xp + (c + 8) * 2048, v1[4 * c], v1[4 * c + 1], v1[4 * c + 2], v1[4 * c + 3], xb);
+        for (int c = 0; c < 8; ++c)
+          st_async_v4(xp + (8 * half + c) * 2048, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], xb);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait_cluster(&x_full[sb], (j >> 1) & 1, a.err));
-      if (!ok) break;
-      float s[64];
+      good = good && __all_sync(0xffffffffu, mbar_wait_cluster(&x_full[sb], (j >> 1) & 1, a.err));
+      float s[32];
+      if (good) {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 pv4 = xcol[sb * (kXBytes / 16) + c * 128];
-        const uint32_t* mine = c < 8 ? &v0[4 * c] : &v1[4 * (c - 8)];
-        s[4 * c + 0] = __uint_as_float(mine[0]) + pv4.x;
-        s[4 * c + 1] = __uint_as_float(mine[1]) + pv4.y;
-        s[4 * c + 2] = __uint_as_float(mine[2]) + pv4.z;
-        s[4 * c + 3] = __uint_as_float(mine[3]) + pv4.w;
+        for (int c = 0; c < 8; ++c) {
+          const float4 pv4 = xcol[sb * (kXBytes / 16) + (8 * half + c) * 128];
+          s[4 * c + 0] = __uint_as_float(v[4 * c]) + pv4.x;
+          s[4 * c + 1] = __uint_as_float(v[4 * c + 1]) + pv4.y;
+          s[4 * c + 2] = __uint_as_float(v[4 * c + 2]) + pv4.z;
+          s[4 * c + 3] = __uint_as_float(v[4 * c + 3]) + pv4.w;
+        }
+        // re-arm receive area sb for block j+2: the peer only stores into it
+        // after its block j+1 completed, which needs every warp's block j+1
+        // stores from here -- issued after this warp's reads above
+        if (sw == 0 && lane == 0 && j + 2 < nblk) mbar_arrive_expect_tx(&x_full[sb], kXBytes);
       }
-      // re-arm receive area sb for block j+2: the peer only stores into it
-      // after its block j+1 completed, which needs every warp's block j+1
-      // stores from here -- issued after this warp's reads above
-      if (qw == 0 && lane == 0 && j + 2 < nblk) mbar_arrive_expect_tx(&x_full[sb], kXBytes);
       // validity of the block's rows (published before the stage completed)
-      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[sb], (j >> 1) & 1, a.err));
-      if (!ok) break;
-      const uint64_t mask = ring_mask[j % kRingBlocks];
-      // masked rows -> -inf; with scale > 0 the scaled maximum is the scaled
-      // raw maximum, and each probability is one FMA and one ex2
+      good = good && __all_sync(0xffffffffu, mbar_wait(&kv_full[sb], (j >> 1) & 1, a.err));
       float mraw = -INFINITY, mneg = INFINITY;
+      if (good) {
+        const uint32_t m32 = (uint32_t)(ring_mask[j % kRingBlocks] >> cb);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const bool on = (mask >> i) & 1ull;
-        s[i] = on ? s[i] : -INFINITY;
-        mraw = fmaxf(mraw, s[i]);
-        mneg = fminf(mneg, on ? s[i] : INFINITY);
+        for (int i = 0; i < 32; ++i) {
+          const bool on = (m32 >> i) & 1u;
+          s[i] = on ? s[i] : -INFINITY;
+          mraw = fmaxf(mraw, s[i]);
+          mneg = fminf(mneg, on ? s[i] : INFINITY);
+        }
+        pair[((j & 1) * 2 + half) * 128 + h] = make_float2(mraw, mneg);
       }
-      const float sc = a.scale_log2;
+      if (bar_red_or(pair_bar, 64, !good)) {  // either half failed: both leave
+        good = false;
+        break;
+      }
+      const float2 other = pair[((j & 1) * 2 + (half ^ 1)) * 128 + h];
+      mraw = fmaxf(mraw, other.x);
+      mneg = fminf(mneg, other.y);
       // scale <= 0 (allowed, if odd): the largest scaled logit comes from the smallest raw one
       const float mblk = mraw == -INFINITY ? -INFINITY : (sc > 0.f ? mraw * sc : mneg * sc);
       const bool move = mblk > m_ref + kRescaleThreshold;
       const float m_new = move ? mblk : m_ref;
       const float alpha = move ? exp2f(m_ref - m_new) : 1.f;  // exp2(-inf) = 0 on the first block
       const float mu = m_new == -INFINITY ? 0.f : m_new;      // nothing unmasked yet: every term is 0
-      uint32_t pk[32], pl[32];
+      uint32_t pk[16], pl[16];
       float psum = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         // masked: s = -inf and sc > 0 give ex2(-inf) = 0; sc <= 0 takes the select
         const float x0 = fmaf(s[2 * i], sc, -mu), x1 = fmaf(s[2 * i + 1], sc, -mu);
         const float e0 = sc > 0.f ? ex2_ftz(x0) : (s[2 * i] == -INFINITY ? 0.f : ex2_ftz(x0));
@@ -377,23 +394,25 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         pk[i] = hb;
         pl[i] = *reinterpret_cast<const uint32_t*>(&lo);
       }
-      tmem_st32(t_lane + kTmemP + 64 * sb, pk);
-      tmem_st32(t_lane + kTmemP + 64 * sb + 32, pl);
+      // P_hi: columns kTmemP + 64 sb + [0, 32), P_lo: + [32, 64); 16 columns per half
+      tmem_st16(t_lane + kTmemP + 64 * sb + 16 * half, pk);
+      tmem_st16(t_lane + kTmemP + 64 * sb + 32 + 16 * half, pl);
       // TMEM loads/stores are warp-wide: if any head of the warp moved its
-      // maximum, the whole warp rescales O (alpha = 1 leaves a row exact),
-      // once PV(j-1) -- the last writer of O -- has completed
+      // maximum, the warp rescales its half of O (alpha = 1 leaves a row
+      // exact), once PV(j-1) -- the last writer of O -- has completed
       if (j >= 1 && __any_sync(0xffffffffu, move && m_ref != -INFINITY)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err));
-        if (!ok) break;
-        tc_fence_after();
+        good = __all_sync(0xffffffffu, mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err));
+        if (good) {
+          tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_lane + 32 * c, o);
-          tmem_ld_wait();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_lane + 128 * half + 32 * c, o);
+            tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(t_lane + 32 * c, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_lane + 128 * half + 32 * c, o);
+          }
         }
       }
       l = l * alpha + psum;
@@ -401,23 +420,29 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (good && lane == 0) mbar_arrive(p_full);
     }
-    // epilogue: O / l for this CTA's 256 value dims.  tcgen05.ld is warp-wide,
-    // so a warp with any valid head loads; only the stores test h < H.
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(&o_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.err));
-    if (ok) {
+    // epilogue: O / l for this half's 128 value dims.  tcgen05.ld is
+    // warp-wide, so a warp with any valid head loads; only the stores test h < H.
+    good = good && __all_sync(0xffffffffu, mbar_wait(&o_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.err));
+    // the sums go through the parity the last block did not use: its maxima
+    // may still be read by the slower warp of the pair
+    const int ep = nblk & 1;
+    pair[(ep * 2 + half) * 128 + h] = make_float2(l, 0.f);
+    const bool failed = bar_red_or(pair_bar, 64, !good);  // also publishes this half's sum
+    if (!failed) {
+      l += pair[(ep * 2 + (half ^ 1)) * 128 + h].x;
       tc_fence_after();
       const bool store = h < a.H;
       if (qw * 32 < a.H) {
         const float m_nat = m_ref * kLn2;
         if (a.splits == 1) {
           const float inv = l > 0.f ? 1.f / l : 0.f;
-          const int64_t base = ((int64_t)t * a.H + h) * kDV + 256 * rank;
+          const int64_t base = ((int64_t)t * a.H + h) * kDV + 256 * rank + 128 * half;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
-            tmem_ld32(t_lane + 32 * c, o);
+            tmem_ld32(t_lane + 128 * half + 32 * c, o);
             tmem_ld_wait();
             if (!store) continue;
             if (a.out_f32) {
@@ -441,14 +466,14 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
               }
             }
           }
-          if (store && rank == 0 && a.lse) a.lse[(int64_t)t * a.H + h] = m_nat + logf(l);
+          if (store && rank == 0 && half == 0 && a.lse) a.lse[(int64_t)t * a.H + h] = m_nat + logf(l);
         } else {
           const int64_t prow = ((int64_t)t * a.splits + sp) * a.H + h;
-          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * kDV + 256 * rank);
+          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * kDV + 256 * rank + 128 * half);
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
-            tmem_ld32(t_lane + 32 * c, o);
+            tmem_ld32(t_lane + 128 * half + 32 * c, o);
             tmem_ld_wait();
             if (!store) continue;
 #pragma unroll
@@ -456,7 +481,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
               dst[8 * c + i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
                                            __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
           }
-          if (store && rank == 0) a.part_ml[prow] = make_float2(m_nat, l);
+          if (store && rank == 0 && half == 0) a.part_ml[prow] = make_float2(m_nat, l);
         }
       }
     } else {
@@ -597,7 +622,7 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16
     attr_dev = dev;
   }
   AttnArgs a{s, tm, kv, idx, K, H, ks, splits, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
-  cudaError_t e = launch_pdl("sparse_mla", k_sparse_mla_tc, dim3(2 * T * splits), dim3(256), (size_t)SMEM_BYTES, st, tq_lat, tq_rope,
+  cudaError_t e = launch_pdl("sparse_mla", k_sparse_mla_tc, dim3(2 * T * splits), dim3(kThreads), (size_t)SMEM_BYTES, st, tq_lat, tq_rope,
                              a);
   if (e == cudaSuccess) e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
