@@ -14,11 +14,11 @@
 // the work of one (token, slice of the index list) goes to a CLUSTER OF TWO
 // CTAs.  CTA r owns value dims [256r, 256r+256) and the key dims
 // {256r..256r+255} u {512+32r..512+32r+31}; it gathers only those 576 bytes of
-// each selected row.  Three warps resolve the rows (index list -> page table)
-// two blocks ahead and copy them with 16-byte cp.async straight into the
-// 128-byte / 64-byte swizzled operand layouts -- many small copies in flight
-// from 96 threads instead of a queue of four-row TMA gathers.  Per block of 64
-// selected rows:
+// each selected row.  Three warps resolve every selected row of the slice
+// up front (index list -> page table, all loads independent) and then copy
+// the rows block by block with 16-byte cp.async straight into the 128-byte /
+// 64-byte swizzled operand layouts -- many small copies in flight instead of
+// a queue of four-row TMA gathers.  Per block of 64 selected rows:
 //   * S_r = Q_r K_r^T (M = 128 heads, N = 64 rows, K = 288 dims) into TMEM;
 //   * the two partial S are exchanged through distributed shared memory
 //     (st.async into the peer's double-buffered receive area, counted on the
@@ -52,13 +52,13 @@ constexpr int kQBytes = 4 * kQLatBytes + 128 * 64;
 constexpr int kKVStage = 4 * kBK * 128 + kBK * 64;  // 36864: 4 latent atoms + rope quarter
 constexpr int kXBytes = 128 * kBK * 4;       // one partial S: [16 column quads][128 heads][4] fp32
 constexpr int kLoaders = 96;                 // warps 0, 2, 3 copy the selected rows
-constexpr int kRingBlocks = 4;               // resolved row ids, blocks j .. j+2 live
+constexpr int kRingBlocks = kMaxK / kBK;     // resolved row ids of every block of a slice
 constexpr int kLoaderBarrier = 1;            // named barrier of the loader warps
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + kQBytes;                 // 73728
 constexpr int OFF_X = OFF_KV + 2 * kKVStage;            // 147456: two receive buffers
-constexpr int OFF_ROWS = OFF_X + 2 * kXBytes;           // 212992: [ring][64] pool rows (-1 = masked)
-constexpr int OFF_MASK = OFF_ROWS + kRingBlocks * kBK * 4;  // [ring] 64-bit validity masks
+constexpr int OFF_ROWS = OFF_X + 2 * kXBytes;           // 212992: [block][64] pool rows (-1 = masked)
+constexpr int OFF_MASK = OFF_ROWS + kRingBlocks * kBK * 4;  // [block] 64-bit validity masks
 constexpr int OFF_BAR = OFF_MASK + kRingBlocks * 8;
 constexpr int kNBars = 14;
 constexpr int OFF_PAIR = OFF_BAR + kNBars * 8;          // [2 parity][2 half][128 heads] float2
@@ -162,6 +162,13 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   cluster_sync();  // the peer's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) {  // q is an input of the call: its load overlaps the wait below
+    prefetch_tmap(&tq_lat);
+    mbar_arrive_expect_tx(q_full, kQBytes);
+    for (int at = 0; at < 4; ++at)
+      tma_load_2d(smem + OFF_Q + at * kQLatBytes, &tq_lat, q_full, 256 * rank + 64 * at, t * a.H);
+    tma_load_2d(smem + OFF_Q + 4 * kQLatBytes, &tq_rope, q_full, 512 + 32 * rank, t * a.H);
+  }
   pdl_wait();  // the token map and the index lists come from earlier kernels
   pdl_trigger();
   const int pos = a.tm.pos[t];
@@ -171,38 +178,51 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   if ((warp == 0 || warp == 2 || warp == 3) && nblk > 0) {
     // ---------------------------------------------------------------- loaders
     const int li = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0 .. 95
-    if (li == 0) {
-      prefetch_tmap(&tq_lat);
-      mbar_arrive_expect_tx(q_full, kQBytes);
-      for (int at = 0; at < 4; ++at)
-        tma_load_2d(smem + OFF_Q + at * kQLatBytes, &tq_lat, q_full, 256 * rank + 64 * at, t * a.H);
-      tma_load_2d(smem + OFF_Q + 4 * kQLatBytes, &tq_rope, q_full, 512 + 32 * rank, t * a.H);
-    }
-    // Pool rows of block j into ring slot j % kRingBlocks: warps 0 and 2 take
-    // one selected row each (index list -> page table -> row, -1 = masked).
-    auto resolve = [&](int j) {
-      if (j >= nblk || warp == 3) return;
-      const int r = (warp == 0 ? 0 : 32) + lane;
-      const int kk = kbeg + j * kBK + r;
-      int row = -1;
-      if (kk < kend) {
-        const int sidx = __ldg(a.idx + (int64_t)t * a.K + kk);
-        if (sidx >= 0 && sidx <= pos) {
-          const int64_t pr = phys_row(a.s.page_table, a.s.max_pages, a.s.num_phys_pages, b, sidx, a.err);
-          if (pr >= 0) row = (int)pr;
-        } else if (sidx != -1) {
-          raise_error(a.err, kErrBadIndex);
-        }
+    const int lw = warp == 0 ? 0 : warp - 1;                // loader warp 0 .. 2
+    // Pool rows of every block of the slice, resolved up front in three
+    // passes whose loads are all independent: the index list, then the page
+    // ids (both staged by cp.async in the KV stage areas, which the first row
+    // copies overwrite only after the last pass), then rows and masks
+    // (row -1 = masked).
+    {
+      const int nkeys = kend - kbeg;
+      int32_t* s_sidx = reinterpret_cast<int32_t*>(smem + OFF_KV);
+      int32_t* s_page = reinterpret_cast<int32_t*>(smem + OFF_KV + kKVStage);
+      const int32_t* idx_row = a.idx + (int64_t)t * a.K + kbeg;
+      for (int k = li; k < nkeys; k += kLoaders) cp_async_4(&s_sidx[k], idx_row + k);
+      cp_async_wait_all();
+      bar_red_or(kLoaderBarrier, kLoaders, false);
+      const int32_t* pt_row = a.s.page_table + (int64_t)b * a.s.max_pages;
+      for (int k = li; k < nkeys; k += kLoaders) {
+        const int sidx = s_sidx[k];
+        if (sidx >= 0 && sidx <= pos) cp_async_4(&s_page[k], pt_row + (sidx >> 6));  // sidx <= pos: inside the table
       }
-      const int slot = j % kRingBlocks;
-      ring_rows[slot * kBK + r] = row;
-      const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
-      if (lane == 0) reinterpret_cast<uint32_t*>(&ring_mask[slot])[warp == 0 ? 0 : 1] = m;
-    };
+      cp_async_wait_all();
+      bar_red_or(kLoaderBarrier, kLoaders, false);
+      for (int k = li; k < nblk * kBK; k += kLoaders) {
+        int row = -1;
+        if (k < nkeys) {
+          const int sidx = s_sidx[k];
+          if (sidx >= 0 && sidx <= pos) {
+            const int page = s_page[k];
+            if (page >= 0 && page < a.s.num_phys_pages)
+              row = page * kPage + (sidx & (kPage - 1));
+            else
+              raise_error(a.err, kErrBadIndex);
+          } else if (sidx != -1) {
+            raise_error(a.err, kErrBadIndex);
+          }
+        }
+        ring_rows[k] = row;
+      }
+      bar_red_or(kLoaderBarrier, kLoaders, false);
+      for (int w32 = lw; w32 < 2 * nblk; w32 += 3) {  // 32 rows per warp -> half a block's mask
+        const uint32_t m = __ballot_sync(0xffffffffu, ring_rows[w32 * 32 + lane] >= 0);
+        if (lane == 0) reinterpret_cast<uint32_t*>(ring_mask)[w32] = m;
+      }
+    }
     const uint32_t kv_smem = smem_u32(smem + OFF_KV);
     const __nv_bfloat16* kv_base = reinterpret_cast<const __nv_bfloat16*>(a.kv);
-    resolve(0);
-    resolve(1);
     bool failed = bar_red_or(kLoaderBarrier, kLoaders, false);
     for (int j = 0; j < nblk && !failed; ++j) {
       const int stage = j & 1, slot = j % kRingBlocks;
@@ -211,7 +231,6 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         // one warp per row: lane k copies latent piece k (16 B = 8 dims) of
         // the CTA's 256 latent dims; rope pieces go 8 rows per instruction
         const uint32_t dst0 = kv_smem + stage * kKVStage;
-        const int lw = warp == 0 ? 0 : warp - 1;  // loader warp 0 .. 2
         for (int r = lw; r < kBK; r += 3) {
           const int row = ring_rows[slot * kBK + r];
           const bool v = row >= 0;
@@ -229,8 +248,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         }
       }
       cp_async_mbar_arrive(&kv_full[stage]);  // counts once this thread's copies land
-      if (li == 0) mbar_arrive(&kv_full[stage]);  // releases the ring mask read by the softmax warps
-      resolve(j + 2);
+      if (li == 0) mbar_arrive(&kv_full[stage]);  // releases the masks read by the softmax warps
       failed = bar_red_or(kLoaderBarrier, kLoaders, !ok);
       if (failed) *abort_flag = 1;
     }
@@ -355,7 +373,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       good = good && __all_sync(0xffffffffu, mbar_wait(&kv_full[sb], (j >> 1) & 1, a.err));
       float mraw = -INFINITY, mneg = INFINITY;
       if (good) {
-        const uint32_t m32 = (uint32_t)(ring_mask[j % kRingBlocks] >> cb);
+        const uint32_t m32 = (uint32_t)(ring_mask[j] >> cb);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const bool on = (m32 >> i) & 1u;
@@ -489,6 +507,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     }
     __syncwarp();
   }
+  if (threadIdx.x == 0 && nblk == 0) mbar_wait(q_full, 0, a.err);  // no copy in flight at exit
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // no peer still writes into this CTA's shared memory
