@@ -56,11 +56,12 @@ constexpr int kRingBlocks = kMaxK / kBK;     // resolved row ids of every block 
 constexpr int kLoaderBarrier = 1;            // named barrier of the loader warps
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + kQBytes;                 // 73728
-constexpr int OFF_X = OFF_KV + 2 * kKVStage;            // 147456: two receive buffers
-constexpr int OFF_ROWS = OFF_X + 2 * kXBytes;           // 212992: [block][64] pool rows (-1 = masked)
+constexpr int kStages = 3;                              // row stages in flight
+constexpr int OFF_X = OFF_KV + kStages * kKVStage;      // 184320: the peer's partial logits
+constexpr int OFF_ROWS = OFF_X + kXBytes;               // 217088: [block][64] pool rows (-1 = masked)
 constexpr int OFF_MASK = OFF_ROWS + kRingBlocks * kBK * 4;  // [block] 64-bit validity masks
 constexpr int OFF_BAR = OFF_MASK + kRingBlocks * 8;
-constexpr int kNBars = 14;
+constexpr int kNBars = 17;
 constexpr int OFF_PAIR = OFF_BAR + kNBars * 8;          // [2 parity][2 half][128 heads] float2
 constexpr int OFF_MISC = OFF_PAIR + 2 * 2 * 128 * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -113,13 +114,14 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;     // [2]
-  uint64_t* s_empty = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* o_done = bars + 10;    // [2] PV of block i (buffer i & 1) has completed
-  uint64_t* x_full = bars + 12;    // [2] the peer's partial S of a block has landed in my X[buffer]
+  uint64_t* kv_full = bars + 1;    // [kStages] rows of block j (stage j % 3) landed
+  uint64_t* kv_empty = bars + 4;   // [kStages] PV of the stage's block completed
+  uint64_t* s_full = bars + 7;     // [2] S of block j (buffer j & 1) in TMEM
+  uint64_t* s_empty = bars + 9;    // [2] S buffer read by every softmax warp
+  uint64_t* p_full = bars + 11;    // [2] P of block j (buffer j & 1) in TMEM
+  uint64_t* o_done = bars + 13;    // [2] PV of block i (buffer i & 1) has completed
+  uint64_t* x_full = bars + 15;    // the peer's partial S of the current block has landed in X
+  uint64_t* x_free = bars + 16;    // the peer's eight softmax warps have read what I sent
   int32_t* ring_rows = reinterpret_cast<int32_t*>(smem + OFF_ROWS);
   uint64_t* ring_mask = reinterpret_cast<uint64_t*>(smem + OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
@@ -135,23 +137,23 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&kv_full[i], kLoaders + 1);  // every loader's copies + the mask's publisher
       mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 8);
-    }
-    mbar_init(p_full, 8);   // one arrival per softmax warp
-    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 8);  // one arrival per softmax warp
       mbar_init(&o_done[i], 1);
-      mbar_init(&x_full[i], 1);  // armed by this CTA (expect_tx), filled by the peer's st.async
     }
+    mbar_init(x_full, 1);   // armed by this CTA (expect_tx), filled by the peer's st.async
+    mbar_init(x_free, 8);   // one arrival per peer softmax warp
     *abort_flag = 0;
     fence_mbar_init();
-    // receive areas of blocks 0 and 1 armed before the cluster barrier below
-    // lets the peer store into them
-    mbar_arrive_expect_tx(&x_full[0], kXBytes);
-    mbar_arrive_expect_tx(&x_full[1], kXBytes);
+    // the receive area for block 0 is armed before the cluster barrier below
+    // lets the peer store into it
+    mbar_arrive_expect_tx(x_full, kXBytes);
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, 512);
@@ -225,8 +227,8 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     const __nv_bfloat16* kv_base = reinterpret_cast<const __nv_bfloat16*>(a.kv);
     bool failed = bar_red_or(kLoaderBarrier, kLoaders, false);
     for (int j = 0; j < nblk && !failed; ++j) {
-      const int stage = j & 1, slot = j % kRingBlocks;
-      bool ok = mbar_wait(&kv_empty[stage], ((j >> 1) & 1) ^ 1, a.err);
+      const int stage = j % kStages, slot = j;
+      bool ok = mbar_wait(&kv_empty[stage], ((j / kStages) & 1) ^ 1, a.err);
       if (ok) {
         // one warp per row: lane k copies latent piece k (16 B = 8 dims) of
         // the CTA's 256 latent dims; rope pieces go 8 rows per instruction
@@ -255,8 +257,8 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     cp_async_wait_all();
     // drain: every stage has been consumed by the MMA before the CTA exits
     if (li == 0 && !*abort_flag) {
-      for (int j = nblk; j < nblk + 2; ++j)
-        if (!mbar_wait(&kv_empty[j & 1], ((j >> 1) & 1) ^ 1, a.err)) break;
+      for (int j = nblk; j < nblk + kStages; ++j)
+        if (!mbar_wait(&kv_empty[j % kStages], ((j / kStages) & 1) ^ 1, a.err)) break;
     }
     __syncwarp();
   } else if (warp == 1 && nblk > 0) {
@@ -265,49 +267,62 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       const uint32_t q_base = smem_u32(smem + OFF_Q);
       const uint32_t kv_base = smem_u32(smem + OFF_KV);
       bool ok = mbar_wait(q_full, 0, a.err);
-      auto pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full, i & 1, a.err)) return false;
-        tc_fence_after();
-        const uint32_t vb = kv_base + (i & 1) * kKVStage;
-        const uint32_t pb = tmem + kTmemP + 64 * (i & 1);  // P_hi at +0, P_lo at +32 (16 keys per 8 columns)
-#pragma unroll
-        for (int term = 0; term < 2; ++term)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts_bf16(tmem, pb + 32 * term + 8 * kk, smem_desc(vb + kk * 2048, 8192, 1024, 2), IDESC_PV,
-                        i > 0 || term > 0 || kk > 0);
-        mma_commit(&kv_empty[i & 1]);
-        mma_commit(&o_done[i & 1]);
-        return true;
-      };
-      for (int j = 0; j < nblk && ok && !*abort_flag; ++j) {
-        const int sb = j & 1;
-        if (!mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err) ||
-            !mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, a.err)) {
+      // Issue whichever is ready, PV first (it frees a row stage):
+      //   PV(i) once P(i) is in TMEM;
+      //   QK(j) once block j's rows have landed, S buffer j & 1 is free and
+      //   PV(j-2) has been issued -- so s_full(j), which tracks every earlier
+      //   MMA, also tells the softmax warps that P buffer j & 1 is free.
+      int nq = 0, np = 0;  // next block to score / to accumulate
+      uint64_t idle_since = 0;
+      while (ok && np < nblk) {
+        if (*abort_flag) {
           ok = false;
           break;
         }
-        fence_proxy_async_smem();  // the rows were written by cp.async (generic proxy)
-        tc_fence_after();
-        const uint32_t d = tmem + kTmemS + kBK * sb;
-        const uint32_t kb = kv_base + (j & 1) * kKVStage;
+        if (np < nq && mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) {
+          tc_fence_after();
+          const uint32_t vb = kv_base + (np % kStages) * kKVStage;
+          const uint32_t pb = tmem + kTmemP + 64 * (np & 1);  // P_hi at +0, P_lo at +32 (16 keys per 8 columns)
 #pragma unroll
-        for (int at = 0; at < 4; ++at)
+          for (int term = 0; term < 2; ++term)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss<true>(d, smem_desc(q_base + at * kQLatBytes + kk * 32, 16, 1024, 2),
-                         smem_desc(kb + at * (kBK * 128) + kk * 32, 16, 1024, 2), IDESC_QK, (at | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts_bf16(tmem, pb + 32 * term + 8 * kk, smem_desc(vb + kk * 2048, 8192, 1024, 2), IDESC_PV,
+                          np > 0 || term > 0 || kk > 0);
+          mma_commit(&kv_empty[np % kStages]);
+          mma_commit(&o_done[np & 1]);
+          ++np;
+          idle_since = 0;
+        } else if (nq < nblk && nq < np + 2 && mbar_test_wait(&kv_full[nq % kStages], (nq / kStages) & 1) &&
+                   mbar_test_wait(&s_empty[nq & 1], ((nq >> 1) & 1) ^ 1)) {
+          fence_proxy_async_smem();  // the rows were written by cp.async (generic proxy)
+          tc_fence_after();
+          const uint32_t d = tmem + kTmemS + kBK * (nq & 1);
+          const uint32_t kb = kv_base + (nq % kStages) * kKVStage;
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk)
-          mma_ss<true>(d, smem_desc(q_base + 4 * kQLatBytes + kk * 32, 16, 512, 4),
-                       smem_desc(kb + 4 * (kBK * 128) + kk * 32, 16, 512, 4), IDESC_QK, true);
-        mma_commit(&s_full[sb]);
-        if (j >= 1 && !pv(j - 1)) {
-          ok = false;
-          break;
+          for (int at = 0; at < 4; ++at)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss<true>(d, smem_desc(q_base + at * kQLatBytes + kk * 32, 16, 1024, 2),
+                           smem_desc(kb + at * (kBK * 128) + kk * 32, 16, 1024, 2), IDESC_QK, (at | kk) != 0);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_ss<true>(d, smem_desc(q_base + 4 * kQLatBytes + kk * 32, 16, 512, 4),
+                         smem_desc(kb + 4 * (kBK * 128) + kk * 32, 16, 512, 4), IDESC_QK, true);
+          mma_commit(&s_full[nq & 1]);
+          ++nq;
+          idle_since = 0;
+        } else {
+          const uint64_t now = globaltimer();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > kWaitLimitNs) {
+            raise_error(a.err, kErrTimeout);
+            ok = false;
+          }
+          __nanosleep(32);
         }
       }
-      if (ok && !*abort_flag) ok = pv(nblk - 1);
       if (!ok) *abort_flag = 1;
     }
     __syncwarp();
@@ -330,6 +345,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     const float4* xcol = reinterpret_cast<const float4*>(smem + OFF_X) + h;
     const uint32_t x_peer = map_peer(smem_u32(smem + OFF_X), peer) + (uint32_t)h * 16u;
     const uint32_t x_full_peer = map_peer(smem_u32(x_full), peer);
+    const uint32_t x_free_peer = map_peer(smem_u32(x_free), peer);
     const float sc = a.scale_log2;
     float m_ref = -INFINITY, l = 0.f;  // l: this half's share of the sum
     bool good = true;
@@ -346,31 +362,36 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[sb]);
-        // my partial logits -> the peer's receive area sb
-        const uint32_t xp = x_peer + (uint32_t)sb * kXBytes;
-        const uint32_t xb = x_full_peer + (uint32_t)sb * 8u;
+      }
+      // the peer's warps have read my previous block: its receive area is free
+      if (j >= 1) good = good && __all_sync(0xffffffffu, mbar_wait_cluster(x_free, (j - 1) & 1, a.err));
+      if (good) {
+        // my partial logits -> the peer's receive area, counted on its x_full
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          st_async_v4(xp + (8 * half + c) * 2048, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], xb);
+          st_async_v4(x_peer + (8 * half + c) * 2048, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3],
+                      x_full_peer);
       }
-      good = good && __all_sync(0xffffffffu, mbar_wait_cluster(&x_full[sb], (j >> 1) & 1, a.err));
+      good = good && __all_sync(0xffffffffu, mbar_wait_cluster(x_full, j & 1, a.err));
       float s[32];
       if (good) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const float4 pv4 = xcol[sb * (kXBytes / 16) + (8 * half + c) * 128];
+          const float4 pv4 = xcol[(8 * half + c) * 128];
           s[4 * c + 0] = __uint_as_float(v[4 * c]) + pv4.x;
           s[4 * c + 1] = __uint_as_float(v[4 * c + 1]) + pv4.y;
           s[4 * c + 2] = __uint_as_float(v[4 * c + 2]) + pv4.z;
           s[4 * c + 3] = __uint_as_float(v[4 * c + 3]) + pv4.w;
         }
-        // re-arm receive area sb for block j+2: the peer only stores into it
-        // after its block j+1 completed, which needs every warp's block j+1
-        // stores from here -- issued after this warp's reads above
-        if (sw == 0 && lane == 0 && j + 2 < nblk) mbar_arrive_expect_tx(&x_full[sb], kXBytes);
+        // re-arm my receive area for block j+1, then tell the peer this
+        // warp is done with it: the peer stores block j+1 only after all
+        // eight signals, the re-arming warp's among them
+        if (sw == 0 && lane == 0 && j + 1 < nblk) mbar_arrive_expect_tx(x_full, kXBytes);
+        __syncwarp();  // every lane's reads of X precede the signal
+        if (lane == 0) mbar_arrive_remote_relaxed(x_free_peer);
       }
       // validity of the block's rows (published before the stage completed)
-      good = good && __all_sync(0xffffffffu, mbar_wait(&kv_full[sb], (j >> 1) & 1, a.err));
+      good = good && __all_sync(0xffffffffu, mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, a.err));
       float mraw = -INFINITY, mneg = INFINITY;
       if (good) {
         const uint32_t m32 = (uint32_t)(ring_mask[j] >> cb);
@@ -438,7 +459,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (good && lane == 0) mbar_arrive(p_full);
+      if (good && lane == 0) mbar_arrive(&p_full[sb]);
     }
     // epilogue: O / l for this half's 128 value dims.  tcgen05.ld is
     // warp-wide, so a warp with any valid head loads; only the stores test h < H.
