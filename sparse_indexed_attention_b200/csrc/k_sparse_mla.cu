@@ -472,56 +472,53 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
     if (!failed) {
       l += pair[(ep * 2 + (half ^ 1)) * 128 + h].x;
       tc_fence_after();
-      const bool store = h < a.H;
-      if (qw * 32 < a.H) {
-        const float m_nat = m_ref * kLn2;
-        if (a.splits == 1) {
-          const float inv = l > 0.f ? 1.f / l : 0.f;
-          const int64_t base = ((int64_t)t * a.H + h) * kDV + 256 * rank + 128 * half;
+      // O / l (or the raw partial) of this warp's 32 heads x 128 value dims,
+      // 32 dims at a time: TMEM -> registers (a row per lane) -> a swizzled
+      // 32 x 32 tile in shared memory -> rows back out, four rows of 128
+      // bytes per warp store instead of 32 scattered 16-byte pieces.  The
+      // tiles use the first row stage: every MMA that read it completed
+      // before the last PV, which this warp has seen complete.
+      float* tile = reinterpret_cast<float*>(smem + OFF_KV) + sw * 1024;
+      const float m_nat = m_ref * kLn2;
+      const bool partial = a.splits > 1;
+      const float inv = partial ? 1.f : (l > 0.f ? 1.f / l : 0.f);
+      const int rsub = lane >> 3, k4 = lane & 7;  // read-back: row 4i + rsub, dims 4 k4 .. 4 k4 + 3
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_lane + 128 * half + 32 * c, o);
-            tmem_ld_wait();
-            if (!store) continue;
-            if (a.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base + 32 * c);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_lane + 128 * half + 32 * c, o);
+        tmem_ld_wait();
+        __syncwarp();  // the previous chunk's tile has been read back
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                                     __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base + 32 * c);
+        for (int k = 0; k < 8; ++k)  // 16-byte piece k of row `lane`, XOR-swizzled by the row
+          *reinterpret_cast<float4*>(tile + lane * 32 + ((k ^ (lane & 7)) << 2)) =
+              make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
+                          __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
+        __syncwarp();
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                uint32_t w[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(o[8 * i + 2 * k]) * inv,
-                                                                  __uint_as_float(o[8 * i + 2 * k + 1]) * inv);
-                  w[k] = *reinterpret_cast<const uint32_t*>(&v2);
-                }
-                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
-              }
-            }
+        for (int i = 0; i < 8; ++i) {
+          const int r = 4 * i + rsub;  // head qw*32 + r
+          const float4 v4 = *reinterpret_cast<const float4*>(tile + r * 32 + ((k4 ^ (r & 7)) << 2));
+          const int hr = qw * 32 + r;
+          if (hr >= a.H) continue;
+          const int dim = 256 * rank + 128 * half + 32 * c + 4 * k4;
+          if (partial) {
+            const int64_t prow = ((int64_t)t * a.splits + sp) * a.H + hr;
+            *reinterpret_cast<float4*>(a.part_o + prow * kDV + dim) = v4;
+          } else if (a.out_f32) {
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + ((int64_t)t * a.H + hr) * kDV + dim) = v4;
+          } else {
+            const __nv_bfloat162 p0 = __floats2bfloat162_rn(v4.x, v4.y), p1 = __floats2bfloat162_rn(v4.z, v4.w);
+            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)t * a.H + hr) * kDV + dim) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1));
           }
-          if (store && rank == 0 && half == 0 && a.lse) a.lse[(int64_t)t * a.H + h] = m_nat + logf(l);
-        } else {
-          const int64_t prow = ((int64_t)t * a.splits + sp) * a.H + h;
-          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * kDV + 256 * rank + 128 * half);
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_lane + 128 * half + 32 * c, o);
-            tmem_ld_wait();
-            if (!store) continue;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[8 * c + i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                           __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
-          }
-          if (store && rank == 0 && half == 0) a.part_ml[prow] = make_float2(m_nat, l);
         }
+      }
+      if (h < a.H && rank == 0 && half == 0) {
+        if (partial)
+          a.part_ml[((int64_t)t * a.splits + sp) * a.H + h] = make_float2(m_nat, l);
+        else if (a.lse)
+          a.lse[(int64_t)t * a.H + h] = m_nat + logf(l);
       }
     } else {
       *abort_flag = 1;
