@@ -241,7 +241,7 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const voi
   TokenMap tm{plan.tok_seq, plan.tok_pos};
   timer_begin(st);
   DSA_CUDA(launch_plan(sd, 1, 0, plan, err, st));  // token geometry only
-  DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
+  DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/false, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
                              out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
   return DSA_OK;
@@ -274,7 +274,7 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const f
   DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, hist, zero,
                       fuse_hist ? topk_zero_words(T) : 0, err, st));
   DSA_CUDA(launch_topk(scores, L.ld, T, nullptr, tm.pos, K, idx, at<void>(ws, L.topk), hist != nullptr, err, st));
-  DSA_CUDA(launch_sparse_mla(sd, tm, reinterpret_cast<const __nv_bfloat16*>(q),
+  DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/true, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
                              out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
   return DSA_OK;

@@ -183,7 +183,8 @@ uint32_t* topk_hist_in_scratch(void* scratch, int T);
 cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, const int32_t* tok_pos,
                         int K, int32_t* idx, void* scratch, bool hist_ready, uint32_t* err, cudaStream_t st);
 size_t sparse_mla_partials_bytes(int T, int K, int H);
-cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16* q, const __nv_bfloat16* kv,
+cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, const __nv_bfloat16* q,
+                              const __nv_bfloat16* kv,
                               const int32_t* idx, int K, int H, float scale, void* out, bool out_f32,
                               float* lse, void* partials, uint32_t* err, cudaStream_t st);
 

@@ -98,6 +98,7 @@ struct AttnArgs {
   const __nv_bfloat16* kv;  // latent pool [rows, 576]
   const int32_t* idx;
   int K, H, ks, splits;
+  bool tm_early;     // the token map was written two or more launches back
   float scale_log2;  // scale * log2(e)
   void* out;
   bool out_f32;
@@ -171,10 +172,15 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       tma_load_2d(smem + OFF_Q + at * kQLatBytes, &tq_lat, q_full, 256 * rank + 64 * at, t * a.H);
     tma_load_2d(smem + OFF_Q + 4 * kQLatBytes, &tq_rope, q_full, 512 + 32 * rank, t * a.H);
   }
-  pdl_wait();  // the token map and the index lists come from earlier kernels
+  // the token map can be read before the wait when it does not come from
+  // the kernel just before; the index lists always do
+  int pos = a.tm_early ? a.tm.pos[t] : 0, b = a.tm_early ? a.tm.seq[t] : 0;
+  pdl_wait();
   pdl_trigger();
-  const int pos = a.tm.pos[t];
-  const int b = a.tm.seq[t];
+  if (!a.tm_early) {
+    pos = a.tm.pos[t];
+    b = a.tm.seq[t];
+  }
   const int nblk = (pos >= 0 && kend > kbeg) ? (kend - kbeg + kBK - 1) / kBK : 0;
 
   if ((warp == 0 || warp == 2 || warp == 3) && nblk > 0) {
@@ -637,9 +643,9 @@ size_t sparse_mla_partials_bytes(int T, int K, int H) {
   return (size_t)T * splits * H * (kDV * sizeof(float) + sizeof(float2));
 }
 
-cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16* q, const __nv_bfloat16* kv,
-                              const int32_t* idx, int K, int H, float scale, void* out, bool out_f32,
-                              float* lse, void* partials, uint32_t* err, cudaStream_t st) {
+cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, const __nv_bfloat16* q,
+                              const __nv_bfloat16* kv, const int32_t* idx, int K, int H, float scale, void* out,
+                              bool out_f32, float* lse, void* partials, uint32_t* err, cudaStream_t st) {
   const int T = s.num_tokens;
   int splits = attn_splits(T, K);
   const int ks = keys_per_split(K, splits);
@@ -658,7 +664,7 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, const __nv_bfloat16
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  AttnArgs a{s, tm, kv, idx, K, H, ks, splits, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
+  AttnArgs a{s, tm, kv, idx, K, H, ks, splits, tm_early, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
   cudaError_t e = launch_pdl("sparse_mla", k_sparse_mla_tc, dim3(2 * T * splits), dim3(kThreads), (size_t)SMEM_BYTES, st, tq_lat, tq_rope,
                              a);
   if (e == cudaSuccess) e = counted(cudaGetLastError());

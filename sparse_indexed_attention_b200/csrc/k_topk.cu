@@ -452,10 +452,12 @@ k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw);
   for (int i = threadIdx.x; i < kD2Bins; i += blockDim.x) sm.hist2[i] = 0;
+  const int t = blockIdx.y, c = blockIdx.x;
+  // row lengths come from the caller or from the call's first kernel, never
+  // from the one just before: read them while it finishes
+  const int n = row_length(row_len, tok_pos, t, ld, nullptr);
   pdl_wait();
   pdl_trigger();
-  const int t = blockIdx.y, c = blockIdx.x;
-  const int n = row_length(row_len, tok_pos, t, ld, nullptr);
   int32_t* __restrict__ out = idx + (int64_t)t * K;
   if (n <= K) {  // every candidate is selected
     if (c == 0)
