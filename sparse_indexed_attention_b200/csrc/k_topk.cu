@@ -47,6 +47,13 @@ constexpr int kPerThread = 8;             // consecutive scores per thread per p
 
 __device__ __forceinline__ uint32_t digit2(uint32_t key) { return (key >> 10) & (kD2Bins - 1); }
 
+// atomicAdd with acquire-release semantics at device scope (fence and add in one).
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Exclusive block-wide prefix sum of v (blockDim.x a multiple of 32, <= 1024);
 // *total receives the sum.  Each warp scans its own values; the warp totals
 // go through `buf` (32 words) and every warp reduces them itself -- two
@@ -79,15 +86,19 @@ __device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* buf, uint32
 // conflicts), a suffix scan over the lanes finds the lane holding the
 // crossing, and a second pass splits that lane's bins over the warp.  If no
 // bin qualifies (need 0 or above the total) the result is bin 0 with nothing
-// above it.  Ends with a barrier; `buf` is unused.
-__device__ __forceinline__ void find_bin(const uint32_t* hist, int bins, uint32_t need, uint32_t* buf,
-                                         uint32_t* out_bin, uint32_t* out_above) {
-  (void)buf;
+// above it.  Ends with a barrier.
+template <int BINS>
+__device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t need, uint32_t* out_bin, uint32_t* out_above) {
+  static_assert(BINS >= 256 && BINS <= 2048 && (BINS & (BINS - 1)) == 0, "bins");
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    const int per = bins >> 5;
+    constexpr int per = BINS >> 5;
+    uint32_t v[per];  // every load issued before the sums
+#pragma unroll
+    for (int j = 0; j < per; ++j) v[j] = hist[lane * per + ((j + lane) & (per - 1))];
     uint32_t sum = 0;
-    for (int j = 0; j < per; ++j) sum += hist[lane * per + ((j + lane) & (per - 1))];
+#pragma unroll
+    for (int j = 0; j < per; ++j) sum += v[j];
     uint32_t incl = sum;  // keys in this lane's bins and every higher lane's
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -103,12 +114,14 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int bins, uint32_
     } else {
       const int L = __ffs(who) - 1;
       const uint32_t above_l = __shfl_sync(0xffffffffu, incl - sum, L);
-      const int q = per >= 32 ? per >> 5 : 1;    // bins per lane in the second pass
+      constexpr int q = per >= 32 ? per >> 5 : 1;  // bins per lane in the second pass
       const int top = L * per + per - 1 - lane * q;  // this lane's bins: top, top-1, ..., top-q+1
       const bool mine = lane * q < per;
       uint32_t s2 = 0;
-      if (mine)
+      if (mine) {
+#pragma unroll
         for (int j = 0; j < q; ++j) s2 += hist[top - j];
+      }
       uint32_t inc2 = s2;  // from the top of L's range down to this lane's bins
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -118,6 +131,7 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int bins, uint32_
       const uint32_t ex = above_l + inc2 - s2;
       if (mine && s2 != 0 && ex < need && need <= ex + s2) {
         uint32_t above = ex;
+#pragma unroll
         for (int j = 0; j < q; ++j) {
           const uint32_t c = hist[top - j];
           if (above + c >= need) {
@@ -187,15 +201,16 @@ __device__ __forceinline__ void emit_selected(int L, uint32_t tau, uint32_t r, i
   for (int base = 0; base < L; base += blockDim.x * 4) {
     const int i0 = base + threadIdx.x * 4;
     uint32_t gt = 0, eq = 0;
+    int2 e[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) e[j] = i0 + j < L ? get(i0 + j) : make_int2(0, 0);
     int32_t pos[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      pos[j] = 0;
+      pos[j] = e[j].x;
       if (i0 + j < L) {
-        const int2 e = get(i0 + j);
-        pos[j] = e.x;
-        gt |= (uint32_t)((uint32_t)e.y > tau) << j;
-        eq |= (uint32_t)((uint32_t)e.y == tau) << j;
+        gt |= (uint32_t)((uint32_t)e[j].y > tau) << j;
+        eq |= (uint32_t)((uint32_t)e[j].y == tau) << j;
       }
     }
     const TwoLists S = scan_two(gt, eq, run_gt, run_eq, buf);
@@ -225,24 +240,27 @@ __device__ __forceinline__ void emit_selected(int L, uint32_t tau, uint32_t r, i
 template <class Get>
 __device__ void resolve_row(Get get, int L, uint32_t b1, uint32_t need, int K, uint32_t* hist, uint32_t* buf,
                             uint32_t* s_bin, uint32_t* s_above, int32_t* out) {
-  find_bin(hist, kD2Bins, need, buf, s_bin, s_above);
+  find_bin<kD2Bins>(hist, need, s_bin, s_above);
   const uint32_t pre22 = (b1 << 11) | *s_bin;
   need -= *s_above;
   __syncthreads();  // every thread has read the result before the histogram is reused
   for (int i = threadIdx.x; i < kD3Bins; i += blockDim.x) hist[i] = 0u;
   __syncthreads();
-  for (int base = 0; base < L; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    uint32_t key = 0;
-    bool act = false;
-    if (i < L) {
-      key = (uint32_t)get(i).y;
-      act = (key >> 10) == pre22;
+  for (int base = 0; base < L; base += 4 * blockDim.x) {
+    uint32_t key[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {  // loads first, then the (rarely active) adds
+      const int i = base + u * blockDim.x + threadIdx.x;
+      key[u] = i < L ? (uint32_t)get(i).y : 0u;
     }
-    hist_add(hist, key & (kD3Bins - 1), act);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * blockDim.x + threadIdx.x;
+      hist_add(hist, key[u] & (kD3Bins - 1), i < L && (key[u] >> 10) == pre22);
+    }
   }
   __syncthreads();
-  find_bin(hist, kD3Bins, need, buf, s_bin, s_above);
+  find_bin<kD3Bins>(hist, need, s_bin, s_above);
   const uint32_t tau = (pre22 << 10) | *s_bin;
   const uint32_t r = need - *s_above;
   emit_selected(L, tau, r, K, get, out, buf);
@@ -268,7 +286,7 @@ __device__ void topk_row_full_radix(const float* __restrict__ row, int n, int K,
       hist_add(hist, (key >> shift) & 0xFFu, act);
     }
     __syncthreads();
-    find_bin(hist, 256, need, buf, s_bin, s_above);
+    find_bin<256>(hist, need, s_bin, s_above);
     prefix |= *s_bin << shift;
     mask |= 0xFFu << shift;
     need -= *s_above;
@@ -315,7 +333,7 @@ k_topk_row(const float* __restrict__ scores, int64_t ld, const int32_t* __restri
     for (int j = 0; j < kPerThread; ++j) hist_add(sm.hist, keys[j] >> kLowBits, (have >> j) & 1u);
   }
   __syncthreads();
-  find_bin(sm.hist, kHistBins, (uint32_t)K, sm.buf, &sm.bin, &sm.above);
+  find_bin<kHistBins>(sm.hist, (uint32_t)K, &sm.bin, &sm.above);
   const uint32_t b1 = sm.bin, above = sm.above;
   const uint32_t L = above + sm.hist[b1];
   if (L > (uint32_t)kRowStage) {  // degenerate distribution: exact radix over the whole row
@@ -474,7 +492,7 @@ k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t
   uint32_t have = load_keys8(row, b0 + threadIdx.x * kPerThread, b1, vec, keys);
   cp_async_wait_all();
   __syncthreads();
-  find_bin(sm.hist, kHistBins, (uint32_t)K, sm.buf, &sm.bin, &sm.above);
+  find_bin<kHistBins>(sm.hist, (uint32_t)K, &sm.bin, &sm.above);
   const uint32_t bstar = sm.bin, above = sm.above;
   int2* my_kept = kept + ((int64_t)t * C + c) * chunk;
   uint32_t run = 0;
@@ -498,15 +516,12 @@ k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t
   for (int i = threadIdx.x; i < kD2Bins; i += blockDim.x)
     if (sm.hist2[i]) atomicAdd(&ghist2[(int64_t)t * kD2Bins + i], sm.hist2[i]);
   // The barrier orders every thread's pairs and histogram adds before thread
-  // 0's device-scope fence and count; the row's last CTA fences after seeing
-  // the count, before its barrier -- a release / acquire pair through row_done.
+  // 0's count, an acquire-release atomic at device scope: it publishes this
+  // CTA's lists and, in the row's last CTA, acquires every other CTA's.
   __syncthreads();
   if (threadIdx.x == 0) {
     counts[(int64_t)t * C + c] = (int)run;
-    __threadfence();
-    const bool last = atomicAdd(&row_done[t], 1) == C - 1;
-    if (last) __threadfence();
-    sm.last = last;
+    sm.last = atom_add_acq_rel_gpu(&row_done[t], 1) == C - 1;
   }
   __syncthreads();
   if (!sm.last) return;
