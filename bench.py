@@ -41,7 +41,7 @@ L2_FLUSH_BYTES = 256 << 20
 # hash to what was captured: any edit turns the figure back into null.
 NCU_TRAFFIC = {
     "index_scores": (143.71e6, ("k_indexer.cu",), "032c38f69f0b5616"),
-    "topk_filter_select": (4.41e6, ("k_topk.cu",), "c122968935f163f0"),
+    "topk_filter": (4.41e6, ("k_topk.cu",), "c122968935f163f0"),
     "sparse_mla": (20.25e6, ("k_sparse_mla.cu",), "60cb7ea372510e1a"),
 }
 CSRC = os.path.join(ROOT, "sparse_indexed_attention_b200", "csrc")
@@ -403,7 +403,7 @@ def run_ours(args, world, rank, local):
     ms_idx = statistics.mean(t_idx)
     score_bytes = n_keys * 4 + T * K * 4                          # Top-K: score rows read, indices written
     roofs = {}
-    for name, nbytes in (("index_scores", idx_bytes), ("topk_filter_select", score_bytes),
+    for name, nbytes in (("index_scores", idx_bytes), ("topk_filter", score_bytes),
                          ("sparse_mla", attn_bytes)):
         if name in kern:
             roofs[name] = roofline_entry(name, kern, nbytes, peak, peak_kind, spec.name)

@@ -175,6 +175,13 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   // the token map can be read before the wait when it does not come from
   // the kernel just before; the index lists always do
   int pos = a.tm_early ? a.tm.pos[t] : 0, b = a.tm_early ? a.tm.seq[t] : 0;
+  if (a.tm_early && warp == 0 && pos >= 0) {
+    // the sequence's page-table row into L2 while the previous kernel ends:
+    // the loaders look selected pages up in it right after the wait
+    const int64_t row_bytes = (int64_t)a.s.max_pages * 4;
+    const char* pt = reinterpret_cast<const char*>(a.s.page_table + (int64_t)b * a.s.max_pages);
+    for (int64_t off = (int64_t)lane * 128; off < row_bytes; off += 32 * 128) prefetch_l2(pt + off);
+  }
   pdl_wait();
   pdl_trigger();
   if (!a.tm_early) {

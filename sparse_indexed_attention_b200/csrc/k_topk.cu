@@ -19,9 +19,10 @@
 //      (the lowest positions);
 //   4. one ordered pass over the kept pairs emits every key > tau and the
 //      first r keys == tau, already in position order.
-// Rows much longer than the number of rows get several CTAs per row (steps 1
-// and 2 split over chunks of the row, the CTA that finishes a row's last
-// chunk does 3 and 4); otherwise one CTA does a row.  A degenerate row that
+// Rows much longer than the number of rows get several CTAs per row: steps 1
+// and 2 run over chunks of the row in one kernel, and in a second kernel
+// every CTA of the row resolves steps 3 and 4 from the row's kept pairs and
+// writes the selections of its own chunk.  Otherwise one CTA does a row.  A degenerate row that
 // keeps more pairs than shared memory holds is resolved from global memory
 // (several CTAs per row) or by four 8-bit radix passes over the row (one CTA).
 #include "sm100.cuh"
@@ -47,12 +48,6 @@ constexpr int kPerThread = 8;             // consecutive scores per thread per p
 
 __device__ __forceinline__ uint32_t digit2(uint32_t key) { return (key >> 10) & (kD2Bins - 1); }
 
-// atomicAdd with acquire-release semantics at device scope (fence and add in one).
-__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
-  int old;
-  asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
 
 // Exclusive block-wide prefix sum of v (blockDim.x a multiple of 32, <= 1024);
 // *total receives the sum.  Each warp scans its own values; the warp totals
@@ -369,9 +364,9 @@ k_topk_row(const float* __restrict__ scores, int64_t ld, const int32_t* __restri
 }
 
 // ---------------------------------------------------------------- several CTAs per row
-// Scratch per call: a zeroed region -- row_done [T] (padded to 16 words), the
-// digit-1 histogram [T][2048], the digit-2 histogram [T][2048] -- then
-// counts [T][C] (pairs kept per chunk) and the kept pairs [T][C][chunk].
+// Several CTAs per row: k_topk_hist (unless the indexer built the digit-1
+// histogram), k_topk_filter, k_topk_emit; their scratch is laid out by
+// launch_topk below.
 
 __global__ void __launch_bounds__(kChunkThreads)
 k_topk_hist(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
@@ -398,77 +393,23 @@ k_topk_hist(const float* __restrict__ scores, int64_t ld, const int32_t* __restr
     if (hist[i]) atomicAdd(&ghist[(int64_t)t * kHistBins + i], hist[i]);
 }
 
-struct SelSmem {
+struct FiltSmem {
   uint32_t hist[kHistBins];
   uint32_t hist2[kD2Bins];
   uint32_t buf[33];
   uint32_t bin, above;
-  int off[kMaxChunks + 1];
-  int last;
-  int2 kept[kSelStage];
 };
 
-// Steps 3 and 4 for row t once every chunk of it is filtered.  The chunks'
-// pairs and histograms were written by other CTAs of this grid: read through
-// L2 (__ldcg).
-__device__ void select_row(int t, int K, int chunk, int C, uint32_t b1, uint32_t above,
-                           const uint32_t* __restrict__ ghist2, const int* __restrict__ counts,
-                           const int2* __restrict__ kept, int32_t* __restrict__ out, SelSmem& sm) {
-  // asynchronous copies: the whole histogram is one round trip, not a chain
-  for (int i = 4 * threadIdx.x; i < kD2Bins; i += 4 * blockDim.x)
-    cp_async_16(&sm.hist2[i], ghist2 + (int64_t)t * kD2Bins + i);
-  if (threadIdx.x < 32) {  // chunk counts -> offsets (two chunks per lane)
-    const int lane = threadIdx.x;
-    const int a0 = 2 * lane < C ? __ldcg(counts + (int64_t)t * C + 2 * lane) : 0;
-    const int a1 = 2 * lane + 1 < C ? __ldcg(counts + (int64_t)t * C + 2 * lane + 1) : 0;
-    int incl = a0 + a1;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += u;
-    }
-    sm.off[2 * lane] = incl - a0 - a1;
-    sm.off[2 * lane + 1] = incl - a1;
-    if (lane == 31) sm.off[kMaxChunks] = incl;
-  }
-  __syncthreads();
-  const int L = sm.off[C];  // offsets past C hold the same total
-  const int2* row_kept = kept + (int64_t)t * C * chunk;
-  if (L <= kSelStage) {
-    // each warp copies whole chunks, every copy in flight at once
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int c = warp; c < C; c += nw) {
-      const int o = sm.off[c], cnt = sm.off[c + 1] - o;
-      for (int i = lane; i < cnt; i += 32) cp_async_8(&sm.kept[o + i], row_kept + (int64_t)c * chunk + i);
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    resolve_row([&](int i) { return sm.kept[i]; }, L, b1, (uint32_t)K - above, K, sm.hist2, sm.buf, &sm.bin,
-                &sm.above, out);
-  } else {  // degenerate row: read the pairs where the chunks left them
-    cp_async_wait_all();  // the histogram
-    __syncthreads();
-    auto get = [&](int i) -> int2 {
-      int lo = 0, hi = C - 1;  // last chunk whose offset <= i
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (sm.off[mid] <= i) lo = mid; else hi = mid - 1;
-      }
-      return __ldcg(row_kept + (int64_t)lo * chunk + (i - sm.off[lo]));
-    };
-    resolve_row(get, L, b1, (uint32_t)K - above, K, sm.hist2, sm.buf, &sm.bin, &sm.above, out);
-  }
-}
-
-// Steps 1-2 on chunk c of row t (digit-1 histogram already complete); the
-// CTA that finishes the row's last chunk then selects the row.
+// Steps 1-2 on chunk c of row t (digit-1 histogram already complete): the
+// chunk's kept pairs, its share of the digit-2 histogram and its count;
+// chunk 0 also records the row's b1 and the count of keys above it.
 __global__ void __launch_bounds__(kChunkThreads)
-k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
-                     const int32_t* __restrict__ tok_pos, int K, int chunk, int C, const uint32_t* __restrict__ ghist,
-                     uint32_t* __restrict__ ghist2, int* __restrict__ counts, int2* __restrict__ kept,
-                     int* __restrict__ row_done, int32_t* __restrict__ idx) {
+k_topk_filter(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ row_len,
+              const int32_t* __restrict__ tok_pos, int K, int chunk, int C, const uint32_t* __restrict__ ghist,
+              uint32_t* __restrict__ ghist2, int* __restrict__ counts, int2* __restrict__ kept,
+              int2* __restrict__ row_info, int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw);
+  FiltSmem& sm = *reinterpret_cast<FiltSmem*>(smem_raw);
   for (int i = threadIdx.x; i < kD2Bins; i += blockDim.x) sm.hist2[i] = 0;
   const int t = blockIdx.y, c = blockIdx.x;
   // row lengths come from the caller or from the call's first kernel, never
@@ -476,8 +417,8 @@ k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t
   const int n = row_length(row_len, tok_pos, t, ld, nullptr);
   pdl_wait();
   pdl_trigger();
-  int32_t* __restrict__ out = idx + (int64_t)t * K;
   if (n <= K) {  // every candidate is selected
+    int32_t* __restrict__ out = idx + (int64_t)t * K;
     if (c == 0)
       for (int i = threadIdx.x; i < K; i += blockDim.x) out[i] = i < n ? i : -1;
     return;
@@ -515,17 +456,132 @@ k_topk_filter_select(const float* __restrict__ scores, int64_t ld, const int32_t
   __syncthreads();
   for (int i = threadIdx.x; i < kD2Bins; i += blockDim.x)
     if (sm.hist2[i]) atomicAdd(&ghist2[(int64_t)t * kD2Bins + i], sm.hist2[i]);
-  // The barrier orders every thread's pairs and histogram adds before thread
-  // 0's count, an acquire-release atomic at device scope: it publishes this
-  // CTA's lists and, in the row's last CTA, acquires every other CTA's.
-  __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0) {  // the next kernel reads these after this grid has completed
     counts[(int64_t)t * C + c] = (int)run;
-    sm.last = atom_add_acq_rel_gpu(&row_done[t], 1) == C - 1;
+    if (c == 0) row_info[t] = make_int2((int)bstar, (int)above);
+  }
+}
+
+struct EmitSmem {
+  uint32_t hist[kD2Bins];  // digit 2, then digit 3
+  uint32_t buf[33];
+  uint32_t bin, above;
+  uint32_t before[2];      // earlier chunks' keys > tau and == tau
+  int2 info;
+  int off[kMaxChunks + 1];
+  int2 kept[kSelStage];
+};
+
+// Steps 3-4 for row t: every CTA of the row resolves tau and r from the whole
+// row's kept pairs (the same result in each), counts the earlier chunks'
+// selections, and writes the selected positions of its own chunk c.
+__global__ void __launch_bounds__(kChunkThreads)
+k_topk_emit(int64_t ld, const int32_t* __restrict__ row_len, const int32_t* __restrict__ tok_pos, int K, int chunk,
+            int C, const uint32_t* __restrict__ ghist2, const int* __restrict__ counts,
+            const int2* __restrict__ kept, const int2* __restrict__ row_info, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  EmitSmem& sm = *reinterpret_cast<EmitSmem*>(smem_raw);
+  const int t = blockIdx.y, c = blockIdx.x;
+  const int n = row_length(row_len, tok_pos, t, ld, nullptr);  // not written by the kernel just before
+  if (threadIdx.x < 2) sm.before[threadIdx.x] = 0u;
+  pdl_wait();
+  pdl_trigger();
+  if (n <= K) return;  // written by the filter
+  for (int i = 4 * threadIdx.x; i < kD2Bins; i += 4 * blockDim.x)
+    cp_async_16(&sm.hist[i], ghist2 + (int64_t)t * kD2Bins + i);
+  if (threadIdx.x < 32) {  // chunk counts -> offsets (two chunks per lane); the row's b1 / above
+    const int lane = threadIdx.x;
+    const int a0 = 2 * lane < C ? counts[(int64_t)t * C + 2 * lane] : 0;
+    const int a1 = 2 * lane + 1 < C ? counts[(int64_t)t * C + 2 * lane + 1] : 0;
+    int incl = a0 + a1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    sm.off[2 * lane] = incl - a0 - a1;
+    sm.off[2 * lane + 1] = incl - a1;
+    if (lane == 31) sm.off[kMaxChunks] = incl;
+    if (lane == 0) sm.info = row_info[t];
   }
   __syncthreads();
-  if (!sm.last) return;
-  select_row(t, K, chunk, C, bstar, above, ghist2, counts, kept, out, sm);
+  const int L = sm.off[C];  // offsets past C hold the same total
+  const uint32_t b1 = (uint32_t)sm.info.x;
+  uint32_t need = (uint32_t)K - (uint32_t)sm.info.y;
+  const int2* row_kept = kept + (int64_t)t * C * chunk;
+  const bool staged = L <= kSelStage;
+  if (staged) {  // each warp copies whole chunks, every copy in flight at once
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int cc = warp; cc < C; cc += nw) {
+      const int o = sm.off[cc], cnt = sm.off[cc + 1] - o;
+      for (int i = lane; i < cnt; i += 32) cp_async_8(&sm.kept[o + i], row_kept + (int64_t)cc * chunk + i);
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  auto get = [&](int i) -> int2 {
+    if (staged) return sm.kept[i];
+    int lo = 0, hi = C - 1;  // degenerate row: last chunk whose offset <= i, read where it was left
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sm.off[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    return __ldcg(row_kept + (int64_t)lo * chunk + (i - sm.off[lo]));
+  };
+  // tau (the K-th largest key) and r (how many tau-valued keys are taken)
+  find_bin<kD2Bins>(sm.hist, need, &sm.bin, &sm.above);
+  const uint32_t pre22 = (b1 << 11) | sm.bin;
+  need -= sm.above;
+  __syncthreads();  // every thread has read the result before the histogram is reused
+  for (int i = threadIdx.x; i < kD3Bins; i += blockDim.x) sm.hist[i] = 0u;
+  __syncthreads();
+  for (int base = 0; base < L; base += 4 * blockDim.x) {
+    uint32_t key[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {  // loads first, then the (rarely active) adds
+      const int i = base + u * blockDim.x + threadIdx.x;
+      key[u] = i < L ? (uint32_t)get(i).y : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * blockDim.x + threadIdx.x;
+      hist_add(sm.hist, key[u] & (kD3Bins - 1), i < L && (key[u] >> 10) == pre22);
+    }
+  }
+  __syncthreads();
+  find_bin<kD3Bins>(sm.hist, need, &sm.bin, &sm.above);
+  const uint32_t tau = (pre22 << 10) | sm.bin;
+  const uint32_t r = need - sm.above;
+  // selections of the earlier chunks: pairs [0, off[c])
+  const int o0 = sm.off[c], o1 = sm.off[c + 1];
+  uint32_t gt = 0, eq = 0;
+  for (int base = 0; base < o0; base += 4 * blockDim.x) {
+    uint32_t key[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * blockDim.x + threadIdx.x;
+      key[u] = i < o0 ? (uint32_t)get(i).y : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * blockDim.x + threadIdx.x;
+      gt += (i < o0 && key[u] > tau) ? 1u : 0u;
+      eq += (i < o0 && key[u] == tau) ? 1u : 0u;
+    }
+  }
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  eq = __reduce_add_sync(0xffffffffu, eq);
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&sm.before[0], gt);
+    atomicAdd(&sm.before[1], eq);
+  }
+  __syncthreads();
+  const uint32_t eq_before = sm.before[1];
+  const uint32_t taken_before = sm.before[0] + min(eq_before, r);
+  const uint32_t r_left = r - min(eq_before, r);  // ties still to take, lowest positions first
+  int32_t* __restrict__ out = idx + (int64_t)t * K + taken_before;
+  emit_selected(
+      o1 - o0, tau, r_left, K - (int)taken_before, [&](int i) { return get(o0 + i); }, out, sm.buf);
 }
 
 // Chunking of a row: several CTAs per row only when there are few rows.
@@ -559,10 +615,10 @@ int64_t pad16(int64_t x) { return (x + 15) / 16 * 16; }
 }  // namespace
 
 // Scratch layout (several CTAs per row): a region zeroed on every call --
-// row_done [T] (padded to 16 words), the digit-1 histogram [T][2048] and the
-// digit-2 histogram [T][2048] -- then counts [T][C] (padded to 16 words) and
-// the kept pairs [T][C][chunk].
-int64_t topk_zero_words(int T) { return pad16(T) + (int64_t)T * (kHistBins + kD2Bins); }
+// the per-row {b1, keys above b1} [T] (padded to 16 words), the digit-1
+// histogram [T][2048] and the digit-2 histogram [T][2048] -- then counts
+// [T][C] (padded to 16 words) and the kept pairs [T][C][chunk].
+int64_t topk_zero_words(int T) { return pad16(2 * (int64_t)T) + (int64_t)T * (kHistBins + kD2Bins); }
 
 size_t topk_scratch_bytes(int T, int64_t ld, int K) {
   (void)K;
@@ -572,7 +628,9 @@ size_t topk_scratch_bytes(int T, int64_t ld, int K) {
   return (size_t)topk_zero_words(T) * 4 + (size_t)pad16((int64_t)T * C) * 4 + (size_t)T * C * chunk * sizeof(int2);
 }
 
-uint32_t* topk_hist_in_scratch(void* scratch, int T) { return reinterpret_cast<uint32_t*>(scratch) + pad16(T); }
+uint32_t* topk_hist_in_scratch(void* scratch, int T) {
+  return reinterpret_cast<uint32_t*>(scratch) + pad16(2 * (int64_t)T);
+}
 
 bool topk_uses_hist(int T, int64_t ld) {
   int C, chunk;
@@ -588,12 +646,12 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* r
     static thread_local int dev_row = -1;
     cudaError_t e = set_smem_once(k_topk_row, (int)sizeof(RowSmem), &dev_row);
     if (e != cudaSuccess) return e;
-    e = launch_pdl("topk_row", k_topk_row, dim3(T), dim3(kRowThreads), sizeof(RowSmem), st, scores, ld, row_len, tok_pos, K, idx,
-                   err);
+    e = launch_pdl("topk_row", k_topk_row, dim3(T), dim3(kRowThreads), sizeof(RowSmem), st, scores, ld, row_len,
+                   tok_pos, K, idx, err);
     if (e != cudaSuccess) return e;
     return counted(cudaGetLastError());
   }
-  int* row_done = reinterpret_cast<int*>(scratch);
+  int2* row_info = reinterpret_cast<int2*>(scratch);
   uint32_t* ghist = topk_hist_in_scratch(scratch, T);
   uint32_t* ghist2 = ghist + (int64_t)T * kHistBins;
   char* p = reinterpret_cast<char*>(scratch) + topk_zero_words(T) * 4;
@@ -604,13 +662,19 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* r
   const dim3 grid(C, T);
   if (!hist_ready) {  // otherwise the caller has zeroed the region and filled the histogram
     if ((e = cudaMemsetAsync(scratch, 0, (size_t)topk_zero_words(T) * 4, st)) != cudaSuccess) return e;
-    e = launch_pdl("topk_hist", k_topk_hist, grid, dim3(kChunkThreads), 0, st, scores, ld, row_len, tok_pos, K, chunk, ghist, err);
+    e = launch_pdl("topk_hist", k_topk_hist, grid, dim3(kChunkThreads), 0, st, scores, ld, row_len, tok_pos, K, chunk,
+                   ghist, err);
     if (e != cudaSuccess || (e = counted(cudaGetLastError())) != cudaSuccess) return e;
   }
-  static thread_local int dev_fs = -1;
-  if ((e = set_smem_once(k_topk_filter_select, (int)sizeof(SelSmem), &dev_fs)) != cudaSuccess) return e;
-  e = launch_pdl("topk_filter_select", k_topk_filter_select, grid, dim3(kChunkThreads), sizeof(SelSmem), st, scores, ld, row_len, tok_pos, K,
-                 chunk, C, (const uint32_t*)ghist, ghist2, counts, kept, row_done, idx);
+  static thread_local int dev_f = -1, dev_e = -1;
+  if ((e = set_smem_once(k_topk_filter, (int)sizeof(FiltSmem), &dev_f)) != cudaSuccess) return e;
+  if ((e = set_smem_once(k_topk_emit, (int)sizeof(EmitSmem), &dev_e)) != cudaSuccess) return e;
+  e = launch_pdl("topk_filter", k_topk_filter, grid, dim3(kChunkThreads), sizeof(FiltSmem), st, scores, ld, row_len,
+                 tok_pos, K, chunk, C, (const uint32_t*)ghist, ghist2, counts, kept, row_info, idx);
+  if (e != cudaSuccess || (e = counted(cudaGetLastError())) != cudaSuccess) return e;
+  e = launch_pdl("topk_emit", k_topk_emit, grid, dim3(kChunkThreads), sizeof(EmitSmem), st, ld, row_len, tok_pos, K,
+                 chunk, C, (const uint32_t*)ghist2, (const int*)counts, (const int2*)kept, (const int2*)row_info,
+                 idx);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }
