@@ -40,9 +40,9 @@ L2_FLUSH_BYTES = 256 << 20
 # (profiles/<kernel>_decode_b8_128k.md), valid only while the kernel's sources
 # hash to what was captured: any edit turns the figure back into null.
 NCU_TRAFFIC = {
-    "index_scores": (143.71e6, ("k_indexer.cu",), "032c38f69f0b5616"),
-    "topk_filter": (4.41e6, ("k_topk.cu",), "c122968935f163f0"),
-    "sparse_mla": (20.25e6, ("k_sparse_mla.cu",), "60cb7ea372510e1a"),
+    "index_scores": (144.11e6, ("k_indexer.cu",), "829dc8b4b29fce72"),
+    "topk_filter": (4.35e6, ("k_topk.cu",), "0b824ddb18426cbe"),
+    "sparse_mla": (20.26e6, ("k_sparse_mla.cu",), "91addb36848b10fd"),
 }
 CSRC = os.path.join(ROOT, "sparse_indexed_attention_b200", "csrc")
 
