@@ -70,6 +70,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage-reps", type=int, default=20)
+    ap.add_argument("--all-configs", action="store_true",
+                    help="one JSON line per workload: fused-call time and the binding roofline of each stage")
     ap.add_argument("--only", choices=["index_scores", "topk", "sparse_mla", "fused"], default=None,
                     help="time one stage (or the fused call, eagerly) alone on the bench workload (profiling aid)")
     return ap.parse_args()
@@ -178,6 +180,17 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def tensor_peak(kind: str):
+    """Measured dense TFLOP/s: bf16 (burst), fp8 = 2 x bf16 (nominal ratio)."""
+    try:
+        with open(PEAKS_FILE) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+        src = "measured"
+    except Exception:
+        bf16, src = 1590.0, "fallback"
+    return (2.0 * bf16 if kind == "fp8" else bf16), src
 
 
 def hbm_peak():
@@ -320,10 +333,88 @@ def run_only(args, dsa, wl, d, dev, stream, flush, world, fused=None):
                           "us_min": 1e3 * min(times), "launches": dsa.dsa_launches_in_last_call()}), flush=True)
 
 
+def run_all_configs(args, dsa, dev, stream, flush):
+    """Every workload once: the fused call (graph replay, L2 flushed before each
+    step) and per-kernel device times, each stage against its binding roofline."""
+    from sparse_indexed_attention_b200.workloads import to_device
+    hbm, hbm_src = hbm_peak()
+    for name in CONFIGS:
+        spec = CONFIGS[name]
+        wl = make_workload(spec)
+        d = to_device(wl)
+        T, H, K = wl.T, spec.heads, spec.topk
+        out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((T, H), dtype=torch.float32, device=dev)
+        ws = torch.zeros(dsa.dsa_workspace_size(dsa.DSA_OP_INDEX_TOPK_ATTN, d.seqs, K, H), dtype=torch.uint8,
+                         device=dev)
+
+        def step():
+            dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse,
+                                    ws=ws)
+
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        if dsa.dsa_check_error(ws) != dsa.DSA_OK:
+            raise RuntimeError(f"device error flag set on {name}")
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        steps = 5 if T > 4096 else 20
+        ms = statistics.mean(time_device(graph.replay, steps, 2, stream, flush))
+        del graph
+        kern = kernel_times(dsa, step, 3, stream, flush)
+        us = {k: 1e3 * statistics.mean(v) for k, v in kern.items()}
+        n = wl.token_pos() + 1
+        pairs = int(n.sum())
+        sel = int(np.minimum(n, K).sum())
+        decode = spec.mode == "decode"
+        stages = {}
+        if "index_scores" in us:
+            t_s = us["index_scores"] * 1e-6
+            if decode:
+                b = pairs * (132 if spec.ki_fp8 else 256)
+                stages["index_scores"] = {"bound": "hbm", "us": us["index_scores"], "achieved": b / t_s / 1e9,
+                                          "peak": hbm, "unit": "GB/s", "frac": b / t_s / 1e9 / hbm}
+            else:
+                pk, src = tensor_peak("fp8" if spec.ki_fp8 else "bf16")
+                f = pairs * 16384
+                stages["index_scores"] = {"bound": "tensor", "us": us["index_scores"], "achieved": f / t_s / 1e12,
+                                          "peak": pk, "unit": "TFLOP/s", "frac": f / t_s / 1e12 / pk,
+                                          "dtype": "fp8" if spec.ki_fp8 else "bf16"}
+        topk_us = sum(v for k, v in us.items() if k.startswith("topk"))
+        b = pairs * 4 + T * K * 4
+        stages["topk"] = {"bound": "latency", "us": topk_us, "hbm_frac_of_one_pass": b / (topk_us * 1e-6) / 1e9 / hbm}
+        attn_us = us.get("sparse_mla", 0.0) + us.get("sparse_mla_combine", 0.0)
+        if attn_us:
+            t_s = attn_us * 1e-6
+            if decode:
+                b = sel * 1152
+                stages["sparse_mla"] = {"bound": "hbm", "us": attn_us, "achieved": b / t_s / 1e9, "peak": hbm,
+                                        "unit": "GB/s", "frac": b / t_s / 1e9 / hbm}
+            else:
+                pk, src = tensor_peak("bf16")
+                f = sel * 2 * H * (576 + 512)
+                stages["sparse_mla"] = {"bound": "tensor", "us": attn_us, "achieved": f / t_s / 1e12, "peak": pk,
+                                        "unit": "TFLOP/s", "frac": f / t_s / 1e12 / pk}
+        line = {"config": name, "tokens": T, "us_per_call": ms * 1e3, "tokens_per_s": T / (ms / 1e3),
+                "launches": dsa.dsa_launches_in_last_call(), "kernels_us": us, "stages": stages,
+                "peak_source": hbm_src, "timing": "graph replay, 256 MiB L2 flush before each step; "
+                "kernels_us from events around each launch (serialised)"}
+        print(json.dumps(line), flush=True)
+        del d, ws, out, lse
+        torch.cuda.empty_cache()
+
+
 def run_ours(args, world, rank, local):
     import sparse_indexed_attention_b200 as dsa
     from sparse_indexed_attention_b200.workloads import to_device
 
+    if args.all_configs:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        run_all_configs(args, dsa, dev, torch.cuda.current_stream(dev),
+                        torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev))
+        return
     spec = CONFIGS[args.config]
     spec = rank_spec(spec, rank)                         # each rank serves its own batch
     wl = make_workload(spec)
