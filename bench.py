@@ -70,6 +70,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage-reps", type=int, default=20)
+    ap.add_argument("--ctx", type=int, default=0,
+                    help="override the workload's context length (profiling a smaller case of the same kernels)")
     ap.add_argument("--all-configs", action="store_true",
                     help="one JSON line per workload: fused-call time and the binding roofline of each stage")
     ap.add_argument("--only", choices=["index_scores", "topk", "sparse_mla", "fused"], default=None,
@@ -416,6 +418,8 @@ def run_ours(args, world, rank, local):
                         torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev))
         return
     spec = CONFIGS[args.config]
+    if args.ctx > 0:
+        spec = spec.scaled(ctx=(args.ctx, args.ctx))
     spec = rank_spec(spec, rank)                         # each rank serves its own batch
     wl = make_workload(spec)
     d = to_device(wl)
