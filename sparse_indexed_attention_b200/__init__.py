@@ -96,6 +96,71 @@ def _stream(device: torch.device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _need(t, name: str, dtypes, shape, device: torch.device, min_rows: int = 0):
+    """Refuse, before any C call, a tensor the kernels would misread: each must
+    be a contiguous tensor on `device` with one of `dtypes`, a shape matching
+    `shape` (None matches any size) and at least `min_rows` rows.  The kernels
+    take bare pointers, so a wrong dtype, a strided view or a short pool would
+    otherwise be read out of bounds."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {[str(d) for d in dtypes]}")
+    if t.dim() != len(shape) or any(w is not None and w != g for g, w in zip(t.shape, shape)):
+        want = "[" + ", ".join("*" if w is None else str(w) for w in shape) + "]"
+        raise ValueError(f"{name}: shape {list(t.shape)}, expected {want}")
+    if t.shape[0] < min_rows:
+        raise ValueError(f"{name}: {t.shape[0]} rows, the page pool needs at least {min_rows}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _cuda_device(t, name: str) -> torch.device:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise TypeError(f"{name}: expected a CUDA tensor")
+    return t.device
+
+
+_I32T, _F32T, _BF16T = (torch.int32,), (torch.float32,), (torch.bfloat16,)
+_FP8T = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _need_seqs(seqs: "Seqs", dev: torch.device):
+    _need(seqs.q_seq_start, "seqs.q_seq_start", _I32T, (seqs.batch + 1,), dev)
+    _need(seqs.ctx_len, "seqs.ctx_len", _I32T, (None,), dev)
+    _need(seqs.page_table, "seqs.page_table", _I32T, (seqs.batch, None), dev)
+
+
+def _need_ws(ws, dev: torch.device):
+    _need(ws, "ws", (torch.uint8,), (None,), dev)
+
+
+def _need_index_inputs(seqs: "Seqs", qI, w, kI, kI_scale) -> torch.device:
+    dev = _cuda_device(qI, "qI")
+    T, rows = seqs.num_q_tokens, seqs.num_phys_pages * 64
+    _need_seqs(seqs, dev)
+    _need(qI, "qI", _BF16T, (T, 64, 128), dev)
+    _need(w, "w", _F32T, (T, 64), dev)
+    _need(kI, "kI", _FP8T if kI_scale is not None else _BF16T, (None, 128), dev, rows)
+    if kI_scale is not None:
+        _need(kI_scale, "kI_scale", _F32T, (None,), dev, rows)
+    return dev
+
+
+def _need_attn_inputs(seqs: "Seqs", q, kv, out, lse) -> torch.device:
+    dev = _cuda_device(q, "q")
+    _need_seqs(seqs, dev)
+    _need(q, "q", _BF16T, (seqs.num_q_tokens, None, 576), dev)
+    T, H = q.shape[0], q.shape[1]
+    _need(kv, "kv", _BF16T, (None, 576), dev, seqs.num_phys_pages * 64)
+    _need(out, "out", (torch.bfloat16, torch.float32), (T, H, 512), dev)
+    if lse is not None:
+        _need(lse, "lse", _F32T, (T, H), dev)
+    return dev
+
+
 # ---------------------------------------------------------------------------
 # Batch geometry
 # ---------------------------------------------------------------------------
@@ -157,34 +222,55 @@ def workspace(nbytes: int, device, key=None) -> torch.Tensor:
 
 
 def dsa_quantize_index_query(qI: torch.Tensor, w: torch.Tensor, codes=None, w_scaled=None):
+    dev = _cuda_device(qI, "qI")
     T = qI.shape[0]
     codes = codes if codes is not None else torch.empty((T, 64, 128), dtype=torch.uint8, device=qI.device)
     w_scaled = w_scaled if w_scaled is not None else torch.empty((T, 64), dtype=torch.float32, device=qI.device)
+    _need(qI, "qI", _BF16T, (T, 64, 128), dev)
+    _need(w, "w", _F32T, (T, 64), dev)
+    _need(codes, "codes", _FP8T, (T, 64, 128), dev)
+    _need(w_scaled, "w_scaled", _F32T, (T, 64), dev)
     _check(_lib.dsa_quantize_index_query(_ptr(qI), _ptr(w), T, _ptr(codes), _ptr(w_scaled), _stream(qI.device)),
            "dsa_quantize_index_query")
     return codes, w_scaled
 
 
 def dsa_index_scores(seqs: Seqs, qI, w, kI, kI_scale=None, scores=None, ld=None, ws=None):
+    """Scores into `scores` [T, ld] fp32 (allocated zeroed when None).  When
+    `scores` is given, ld defaults to its row stride and must equal it."""
+    dev = _need_index_inputs(seqs, qI, w, kI, kI_scale)
     T = seqs.num_q_tokens
-    ld = ld or (seqs.max_ctx + 3) // 4 * 4
     if scores is None:
+        ld = ld or (seqs.max_ctx + 3) // 4 * 4
         scores = torch.zeros((T, ld), dtype=torch.float32, device=qI.device)
+    else:
+        _need(scores, "scores", _F32T, (T, None), dev)
+        if ld is not None and ld != scores.stride(0):
+            raise ValueError(f"ld={ld} differs from the row stride {scores.stride(0)} of scores")
+        ld = scores.stride(0)
     ki_dtype = DSA_KI_FP8_E4M3 if kI_scale is not None else DSA_KI_BF16
     c = seqs.c()
     need = _lib.dsa_workspace_size(DSA_OP_INDEX_SCORES, ctypes.byref(c), 1, 16)
     ws = ws if ws is not None else workspace(need, qI.device, "index_scores")
+    _need_ws(ws, dev)
     _check(_lib.dsa_index_scores(ctypes.byref(c), _ptr(qI), _ptr(w), _ptr(kI), _ptr(kI_scale), ki_dtype, _ptr(scores),
                                  ld, _ptr(ws), ws.numel(), _stream(qI.device)), "dsa_index_scores")
     return scores
 
 
 def dsa_topk(scores: torch.Tensor, row_len: torch.Tensor, K: int, idx=None, ws=None):
+    """Top-K of each fp32 row of `scores` [T, ld] (contiguous) over its first
+    row_len[t] entries, into idx [T, K] int32."""
+    dev = _cuda_device(scores, "scores")
+    _need(scores, "scores", _F32T, (None, None), dev)
     T, ld = scores.shape
     idx = idx if idx is not None else torch.empty((T, K), dtype=torch.int32, device=scores.device)
+    _need(row_len, "row_len", _I32T, (T,), dev)
+    _need(idx, "idx", _I32T, (T, K), dev)
     c = DsaSeqsC(1, T, 64, 1, 1, ld, None, None, None)
     need = _lib.dsa_workspace_size(DSA_OP_TOPK, ctypes.byref(c), K, 16)
     ws = ws if ws is not None else workspace(need, scores.device, "topk")
+    _need_ws(ws, dev)
     _check(_lib.dsa_topk(_ptr(scores), ld, T, _ptr(row_len), K, _ptr(idx), _ptr(ws), ws.numel(),
                          _stream(scores.device)), "dsa_topk")
     return idx
@@ -205,9 +291,12 @@ def dsa_sparse_mla_fwd(seqs: Seqs, q, kv, idx, scale: float, out=None, lse=None,
     out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    dev = _need_attn_inputs(seqs, q, kv, out, lse)
+    _need(idx, "idx", _I32T, (T, K), dev)
     c = seqs.c()
     need = _lib.dsa_workspace_size(DSA_OP_SPARSE_MLA, ctypes.byref(c), K, H)
     ws = ws if ws is not None else workspace(need, q.device, "sparse_mla")
+    _need_ws(ws, dev)
     _check(_lib.dsa_sparse_mla_fwd(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(idx), K, H, scale, _ptr(out),
                                    _out_dtype(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)),
            "dsa_sparse_mla_fwd")
@@ -224,6 +313,8 @@ def dsa_sparse_mla_fwd_noalloc(seqs: Seqs, q, kv, idx, scale: float, out=None, l
     out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    dev = _need_attn_inputs(seqs, q, kv, out, lse)
+    _need(idx, "idx", _I32T, (T, K), dev)
     c = seqs.c()
     _check(_lib.dsa_sparse_mla_fwd_noalloc(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(idx), K, H, scale, _ptr(out),
                                            _out_dtype(out), _ptr(lse), _stream(q.device)),
@@ -237,10 +328,16 @@ def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: f
     out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    dev = _need_attn_inputs(seqs, q, kv, out, lse)
+    if _need_index_inputs(seqs, qI, w, kI, kI_scale) != dev:
+        raise ValueError("qI and q are on different devices")
+    if idx_out is not None:
+        _need(idx_out, "idx_out", _I32T, (T, K), dev)
     ki_dtype = DSA_KI_FP8_E4M3 if kI_scale is not None else DSA_KI_BF16
     c = seqs.c()
     need = _lib.dsa_workspace_size(DSA_OP_INDEX_TOPK_ATTN, ctypes.byref(c), K, H)
     ws = ws if ws is not None else workspace(need, q.device, "index_topk_attn")
+    _need_ws(ws, dev)
     _check(_lib.dsa_index_topk_attn(ctypes.byref(c), _ptr(qI), _ptr(w), _ptr(kI), _ptr(kI_scale), ki_dtype, _ptr(q),
                                     _ptr(kv), K, H, scale, _ptr(out), _out_dtype(out), _ptr(lse), _ptr(idx_out),
                                     _ptr(ws), ws.numel(), _stream(q.device)), "dsa_index_topk_attn")

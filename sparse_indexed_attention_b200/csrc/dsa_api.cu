@@ -315,8 +315,16 @@ dsa_status_t dsa_launch_timing(int enable) {
   if (!enable) return DSA_OK;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
-  for (cudaEvent_t& e : tm.ev)
-    if (cudaEventCreate(&e) != cudaSuccess) return DSA_ERR_CUDA;
+  for (cudaEvent_t& e : tm.ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      e = nullptr;
+      for (cudaEvent_t& f : tm.ev) {  // release the ones already made: timing stays off
+        if (f) cudaEventDestroy(f);
+        f = nullptr;
+      }
+      return DSA_ERR_CUDA;
+    }
+  }
   tm.device = dev;
   return DSA_OK;
 }

@@ -1,0 +1,58 @@
+"""The Python binding refuses tensors the kernels would misread before any C
+call: wrong device, dtype, shape, stride or pool size.  CPU only -- every
+refusal here happens before the library is entered."""
+import pytest
+import torch
+
+import sparse_indexed_attention_b200 as dsa
+
+CPU = torch.device("cpu")
+
+
+def test_need_accepts_a_matching_tensor():
+    dsa._need(torch.zeros(3, 64, dtype=torch.float32), "w", dsa._F32T, (3, 64), CPU)
+    dsa._need(torch.zeros(128, 128, dtype=torch.uint8), "kI", dsa._FP8T, (None, 128), CPU, 128)
+    dsa._need(torch.zeros(128, 128, dtype=torch.float8_e4m3fn), "kI", dsa._FP8T, (None, 128), CPU, 64)
+
+
+@pytest.mark.parametrize("bad, err, what", [
+    (torch.zeros(3, 64, dtype=torch.float64), TypeError, "dtype"),
+    (torch.zeros(3, 65, dtype=torch.float32), ValueError, "shape"),
+    (torch.zeros(3, 64, 1, dtype=torch.float32), ValueError, "shape"),
+    (torch.zeros(64, 3, dtype=torch.float32).t(), ValueError, "contiguous"),
+    ([0.0] * 64, TypeError, "torch.Tensor"),
+])
+def test_need_refuses(bad, err, what):
+    with pytest.raises(err, match=what):
+        dsa._need(bad, "w", dsa._F32T, (3, 64), CPU)
+
+
+def test_need_refuses_a_short_pool_and_another_device():
+    with pytest.raises(ValueError, match="at least 128"):
+        dsa._need(torch.zeros(127, 576, dtype=torch.bfloat16), "kv", dsa._BF16T, (None, 576), CPU, 128)
+    with pytest.raises(ValueError, match="expected meta"):
+        dsa._need(torch.zeros(4, dtype=torch.int32), "row_len", dsa._I32T, (4,), torch.device("meta"))
+
+
+def test_entry_points_want_cuda_tensors():
+    T, K = 2, 16
+    seqs = dsa.Seqs(torch.tensor([0, 1, 2], dtype=torch.int32), torch.tensor([5, 7], dtype=torch.int32),
+                    torch.zeros(2, 1, dtype=torch.int32), 2, 7, T)
+    qI = torch.zeros(T, 64, 128, dtype=torch.bfloat16)
+    w = torch.zeros(T, 64)
+    kI = torch.zeros(128, 128, dtype=torch.bfloat16)
+    q = torch.zeros(T, 16, 576, dtype=torch.bfloat16)
+    kv = torch.zeros(128, 576, dtype=torch.bfloat16)
+    idx = torch.zeros(T, K, dtype=torch.int32)
+    with pytest.raises(TypeError, match="CUDA"):
+        dsa.dsa_quantize_index_query(qI, w)
+    with pytest.raises(TypeError, match="CUDA"):
+        dsa.dsa_index_scores(seqs, qI, w, kI)
+    with pytest.raises(TypeError, match="CUDA"):
+        dsa.dsa_topk(torch.zeros(T, 8), torch.full((T,), 8, dtype=torch.int32), K)
+    with pytest.raises(TypeError, match="CUDA"):
+        dsa.dsa_sparse_mla_fwd(seqs, q, kv, idx, 0.1)
+    with pytest.raises(TypeError, match="CUDA"):
+        dsa.dsa_sparse_mla_fwd_noalloc(seqs, q, kv, idx, 0.1)
+    with pytest.raises(TypeError, match="CUDA"):
+        dsa.dsa_index_topk_attn(seqs, qI, w, kI, None, q, kv, K, 0.1)
