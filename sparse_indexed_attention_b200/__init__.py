@@ -102,6 +102,22 @@ def _need(t, name: str, dtypes, shape, device: torch.device, min_rows: int = 0):
     `shape` (None matches any size) and at least `min_rows` rows.  The kernels
     take bare pointers, so a wrong dtype, a strided view or a short pool would
     otherwise be read out of bounds."""
+    try:  # fast path: one pass over the metadata, no message building
+        sz = t.shape
+        ok = t.device == device and t.dtype in dtypes and len(sz) == len(shape) and sz[0] >= min_rows \
+            and t.is_contiguous()
+        if ok:
+            for g, w in zip(sz, shape):
+                if w is not None and g != w:
+                    ok = False
+                    break
+    except (AttributeError, IndexError):
+        ok = False
+    if not ok:
+        _refuse(t, name, dtypes, shape, device, min_rows)
+
+
+def _refuse(t, name, dtypes, shape, device, min_rows):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
     if t.device != device:
@@ -113,8 +129,7 @@ def _need(t, name: str, dtypes, shape, device: torch.device, min_rows: int = 0):
         raise ValueError(f"{name}: shape {list(t.shape)}, expected {want}")
     if t.shape[0] < min_rows:
         raise ValueError(f"{name}: {t.shape[0]} rows, the page pool needs at least {min_rows}")
-    if not t.is_contiguous():
-        raise ValueError(f"{name}: must be contiguous")
+    raise ValueError(f"{name}: must be contiguous")
 
 
 def _cuda_device(t, name: str) -> torch.device:
@@ -137,10 +152,11 @@ def _need_ws(ws, dev: torch.device):
     _need(ws, "ws", (torch.uint8,), (None,), dev)
 
 
-def _need_index_inputs(seqs: "Seqs", qI, w, kI, kI_scale) -> torch.device:
+def _need_index_inputs(seqs: "Seqs", qI, w, kI, kI_scale, check_seqs: bool = True) -> torch.device:
     dev = _cuda_device(qI, "qI")
     T, rows = seqs.num_q_tokens, seqs.num_phys_pages * 64
-    _need_seqs(seqs, dev)
+    if check_seqs:
+        _need_seqs(seqs, dev)
     _need(qI, "qI", _BF16T, (T, 64, 128), dev)
     _need(w, "w", _F32T, (T, 64), dev)
     _need(kI, "kI", _FP8T if kI_scale is not None else _BF16T, (None, 128), dev, rows)
@@ -329,7 +345,7 @@ def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: f
     if lse is None and want_lse:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
     dev = _need_attn_inputs(seqs, q, kv, out, lse)
-    if _need_index_inputs(seqs, qI, w, kI, kI_scale) != dev:
+    if _need_index_inputs(seqs, qI, w, kI, kI_scale, check_seqs=False) != dev:
         raise ValueError("qI and q are on different devices")
     if idx_out is not None:
         _need(idx_out, "idx_out", _I32T, (T, K), dev)
