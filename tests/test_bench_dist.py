@@ -70,3 +70,11 @@ def test_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    # the line carries every key of the bench contract
+    keys = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+            "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
+    assert keys <= set(d), keys - set(d)
+    assert d["steps"] == 1 and d["warmup"] == 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny_prefill_1k"
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["unit"] == d["unit"] == d["cpu_baseline"]["unit"]
+    assert {"value", "cores", "sample"} <= set(d["cpu_baseline"]) and d["cpu_baseline"]["value"] == d["value"]
