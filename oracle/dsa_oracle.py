@@ -31,8 +31,8 @@ library's specification fixes it, and this module writes it out literally:
 
 Readings taken where the pages are silent (each repeated at its function):
   * candidates of query t are the positions 0..pos(t), the token itself
-    included ("all historical positions", [P1] Understanding the New
-    Architecture item 2; [P2] §2 item 2);
+    included (the indexer scores every earlier position: [P1] Understanding
+    the New Architecture item 2; [P2] §2 item 2);
   * a row with fewer than K candidates takes all of them, index list padded
     with -1, and the selected indices are emitted in ascending order;
   * the FP8 index cache is OCP E4M3 with one fp32 scale per token row; the bf16
