@@ -29,16 +29,16 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from sparse_indexed_attention_b200.workloads import CONFIGS, make_workload  # noqa: E402
+from dsa_workloads import CONFIGS, make_workload  # noqa: E402
 
 METRIC = "DSA decode tokens/s at 128K ctx"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
-# DRAM bytes (read + write) per launch from one ncu capture on this workload
-# (profiles/<kernel>_decode_b8_128k.md), valid only while the kernel's sources
-# hash to what was captured: any edit turns the figure back into null.
+# DRAM bytes (read + write) per launch from one ncu capture on this workload,
+# valid only while the kernel's sources hash to what was captured: any edit
+# turns the figure back into null.
 NCU_TRAFFIC = {
     "index_scores": (144.11e6, ("k_indexer.cu",), "829dc8b4b29fce72"),
     "topk_filter": (4.35e6, ("k_topk.cu",), "0b824ddb18426cbe"),
@@ -218,7 +218,7 @@ def cpu_threads() -> int:
 def cpu_baseline(wl, n_tokens: int):
     """The fp64 oracle on a bounded sample (the first n_tokens query tokens)."""
     from oracle import dsa_oracle as O
-    from sparse_indexed_attention_b200.workloads import bits16
+    from dsa_workloads import bits16
     seqs = O.Seqs(ctx_len=wl.ctx_len.astype(np.int64), q_seq_start=wl.q_seq_start.astype(np.int64),
                   page_table=wl.page_table, page_size=wl.spec.page_size)
     if wl.kI_scale is None:
@@ -236,6 +236,15 @@ def cpu_baseline(wl, n_tokens: int):
 # ---------------------------------------------------------------------------
 # reference arm: the oracle on the host cores
 # ---------------------------------------------------------------------------
+
+
+def workload_config(spec, wl, world: int) -> dict:
+    """The `config` object of the JSON line, the same for both arms."""
+    return {"workload": spec.name, "batch_per_gpu": spec.batch, "global_batch": wl.T * world,
+            "ctx": int(wl.ctx_len[0]), "topk": spec.topk, "heads": spec.heads, "index_heads": spec.index_heads,
+            "index_dim": spec.index_dim, "page_size": spec.page_size, "pool_tokens": wl.num_phys_pages * 64,
+            "index_cache": "fp8_e4m3" if spec.ki_fp8 else "bf16", "parallelism": f"dp{world}",
+            "l2": "256 MiB buffer written before every timed GPU step"}
 
 
 def run_reference(args, world, rank):
@@ -257,8 +266,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": spec.name, "batch": spec.batch, "ctx": int(wl.ctx_len[0]), "topk": spec.topk,
-                       "heads": spec.heads, "index_cache": "fp8_e4m3" if spec.ki_fp8 else "bf16"},
+            "config": workload_config(spec, wl, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -338,7 +346,7 @@ def run_only(args, dsa, wl, d, dev, stream, flush, world, fused=None):
 def run_all_configs(args, dsa, dev, stream, flush):
     """Every workload once: the fused call (graph replay, L2 flushed before each
     step) and per-kernel device times, each stage against its binding roofline."""
-    from sparse_indexed_attention_b200.workloads import to_device
+    from dsa_workloads import to_device
     hbm, hbm_src = hbm_peak()
     for name in CONFIGS:
         spec = CONFIGS[name]
@@ -410,7 +418,7 @@ def run_all_configs(args, dsa, dev, stream, flush):
 
 def run_ours(args, world, rank, local):
     import sparse_indexed_attention_b200 as dsa
-    from sparse_indexed_attention_b200.workloads import to_device
+    from dsa_workloads import to_device
 
     if args.all_configs:
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -547,11 +555,8 @@ def run_ours(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 index / bf16 attention / fp32 accum",
             "data": "synthetic (seeded, 64 planted keys per sequence)",
-            "config": {"workload": spec.name, "batch_per_gpu": spec.batch, "global_batch": T * world,
-                       "ctx": int(wl.ctx_len[0]), "topk": K, "heads": H, "index_heads": 64, "index_dim": 128,
-                       "page_size": 64, "pool_tokens": wl.num_phys_pages * 64, "parallelism": f"dp{world}",
-                       "l2": "256 MiB buffer written before every timed step",
-                       "launch": launch_mode},
+            "config": workload_config(spec, wl, world),
+            "launch": launch_mode,
             "stages_us": {"index_scores": ms_idx * 1e3, "topk": statistics.mean(t_topk) * 1e3,
                           "sparse_mla": statistics.mean(t_attn) * 1e3},
             "roofline": dominant,

@@ -269,7 +269,7 @@ class DeviceWorkload:
 
 
 def to_device(wl: Workload, device="cuda") -> DeviceWorkload:
-    from . import Seqs
+    from sparse_indexed_attention_b200 import Seqs
     seqs = Seqs.from_host(wl.q_seq_start, wl.ctx_len, wl.page_table, wl.num_phys_pages, device=device)
     dev = lambda x: None if x is None else x.contiguous().to(device)  # noqa: E731
     return DeviceWorkload(wl, seqs, dev(wl.qI), dev(wl.w), dev(wl.kI), dev(wl.kI_scale), dev(wl.q), dev(wl.kv))

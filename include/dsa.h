@@ -204,11 +204,12 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t *seqs, const void *q,
  * a fixed array of DSA_NOALLOC_SCRATCH_BYTES in the library's device image:
  *   - every GPU that loads the library holds that memory until the process exits;
  *   - a geometry whose scratch (dsa_workspace_size(DSA_OP_SPARSE_MLA, ...))
- *     exceeds it returns DSA_ERR_WORKSPACE before any CUDA call (decode batches
- *     below 74 tokens need at most ~20 MiB; larger batches need only 8 bytes per
- *     token plus 4 per sequence);
- *   - the first call on each device, with that device current, looks up the
- *     array's device address; make that first call before any stream capture;
+ *     exceeds it returns DSA_ERR_WORKSPACE before any CUDA call (a batch whose
+ *     index lists are split over several CTAs -- fewer than 148 (token, 64-head
+ *     group) pairs -- needs at most ~20 MiB; larger batches need only 8 bytes
+ *     per token plus 4 per sequence);
+ *   - each call looks up the array's device address in the current context
+ *     (a host-side runtime query; the device must be current);
  *   - nothing is allocated or freed (no cudaMalloc, cudaFree or allocating
  *     library routine); the array's error word is cleared at the start of each
  *     call with an asynchronous memset;
@@ -216,12 +217,20 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t *seqs, const void *q,
  *     calls that overlap on the GPU (other streams, other host threads) race
  *     and corrupt each other's results, so serialise them;
  *   - bad device-side indices or page ids are skipped as in dsa_sparse_mla_fwd,
- *     but cannot be reported: the error word lives in the shared array. */
+ *     and a bounded in-kernel wait that runs out abandons its slice, whose
+ *     partial result the merge may then take from an earlier call; both set the
+ *     array's error word, which only dsa_check_error_noalloc reads: call it
+ *     after the call (before the next one) to know the result is sound. */
 dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_seqs_t *seqs, const void *q,
                                         const void *kv, const int32_t *idx,
                                         int K, int H, float scale, void *out,
                                         dsa_out_dtype_t out_dtype, float *lse,
                                         dsa_stream_t stream);
+
+/* dsa_check_error for dsa_sparse_mla_fwd_noalloc: synchronises `stream`, then
+ * reads and clears the error word of the built-in scratch array (the device
+ * must be current).  Same results as dsa_check_error. */
+dsa_status_t dsa_check_error_noalloc(dsa_stream_t stream);
 
 /* The whole path in one call ([P1] Layer 1, "Sparse attention": scoring,
  * selection, gathering and attention integrated; [P3] section 3 pseudocode):
@@ -241,6 +250,14 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t *seqs, const void *qI,
  * flag.  Returns DSA_OK, DSA_ERR_BAD_INDEX, DSA_ERR_TIMEOUT or DSA_ERR_CUDA
  * (a pending CUDA error on the stream). */
 dsa_status_t dsa_check_error(void *ws, dsa_stream_t stream);
+
+/* Limit, in nanoseconds, of every bounded in-kernel wait for another part of
+ * the kernel to make progress, for the launches of later calls made by the
+ * calling host thread (0 restores the default of 2 s).  A wait that runs out
+ * sets DSA_ERR_TIMEOUT and its CTA winds down (waiting, under a fixed 2 s
+ * bound, only for copies and MMAs it has already issued).  A failure-handling
+ * aid: a short limit makes waits run out on purpose.  Host only; DSA_OK. */
+dsa_status_t dsa_set_wait_limit_ns(uint64_t ns);
 
 /* Number of kernels the calling host thread's most recent entry-point call
  * (dsa_quantize_index_query .. dsa_index_topk_attn) launched.  Host only. */

@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY.  The library never imports, links or calls anything
 here; only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may.  It shares no code, header, table or constant generator with
 the CUDA path: the only thing both sides see is the seeded synthetic input
-(``sparse_indexed_attention_b200.workloads``), which holds none of the method's
+(``dsa_workloads``), which holds none of the method's
 arithmetic.
 
 Sources.  Five web pages describe one engineering effort on DSA; they are cited

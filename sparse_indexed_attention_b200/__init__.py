@@ -37,8 +37,9 @@ DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA
 
 # Names the C header declares (checked against include/dsa.h by the tests).
 EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_index_scores", "dsa_topk",
-           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_noalloc", "dsa_index_topk_attn", "dsa_check_error", "dsa_launches_in_last_call",
-           "dsa_launch_timing", "dsa_last_launch_times", "dsa_status_string")
+           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_noalloc", "dsa_check_error_noalloc", "dsa_index_topk_attn",
+           "dsa_check_error", "dsa_set_wait_limit_ns", "dsa_launches_in_last_call", "dsa_launch_timing",
+           "dsa_last_launch_times", "dsa_status_string")
 
 
 class DsaSeqsC(ctypes.Structure):
@@ -62,6 +63,8 @@ _sig = {
     "dsa_index_topk_attn": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
                                            _F, _P, ctypes.c_int, _P, _P, _P, _SZ, _P]),
     "dsa_check_error": (ctypes.c_int, [_P, _P]),
+    "dsa_check_error_noalloc": (ctypes.c_int, [_P]),
+    "dsa_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
     "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dsa_launches_in_last_call": (ctypes.c_int, []),
     "dsa_launch_timing": (ctypes.c_int, [ctypes.c_int]),
@@ -363,6 +366,18 @@ def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: f
 def dsa_check_error(ws: torch.Tensor) -> int:
     """Synchronise the current stream and return (and clear) the device error status."""
     return int(_lib.dsa_check_error(_ptr(ws), _stream(ws.device)))
+
+
+def dsa_check_error_noalloc(device=None) -> int:
+    """dsa_check_error for the built-in scratch of dsa_sparse_mla_fwd_noalloc
+    (synchronises the current stream of `device`)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(_lib.dsa_check_error_noalloc(_stream(dev)))
+
+
+def dsa_set_wait_limit_ns(ns: int) -> None:
+    """Limit of every bounded in-kernel wait of this thread's later calls (0 = the 2 s default)."""
+    _check(_lib.dsa_set_wait_limit_ns(int(ns)), "dsa_set_wait_limit_ns")
 
 
 def dsa_launches_in_last_call() -> int:

@@ -10,6 +10,7 @@ using namespace dsa;
 namespace dsa {
 thread_local int g_launches = 0;
 thread_local LaunchTimer g_timer;
+thread_local uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 }
 
 namespace {
@@ -296,6 +297,11 @@ dsa_status_t dsa_check_error(void* ws, dsa_stream_t stream) {
 }
 
 int dsa_launches_in_last_call(void) { return g_launches; }
+
+dsa_status_t dsa_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns = ns == 0 ? kDefaultWaitLimitNs : ns;
+  return DSA_OK;
+}
 
 dsa_status_t dsa_launch_timing(int enable) {
   LaunchTimer& tm = g_timer;

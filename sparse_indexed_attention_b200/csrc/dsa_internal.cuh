@@ -127,6 +127,12 @@ inline cudaError_t launch_pdl(const char* name, void (*kernel)(KArgs...), dim3 g
   return e;
 }
 
+// Limit of every in-kernel wait for another role's progress, for launches
+// made by the current host thread (dsa_set_wait_limit_ns; default 2 s).
+constexpr uint64_t kDefaultWaitLimitNs = 2000ull * 1000ull * 1000ull;
+extern thread_local uint64_t g_wait_limit_ns;
+__host__ inline uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+
 // Kernels launched by the current host thread since its last entry-point call
 // began (reported by dsa_launches_in_last_call).
 extern thread_local int g_launches;

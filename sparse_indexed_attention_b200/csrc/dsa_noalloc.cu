@@ -2,8 +2,6 @@
 // allocate device memory (see include/dsa.h).  The scratch that
 // dsa_sparse_mla_fwd takes from the caller lives here in a fixed array of the
 // library's device image instead; everything else is the regular entry point.
-#include <atomic>
-
 #include "dsa_internal.cuh"
 
 namespace {
@@ -12,8 +10,15 @@ namespace {
 // library's device image is loaded; kept by each GPU that loads it until exit.
 __device__ __align__(256) unsigned char g_noalloc_scratch[DSA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];  // device address of the array, per device
+// Device address of the array in the current context.  Looked up on every
+// call (a cheap host-side query): a cached address would go stale if the
+// library's module were reloaded in a new primary context.
+dsa_status_t scratch_address(void** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+  *out = p;
+  return DSA_OK;
+}
 
 }  // namespace
 
@@ -25,21 +30,19 @@ extern "C" dsa_status_t dsa_sparse_mla_fwd_noalloc(const dsa_seqs_t* seqs, const
   const size_t need = dsa_workspace_size(DSA_OP_SPARSE_MLA, seqs, K, H);
   if (need > (size_t)DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE;
   // need == 0 means invalid sizes; the regular entry point reports which.
-
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
-  void* scratch = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!scratch) {
-    // One-time set-up on this device (the device is current): the host-side
-    // name of the array is not a device address, so ask the runtime for it.
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
-    g_scratch_addr[dev].store(p, std::memory_order_release);
-    scratch = p;
-  }
+  void* scratch = nullptr;
+  const dsa_status_t st = scratch_address(&scratch);
+  if (st != DSA_OK) return st;
   // The error word at the head of the scratch is the only part that has to
-  // start at zero; earlier calls may have left bits in it.
+  // start at zero: the previous call may have left bits in it.
   if (cudaMemsetAsync(scratch, 0, 256, (cudaStream_t)stream) != cudaSuccess) return DSA_ERR_CUDA;
   return dsa_sparse_mla_fwd(seqs, q, kv, idx, K, H, scale, out, out_dtype, lse, scratch,
                             (size_t)DSA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" dsa_status_t dsa_check_error_noalloc(dsa_stream_t stream) {
+  void* scratch = nullptr;
+  const dsa_status_t st = scratch_address(&scratch);
+  if (st != DSA_OK) return st;
+  return dsa_check_error(scratch, stream);
 }

@@ -54,7 +54,7 @@ struct IdxCfg {
   static constexpr int OFF_HIST = OFF_W + 2 * TG * 256;   // TG == 1: per-epilogue-warp Top-K histograms
   static constexpr int OFF_RING = OFF_HIST + (TG == 1 ? kEpiWarps * kTopkHistBins * 4 : 0);
   static constexpr int OFF_BAR = OFF_RING + kRingSlots * (32 + 128);  // producer's item records + page ids
-  static constexpr int NBARS = 2 * NS + 4 + 2 * NACC;
+  static constexpr int NBARS = 2 * NS + 4 + 2 * NACC + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;                // slack for 1024-byte alignment
@@ -72,6 +72,7 @@ struct IdxArgs {
   int64_t ld;
   uint32_t* hist;          // TG == 1 only, may be null: Top-K first-digit histogram [T][2048]
   uint32_t* err;
+  uint64_t wait_ns;        // limit of each wait for another role's progress
 };
 
 // Adds one epilogue warp's histogram of the current token to the global one
@@ -102,6 +103,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
   uint64_t* b_empty = b_full + 2;             // [2]   group operands released
   uint64_t* acc_full = b_empty + 2;           // [NACC]
   uint64_t* acc_empty = acc_full + C::NACC;   // [NACC]
+  uint64_t* mma_drain = acc_empty + C::NACC;  // every MMA this CTA issued has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   const float* sc_smem = reinterpret_cast<const float*>(smem + C::OFF_SC);
@@ -121,6 +123,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
     }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -175,6 +178,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
       cp_async_commit();
     }
     int stage = 0, sphase = 0, prev_g = -1, gcount = 0;
+    int issued = 0, b_issued = 0;  // tiles / group operand loads with copies in flight or landed (lane 0)
     bool ok = true;
     for (int it = it_lo; it < it_hi && ok; ++it) {
       // groups so far: the page ids of it_lo .. it_lo+kPgAhead-1, then one
@@ -191,7 +195,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
       if (cb.z != prev_g) {
         if (lane == 0) {
           const int slot = gcount & 1, use = gcount >> 1;
-          if (!mbar_wait(&b_empty[slot], (use & 1) ^ 1, a.err)) {
+          if (!mbar_wait(&b_empty[slot], (use & 1) ^ 1, a.err, a.wait_ns)) {
             *abort_flag = 1;
           } else {
             const uint32_t wbytes = (uint32_t)grp.z * 256u;
@@ -204,6 +208,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
               tma_load_2d(bdst, &tmap_q, &b_full[slot], 0, grp.y * 64);
             }
             bulk_load(smem + C::OFF_W + slot * TG * 256, a.w_operand + (int64_t)grp.y * 64, wbytes, &b_full[slot]);
+            ++b_issued;
           }
         }
         prev_g = cb.z;
@@ -214,7 +219,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
         const int pg0 = __shfl_sync(0xffffffffu, pages, 2 * j);
         const int pg1 = __shfl_sync(0xffffffffu, pages, 2 * j + 1);
         if (lane == 0 && !*abort_flag) {
-          if (!mbar_wait(&empty[stage], sphase ^ 1, a.err)) {
+          if (!mbar_wait(&empty[stage], sphase ^ 1, a.err, a.wait_ns)) {
             *abort_flag = 1;
           } else {
             const int last = grp.w + grp.z - 1;
@@ -234,6 +239,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
               }
             }
             mbar_arrive_expect_tx(&full[stage], bytes);
+            ++issued;
             uint8_t* adst = smem + C::OFF_A + stage * C::A_BYTES;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -253,12 +259,14 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
       ok = __shfl_sync(0xffffffffu, (int)(*abort_flag == 0), 0) != 0;  // lane 0's view, warp-uniform
     }
     cp_async_wait<0>();  // no copy into the ring is still in flight at exit
-    // drain: every issued stage has been consumed before the CTA exits
+    // drain, also after a failed wait: every copy this warp issued has landed
+    // before the CTA exits (tile i used stage i % NS in phase i / NS; a stage's
+    // last use is its only phase that can still be pending)
     if (lane == 0) {
-      for (int i = 0; i < C::NS && !*abort_flag; ++i) {
-        if (!mbar_wait(&empty[stage], sphase ^ 1, a.err)) break;
-        if (++stage == C::NS) { stage = 0; sphase ^= 1; }
-      }
+      for (int i = issued > C::NS ? issued - C::NS : 0; i < issued; ++i)
+        if (!mbar_wait(&full[i % C::NS], (uint32_t)((i / C::NS) & 1), a.err, kDrainLimitNs)) break;
+      for (int i = b_issued > 2 ? b_issued - 2 : 0; i < b_issued; ++i)
+        if (!mbar_wait(&b_full[i & 1], (uint32_t)((i >> 1) & 1), a.err, kDrainLimitNs)) break;
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -272,14 +280,14 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
         if (item.x != prev_g) {
           if (prev_g >= 0) mma_commit(&b_empty[slot]);  // previous group's operands free once its MMAs finish
           slot = gcount & 1;
-          if (!mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err)) { *abort_flag = 1; break; }
+          if (!mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err, a.wait_ns)) { *abort_flag = 1; break; }
           prev_g = item.x;
           ++gcount;
         }
         const uint32_t b_base = smem_u32(smem + C::OFF_B + slot * C::B_BYTES);
         for (int tile = item.y; tile < item.z; ++tile) {
-          if (!mbar_wait(&full[stage], sphase, a.err)) { *abort_flag = 1; break; }
-          if (!mbar_wait(&acc_empty[acc], aphase ^ 1, a.err)) { *abort_flag = 1; break; }
+          if (!mbar_wait(&full[stage], sphase, a.err, a.wait_ns)) { *abort_flag = 1; break; }
+          if (!mbar_wait(&acc_empty[acc], aphase ^ 1, a.err, a.wait_ns)) { *abort_flag = 1; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
 #pragma unroll
@@ -296,6 +304,10 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
           if (++acc == C::NACC) { acc = 0; aphase ^= 1; }
         }
       }
+      // drain, also after a failed wait: no MMA of this CTA still reads shared
+      // memory or writes TMEM when the CTA deallocates and exits
+      mma_commit(mma_drain);
+      mbar_wait(mma_drain, 0, a.err, kDrainLimitNs);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -328,7 +340,10 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
         if (do_hist && prev_t >= 0 && prev_t != grp.y) flush_hist(sh_hist, a.hist, prev_t, lane);
         prev_t = grp.y;
         slot = gcount & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err))) { *abort_flag = 1; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err, a.wait_ns))) {
+          *abort_flag = 1;
+          break;
+        }
         if constexpr (TG == 1) {
 #pragma unroll
           for (int h = 0; h < 64; ++h) wreg[h] = w_smem[slot * TG * 64 + h];
@@ -338,9 +353,9 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
       }
       for (int tile = item.y; tile < item.z; ++tile, ++ti) {
         if ((ti & 1) == wg) {
-          bool okw = mbar_wait(&acc_full[acc], aphase, a.err);
+          bool okw = mbar_wait(&acc_full[acc], aphase, a.err, a.wait_ns);
           // the row scales arrived with the stage's TMA; observe that completion here too
-          if (!kBf16) okw = okw && mbar_wait(&full[stage], sphase, a.err);
+          if (!kBf16) okw = okw && mbar_wait(&full[stage], sphase, a.err, a.wait_ns);
           if (!__all_sync(0xffffffffu, okw)) { *abort_flag = 1; break; }
           tc_fence_after();
           const float sk = kBf16 ? 1.f : sc_smem[stage * 128 + r];
@@ -456,7 +471,7 @@ cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, 
   CUtensorMap mk, mq;
   if (!make_map(&mk, kI, bf16, kDI, R, bf16 ? 64 : 128, 64)) return cudaErrorInvalidValue;
   if (!make_map(&mq, q_operand, bf16, kDI, qrows, bf16 ? 64 : 128, 64 * tg)) return cudaErrorInvalidValue;
-  IdxArgs a{s, plan, w_operand, kI_scale, scores, ld, tg == 1 ? hist : nullptr, err};
+  IdxArgs a{s, plan, w_operand, kI_scale, scores, ld, tg == 1 ? hist : nullptr, err, wait_limit_ns()};
   if (fp8) {
     if (tg == 1) return launch_tc<false, 1>(mk, mq, a, st);
     if (tg == 4) return launch_tc<false, 4>(mk, mq, a, st);

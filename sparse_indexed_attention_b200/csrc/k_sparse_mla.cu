@@ -10,34 +10,33 @@
 //   out[t,h,:] = sum_{s in idx[t]} p_s KV[s,0:512],
 //   p = softmax_s(scale * q[t,h,:] . KV[s,0:576]),   lse = ln sum exp(...)
 //
-// The fp32 accumulator of 128 heads x 512 value dims fills all of TMEM, so
-// the work of one (token, slice of the index list) goes to a CLUSTER OF TWO
-// CTAs.  CTA r owns value dims [256r, 256r+256) and the key dims
-// {256r..256r+255} u {512+32r..512+32r+31}; it gathers only those 576 bytes of
-// each selected row.  Three warps resolve every selected row of the slice
-// up front (index list -> page table, all loads independent) and then copy
-// the rows block by block with 16-byte cp.async straight into the 128-byte /
-// 64-byte swizzled operand layouts -- many small copies in flight instead of
-// a queue of four-row TMA gathers.  Per block of 64 selected rows:
-//   * S_r = Q_r K_r^T (M = 128 heads, N = 64 rows, K = 288 dims) into TMEM;
-//   * the two partial S are exchanged through distributed shared memory
-//     (st.async into the peer's double-buffered receive area, counted on the
-//     peer's mbarrier, so no cluster-scope fence sits on the path) and summed
-//     (a + b = b + a, so both CTAs hold bit-identical logits and take
-//     identical softmax decisions);
-//   * online softmax in registers (one head row per thread, base-2 exponent,
-//     the running maximum is only moved -- and O rescaled in TMEM -- when it
-//     grows by more than 2^8, which is exact because O and l share it);
-//   * P goes to TMEM as two bf16 terms, P = P_hi + P_lo (together within
-//     2^-17 of the fp32 value; one bf16 term alone would leave a relative
-//     error of 2^-9 on rows dominated by a few selected keys), and
-//     O_r += P_hi V_r + P_lo V_r (M = 128, N = 256, K = 64) accumulates in
-//     TMEM with P read from TMEM, V_r being the same gathered bytes read as an
-//     MN-major operand.  TMEM columns: O [0, 256), S [256, 384) (two
-//     buffers), P [384, 512) (two buffers of hi + lo).
-// Slices of one token are merged by k_combine (log-sum-exp weights).
-#include <cudaTypedefs.h>
-
+// One CTA takes 64 heads of one token and one slice of its index list, and
+// works on whole 576-dim rows, so no logit ever leaves the CTA.  An M = 64
+// MMA keeps its rows in 16 of the 32 lanes of each TMEM lane quarter, so
+// tensor memory holds, side by side:
+//   lanes 0-15 of each quarter:  Q (64 heads x 576 bf16, 288 columns) -- the
+//                                A operand of S = Q K^T, read from TMEM --
+//                                and two logit buffers S (64 columns each);
+//   lanes 16-31:                 O (64 heads x 512 fp32, all 512 columns).
+// Shared memory then holds only rows and probabilities:
+//   * four loader warps resolve every selected row of the slice up front
+//     (index list -> page table -> pool row, all loads independent) and copy
+//     the rows block by block (64 rows, two stages) with 16-byte cp.async
+//     straight into the 128-byte-swizzled operand layout: nine 8 KB atoms of
+//     64 dims each;
+//   * one thread issues S = Q K^T (M = 64 heads, N = 64 rows, K = 576) and
+//     O += P V (M = 64, N = 256, twice, K = 64 rows) -- V is the same gathered
+//     bytes read as an MN-major operand;
+//   * four softmax warps, one per lane quarter: thread i and i + 16 share a
+//     head and take 32 of the block's 64 logits each (online softmax, base-2
+//     exponent; the running maximum only moves -- and O is rescaled in TMEM --
+//     when it grows by more than 2^8, exact because O and l share it).  P goes
+//     to shared memory as two bf16 terms, P = P_hi + P_lo (within 2^-16 of the
+//     fp32 value), and PV runs once per term: one bf16 term alone misses the
+//     accuracy bound on rows that a few selected keys dominate (relative
+//     error up to 2^-8 of the spread of V, measured on the 1024-token prefill).
+// Decode batches split the index list over several CTAs per (token, head
+// group); k_combine merges their partials (log-sum-exp weights).
 #include "sm100.cuh"
 
 namespace dsa {
@@ -46,36 +45,36 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBK = 64;                      // selected rows per block
-constexpr int kQLatBytes = 128 * 128;        // one 64-dim swizzle atom of 128 head rows
-constexpr int kQBytes = 4 * kQLatBytes + 128 * 64;
-constexpr int kKVStage = 4 * kBK * 128 + kBK * 64;  // 36864: 4 latent atoms + rope quarter
-constexpr int kXBytes = 128 * kBK * 4;       // one partial S: [16 column quads][128 heads][4] fp32
-constexpr int kLoaders = 96;                 // warps 0, 2, 3 copy the selected rows
-constexpr int kRingBlocks = kMaxK / kBK;     // resolved row ids of every block of a slice
-constexpr int kLoaderBarrier = 1;            // named barrier of the loader warps
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + kQBytes;                 // 73728
-constexpr int kStages = 3;                              // row stages in flight
-constexpr int OFF_X = OFF_KV + kStages * kKVStage;      // 184320: the peer's partial logits
-constexpr int OFF_ROWS = OFF_X + kXBytes;               // 217088: [block][64] pool rows (-1 = masked)
-constexpr int OFF_MASK = OFF_ROWS + kRingBlocks * kBK * 4;  // [block] 64-bit validity masks
-constexpr int OFF_BAR = OFF_MASK + kRingBlocks * 8;
-constexpr int kNBars = 17;
-constexpr int OFF_PAIR = OFF_BAR + kNBars * 8;          // [2 parity][2 half][128 heads] float2
-constexpr int OFF_MISC = OFF_PAIR + 2 * 2 * 128 * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-constexpr int kThreads = 384;                // warps 0, 2, 3 load; 1 issues MMAs; 4-11 softmax
-constexpr int kPairBarrier = 2;              // named barriers 2..5: softmax warps w and w+4
+constexpr int kBK = 64;                       // selected rows per block
+constexpr int kHG = 64;                       // heads per CTA (one M = 64 tile)
+constexpr int kAtom = 64 * 128;               // 64 rows x 64 bf16 dims, 128-byte swizzle
+constexpr int kNAtoms = kDQK / 64;            // 9: eight latent atoms + the rope atom
+constexpr int kStageBytes = kNAtoms * kAtom;  // 73728
+constexpr int kStages = 2;
+constexpr int kPTerm = kHG * kBK * 2;         // one bf16 term of P: 64 heads x 64 rows, 128-byte swizzle
+constexpr int kLoaders = 128;                 // warps 4-7
+constexpr int kLoaderBarrier = 1;             // named barrier of the loader warps
+constexpr int OFF_KV = 0;
+constexpr int OFF_P = OFF_KV + kStages * kStageBytes;     // [2 buffers][hi, lo]
+constexpr int OFF_ROWS = OFF_P + 2 * 2 * kPTerm;          // [block][64] pool rows of the slice (-1 = masked)
+constexpr int OFF_MASK = OFF_ROWS + kMaxK * 4;            // [block] 64-bit validity masks
+constexpr int OFF_BAR = OFF_MASK + (kMaxK / kBK) * 8;
+constexpr int kNBars = 14;
+constexpr int OFF_MISC = OFF_BAR + kNBars * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;          // slack for 1024-byte alignment
+constexpr int kThreads = 288;  // warps 0-3 softmax + epilogue, 4-7 load, 8 issues MMAs and owns TMEM
+constexpr int kMmaWarp = 8;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-static_assert(OFF_KV % 1024 == 0 && kKVStage % 1024 == 0, "swizzle atoms need 1024-B alignment");
-constexpr uint32_t kTmemS = 256, kTmemP = 384;  // TMEM column bases (O at 0)
+static_assert(kStageBytes % 1024 == 0 && OFF_P % 1024 == 0 && kPTerm % 1024 == 0, "swizzle atoms need 1024-B alignment");
+// TMEM map: lane offset << 16 | column
+constexpr uint32_t kTmemS = 288;             // S buffers at columns 288 and 352 of lanes 0-15 (Q at 0)
+constexpr uint32_t kTmemO = 16u << 16;       // O: lanes 16-31, columns 0-511
 
-constexpr uint32_t IDESC_QK = make_idesc_major(true, 128, kBK, 0, 0);  // S = Q K^T, both K-major
-constexpr uint32_t IDESC_PV = make_idesc_major(true, 128, 256, 0, 1);  // O += P V, V MN-major
+constexpr uint32_t IDESC_QK = make_idesc_major(true, kHG, kBK, 0, 0);  // S = Q K^T, both K-major
+constexpr uint32_t IDESC_PV = make_idesc_major(true, kHG, 256, 0, 1);  // O += P V, V MN-major
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;    // log2 units
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 // 2^x from the MUFU unit (approximate, subnormal results flushed to 0;
 // ex2(-inf) = +0).
@@ -92,90 +91,122 @@ __device__ __forceinline__ void store_out(void* out, bool f32, int64_t i, float 
     reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16(v);
 }
 
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc(saddr, lbo, sbo, 2);
+}
+
 struct AttnArgs {
   SeqsDev s;
   TokenMap tm;
+  const __nv_bfloat16* q;   // [T, H, 576]
   const __nv_bfloat16* kv;  // latent pool [rows, 576]
   const int32_t* idx;
-  int K, H, ks, splits;
-  bool tm_early;     // the token map was written two or more launches back
-  float scale_log2;  // scale * log2(e)
+  int K, H, G, ks, splits;  // G head groups of 64; ks selected slots per split
+  bool tm_early;            // the token map was written two or more launches back
+  float scale_log2;         // scale * log2(e)
   void* out;
   bool out_f32;
   float* lse;
   float* part_o;
   float2* part_ml;
   uint32_t* err;
+  uint64_t wait_ns;         // limit of each wait for another role's progress
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constant__ CUtensorMap tq_rope,
-                const AttnArgs a) {
+// Query rows of the CTA's 64 heads into TMEM (A operand of S = Q K^T): warp q
+// writes heads 16q .. 16q+15, thread i (i < 16) dims [0, 288) and thread
+// i + 16 dims [288, 576) of head 16q + i, as bf16 pairs (column c = dims 2c,
+// 2c + 1).  Heads at or past H are zero.  Two rounds of loads, each issued
+// together.
+__device__ __forceinline__ void load_query_to_tmem(const AttnArgs& a, int t, int g, uint32_t t_q, int lane, int q) {
+  const int hr = 16 * q + (lane & 15), half = lane >> 4;
+  const int head = kHG * g + hr;
+  const bool valid = head < a.H;
+  const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)t * a.H + (valid ? head : 0)) * kDQK + 288 * half);
+#pragma unroll
+  for (int round = 0; round < 2; ++round) {
+    constexpr int kChunks = 5;  // chunk = 32 dims = 64 bytes = 16 TMEM columns
+    uint4 v[kChunks * 4];
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+      const int chunk = round * kChunks + c;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v[4 * c + k] = (valid && chunk < 9) ? __ldg(src + 4 * chunk + k) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+      const int chunk = round * kChunks + c;
+      if (chunk >= 9) break;
+      const uint32_t r[16] = {v[4 * c].x,     v[4 * c].y,     v[4 * c].z,     v[4 * c].w,
+                              v[4 * c + 1].x, v[4 * c + 1].y, v[4 * c + 1].z, v[4 * c + 1].w,
+                              v[4 * c + 2].x, v[4 * c + 2].y, v[4 * c + 2].z, v[4 * c + 2].w,
+                              v[4 * c + 3].x, v[4 * c + 3].y, v[4 * c + 3].z, v[4 * c + 3].w};
+      tmem_st16x2_16<144>(t_q + 16 * chunk, r);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+k_sparse_mla_tc(const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [kStages] rows of block j (stage j % 3) landed
-  uint64_t* kv_empty = bars + 4;   // [kStages] PV of the stage's block completed
-  uint64_t* s_full = bars + 7;     // [2] S of block j (buffer j & 1) in TMEM
-  uint64_t* s_empty = bars + 9;    // [2] S buffer read by every softmax warp
-  uint64_t* p_full = bars + 11;    // [2] P of block j (buffer j & 1) in TMEM
-  uint64_t* o_done = bars + 13;    // [2] PV of block i (buffer i & 1) has completed
-  uint64_t* x_full = bars + 15;    // the peer's partial S of the current block has landed in X
-  uint64_t* x_free = bars + 16;    // the peer's eight softmax warps have read what I sent
+  uint64_t* q_full = bars + 0;     // the query rows are in TMEM (one arrival per softmax warp)
+  uint64_t* kv_full = bars + 1;    // [kStages] rows of block j (stage j % 2) landed
+  uint64_t* kv_empty = bars + 3;   // [kStages] PV of the stage's block completed
+  uint64_t* s_full = bars + 5;     // [2] S of block j (buffer j & 1) in TMEM
+  uint64_t* s_empty = bars + 7;    // [2] S buffer read by every softmax warp
+  uint64_t* p_full = bars + 9;     // [2] P of block j (buffer j & 1) in shared memory
+  uint64_t* o_done = bars + 11;    // [2] PV of block i (parity by i & 1) has completed
+  uint64_t* mma_drain = bars + 13; // every MMA this CTA issued has completed
   int32_t* ring_rows = reinterpret_cast<int32_t*>(smem + OFF_ROWS);
   uint64_t* ring_mask = reinterpret_cast<uint64_t*>(smem + OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const uint32_t peer = rank ^ 1u;
-  const int cluster = blockIdx.x >> 1;
-  const int t = cluster / a.splits, sp = cluster % a.splits;
+  const int cta = blockIdx.x;
+  const int sp = cta % a.splits, tg = cta / a.splits;
+  const int g = tg % a.G, t = tg / a.G;
   const int kbeg = sp * a.ks;
   const int kend = min(a.K, kbeg + a.ks);
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, 4);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&kv_full[i], kLoaders + 1);  // every loader's copies + the mask's publisher
       mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 8);
-      mbar_init(&p_full[i], 8);  // one arrival per softmax warp
+      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
       mbar_init(&o_done[i], 1);
     }
-    mbar_init(x_full, 1);   // armed by this CTA (expect_tx), filled by the peer's st.async
-    mbar_init(x_free, 8);   // one arrival per peer softmax warp
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // the receive area for block 0 is armed before the cluster barrier below
-    // lets the peer store into it
-    mbar_arrive_expect_tx(x_full, kXBytes);
   }
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // the peer's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) {  // q is an input of the call: its load overlaps the wait below
-    prefetch_tmap(&tq_lat);
-    mbar_arrive_expect_tx(q_full, kQBytes);
-    for (int at = 0; at < 4; ++at)
-      tma_load_2d(smem + OFF_Q + at * kQLatBytes, &tq_lat, q_full, 256 * rank + 64 * at, t * a.H);
-    tma_load_2d(smem + OFF_Q + 4 * kQLatBytes, &tq_rope, q_full, 512 + 32 * rank, t * a.H);
+  if (warp < 4) {  // q is an input of the call: its load overlaps the wait below
+    load_query_to_tmem(a, t, g, tmem + ((uint32_t)(32 * warp) << 16), lane, warp);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_full);
   }
   // the token map can be read before the wait when it does not come from
   // the kernel just before; the index lists always do
   int pos = a.tm_early ? a.tm.pos[t] : 0, b = a.tm_early ? a.tm.seq[t] : 0;
-  if (a.tm_early && warp == 0 && pos >= 0) {
+  if (a.tm_early && warp == 4 && pos >= 0) {
     // the sequence's page-table row into L2 while the previous kernel ends:
     // the loaders look selected pages up in it right after the wait
     const int64_t row_bytes = (int64_t)a.s.max_pages * 4;
@@ -190,19 +221,19 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
   }
   const int nblk = (pos >= 0 && kend > kbeg) ? (kend - kbeg + kBK - 1) / kBK : 0;
 
-  if ((warp == 0 || warp == 2 || warp == 3) && nblk > 0) {
+  if (warp >= 4 && warp < kMmaWarp && nblk > 0) {
     // ---------------------------------------------------------------- loaders
-    const int li = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0 .. 95
-    const int lw = warp == 0 ? 0 : warp - 1;                // loader warp 0 .. 2
+    const int li = threadIdx.x - 128;  // 0 .. 127
+    const int lw = warp - 4;           // loader warp 0 .. 3
     // Pool rows of every block of the slice, resolved up front in three
     // passes whose loads are all independent: the index list, then the page
-    // ids (both staged by cp.async in the KV stage areas, which the first row
+    // ids (both staged by cp.async in the row stages, which the first row
     // copies overwrite only after the last pass), then rows and masks
     // (row -1 = masked).
     {
       const int nkeys = kend - kbeg;
       int32_t* s_sidx = reinterpret_cast<int32_t*>(smem + OFF_KV);
-      int32_t* s_page = reinterpret_cast<int32_t*>(smem + OFF_KV + kKVStage);
+      int32_t* s_page = reinterpret_cast<int32_t*>(smem + OFF_KV + kStageBytes);
       const int32_t* idx_row = a.idx + (int64_t)t * a.K + kbeg;
       for (int k = li; k < nkeys; k += kLoaders) cp_async_4(&s_sidx[k], idx_row + k);
       cp_async_wait_all();
@@ -231,60 +262,49 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         ring_rows[k] = row;
       }
       bar_red_or(kLoaderBarrier, kLoaders, false);
-      for (int w32 = lw; w32 < 2 * nblk; w32 += 3) {  // 32 rows per warp -> half a block's mask
+      for (int w32 = lw; w32 < 2 * nblk; w32 += 4) {  // 32 rows per warp -> half a block's mask
         const uint32_t m = __ballot_sync(0xffffffffu, ring_rows[w32 * 32 + lane] >= 0);
         if (lane == 0) reinterpret_cast<uint32_t*>(ring_mask)[w32] = m;
       }
     }
     const uint32_t kv_smem = smem_u32(smem + OFF_KV);
-    const __nv_bfloat16* kv_base = reinterpret_cast<const __nv_bfloat16*>(a.kv);
+    const __nv_bfloat16* kv_base = a.kv;
+    const int rsub = lane >> 3, piece = lane & 7;  // a warp copies 4 rows x 128 bytes of one atom
     bool failed = bar_red_or(kLoaderBarrier, kLoaders, false);
     for (int j = 0; j < nblk && !failed; ++j) {
-      const int stage = j % kStages, slot = j;
-      bool ok = mbar_wait(&kv_empty[stage], ((j / kStages) & 1) ^ 1, a.err);
+      const int stage = j % kStages;
+      const bool ok = mbar_wait(&kv_empty[stage], ((j / kStages) & 1) ^ 1, a.err, a.wait_ns);
       if (ok) {
-        // one warp per row: lane k copies latent piece k (16 B = 8 dims) of
-        // the CTA's 256 latent dims; rope pieces go 8 rows per instruction
-        const uint32_t dst0 = kv_smem + stage * kKVStage;
-        for (int r = lw; r < kBK; r += 3) {
-          const int row = ring_rows[slot * kBK + r];
+        // task = (atom, quad of rows): the warp's 32 copies fill 512
+        // contiguous bytes of the atom (no bank conflict) from four 128-byte
+        // pieces of the pool
+        const uint32_t dst0 = kv_smem + stage * kStageBytes;
+        for (int task = lw; task < kNAtoms * (kBK / 4); task += 4) {
+          const int at = task / (kBK / 4);
+          const int r = 4 * (task % (kBK / 4)) + rsub;
+          const int row = ring_rows[j * kBK + r];
           const bool v = row >= 0;
-          const uint32_t dst = dst0 + (lane >> 3) * (kBK * 128) + r * 128 +
-                               ((((uint32_t)lane & 7u) ^ ((uint32_t)r & 7u)) << 4);
-          cp_async_16_zfill(dst, kv_base + (v ? (int64_t)row * kDQK + 256 * rank + 8 * lane : 0), v ? 16u : 0u);
-        }
-        for (int g8 = lw; g8 < kBK / 8; g8 += 3) {
-          const int r = 8 * g8 + (lane >> 2);
-          const uint32_t kr = (uint32_t)lane & 3u;
-          const int row = ring_rows[slot * kBK + r];
-          const bool v = row >= 0;
-          const uint32_t dst = dst0 + 4 * (kBK * 128) + r * 64 + ((kr ^ (((uint32_t)r >> 1) & 3u)) << 4);
-          cp_async_16_zfill(dst, kv_base + (v ? (int64_t)row * kDQK + 512 + 32 * rank + 8 * kr : 0), v ? 16u : 0u);
+          const uint32_t dst = dst0 + at * kAtom + r * 128 + ((((uint32_t)piece) ^ ((uint32_t)r & 7u)) << 4);
+          cp_async_16_zfill(dst, kv_base + (v ? (int64_t)row * kDQK + 64 * at + 8 * piece : 0), v ? 16u : 0u);
         }
       }
-      cp_async_mbar_arrive(&kv_full[stage]);  // counts once this thread's copies land
+      cp_async_mbar_arrive(&kv_full[stage]);     // counts once this thread's copies land
       if (li == 0) mbar_arrive(&kv_full[stage]);  // releases the masks read by the softmax warps
       failed = bar_red_or(kLoaderBarrier, kLoaders, !ok);
       if (failed) *abort_flag = 1;
     }
-    cp_async_wait_all();
-    // drain: every stage has been consumed by the MMA before the CTA exits
-    if (li == 0 && !*abort_flag) {
-      for (int j = nblk; j < nblk + kStages; ++j)
-        if (!mbar_wait(&kv_empty[j % kStages], ((j / kStages) & 1) ^ 1, a.err)) break;
-    }
+    cp_async_wait_all();  // nothing this thread copies is still in flight at exit
     __syncwarp();
-  } else if (warp == 1 && nblk > 0) {
+  } else if (warp == kMmaWarp && nblk > 0) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t q_base = smem_u32(smem + OFF_Q);
       const uint32_t kv_base = smem_u32(smem + OFF_KV);
-      bool ok = mbar_wait(q_full, 0, a.err);
+      const uint32_t p_base = smem_u32(smem + OFF_P);
+      bool ok = mbar_wait(q_full, 0, a.err, a.wait_ns);
+      tc_fence_after();
       // Issue whichever is ready, PV first (it frees a row stage):
-      //   PV(i) once P(i) is in TMEM;
-      //   QK(j) once block j's rows have landed, S buffer j & 1 is free and
-      //   PV(j-2) has been issued -- so s_full(j), which tracks every earlier
-      //   MMA, also tells the softmax warps that P buffer j & 1 is free.
+      //   PV(i) once P(i) is in shared memory;
+      //   QK(j) once block j's rows have landed and S buffer j & 1 is free.
       int nq = 0, np = 0;  // next block to score / to accumulate
       uint64_t idle_since = 0;
       while (ok && np < nblk) {
@@ -293,15 +313,19 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
           break;
         }
         if (np < nq && mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) {
+          fence_proxy_async_smem();  // P was written by the softmax threads (generic proxy)
           tc_fence_after();
-          const uint32_t vb = kv_base + (np % kStages) * kKVStage;
-          const uint32_t pb = tmem + kTmemP + 64 * (np & 1);  // P_hi at +0, P_lo at +32 (16 keys per 8 columns)
+          const uint32_t vb = kv_base + (np % kStages) * kStageBytes;
+          const uint32_t pb = p_base + (np & 1) * 2 * kPTerm;
 #pragma unroll
           for (int term = 0; term < 2; ++term)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ts_bf16(tmem, pb + 32 * term + 8 * kk, smem_desc(vb + kk * 2048, 8192, 1024, 2), IDESC_PV,
-                          np > 0 || term > 0 || kk > 0);
+            for (int half = 0; half < 2; ++half)
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk)
+                mma_ss<true>(tmem + kTmemO + 256 * half, sw128_desc(pb + term * kPTerm + kk * 32, 16, 1024),
+                             sw128_desc(vb + 4 * half * kAtom + kk * 2048, kAtom, 1024), IDESC_PV,
+                             np > 0 || term > 0 || kk > 0);
           mma_commit(&kv_empty[np % kStages]);
           mma_commit(&o_done[np & 1]);
           ++np;
@@ -311,17 +335,13 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
           fence_proxy_async_smem();  // the rows were written by cp.async (generic proxy)
           tc_fence_after();
           const uint32_t d = tmem + kTmemS + kBK * (nq & 1);
-          const uint32_t kb = kv_base + (nq % kStages) * kKVStage;
+          const uint32_t kb = kv_base + (nq % kStages) * kStageBytes;
 #pragma unroll
-          for (int at = 0; at < 4; ++at)
+          for (int at = 0; at < kNAtoms; ++at)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ss<true>(d, smem_desc(q_base + at * kQLatBytes + kk * 32, 16, 1024, 2),
-                           smem_desc(kb + at * (kBK * 128) + kk * 32, 16, 1024, 2), IDESC_QK, (at | kk) != 0);
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_ss<true>(d, smem_desc(q_base + 4 * kQLatBytes + kk * 32, 16, 512, 4),
-                         smem_desc(kb + 4 * (kBK * 128) + kk * 32, 16, 512, 4), IDESC_QK, true);
+            for (int kk = 0; kk < 4; ++kk)  // K step of 16 dims = 8 TMEM columns of Q
+              mma_ts_bf16(d, tmem + 32 * at + 8 * kk, sw128_desc(kb + at * kAtom + kk * 32, 16, 1024), IDESC_QK,
+                          (at | kk) != 0);
           mma_commit(&s_full[nq & 1]);
           ++nq;
           idle_since = 0;
@@ -329,7 +349,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
           const uint64_t now = globaltimer();
           if (idle_since == 0) {
             idle_since = now;
-          } else if (now - idle_since > kWaitLimitNs) {
+          } else if (now - idle_since > a.wait_ns) {
             raise_error(a.err, kErrTimeout);
             ok = false;
           }
@@ -337,93 +357,53 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         }
       }
       if (!ok) *abort_flag = 1;
+      // drain, also after a failed wait: no MMA still reads shared memory or
+      // writes TMEM when the CTA deallocates and exits
+      mma_commit(mma_drain);
+      mbar_wait(mma_drain, 0, a.err, kDrainLimitNs);
     }
     __syncwarp();
-  } else if (warp >= 4 && nblk > 0) {
-    // ---------------------------------------------------------------- softmax / exchange / epilogue
-    // Eight warps: warp 4+q and warp 8+q share TMEM lane quarter q (heads
-    // 32q .. 32q+31); half g = 0 / 1 takes logits 32g .. 32g+31 of every
-    // block and value dims 128g .. 128g+127 of O.  The two halves of a head
-    // combine their maxima (and at the end their sums) through shared memory
-    // at a 64-thread named barrier, which also carries any failure, so both
-    // warps of a pair always leave together.
-    const int sw = warp - 4, half = sw >> 2, qw = sw & 3;
-    const int h = qw * 32 + lane;  // head row = TMEM lane
-    const int cb = 32 * half;      // this half's first logit of a block
-    const uint32_t t_lane = tmem + ((uint32_t)(qw * 32) << 16);
-    const int pair_bar = kPairBarrier + qw;
-    float2* pair = reinterpret_cast<float2*>(smem + OFF_PAIR);  // [parity][half][head]
-    // X[b][c][h] holds logits 4c .. 4c+3 of head h: a warp's stores of one c
-    // are 512 contiguous bytes
-    const float4* xcol = reinterpret_cast<const float4*>(smem + OFF_X) + h;
-    const uint32_t x_peer = map_peer(smem_u32(smem + OFF_X), peer) + (uint32_t)h * 16u;
-    const uint32_t x_full_peer = map_peer(smem_u32(x_full), peer);
-    const uint32_t x_free_peer = map_peer(smem_u32(x_free), peer);
+  } else if (warp < 4 && nblk > 0) {
+    // ---------------------------------------------------------------- softmax / epilogue
+    // Warp q reads lane quarter q: S rows at lanes 0-15, O rows at lanes
+    // 16-31, head hr = 16q + (lane & 15).  Lanes i and i + 16 share the head:
+    // kh = 0 / 1 takes logits [0, 32) / [32, 64) of every block and value
+    // dims [0, 256) / [256, 512) of O.
+    const int q = warp;
+    const int hr = 16 * q + (lane & 15);
+    const int kh = lane >> 4;
+    const uint32_t t_s = tmem + ((uint32_t)(32 * q) << 16) + kTmemS;
+    const uint32_t t_o = tmem + ((uint32_t)(32 * q) << 16) + kTmemO;
     const float sc = a.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;  // l: this half's share of the sum
+    float m_ref = -INFINITY, l = 0.f;  // l: this thread's share of the head's sum
     bool good = true;
-    for (int j = 0; j < nblk; ++j) {
+    for (int j = 0; j < nblk && good; ++j) {
       const int sb = j & 1;
-      // s_full(j) also means PV(j-2) is complete (it was issued before QK(j)),
-      // so P's buffer sb is free
-      good = good && __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&s_full[sb], (j >> 1) & 1, a.err));
+      const int stage = j % kStages;
+      good = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&s_full[sb], (j >> 1) & 1, a.err, a.wait_ns));
+      if (!good) break;
       uint32_t v[32];
-      if (good) {
-        tc_fence_after();
-        tmem_ld32(t_lane + kTmemS + kBK * sb + cb, v);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[sb]);
-      }
-      // the peer's warps have read my previous block: its receive area is free
-      if (j >= 1) good = good && __all_sync(0xffffffffu, mbar_wait_cluster(x_free, (j - 1) & 1, a.err));
-      if (good) {
-        // my partial logits -> the peer's receive area, counted on its x_full
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_async_v4(x_peer + (8 * half + c) * 2048, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3],
-                      x_full_peer);
-      }
-      good = good && __all_sync(0xffffffffu, mbar_wait_cluster(x_full, j & 1, a.err));
-      float s[32];
-      if (good) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 pv4 = xcol[(8 * half + c) * 128];
-          s[4 * c + 0] = __uint_as_float(v[4 * c]) + pv4.x;
-          s[4 * c + 1] = __uint_as_float(v[4 * c + 1]) + pv4.y;
-          s[4 * c + 2] = __uint_as_float(v[4 * c + 2]) + pv4.z;
-          s[4 * c + 3] = __uint_as_float(v[4 * c + 3]) + pv4.w;
-        }
-        // re-arm my receive area for block j+1, then tell the peer this
-        // warp is done with it: the peer stores block j+1 only after all
-        // eight signals, the re-arming warp's among them
-        if (sw == 0 && lane == 0 && j + 1 < nblk) mbar_arrive_expect_tx(x_full, kXBytes);
-        __syncwarp();  // every lane's reads of X precede the signal
-        if (lane == 0) mbar_arrive_remote_relaxed(x_free_peer);
-      }
+      tc_fence_after();
+      tmem_ld16x2_32<32>(t_s + kBK * sb, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
       // validity of the block's rows (published before the stage completed)
-      good = good && __all_sync(0xffffffffu, mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, a.err));
+      good = __all_sync(0xffffffffu, mbar_wait(&kv_full[stage], (j / kStages) & 1, a.err, a.wait_ns));
+      if (!good) break;
+      const uint32_t m32 = (uint32_t)(ring_mask[j] >> (32 * kh));
+      float s[32];
       float mraw = -INFINITY, mneg = INFINITY;
-      if (good) {
-        const uint32_t m32 = (uint32_t)(ring_mask[j] >> cb);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const bool on = (m32 >> i) & 1u;
-          s[i] = on ? s[i] : -INFINITY;
-          mraw = fmaxf(mraw, s[i]);
-          mneg = fminf(mneg, on ? s[i] : INFINITY);
-        }
-        pair[((j & 1) * 2 + half) * 128 + h] = make_float2(mraw, mneg);
+      for (int i = 0; i < 32; ++i) {
+        const bool on = (m32 >> i) & 1u;
+        s[i] = on ? __uint_as_float(v[i]) : -INFINITY;
+        mraw = fmaxf(mraw, s[i]);
+        mneg = fminf(mneg, on ? s[i] : INFINITY);
       }
-      if (bar_red_or(pair_bar, 64, !good)) {  // either half failed: both leave
-        good = false;
-        break;
-      }
-      const float2 other = pair[((j & 1) * 2 + (half ^ 1)) * 128 + h];
-      mraw = fmaxf(mraw, other.x);
-      mneg = fminf(mneg, other.y);
+      mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
+      mneg = fminf(mneg, __shfl_xor_sync(0xffffffffu, mneg, 16));
       // scale <= 0 (allowed, if odd): the largest scaled logit comes from the smallest raw one
       const float mblk = mraw == -INFINITY ? -INFINITY : (sc > 0.f ? mraw * sc : mneg * sc);
       const bool move = mblk > m_ref + kRescaleThreshold;
@@ -446,25 +426,33 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
         pk[i] = hb;
         pl[i] = *reinterpret_cast<const uint32_t*>(&lo);
       }
-      // P_hi: columns kTmemP + 64 sb + [0, 32), P_lo: + [32, 64); 16 columns per half
-      tmem_st16(t_lane + kTmemP + 64 * sb + 16 * half, pk);
-      tmem_st16(t_lane + kTmemP + 64 * sb + 32 + 16 * half, pl);
-      // TMEM loads/stores are warp-wide: if any head of the warp moved its
-      // maximum, the warp rescales its half of O (alpha = 1 leaves a row
-      // exact), once PV(j-1) -- the last writer of O -- has completed
-      if (j >= 1 && __any_sync(0xffffffffu, move && m_ref != -INFINITY)) {
-        good = __all_sync(0xffffffffu, mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err));
-        if (good) {
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_lane + 128 * half + 32 * c, o);
-            tmem_ld_wait();
+      // P(j) into buffer j & 1 (PV(j-2), its last reader, completed before
+      // QK(j) could start): row hr, this thread's four 16-byte pieces of keys
+      // [32 kh, 32 kh + 32), each term in its own 128-byte-swizzled tile
+      uint8_t* prow = smem + OFF_P + sb * 2 * kPTerm + hr * 128;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(t_lane + 128 * half + 32 * c, o);
-          }
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t off = (((uint32_t)(4 * kh + c)) ^ ((uint32_t)hr & 7u)) << 4;
+        *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(prow + kPTerm + off) =
+            make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+      }
+      fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+      // TMEM loads/stores are warp-wide: if any head of the warp moved its
+      // maximum, the warp rescales its heads' rows of O (alpha = 1 leaves a
+      // row exact), once PV(j-1) -- the last writer of O -- has completed
+      if (j >= 1 && __any_sync(0xffffffffu, move && m_ref != -INFINITY)) {
+        good = __all_sync(0xffffffffu, mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err, a.wait_ns));
+        if (!good) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          tmem_ld16x2_32<256>(t_o + 32 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st16x2_32<256>(t_o + 32 * c, o);
         }
       }
       l = l * alpha + psum;
@@ -472,77 +460,63 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq_lat, const __grid_constan
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (good && lane == 0) mbar_arrive(&p_full[sb]);
+      if (lane == 0) mbar_arrive(&p_full[sb]);
     }
-    // epilogue: O / l for this half's 128 value dims.  tcgen05.ld is
-    // warp-wide, so a warp with any valid head loads; only the stores test h < H.
-    good = good && __all_sync(0xffffffffu, mbar_wait(&o_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.err));
-    // the sums go through the parity the last block did not use: its maxima
-    // may still be read by the slower warp of the pair
-    const int ep = nblk & 1;
-    pair[(ep * 2 + half) * 128 + h] = make_float2(l, 0.f);
-    const bool failed = bar_red_or(pair_bar, 64, !good);  // also publishes this half's sum
-    if (!failed) {
-      l += pair[(ep * 2 + (half ^ 1)) * 128 + h].x;
+    // epilogue: O / l for this thread's head and 256 value dims
+    good = good && __all_sync(0xffffffffu, mbar_wait(&o_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.err,
+                                                     a.wait_ns));
+    const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
+    if (good) {
       tc_fence_after();
-      // O / l (or the raw partial) of this warp's 32 heads x 128 value dims,
-      // 32 dims at a time: TMEM -> registers (a row per lane) -> a swizzled
-      // 32 x 32 tile in shared memory -> rows back out, four rows of 128
-      // bytes per warp store instead of 32 scattered 16-byte pieces.  The
-      // tiles use the first row stage: every MMA that read it completed
-      // before the last PV, which this warp has seen complete.
-      float* tile = reinterpret_cast<float*>(smem + OFF_KV) + sw * 1024;
-      const float m_nat = m_ref * kLn2;
       const bool partial = a.splits > 1;
-      const float inv = partial ? 1.f : (l > 0.f ? 1.f / l : 0.f);
-      const int rsub = lane >> 3, k4 = lane & 7;  // read-back: row 4i + rsub, dims 4 k4 .. 4 k4 + 3
+      const float inv = partial ? 1.f : (lt > 0.f ? 1.f / lt : 0.f);
+      const int head = kHG * g + hr;
+      const bool mine = head < a.H;
+      const int64_t orow = partial ? (((int64_t)t * a.splits + sp) * a.H + head) : ((int64_t)t * a.H + head);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 8; ++c) {
         uint32_t o[32];
-        tmem_ld32(t_lane + 128 * half + 32 * c, o);
+        tmem_ld16x2_32<256>(t_o + 32 * c, o);
         tmem_ld_wait();
-        __syncwarp();  // the previous chunk's tile has been read back
+        if (!mine) continue;
+        const int dim = 256 * kh + 32 * c;
+        if (partial || a.out_f32) {
+          float* dst = (partial ? a.part_o : reinterpret_cast<float*>(a.out)) + orow * kDV + dim;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)  // 16-byte piece k of row `lane`, XOR-swizzled by the row
-          *reinterpret_cast<float4*>(tile + lane * 32 + ((k ^ (lane & 7)) << 2)) =
-              make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
-                          __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
-        __syncwarp();
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(dst)[i] =
+                make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                            __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+        } else {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + orow * kDV + dim;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = 4 * i + rsub;  // head qw*32 + r
-          const float4 v4 = *reinterpret_cast<const float4*>(tile + r * 32 + ((k4 ^ (r & 7)) << 2));
-          const int hr = qw * 32 + r;
-          if (hr >= a.H) continue;
-          const int dim = 256 * rank + 128 * half + 32 * c + 4 * k4;
-          if (partial) {
-            const int64_t prow = ((int64_t)t * a.splits + sp) * a.H + hr;
-            *reinterpret_cast<float4*>(a.part_o + prow * kDV + dim) = v4;
-          } else if (a.out_f32) {
-            *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + ((int64_t)t * a.H + hr) * kDV + dim) = v4;
-          } else {
-            const __nv_bfloat162 p0 = __floats2bfloat162_rn(v4.x, v4.y), p1 = __floats2bfloat162_rn(v4.z, v4.w);
-            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)t * a.H + hr) * kDV + dim) =
-                make_uint2(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1));
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(o[8 * i + 2 * k]) * inv,
+                                                               __uint_as_float(o[8 * i + 2 * k + 1]) * inv);
+              w[k] = *reinterpret_cast<const uint32_t*>(&p2);
+            }
+            reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
-      if (h < a.H && rank == 0 && half == 0) {
+      if (mine && kh == 0) {
+        const float m_nat = m_ref * kLn2;
         if (partial)
-          a.part_ml[((int64_t)t * a.splits + sp) * a.H + h] = make_float2(m_nat, l);
+          a.part_ml[orow] = make_float2(m_nat, lt);
         else if (a.lse)
-          a.lse[(int64_t)t * a.H + h] = m_nat + logf(l);
+          a.lse[orow] = m_nat + logf(lt);
       }
     } else {
       *abort_flag = 1;
     }
     __syncwarp();
   }
-  if (threadIdx.x == 0 && nblk == 0) mbar_wait(q_full, 0, a.err);  // no copy in flight at exit
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // no peer still writes into this CTA's shared memory
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -603,10 +577,14 @@ k_combine(int H, int splits, const float* __restrict__ part_o, const float2* __r
   if (lse && tid == 0) lse[(int64_t)t * H + h] = M + logf(L);
 }
 
-int attn_splits(int T, int K) {
-  const int clusters = 74;  // 148 SMs / 2
-  if (T >= clusters) return 1;
-  const int want = clusters / T;
+constexpr int kSplitSms = 148;  // SMs the split decision fills (a host-only constant: no device query)
+
+int head_groups(int H) { return (H + kHG - 1) / kHG; }
+
+int attn_splits(int T, int K, int H) {
+  const int units = T * head_groups(H);
+  if (units >= kSplitSms) return 1;
+  const int want = kSplitSms / units;
   const int most = (K + kBK - 1) / kBK;
   return want < 1 ? 1 : (want < most ? want : most);
 }
@@ -616,36 +594,10 @@ int keys_per_split(int K, int splits) {
   return (ks + kBK - 1) / kBK * kBK;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// bf16 [rows, 576] map with a box of box_x x box_y and the given swizzle.
-bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_x, uint32_t box_y,
-                  CUtensorMapSwizzle sw) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)kDQK, rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)kDQK * 2};
-  const cuuint32_t box[2] = {box_x, box_y};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 size_t sparse_mla_partials_bytes(int T, int K, int H) {
-  const int splits = attn_splits(T, K);
+  const int splits = attn_splits(T, K, H);
   if (splits == 1) return 0;
   return (size_t)T * splits * H * (kDV * sizeof(float) + sizeof(float2));
 }
@@ -654,15 +606,12 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, cons
                               const __nv_bfloat16* kv, const int32_t* idx, int K, int H, float scale, void* out,
                               bool out_f32, float* lse, void* partials, uint32_t* err, cudaStream_t st) {
   const int T = s.num_tokens;
-  int splits = attn_splits(T, K);
+  const int G = head_groups(H);
+  int splits = attn_splits(T, K, H);
   const int ks = keys_per_split(K, splits);
   splits = (K + ks - 1) / ks;
   float* part_o = reinterpret_cast<float*>(partials);
   float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)T * splits * H * kDV);
-  CUtensorMap tq_lat, tq_rope;
-  if (!make_map_576(&tq_lat, q, (uint64_t)T * H, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_576(&tq_rope, q, (uint64_t)T * H, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
-    return cudaErrorInvalidValue;
   static thread_local int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -671,13 +620,16 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, cons
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  AttnArgs a{s, tm, kv, idx, K, H, ks, splits, tm_early, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err};
-  cudaError_t e = launch_pdl("sparse_mla", k_sparse_mla_tc, dim3(2 * T * splits), dim3(kThreads), (size_t)SMEM_BYTES, st, tq_lat, tq_rope,
-                             a);
+  AttnArgs a{s, tm, q, kv, idx, K, H, G, ks, splits, tm_early, scale * kLog2e, out, out_f32, lse, part_o, part_ml,
+             err, wait_limit_ns()};
+  const int64_t ctas = (int64_t)T * G * splits;
+  if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
+  cudaError_t e = launch_pdl("sparse_mla", k_sparse_mla_tc, dim3((unsigned)ctas), dim3(kThreads), (size_t)SMEM_BYTES,
+                             st, a);
   if (e == cudaSuccess) e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
-  e = launch_pdl("sparse_mla_combine", k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o, (const float2*)part_ml,
-                 tm.pos, out, out_f32, lse);
+  e = launch_pdl("sparse_mla_combine", k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o,
+                 (const float2*)part_ml, tm.pos, out, out_f32, lse);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }

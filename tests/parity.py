@@ -20,7 +20,7 @@ import numpy as np
 import torch
 
 from oracle import dsa_oracle as O
-from sparse_indexed_attention_b200.workloads import Workload, bits16
+from dsa_workloads import Workload, bits16
 
 SCORE_TOL = 1e-2
 TIE_TOL = 1e-3

@@ -1,7 +1,7 @@
 """Workload shapes used by the GPU parity tests: the five measured workloads
 (some at full size) and reduced versions that the oracle finishes in seconds
 while still spanning several tiles and ragged tails."""
-from sparse_indexed_attention_b200.workloads import CONFIGS
+from dsa_workloads import CONFIGS
 
 SMALL = {
     "tiny_prefill_1k": CONFIGS["tiny_prefill_1k"],
@@ -22,7 +22,7 @@ _cache: dict = {}
 
 def workload(spec):
     """make_workload with a small host-side cache (full-size workloads take seconds to draw)."""
-    from sparse_indexed_attention_b200.workloads import make_workload
+    from dsa_workloads import make_workload
     if spec not in _cache:
         if len(_cache) >= 2:
             _cache.pop(next(iter(_cache)))

@@ -27,7 +27,7 @@ def _rank_main(rank, world, port, q):
                       LOCAL_RANK=str(rank))
     sys.path.insert(0, ROOT)
     import bench
-    from sparse_indexed_attention_b200.workloads import CONFIGS, make_workload
+    from dsa_workloads import CONFIGS, make_workload
     import torch.distributed as dist
     w, r, _ = bench.dist_setup(None, backend="gloo")
     try:

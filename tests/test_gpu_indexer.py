@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from oracle import dsa_oracle as O
-from sparse_indexed_attention_b200.workloads import bits16, to_device
+from dsa_workloads import bits16, to_device
 from tests import parity as P
 from tests.specs import FULL, SMALL, workload as make_workload
 

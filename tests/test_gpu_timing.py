@@ -3,7 +3,7 @@ per kernel of a fused call while enabled, and a call with identical results."""
 import pytest
 import torch
 
-from sparse_indexed_attention_b200.workloads import to_device
+from dsa_workloads import to_device
 from tests.specs import SMALL, workload as make_workload
 
 pytestmark = pytest.mark.gpu

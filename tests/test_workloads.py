@@ -2,7 +2,7 @@
 import numpy as np
 import torch
 
-from sparse_indexed_attention_b200.workloads import CONFIGS, make_workload
+from dsa_workloads import CONFIGS, make_workload
 
 SMALL = {
     "prefill": CONFIGS["tiny_prefill_1k"].scaled(ctx=(300, 300), topk=64),

@@ -3,9 +3,10 @@ allocate device memory (a plugin whose host framework owns every device
 allocation, or code running where cudaMalloc is not allowed).  Instead of a
 caller workspace it uses a fixed scratch array inside the library.
 
-Its results must be those of dsa_sparse_mla_fwd on the same inputs; two
-calls in a row check that the shared array carries no state from one call
-into the next.  The file sorts last so that a run stopping at the first
+Its results must be those of dsa_sparse_mla_fwd on the same inputs and
+match the oracle; two calls in a row check that the shared array carries no
+state from one call into the next, and dsa_check_error_noalloc reads the
+array's error word.  The file sorts last so that a run stopping at the first
 failure has already run every other test."""
 import ctypes
 
@@ -14,7 +15,8 @@ import pytest
 import torch
 
 import sparse_indexed_attention_b200 as dsa
-from sparse_indexed_attention_b200.workloads import to_device
+from dsa_workloads import bits16, to_device
+from oracle import dsa_oracle as O
 from tests import parity as P
 from tests.specs import SMALL, workload as make_workload
 
@@ -46,12 +48,18 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         got_out, got_lse = dsa.dsa_sparse_mla_fwd_noalloc(d.seqs, d.q, d.kv, idx, wl.scale, out_dtype=torch.float32)
         torch.cuda.synchronize()
         assert dsa.dsa_check_error(ws) == dsa.DSA_OK
+        assert dsa.dsa_check_error_noalloc() == dsa.DSA_OK
         ref = ref_out.double().cpu().numpy()
         rms = float(np.sqrt(np.mean(ref * ref)))
         err = float(np.abs(got_out.double().cpu().numpy() - ref).max())
         assert err <= P.OUT_TOL * rms, f"{spec.name}: max err {err:.3e} vs rms {rms:.3e}"
         lerr = (got_lse.double() - ref_lse.double()).abs().max().item()
         assert lerr <= P.LSE_TOL
+        # and the oracle on the same index lists
+        tokens = np.arange(wl.T)
+        o_out, o_lse = O.sparse_mla(P.oracle_seqs(wl), bits16(wl.q), bits16(wl.kv), idx.cpu().numpy(), wl.scale,
+                                    tokens=tokens)
+        P.assert_attention_close(got_out, got_lse, o_out, o_lse)
 
 
 def test_noalloc_rejects_geometry_beyond_its_scratch():
