@@ -367,7 +367,8 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
             uint32_t v0[32], v1[32];
             tmem_ld32(t_lane + acc * C::N + k * 64, v0);
             tmem_ld32(t_lane + acc * C::N + k * 64 + 32, v1);
-            tmem_ld_wait();
+            tmem_ld_wait_regs(v0);
+            tmem_ld_wait_regs(v1);
             if (k == TG - 1) {  // every TMEM read of this accumulator is complete
               tc_fence_before();
               __syncwarp();

@@ -16,9 +16,13 @@
 // tensor memory holds, side by side:
 //   lanes 0-15 of each quarter:  Q (64 heads x 576 bf16, 288 columns) -- the
 //                                A operand of S = Q K^T, read from TMEM --
-//                                and two logit buffers S (64 columns each);
+//                                and S as three partial sums (64 columns
+//                                each: K dims split by 64-dim atom, atom a
+//                                into partial a % 3);
 //   lanes 16-31:                 O (64 heads x 512 fp32, all 512 columns).
-// Shared memory then holds only rows and probabilities:
+// The three partials are independent accumulation chains that the tensor
+// core overlaps: one chain of 36 small MMAs into a single S is bound by the
+// latency of each MMA, not by its arithmetic.
 //   * four loader warps resolve every selected row of the slice up front
 //     (index list -> page table -> pool row, all loads independent) and copy
 //     the rows block by block (64 rows, two stages) with 16-byte cp.async
@@ -35,8 +39,13 @@
 //     fp32 value), and PV runs once per term: one bf16 term alone misses the
 //     accuracy bound on rows that a few selected keys dominate (relative
 //     error up to 2^-8 of the spread of V, measured on the 1024-token prefill).
+//   * the query tile arrives by TMA in the second row stage and the softmax
+//     warps move it into TMEM before that stage's first rows; the output rows
+//     leave through shared memory with one bulk copy per head row.
 // Decode batches split the index list over several CTAs per (token, head
 // group); k_combine merges their partials (log-sum-exp weights).
+#include <cudaTypedefs.h>
+
 #include "sm100.cuh"
 
 namespace dsa {
@@ -51,23 +60,28 @@ constexpr int kAtom = 64 * 128;               // 64 rows x 64 bf16 dims, 128-byt
 constexpr int kNAtoms = kDQK / 64;            // 9: eight latent atoms + the rope atom
 constexpr int kStageBytes = kNAtoms * kAtom;  // 73728
 constexpr int kStages = 2;
+constexpr int kSParts = 3;                    // partial sums of S
 constexpr int kPTerm = kHG * kBK * 2;         // one bf16 term of P: 64 heads x 64 rows, 128-byte swizzle
 constexpr int kLoaders = 128;                 // warps 4-7
 constexpr int kLoaderBarrier = 1;             // named barrier of the loader warps
-constexpr int OFF_KV = 0;
-constexpr int OFF_P = OFF_KV + kStages * kStageBytes;     // [2 buffers][hi, lo]
+constexpr int OFF_KV = 0;                     // stage 1 holds the query tile until it is in TMEM
+constexpr int OFF_P = OFF_KV + kStages * kStageBytes;     // [2 buffers][hi, lo]; index staging at first
 constexpr int OFF_ROWS = OFF_P + 2 * 2 * kPTerm;          // [block][64] pool rows of the slice (-1 = masked)
 constexpr int OFF_MASK = OFF_ROWS + kMaxK * 4;            // [block] 64-bit validity masks
 constexpr int OFF_BAR = OFF_MASK + (kMaxK / kBK) * 8;
-constexpr int kNBars = 14;
+constexpr int kNBars = 13;
 constexpr int OFF_MISC = OFF_BAR + kNBars * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;          // slack for 1024-byte alignment
 constexpr int kThreads = 288;  // warps 0-3 softmax + epilogue, 4-7 load, 8 issues MMAs and owns TMEM
 constexpr int kMmaWarp = 8;
+constexpr int kOutRowF32 = kDV * 4 + 16;      // epilogue staging row (padded: no bank conflicts)
+constexpr int kOutRowBf16 = kDV * 2 + 16;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 static_assert(kStageBytes % 1024 == 0 && OFF_P % 1024 == 0 && kPTerm % 1024 == 0, "swizzle atoms need 1024-B alignment");
+static_assert(kHG * kOutRowF32 <= kStages * kStageBytes, "epilogue staging fits in the row stages");
+static_assert(2 * kMaxK * 4 <= 2 * 2 * kPTerm, "index staging fits in the P buffers");
 // TMEM map: lane offset << 16 | column
-constexpr uint32_t kTmemS = 288;             // S buffers at columns 288 and 352 of lanes 0-15 (Q at 0)
+constexpr uint32_t kTmemS = 288;             // S partials at columns 288, 352, 416 of lanes 0-15 (Q at 0)
 constexpr uint32_t kTmemO = 16u << 16;       // O: lanes 16-31, columns 0-511
 
 constexpr uint32_t IDESC_QK = make_idesc_major(true, kHG, kBK, 0, 0);  // S = Q K^T, both K-major
@@ -95,10 +109,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   return smem_desc(saddr, lbo, sbo, 2);
 }
 
+// A descriptor moved by `bytes` (a compile-time offset inside the operand):
+// the start address sits in the low 14 bits as address / 16 and stays below
+// 2^14 for any shared-memory address, so the move is one add.  The issuing
+// thread builds each operand's base descriptor once per block.
+__device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t bytes) { return base + (bytes >> 4); }
+
 struct AttnArgs {
   SeqsDev s;
   TokenMap tm;
-  const __nv_bfloat16* q;   // [T, H, 576]
   const __nv_bfloat16* kv;  // latent pool [rows, 576]
   const int32_t* idx;
   int K, H, G, ks, splits;  // G head groups of 64; ks selected slots per split
@@ -113,53 +132,44 @@ struct AttnArgs {
   uint64_t wait_ns;         // limit of each wait for another role's progress
 };
 
-// Query rows of the CTA's 64 heads into TMEM (A operand of S = Q K^T): warp q
-// writes heads 16q .. 16q+15, thread i (i < 16) dims [0, 288) and thread
-// i + 16 dims [288, 576) of head 16q + i, as bf16 pairs (column c = dims 2c,
-// 2c + 1).  Heads at or past H are zero.  Two rounds of loads, each issued
-// together.
-__device__ __forceinline__ void load_query_to_tmem(const AttnArgs& a, int t, int g, uint32_t t_q, int lane, int q) {
-  const int hr = 16 * q + (lane & 15), half = lane >> 4;
-  const int head = kHG * g + hr;
-  const bool valid = head < a.H;
-  const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)t * a.H + (valid ? head : 0)) * kDQK + 288 * half);
+// The query tile (64 heads x 576 dims, 128-byte-swizzled atoms in shared
+// memory) into TMEM as the A operand of S = Q K^T: warp q writes heads
+// 16q .. 16q+15, thread i (i < 16) dims [0, 288) and thread i + 16 dims
+// [288, 576) of head 16q + i, as bf16 pairs (column c = dims 2c, 2c + 1).
+// Heads at or past H are zero.
+__device__ __forceinline__ void query_to_tmem(const uint8_t* qs, bool valid, int hr, int half, uint32_t t_q) {
 #pragma unroll
-  for (int round = 0; round < 2; ++round) {
-    constexpr int kChunks = 5;  // chunk = 32 dims = 64 bytes = 16 TMEM columns
-    uint4 v[kChunks * 4];
+  for (int chunk = 0; chunk < 9; ++chunk) {  // 32 dims = 4 pieces of 16 bytes = 16 TMEM columns
+    uint32_t r[16];
 #pragma unroll
-    for (int c = 0; c < kChunks; ++c) {
-      const int chunk = round * kChunks + c;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        v[4 * c + k] = (valid && chunk < 9) ? __ldg(src + 4 * chunk + k) : make_uint4(0u, 0u, 0u, 0u);
+    for (int k = 0; k < 4; ++k) {
+      const int d = 288 * half + 32 * chunk + 8 * k;  // first dim of the piece
+      const int at = d >> 6, piece = (d & 63) >> 3;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) v = *reinterpret_cast<const uint4*>(qs + at * kAtom + hr * 128 + ((piece ^ (hr & 7)) << 4));
+      r[4 * k] = v.x;
+      r[4 * k + 1] = v.y;
+      r[4 * k + 2] = v.z;
+      r[4 * k + 3] = v.w;
     }
-#pragma unroll
-    for (int c = 0; c < kChunks; ++c) {
-      const int chunk = round * kChunks + c;
-      if (chunk >= 9) break;
-      const uint32_t r[16] = {v[4 * c].x,     v[4 * c].y,     v[4 * c].z,     v[4 * c].w,
-                              v[4 * c + 1].x, v[4 * c + 1].y, v[4 * c + 1].z, v[4 * c + 1].w,
-                              v[4 * c + 2].x, v[4 * c + 2].y, v[4 * c + 2].z, v[4 * c + 2].w,
-                              v[4 * c + 3].x, v[4 * c + 3].y, v[4 * c + 3].z, v[4 * c + 3].w};
-      tmem_st16x2_16<144>(t_q + 16 * chunk, r);
-    }
+    tmem_st16x2_16<144>(t_q + 16 * chunk, r);
   }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-k_sparse_mla_tc(const AttnArgs a) {
+k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* q_full = bars + 0;     // the query rows are in TMEM (one arrival per softmax warp)
-  uint64_t* kv_full = bars + 1;    // [kStages] rows of block j (stage j % 2) landed
-  uint64_t* kv_empty = bars + 3;   // [kStages] PV of the stage's block completed
-  uint64_t* s_full = bars + 5;     // [2] S of block j (buffer j & 1) in TMEM
-  uint64_t* s_empty = bars + 7;    // [2] S buffer read by every softmax warp
-  uint64_t* p_full = bars + 9;     // [2] P of block j (buffer j & 1) in shared memory
-  uint64_t* o_done = bars + 11;    // [2] PV of block i (parity by i & 1) has completed
-  uint64_t* mma_drain = bars + 13; // every MMA this CTA issued has completed
+  uint64_t* q_tma = bars + 0;      // the query tile has landed in stage 1
+  uint64_t* q_full = bars + 1;     // the query is in TMEM and stage 1 is free (one arrival per softmax warp)
+  uint64_t* kv_full = bars + 2;    // [kStages] rows of block j (stage j % 2) landed
+  uint64_t* kv_empty = bars + 4;   // [kStages] PV of the stage's block completed
+  uint64_t* s_full = bars + 6;     // S of block j in TMEM
+  uint64_t* s_empty = bars + 7;    // S read by every softmax warp
+  uint64_t* p_full = bars + 8;     // [2] P of block j (buffer j & 1) in shared memory
+  uint64_t* o_done = bars + 10;    // [2] PV of block i (parity by i & 1) has completed
+  uint64_t* mma_drain = bars + 12; // every MMA this CTA issued has completed
   int32_t* ring_rows = reinterpret_cast<int32_t*>(smem + OFF_ROWS);
   uint64_t* ring_mask = reinterpret_cast<uint64_t*>(smem + OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
@@ -173,14 +183,15 @@ k_sparse_mla_tc(const AttnArgs a) {
   const int kend = min(a.K, kbeg + a.ks);
 
   if (threadIdx.x == 0) {
+    mbar_init(q_tma, 1);
     mbar_init(q_full, 4);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&kv_full[i], kLoaders + 1);  // every loader's copies + the mask's publisher
       mbar_init(&kv_empty[i], 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
       mbar_init(&p_full[i], 4);  // one arrival per softmax warp
       mbar_init(&o_done[i], 1);
     }
@@ -196,12 +207,11 @@ k_sparse_mla_tc(const AttnArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp < 4) {  // q is an input of the call: its load overlaps the wait below
-    load_query_to_tmem(a, t, g, tmem + ((uint32_t)(32 * warp) << 16), lane, warp);
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(q_full);
+  if (threadIdx.x == 0) {  // q is an input of the call: its load overlaps the wait below
+    prefetch_tmap(&tq);
+    mbar_arrive_expect_tx(q_tma, kStageBytes);
+    for (int at = 0; at < kNAtoms; ++at)
+      tma_load_2d(smem + OFF_KV + kStageBytes + at * kAtom, &tq, q_tma, 64 * at, t * a.H + kHG * g);
   }
   // the token map can be read before the wait when it does not come from
   // the kernel just before; the index lists always do
@@ -227,13 +237,12 @@ k_sparse_mla_tc(const AttnArgs a) {
     const int lw = warp - 4;           // loader warp 0 .. 3
     // Pool rows of every block of the slice, resolved up front in three
     // passes whose loads are all independent: the index list, then the page
-    // ids (both staged by cp.async in the row stages, which the first row
-    // copies overwrite only after the last pass), then rows and masks
-    // (row -1 = masked).
+    // ids (both staged by cp.async in the P buffers, which are first written
+    // after block 0 has been scored), then rows and masks (row -1 = masked).
     {
       const int nkeys = kend - kbeg;
-      int32_t* s_sidx = reinterpret_cast<int32_t*>(smem + OFF_KV);
-      int32_t* s_page = reinterpret_cast<int32_t*>(smem + OFF_KV + kStageBytes);
+      int32_t* s_sidx = reinterpret_cast<int32_t*>(smem + OFF_P);
+      int32_t* s_page = s_sidx + kMaxK;
       const int32_t* idx_row = a.idx + (int64_t)t * a.K + kbeg;
       for (int k = li; k < nkeys; k += kLoaders) cp_async_4(&s_sidx[k], idx_row + k);
       cp_async_wait_all();
@@ -273,7 +282,9 @@ k_sparse_mla_tc(const AttnArgs a) {
     bool failed = bar_red_or(kLoaderBarrier, kLoaders, false);
     for (int j = 0; j < nblk && !failed; ++j) {
       const int stage = j % kStages;
-      const bool ok = mbar_wait(&kv_empty[stage], ((j / kStages) & 1) ^ 1, a.err, a.wait_ns);
+      bool ok = mbar_wait(&kv_empty[stage], ((j / kStages) & 1) ^ 1, a.err, a.wait_ns);
+      // stage 1 first holds the query tile
+      if (j == 1) ok = ok && mbar_wait(q_full, 0, a.err, a.wait_ns);
       if (ok) {
         // task = (atom, quad of rows): the warp's 32 copies fill 512
         // contiguous bytes of the atom (no bank conflict) from four 128-byte
@@ -304,7 +315,7 @@ k_sparse_mla_tc(const AttnArgs a) {
       tc_fence_after();
       // Issue whichever is ready, PV first (it frees a row stage):
       //   PV(i) once P(i) is in shared memory;
-      //   QK(j) once block j's rows have landed and S buffer j & 1 is free.
+      //   QK(j) once block j's rows have landed and S(j-1) has been read.
       int nq = 0, np = 0;  // next block to score / to accumulate
       uint64_t idle_since = 0;
       while (ok && np < nblk) {
@@ -315,34 +326,38 @@ k_sparse_mla_tc(const AttnArgs a) {
         if (np < nq && mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) {
           fence_proxy_async_smem();  // P was written by the softmax threads (generic proxy)
           tc_fence_after();
-          const uint32_t vb = kv_base + (np % kStages) * kStageBytes;
-          const uint32_t pb = p_base + (np & 1) * 2 * kPTerm;
+          const uint64_t vd = sw128_desc(kv_base + (np % kStages) * kStageBytes, kAtom, 1024);
+          const uint64_t pd = sw128_desc(p_base + (np & 1) * 2 * kPTerm, 16, 1024);
+          const bool acc0 = np > 0;
 #pragma unroll
           for (int term = 0; term < 2; ++term)
 #pragma unroll
-            for (int half = 0; half < 2; ++half)
+            for (int kk = 0; kk < kBK / 16; ++kk)
 #pragma unroll
-              for (int kk = 0; kk < kBK / 16; ++kk)
-                mma_ss<true>(tmem + kTmemO + 256 * half, sw128_desc(pb + term * kPTerm + kk * 32, 16, 1024),
-                             sw128_desc(vb + 4 * half * kAtom + kk * 2048, kAtom, 1024), IDESC_PV,
-                             np > 0 || term > 0 || kk > 0);
+              for (int half = 0; half < 2; ++half)  // the halves alternate: independent chains
+                mma_ss<true>(tmem + kTmemO + 256 * half, desc_at(pd, term * kPTerm + kk * 32),
+                             desc_at(vd, 4 * half * kAtom + kk * 2048), IDESC_PV, acc0 || term > 0 || kk > 0);
           mma_commit(&kv_empty[np % kStages]);
           mma_commit(&o_done[np & 1]);
           ++np;
           idle_since = 0;
         } else if (nq < nblk && nq < np + 2 && mbar_test_wait(&kv_full[nq % kStages], (nq / kStages) & 1) &&
-                   mbar_test_wait(&s_empty[nq & 1], ((nq >> 1) & 1) ^ 1)) {
+                   (nq == 0 || mbar_test_wait(s_empty, (nq - 1) & 1))) {
           fence_proxy_async_smem();  // the rows were written by cp.async (generic proxy)
           tc_fence_after();
-          const uint32_t d = tmem + kTmemS + kBK * (nq & 1);
-          const uint32_t kb = kv_base + (nq % kStages) * kStageBytes;
+          const uint64_t kd = sw128_desc(kv_base + (nq % kStages) * kStageBytes, 16, 1024);
+          // atom at -> partial at % 3; consecutive MMAs go to different partials
 #pragma unroll
-          for (int at = 0; at < kNAtoms; ++at)
+          for (int grp = 0; grp < kNAtoms / kSParts; ++grp)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // K step of 16 dims = 8 TMEM columns of Q
-              mma_ts_bf16(d, tmem + 32 * at + 8 * kk, sw128_desc(kb + at * kAtom + kk * 32, 16, 1024), IDESC_QK,
-                          (at | kk) != 0);
-          mma_commit(&s_full[nq & 1]);
+#pragma unroll
+              for (int part = 0; part < kSParts; ++part) {
+                const int at = kSParts * grp + part;
+                mma_ts_bf16(tmem + kTmemS + kBK * part, tmem + 32 * at + 8 * kk, desc_at(kd, at * kAtom + kk * 32),
+                            IDESC_QK, (grp | kk) != 0);
+              }
+          mma_commit(s_full);
           ++nq;
           idle_since = 0;
         } else {
@@ -363,62 +378,95 @@ k_sparse_mla_tc(const AttnArgs a) {
       mbar_wait(mma_drain, 0, a.err, kDrainLimitNs);
     }
     __syncwarp();
-  } else if (warp < 4 && nblk > 0) {
+  } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax / epilogue
-    // Warp q reads lane quarter q: S rows at lanes 0-15, O rows at lanes
-    // 16-31, head hr = 16q + (lane & 15).  Lanes i and i + 16 share the head:
-    // kh = 0 / 1 takes logits [0, 32) / [32, 64) of every block and value
-    // dims [0, 256) / [256, 512) of O.
+    // Warp q reads lane quarter q: Q and S rows at lanes 0-15, O rows at
+    // lanes 16-31, head hr = 16q + (lane & 15).  Lanes i and i + 16 share the
+    // head: kh = 0 / 1 takes logits [0, 32) / [32, 64) of every block and
+    // value dims [0, 256) / [256, 512) of O.
     const int q = warp;
     const int hr = 16 * q + (lane & 15);
     const int kh = lane >> 4;
+    const int head = kHG * g + hr;
+    const bool mine = head < a.H;
     const uint32_t t_s = tmem + ((uint32_t)(32 * q) << 16) + kTmemS;
     const uint32_t t_o = tmem + ((uint32_t)(32 * q) << 16) + kTmemO;
+    bool good = true;
+    if (nblk > 0) {
+      good = __all_sync(0xffffffffu, mbar_wait(q_tma, 0, a.err, a.wait_ns));
+      if (good) {
+        query_to_tmem(smem + OFF_KV + kStageBytes, mine, hr, kh, tmem + ((uint32_t)(32 * q) << 16));
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (good && lane == 0) mbar_arrive(q_full);
+    }
     const float sc = a.scale_log2;
     float m_ref = -INFINITY, l = 0.f;  // l: this thread's share of the head's sum
-    bool good = true;
     for (int j = 0; j < nblk && good; ++j) {
       const int sb = j & 1;
       const int stage = j % kStages;
-      good = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&s_full[sb], (j >> 1) & 1, a.err, a.wait_ns));
+      good = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(s_full, j & 1, a.err, a.wait_ns));
       if (!good) break;
-      uint32_t v[32];
+      uint32_t v[32], w[32];
+      float s[32];
       tc_fence_after();
-      tmem_ld16x2_32<32>(t_s + kBK * sb, v);
-      tmem_ld_wait();
+      tmem_ld16x2_32<32>(t_s, v);
+      tmem_ld16x2_32<32>(t_s + kBK, w);
+      tmem_ld_wait_regs(v);
+      tmem_ld_wait_regs(w);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(v[i]) + __uint_as_float(w[i]);
+      tmem_ld16x2_32<32>(t_s + 2 * kBK, v);
+      tmem_ld_wait_regs(v);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      if (lane == 0) mbar_arrive(s_empty);
       // validity of the block's rows (published before the stage completed)
       good = __all_sync(0xffffffffu, mbar_wait(&kv_full[stage], (j / kStages) & 1, a.err, a.wait_ns));
       if (!good) break;
       const uint32_t m32 = (uint32_t)(ring_mask[j] >> (32 * kh));
-      float s[32];
-      float mraw = -INFINITY, mneg = INFINITY;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool on = (m32 >> i) & 1u;
-        s[i] = on ? __uint_as_float(v[i]) : -INFINITY;
-        mraw = fmaxf(mraw, s[i]);
-        mneg = fminf(mneg, on ? s[i] : INFINITY);
+      for (int i = 0; i < 32; ++i) s[i] += __uint_as_float(v[i]);
+      if (m32 != 0xffffffffu) {  // masked rows (padding, bad indices) never count
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[i] = ((m32 >> i) & 1u) ? s[i] : -INFINITY;
       }
-      mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 16));
-      mneg = fminf(mneg, __shfl_xor_sync(0xffffffffu, mneg, 16));
-      // scale <= 0 (allowed, if odd): the largest scaled logit comes from the smallest raw one
-      const float mblk = mraw == -INFINITY ? -INFINITY : (sc > 0.f ? mraw * sc : mneg * sc);
+      // maxima as trees (depth 5), not chains
+      float mx[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mx[i] = fmaxf(s[i], s[i + 16]);
+#pragma unroll
+      for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+      float mraw = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], 16));
+      float mblk;
+      if (sc > 0.f) {
+        mblk = mraw == -INFINITY ? -INFINITY : mraw * sc;
+      } else {
+        // scale <= 0 (allowed, if odd): the largest scaled logit comes from
+        // the smallest unmasked raw one
+        float mneg = INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mneg = fminf(mneg, s[i] == -INFINITY ? INFINITY : s[i]);
+        mneg = fminf(mneg, __shfl_xor_sync(0xffffffffu, mneg, 16));
+        mblk = mraw == -INFINITY ? -INFINITY : mneg * sc;
+      }
       const bool move = mblk > m_ref + kRescaleThreshold;
       const float m_new = move ? mblk : m_ref;
       const float alpha = move ? exp2f(m_ref - m_new) : 1.f;  // exp2(-inf) = 0 on the first block
       const float mu = m_new == -INFINITY ? 0.f : m_new;      // nothing unmasked yet: every term is 0
       uint32_t pk[16], pl[16];
-      float psum = 0.f;
+      float ps[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         // masked: s = -inf and sc > 0 give ex2(-inf) = 0; sc <= 0 takes the select
         const float x0 = fmaf(s[2 * i], sc, -mu), x1 = fmaf(s[2 * i + 1], sc, -mu);
         const float e0 = sc > 0.f ? ex2_ftz(x0) : (s[2 * i] == -INFINITY ? 0.f : ex2_ftz(x0));
         const float e1 = sc > 0.f ? ex2_ftz(x1) : (s[2 * i + 1] == -INFINITY ? 0.f : ex2_ftz(x1));
-        psum += e0 + e1;
+        ps[i] = e0 + e1;
         const __nv_bfloat162 hi = __floats2bfloat162_rn(e0, e1);
         const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hi);
         const __nv_bfloat162 lo =
@@ -426,6 +474,11 @@ k_sparse_mla_tc(const AttnArgs a) {
         pk[i] = hb;
         pl[i] = *reinterpret_cast<const uint32_t*>(&lo);
       }
+#pragma unroll
+      for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) ps[i] += ps[i + w];
+      const float psum = ps[0];
       // P(j) into buffer j & 1 (PV(j-2), its last reader, completed before
       // QK(j) could start): row hr, this thread's four 16-byte pieces of keys
       // [32 kh, 32 kh + 32), each term in its own 128-byte-swizzled tile
@@ -449,7 +502,7 @@ k_sparse_mla_tc(const AttnArgs a) {
         for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
           tmem_ld16x2_32<256>(t_o + 32 * c, o);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st16x2_32<256>(t_o + 32 * c, o);
@@ -462,58 +515,74 @@ k_sparse_mla_tc(const AttnArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
     }
-    // epilogue: O / l for this thread's head and 256 value dims
-    good = good && __all_sync(0xffffffffu, mbar_wait(&o_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.err,
-                                                     a.wait_ns));
-    const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
-    if (good) {
-      tc_fence_after();
-      const bool partial = a.splits > 1;
-      const float inv = partial ? 1.f : (lt > 0.f ? 1.f / lt : 0.f);
-      const int head = kHG * g + hr;
-      const bool mine = head < a.H;
-      const int64_t orow = partial ? (((int64_t)t * a.splits + sp) * a.H + head) : ((int64_t)t * a.H + head);
+    // epilogue: O / l for this thread's head and 256 value dims, staged in
+    // the row stages (every MMA that read them has completed: o_done of the
+    // last block tracks all of them) and written with one bulk copy per row
+    if (nblk > 0) {
+      good = good && __all_sync(0xffffffffu, mbar_wait(&o_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.err,
+                                                       a.wait_ns));
+      const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      if (good) {
+        tc_fence_after();
+        const bool partial = a.splits > 1;
+        const bool f32 = partial || a.out_f32;
+        const float inv = partial ? 1.f : (lt > 0.f ? 1.f / lt : 0.f);
+        const int64_t orow = partial ? (((int64_t)t * a.splits + sp) * a.H + head) : ((int64_t)t * a.H + head);
+        uint8_t* srow = smem + OFF_KV + hr * (f32 ? kOutRowF32 : kOutRowBf16);
+        uint32_t on[32];
+        tmem_ld16x2_32<256>(t_o, on);
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        tmem_ld16x2_32<256>(t_o + 32 * c, o);
-        tmem_ld_wait();
-        if (!mine) continue;
-        const int dim = 256 * kh + 32 * c;
-        if (partial || a.out_f32) {
-          float* dst = (partial ? a.part_o : reinterpret_cast<float*>(a.out)) + orow * kDV + dim;
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          tmem_ld_wait_regs(on);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(dst)[i] =
-                make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                            __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
-        } else {
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + orow * kDV + dim;
+          for (int i = 0; i < 32; ++i) o[i] = on[i];
+          if (c + 1 < 8) tmem_ld16x2_32<256>(t_o + 32 * (c + 1), on);  // the next chunk's load overlaps this one's stores
+          const int dim = 256 * kh + 32 * c;
+          if (f32) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t w[4];
+            for (int i = 0; i < 8; ++i)
+              *reinterpret_cast<float4*>(srow + dim * 4 + 16 * i) =
+                  make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                              __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(o[8 * i + 2 * k]) * inv,
-                                                               __uint_as_float(o[8 * i + 2 * k + 1]) * inv);
-              w[k] = *reinterpret_cast<const uint32_t*>(&p2);
+            for (int i = 0; i < 4; ++i) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(o[8 * i + 2 * k]) * inv,
+                                                                 __uint_as_float(o[8 * i + 2 * k + 1]) * inv);
+                w4[k] = *reinterpret_cast<const uint32_t*>(&p2);
+              }
+              *reinterpret_cast<uint4*>(srow + dim * 2 + 16 * i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
+        fence_proxy_async_smem();  // the bulk copy reads the staged row (async proxy)
+        __syncwarp();
+        if (mine && kh == 0) {
+          void* dst = partial ? (void*)(a.part_o + orow * kDV)
+                              : (a.out_f32 ? (void*)(reinterpret_cast<float*>(a.out) + orow * kDV)
+                                           : (void*)(reinterpret_cast<__nv_bfloat16*>(a.out) + orow * kDV));
+          bulk_store(dst, srow, f32 ? kDV * 4 : kDV * 2);
+          bulk_commit();
+          const float m_nat = m_ref * kLn2;
+          if (partial)
+            a.part_ml[orow] = make_float2(m_nat, lt);
+          else if (a.lse)
+            a.lse[orow] = m_nat + logf(lt);
+          bulk_wait_read();  // the staged row stays until the copy has read it
+        }
+      } else {
+        *abort_flag = 1;
       }
-      if (mine && kh == 0) {
-        const float m_nat = m_ref * kLn2;
-        if (partial)
-          a.part_ml[orow] = make_float2(m_nat, lt);
-        else if (a.lse)
-          a.lse[orow] = m_nat + logf(lt);
-      }
-    } else {
-      *abort_flag = 1;
     }
     __syncwarp();
   }
+  // drain: the query tile's copy has landed before the CTA exits (its
+  // consumers may have given up waiting, or never run when nblk == 0)
+  if (threadIdx.x == 0) mbar_wait(q_tma, 0, a.err, kDrainLimitNs);
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -594,6 +663,31 @@ int keys_per_split(int K, int splits) {
   return (ks + kBK - 1) / kBK * kBK;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 [rows, 576] map with a box of 64 dims x 64 rows and the 128-byte swizzle.
+bool make_map_576(CUtensorMap* m, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kDQK, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kDQK * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kHG};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 size_t sparse_mla_partials_bytes(int T, int K, int H) {
@@ -620,12 +714,14 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, cons
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  AttnArgs a{s, tm, q, kv, idx, K, H, G, ks, splits, tm_early, scale * kLog2e, out, out_f32, lse, part_o, part_ml,
+  CUtensorMap tq;
+  if (!make_map_576(&tq, q, (uint64_t)T * H)) return cudaErrorInvalidValue;
+  AttnArgs a{s, tm, kv, idx, K, H, G, ks, splits, tm_early, scale * kLog2e, out, out_f32, lse, part_o, part_ml,
              err, wait_limit_ns()};
   const int64_t ctas = (int64_t)T * G * splits;
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
   cudaError_t e = launch_pdl("sparse_mla", k_sparse_mla_tc, dim3((unsigned)ctas), dim3(kThreads), (size_t)SMEM_BYTES,
-                             st, a);
+                             st, tq, a);
   if (e == cudaSuccess) e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
   e = launch_pdl("sparse_mla_combine", k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o,
