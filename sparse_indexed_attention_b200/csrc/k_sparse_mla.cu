@@ -54,37 +54,53 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBK = 64;                       // selected rows per block
 constexpr int kHG = 64;                       // heads per CTA (one M = 64 tile)
-constexpr int kAtom = 64 * 128;               // 64 rows x 64 bf16 dims, 128-byte swizzle
 constexpr int kNAtoms = kDQK / 64;            // 9: eight latent atoms + the rope atom
-constexpr int kStageBytes = kNAtoms * kAtom;  // 73728
-constexpr int kStages = 2;
+constexpr int kQAtom = kHG * 128;             // query atom: 64 heads x 64 dims
+constexpr int kQBytes = kNAtoms * kQAtom;     // 73728
 constexpr int kSParts = 3;                    // partial sums of S
-constexpr int kPTerm = kHG * kBK * 2;         // one bf16 term of P: 64 heads x 64 rows, 128-byte swizzle
+constexpr int kSCols = 64;                    // TMEM columns per partial (and P row width in keys)
+constexpr int kPTerm = kHG * kSCols * 2;      // one bf16 term of P: 64 heads x 64 keys, 128-byte swizzle
 constexpr int kLoaders = 128;                 // warps 4-7
 constexpr int kLoaderBarrier = 1;             // named barrier of the loader warps
-constexpr int OFF_KV = 0;                     // stage 1 holds the query tile until it is in TMEM
-constexpr int OFF_P = OFF_KV + kStages * kStageBytes;     // [2 buffers][hi, lo]; index staging at first
-constexpr int OFF_ROWS = OFF_P + 2 * 2 * kPTerm;          // [block][64] pool rows of the slice (-1 = masked)
-constexpr int OFF_MASK = OFF_ROWS + kMaxK * 4;            // [block] 64-bit validity masks
-constexpr int OFF_BAR = OFF_MASK + (kMaxK / kBK) * 8;
-constexpr int kNBars = 13;
-constexpr int OFF_MISC = OFF_BAR + kNBars * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;          // slack for 1024-byte alignment
+constexpr int kNBars = 15;
 constexpr int kThreads = 288;  // warps 0-3 softmax + epilogue, 4-7 load, 8 issues MMAs and owns TMEM
 constexpr int kMmaWarp = 8;
 constexpr int kOutRowF32 = kDV * 4 + 16;      // epilogue staging row (padded: no bank conflicts)
 constexpr int kOutRowBf16 = kDV * 2 + 16;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-static_assert(kStageBytes % 1024 == 0 && OFF_P % 1024 == 0 && kPTerm % 1024 == 0, "swizzle atoms need 1024-B alignment");
-static_assert(kHG * kOutRowF32 <= kStages * kStageBytes, "epilogue staging fits in the row stages");
-static_assert(2 * kMaxK * 4 <= 2 * 2 * kPTerm, "index staging fits in the P buffers");
+
+// Block shape: BK selected rows per block (a multiple of 16, at most 64),
+// NS row stages.  The library uses (64, 2): measured on all five workloads
+// it beat (48, 3), whose deeper gather pipeline did not repay the larger
+// number of (issue-bound) QK MMAs per selected row.
+template <int BK_, int NS_>
+struct AttnCfg {
+  static constexpr int BK = BK_, NS = NS_;
+  static constexpr int ATOM = BK * 128;                    // BK rows x 64 bf16 dims, 128-byte swizzle
+  static constexpr int STAGE = kNAtoms * ATOM;
+  static constexpr int MAX_BLOCKS = (kMaxK + BK - 1) / BK;
+  static constexpr int OFF_KV = 0;                         // stage 0 stages the index lists at first
+  static constexpr int OFF_Q = (NS - 1) * STAGE;           // the query tile lands in the last stage (and on)
+  static constexpr int OFF_P = NS * STAGE;                 // [2 buffers][hi, lo]
+  static constexpr int OFF_ROWS = OFF_P + 2 * 2 * kPTerm;  // [block][BK] pool rows of the slice (-1 = masked)
+  static constexpr int OFF_MASK = OFF_ROWS + MAX_BLOCKS * BK * 4;  // [block] 64-bit validity masks
+  static constexpr int OFF_BAR = OFF_MASK + MAX_BLOCKS * 8;
+  static constexpr int OFF_MISC = OFF_BAR + kNBars * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;        // slack for 1024-byte alignment
+  static constexpr uint32_t IDESC_QK = make_idesc_major(true, kHG, BK, 0, 0);  // S = Q K^T, both K-major
+  static_assert(BK % 16 == 0 && BK <= kSCols, "block shape");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(ATOM % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms need 1024-B alignment");
+  static_assert(OFF_Q + kQBytes <= OFF_ROWS, "the query tile fits in the last stage and the P buffers");
+  static_assert(kHG * kOutRowF32 <= NS * STAGE, "epilogue staging fits in the row stages");
+  static_assert(2 * kMaxK * 4 <= STAGE, "index staging fits in stage 0");
+};
+using Cfg = AttnCfg<64, 2>;
+
 // TMEM map: lane offset << 16 | column
 constexpr uint32_t kTmemS = 288;             // S partials at columns 288, 352, 416 of lanes 0-15 (Q at 0)
 constexpr uint32_t kTmemO = 16u << 16;       // O: lanes 16-31, columns 0-511
 
-constexpr uint32_t IDESC_QK = make_idesc_major(true, kHG, kBK, 0, 0);  // S = Q K^T, both K-major
 constexpr uint32_t IDESC_PV = make_idesc_major(true, kHG, 256, 0, 1);  // O += P V, V MN-major
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -146,7 +162,7 @@ __device__ __forceinline__ void query_to_tmem(const uint8_t* qs, bool valid, int
       const int d = 288 * half + 32 * chunk + 8 * k;  // first dim of the piece
       const int at = d >> 6, piece = (d & 63) >> 3;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (valid) v = *reinterpret_cast<const uint4*>(qs + at * kAtom + hr * 128 + ((piece ^ (hr & 7)) << 4));
+      if (valid) v = *reinterpret_cast<const uint4*>(qs + at * kQAtom + hr * 128 + ((piece ^ (hr & 7)) << 4));
       r[4 * k] = v.x;
       r[4 * k + 1] = v.y;
       r[4 * k + 2] = v.z;
@@ -156,29 +172,33 @@ __device__ __forceinline__ void query_to_tmem(const uint8_t* qs, bool valid, int
   }
 }
 
+template <int BK, int NS>
 __global__ void __launch_bounds__(kThreads, 1)
 k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
+  using C = AttnCfg<BK, NS>;
+  constexpr int OFF_KV = C::OFF_KV, OFF_P = C::OFF_P;
+  constexpr int kAtom = C::ATOM, kStageBytes = C::STAGE, kStages = NS, kBK = BK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_tma = bars + 0;      // the query tile has landed in stage 1
   uint64_t* q_full = bars + 1;     // the query is in TMEM and stage 1 is free (one arrival per softmax warp)
-  uint64_t* kv_full = bars + 2;    // [kStages] rows of block j (stage j % 2) landed
-  uint64_t* kv_empty = bars + 4;   // [kStages] PV of the stage's block completed
-  uint64_t* s_full = bars + 6;     // S of block j in TMEM
-  uint64_t* s_empty = bars + 7;    // S read by every softmax warp
-  uint64_t* p_full = bars + 8;     // [2] P of block j (buffer j & 1) in shared memory
-  uint64_t* o_done = bars + 10;    // [2] PV of block i (parity by i & 1) has completed
-  uint64_t* mma_drain = bars + 12; // every MMA this CTA issued has completed
-  int32_t* ring_rows = reinterpret_cast<int32_t*>(smem + OFF_ROWS);
-  uint64_t* ring_mask = reinterpret_cast<uint64_t*>(smem + OFF_MASK);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+  uint64_t* kv_full = bars + 2;    // [NS] rows of block j (stage j % NS) landed
+  uint64_t* kv_empty = bars + 5;   // [NS] PV of the stage's block completed
+  uint64_t* s_full = bars + 8;     // S of block j in TMEM
+  uint64_t* s_empty = bars + 9;    // S read by every softmax warp
+  uint64_t* p_full = bars + 10;    // [2] P of block j (buffer j & 1) in shared memory
+  uint64_t* o_done = bars + 12;    // [2] PV of block i (parity by i & 1) has completed
+  uint64_t* mma_drain = bars + 14; // every MMA this CTA issued has completed
+  int32_t* ring_rows = reinterpret_cast<int32_t*>(smem + C::OFF_ROWS);
+  uint64_t* ring_mask = reinterpret_cast<uint64_t*>(smem + C::OFF_MASK);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  const int sp = cta % a.splits, tg = cta / a.splits;
-  const int g = tg % a.G, t = tg / a.G;
+  const int g = cta % a.G, rest = cta / a.G;  // the head groups of a (token, slice) are neighbours (shared rows in L2)
+  const int sp = rest % a.splits, t = rest / a.splits;
   const int kbeg = sp * a.ks;
   const int kend = min(a.K, kbeg + a.ks);
 
@@ -209,9 +229,9 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) {  // q is an input of the call: its load overlaps the wait below
     prefetch_tmap(&tq);
-    mbar_arrive_expect_tx(q_tma, kStageBytes);
+    mbar_arrive_expect_tx(q_tma, kQBytes);
     for (int at = 0; at < kNAtoms; ++at)
-      tma_load_2d(smem + OFF_KV + kStageBytes + at * kAtom, &tq, q_tma, 64 * at, t * a.H + kHG * g);
+      tma_load_2d(smem + C::OFF_Q + at * kQAtom, &tq, q_tma, 64 * at, t * a.H + kHG * g);
   }
   // the token map can be read before the wait when it does not come from
   // the kernel just before; the index lists always do
@@ -237,11 +257,11 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
     const int lw = warp - 4;           // loader warp 0 .. 3
     // Pool rows of every block of the slice, resolved up front in three
     // passes whose loads are all independent: the index list, then the page
-    // ids (both staged by cp.async in the P buffers, which are first written
-    // after block 0 has been scored), then rows and masks (row -1 = masked).
+    // ids (both staged by cp.async in stage 0, which block 0's copies fill
+    // only after the last pass), then rows and masks (row -1 = masked).
     {
       const int nkeys = kend - kbeg;
-      int32_t* s_sidx = reinterpret_cast<int32_t*>(smem + OFF_P);
+      int32_t* s_sidx = reinterpret_cast<int32_t*>(smem + OFF_KV);
       int32_t* s_page = s_sidx + kMaxK;
       const int32_t* idx_row = a.idx + (int64_t)t * a.K + kbeg;
       for (int k = li; k < nkeys; k += kLoaders) cp_async_4(&s_sidx[k], idx_row + k);
@@ -272,36 +292,41 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
       }
       bar_red_or(kLoaderBarrier, kLoaders, false);
       for (int w32 = lw; w32 < 2 * nblk; w32 += 4) {  // 32 rows per warp -> half a block's mask
-        const uint32_t m = __ballot_sync(0xffffffffu, ring_rows[w32 * 32 + lane] >= 0);
+        const int r = 32 * (w32 & 1) + lane;         // row of block w32 / 2 (rows >= BK never count)
+        const uint32_t m = __ballot_sync(0xffffffffu, r < kBK && ring_rows[(w32 >> 1) * kBK + r] >= 0);
         if (lane == 0) reinterpret_cast<uint32_t*>(ring_mask)[w32] = m;
       }
     }
     const uint32_t kv_smem = smem_u32(smem + OFF_KV);
-    const __nv_bfloat16* kv_base = a.kv;
-    const int rsub = lane >> 3, piece = lane & 7;  // a warp copies 4 rows x 128 bytes of one atom
+    const char* kv_base = reinterpret_cast<const char*>(a.kv);
+    const int rsub = lane >> 3, piece = lane & 7;  // a warp copies 4 rows x 128 bytes of one atom at a time
+    constexpr int kQuads = BK / 4;  // row quads per block
     bool failed = bar_red_or(kLoaderBarrier, kLoaders, false);
     for (int j = 0; j < nblk && !failed; ++j) {
       const int stage = j % kStages;
+      // the PV of the stage's previous block has completed
       bool ok = mbar_wait(&kv_empty[stage], ((j / kStages) & 1) ^ 1, a.err, a.wait_ns);
-      // stage 1 first holds the query tile
-      if (j == 1) ok = ok && mbar_wait(q_full, 0, a.err, a.wait_ns);
+      // the last stage first holds the query tile
+      if (j == NS - 1) ok = ok && mbar_wait(q_full, 0, a.err, a.wait_ns);
       if (ok) {
-        // task = (atom, quad of rows): the warp's 32 copies fill 512
-        // contiguous bytes of the atom (no bank conflict) from four 128-byte
-        // pieces of the pool
+        // one row per (warp, quad): its pool row is looked up once, then the
+        // nine 128-byte pieces (one per atom) go out back to back; a warp's
+        // 32 copies of one atom fill 512 contiguous bytes (no bank conflict)
         const uint32_t dst0 = kv_smem + stage * kStageBytes;
-        for (int task = lw; task < kNAtoms * (kBK / 4); task += 4) {
-          const int at = task / (kBK / 4);
-          const int r = 4 * (task % (kBK / 4)) + rsub;
+#pragma unroll 1
+        for (int qd = lw; qd < kQuads; qd += 4) {
+          const int r = 4 * qd + rsub;
           const int row = ring_rows[j * kBK + r];
           const bool v = row >= 0;
-          const uint32_t dst = dst0 + at * kAtom + r * 128 + ((((uint32_t)piece) ^ ((uint32_t)r & 7u)) << 4);
-          cp_async_16_zfill(dst, kv_base + (v ? (int64_t)row * kDQK + 64 * at + 8 * piece : 0), v ? 16u : 0u);
+          const char* src = kv_base + (v ? (int64_t)row * (kDQK * 2) : 0) + 16 * piece;
+          const uint32_t dst = dst0 + r * 128 + ((((uint32_t)piece) ^ ((uint32_t)r & 7u)) << 4);
+#pragma unroll
+          for (int at = 0; at < kNAtoms; ++at) cp_async_16_zfill(dst + at * kAtom, src + 128 * at, v ? 16u : 0u);
         }
       }
       cp_async_mbar_arrive(&kv_full[stage]);     // counts once this thread's copies land
       if (li == 0) mbar_arrive(&kv_full[stage]);  // releases the masks read by the softmax warps
-      failed = bar_red_or(kLoaderBarrier, kLoaders, !ok);
+      failed = bar_red_or(kLoaderBarrier, kLoaders, !ok || *abort_flag != 0);
       if (failed) *abort_flag = 1;
     }
     cp_async_wait_all();  // nothing this thread copies is still in flight at exit
@@ -354,8 +379,8 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
 #pragma unroll
               for (int part = 0; part < kSParts; ++part) {
                 const int at = kSParts * grp + part;
-                mma_ts_bf16(tmem + kTmemS + kBK * part, tmem + 32 * at + 8 * kk, desc_at(kd, at * kAtom + kk * 32),
-                            IDESC_QK, (grp | kk) != 0);
+                mma_ts_bf16(tmem + kTmemS + kSCols * part, tmem + 32 * at + 8 * kk,
+                            desc_at(kd, at * kAtom + kk * 32), C::IDESC_QK, (grp | kk) != 0);
               }
           mma_commit(s_full);
           ++nq;
@@ -395,7 +420,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
     if (nblk > 0) {
       good = __all_sync(0xffffffffu, mbar_wait(q_tma, 0, a.err, a.wait_ns));
       if (good) {
-        query_to_tmem(smem + OFF_KV + kStageBytes, mine, hr, kh, tmem + ((uint32_t)(32 * q) << 16));
+        query_to_tmem(smem + C::OFF_Q, mine, hr, kh, tmem + ((uint32_t)(32 * q) << 16));
         tmem_st_wait();
       }
       tc_fence_before();
@@ -413,12 +438,12 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
       float s[32];
       tc_fence_after();
       tmem_ld16x2_32<32>(t_s, v);
-      tmem_ld16x2_32<32>(t_s + kBK, w);
+      tmem_ld16x2_32<32>(t_s + kSCols, w);
       tmem_ld_wait_regs(v);
       tmem_ld_wait_regs(w);
 #pragma unroll
       for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(v[i]) + __uint_as_float(w[i]);
-      tmem_ld16x2_32<32>(t_s + 2 * kBK, v);
+      tmem_ld16x2_32<32>(t_s + 2 * kSCols, v);
       tmem_ld_wait_regs(v);
       tc_fence_before();
       __syncwarp();
@@ -479,9 +504,14 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
 #pragma unroll
         for (int i = 0; i < w; ++i) ps[i] += ps[i + w];
       const float psum = ps[0];
-      // P(j) into buffer j & 1 (PV(j-2), its last reader, completed before
-      // QK(j) could start): row hr, this thread's four 16-byte pieces of keys
-      // [32 kh, 32 kh + 32), each term in its own 128-byte-swizzled tile
+      // P(j) into buffer j & 1 once PV(j-2), its last reader, has completed
+      // (with two stages QK(j) could not start before that): row hr, this
+      // thread's four 16-byte pieces of keys [32 kh, 32 kh + 32), each term in
+      // its own 128-byte-swizzled tile
+      if (NS > 2 && j >= 2) {
+        good = __all_sync(0xffffffffu, mbar_wait(&o_done[j & 1], ((j - 2) >> 1) & 1, a.err, a.wait_ns));
+        if (!good) break;
+      }
       uint8_t* prow = smem + OFF_P + sb * 2 * kPTerm + hr * 128;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -650,17 +680,36 @@ constexpr int kSplitSms = 148;  // SMs the split decision fills (a host-only con
 
 int head_groups(int H) { return (H + kHG - 1) / kHG; }
 
+// Batches with fewer (token, head group) units than SMs split each index
+// list over several CTAs (whose partials k_combine merges).
 int attn_splits(int T, int K, int H) {
-  const int units = T * head_groups(H);
+  const int64_t units = (int64_t)T * head_groups(H);
   if (units >= kSplitSms) return 1;
-  const int want = kSplitSms / units;
-  const int most = (K + kBK - 1) / kBK;
+  const int want = kSplitSms / (int)units;
+  int most = (K + Cfg::BK - 1) / Cfg::BK;
+  if (most > kMaxSplits) most = kMaxSplits;
   return want < 1 ? 1 : (want < most ? want : most);
 }
 
-int keys_per_split(int K, int splits) {
+int keys_per_split(int K, int splits, int bk) {
   const int ks = (K + splits - 1) / splits;
-  return (ks + kBK - 1) / kBK * kBK;
+  return (ks + bk - 1) / bk * bk;
+}
+
+template <int BK, int NS>
+cudaError_t launch_attn(const CUtensorMap& tq, const AttnArgs& a, int64_t ctas, cudaStream_t st) {
+  using C = AttnCfg<BK, NS>;
+  static thread_local int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_sparse_mla_tc<BK, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_dev = dev;
+  }
+  return launch_pdl("sparse_mla", k_sparse_mla_tc<BK, NS>, dim3((unsigned)ctas), dim3(kThreads), (size_t)C::SMEM, st,
+                    tq, a);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -702,26 +751,17 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, cons
   const int T = s.num_tokens;
   const int G = head_groups(H);
   int splits = attn_splits(T, K, H);
-  const int ks = keys_per_split(K, splits);
+  const int ks = keys_per_split(K, splits, Cfg::BK);
   splits = (K + ks - 1) / ks;
   float* part_o = reinterpret_cast<float*>(partials);
   float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)T * splits * H * kDV);
-  static thread_local int attr_dev = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (attr_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(k_sparse_mla_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_dev = dev;
-  }
   CUtensorMap tq;
   if (!make_map_576(&tq, q, (uint64_t)T * H)) return cudaErrorInvalidValue;
   AttnArgs a{s, tm, kv, idx, K, H, G, ks, splits, tm_early, scale * kLog2e, out, out_f32, lse, part_o, part_ml,
              err, wait_limit_ns()};
   const int64_t ctas = (int64_t)T * G * splits;
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
-  cudaError_t e = launch_pdl("sparse_mla", k_sparse_mla_tc, dim3((unsigned)ctas), dim3(kThreads), (size_t)SMEM_BYTES,
-                             st, tq, a);
+  cudaError_t e = launch_attn<Cfg::BK, Cfg::NS>(tq, a, ctas, st);
   if (e == cudaSuccess) e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
   e = launch_pdl("sparse_mla_combine", k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o,
