@@ -74,6 +74,8 @@ def parse():
                     help="override the workload's context length (profiling a smaller case of the same kernels)")
     ap.add_argument("--all-configs", action="store_true",
                     help="one JSON line per workload: fused-call time and the binding roofline of each stage")
+    ap.add_argument("--select-in-indexer", action="store_true",
+                    help="decode: select the Top-K inside the indexer kernel (DSA_SELECT_IN_INDEXER)")
     ap.add_argument("--only", choices=["index_scores", "topk", "sparse_mla", "fused"], default=None,
                     help="time one stage (or the fused call, eagerly) alone on the bench workload (profiling aid)")
     return ap.parse_args()
@@ -355,12 +357,12 @@ def run_all_configs(args, dsa, dev, stream, flush):
         T, H, K = wl.T, spec.heads, spec.topk
         out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((T, H), dtype=torch.float32, device=dev)
-        ws = torch.zeros(dsa.dsa_workspace_size(dsa.DSA_OP_INDEX_TOPK_ATTN, d.seqs, K, H), dtype=torch.uint8,
-                         device=dev)
+        op = dsa.DSA_OP_INDEX_TOPK_ATTN_FUSED if args.select_in_indexer else dsa.DSA_OP_INDEX_TOPK_ATTN
+        ws = torch.zeros(dsa.dsa_workspace_size(op, d.seqs, K, H), dtype=torch.uint8, device=dev)
 
         def step():
             dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse,
-                                    ws=ws)
+                                    ws=ws, select_in_indexer=args.select_in_indexer)
 
         for _ in range(2):
             step()
@@ -394,7 +396,11 @@ def run_all_configs(args, dsa, dev, stream, flush):
                                           "dtype": "fp8" if spec.ki_fp8 else "bf16"}
         topk_us = sum(v for k, v in us.items() if k.startswith("topk"))
         b = pairs * 4 + T * K * 4
-        stages["topk"] = {"bound": "latency", "us": topk_us, "hbm_frac_of_one_pass": b / (topk_us * 1e-6) / 1e9 / hbm}
+        if topk_us > 0:
+            stages["topk"] = {"bound": "latency", "us": topk_us,
+                              "hbm_frac_of_one_pass": b / (topk_us * 1e-6) / 1e9 / hbm}
+        else:  # decode: the indexer kernel selects the Top-K itself
+            stages["topk"] = {"bound": "latency", "us": 0.0, "inside": "index_scores"}
         attn_us = us.get("sparse_mla", 0.0) + us.get("sparse_mla_combine", 0.0)
         if attn_us:
             t_s = attn_us * 1e-6
@@ -409,6 +415,7 @@ def run_all_configs(args, dsa, dev, stream, flush):
                                         "unit": "TFLOP/s", "frac": f / t_s / 1e12 / pk}
         line = {"config": name, "tokens": T, "us_per_call": ms * 1e3, "tokens_per_s": T / (ms / 1e3),
                 "launches": dsa.dsa_launches_in_last_call(), "kernels_us": us, "stages": stages,
+                "select_in_indexer": args.select_in_indexer,
                 "peak_source": hbm_src, "timing": "graph replay, 256 MiB L2 flush before each step; "
                 "kernels_us from events around each launch (serialised)"}
         print(json.dumps(line), flush=True)
@@ -436,12 +443,14 @@ def run_ours(args, world, rank, local):
     T, H, K = wl.T, spec.heads, spec.topk
     out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((T, H), dtype=torch.float32, device=dev)
-    ws = torch.zeros(dsa.dsa_workspace_size(dsa.DSA_OP_INDEX_TOPK_ATTN, d.seqs, K, H), dtype=torch.uint8,
-                     device=dev)
+    sel = args.select_in_indexer
+    op = dsa.DSA_OP_INDEX_TOPK_ATTN_FUSED if sel else dsa.DSA_OP_INDEX_TOPK_ATTN
+    ws = torch.zeros(dsa.dsa_workspace_size(op, d.seqs, K, H), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step():
-        dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse, ws=ws)
+        dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse, ws=ws,
+                                select_in_indexer=sel)
 
     if args.only:
         run_only(args, dsa, wl, d, dev, stream, flush, world, fused=step)
@@ -520,13 +529,23 @@ def run_ours(args, world, rank, local):
     h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     d_meta = [d.seqs.q_seq_start, d.seqs.ctx_len, d.seqs.page_table]
 
+    side = torch.cuda.Stream(dev)
+    q_ready = torch.cuda.Event()
+
     def e2e_step():
+        # the indexer's inputs on the call's stream; the attention query on a
+        # side stream (once the previous step's attention is done with it),
+        # overlapping the indexer: the attention launch waits on q_ready
         d.qI.copy_(h_qI, non_blocking=True)
         d.w.copy_(h_w, non_blocking=True)
-        d.q.copy_(h_q, non_blocking=True)
         for dm, hm in zip(d_meta, h_meta):
             dm.copy_(hm, non_blocking=True)
-        step()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            d.q.copy_(h_q, non_blocking=True)
+            q_ready.record(side)
+        dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse, ws=ws,
+                                q_ready=q_ready, select_in_indexer=sel)
         h_out.copy_(out, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
 

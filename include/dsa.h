@@ -77,6 +77,8 @@ extern "C" {
 
 /* An opaque cudaStream_t (struct CUstream_st*).  NULL = legacy default stream. */
 typedef struct CUstream_st *dsa_stream_t;
+/* An opaque cudaEvent_t (struct CUevent_st*). */
+typedef struct CUevent_st *dsa_event_t;
 
 typedef enum {
   DSA_OK = 0,
@@ -103,8 +105,20 @@ typedef enum {
   DSA_OP_INDEX_SCORES = 1,
   DSA_OP_TOPK = 2,
   DSA_OP_SPARSE_MLA = 3,
-  DSA_OP_INDEX_TOPK_ATTN = 4
+  DSA_OP_INDEX_TOPK_ATTN = 4,
+  DSA_OP_INDEX_TOPK_ATTN_FUSED = 5  /* dsa_index_topk_attn_ex with DSA_SELECT_IN_INDEXER */
 } dsa_op_t;
+
+/* Flags of dsa_index_topk_attn_ex. */
+enum {
+  /* Decode batches (one query token per sequence) whose rows fit: the indexer
+   * kernel selects the Top-K itself -- the fused scoring-weighting-selection
+   * operator of [P2] section 4(1) / [P4] section 3.1 -- so no score array
+   * exists and the call is at most four launches.  Workspace: size it with
+   * DSA_OP_INDEX_TOPK_ATTN_FUSED.  Other geometries ignore the flag.  The
+   * selected sets are the same as without it. */
+  DSA_SELECT_IN_INDEXER = 1
+};
 
 /* Batch geometry (host struct; the three arrays are device memory).
  *   batch          B >= 1 sequences
@@ -245,6 +259,25 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t *seqs, const void *qI,
                                  dsa_out_dtype_t out_dtype, float *lse,
                                  int32_t *idx_out, void *ws, size_t ws_bytes,
                                  dsa_stream_t stream);
+
+/* dsa_index_topk_attn with options.  `flags`: 0 or DSA_SELECT_IN_INDEXER.
+ * `q_ready`: for a caller whose attention query q is still being
+ * produced or copied on another stream when the call is made ([P2] section
+ * 4(2): the indexer's inputs are prepared apart from the attention's, so the
+ * two overlap).  Everything up to the attention stage is launched at once;
+ * the attention launch first waits on `q_ready` (cudaStreamWaitEvent on
+ * `stream`), so q must hold its final values when the event completes.
+ * q_ready NULL is dsa_index_topk_attn.  The event must have been recorded
+ * before the call. */
+dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t *seqs, const void *qI,
+                                    const float *w, const void *kI,
+                                    const float *kI_scale, dsa_ki_dtype_t ki_dtype,
+                                    const void *q, const void *kv, int K, int H,
+                                    float scale, void *out,
+                                    dsa_out_dtype_t out_dtype, float *lse,
+                                    int32_t *idx_out, void *ws, size_t ws_bytes,
+                                    unsigned flags, dsa_event_t q_ready,
+                                    dsa_stream_t stream);
 
 /* Synchronises `stream`, reads and clears the workspace's sticky device error
  * flag.  Returns DSA_OK, DSA_ERR_BAD_INDEX, DSA_ERR_TIMEOUT or DSA_ERR_CUDA

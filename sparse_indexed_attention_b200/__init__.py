@@ -33,11 +33,14 @@ DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUD
 DSA_KI_BF16, DSA_KI_FP8_E4M3 = 0, 1
 DSA_OUT_BF16, DSA_OUT_F32 = 0, 1
 DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
-DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_INDEX_TOPK_ATTN = range(5)
+DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_INDEX_TOPK_ATTN, \
+    DSA_OP_INDEX_TOPK_ATTN_FUSED = range(6)
+DSA_SELECT_IN_INDEXER = 1
 
 # Names the C header declares (checked against include/dsa.h by the tests).
 EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_index_scores", "dsa_topk",
            "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_noalloc", "dsa_check_error_noalloc", "dsa_index_topk_attn",
+           "dsa_index_topk_attn_ex",
            "dsa_check_error", "dsa_set_wait_limit_ns", "dsa_launches_in_last_call", "dsa_launch_timing",
            "dsa_last_launch_times", "dsa_status_string")
 
@@ -62,6 +65,8 @@ _sig = {
                                                   _P, _P]),
     "dsa_index_topk_attn": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
                                            _F, _P, ctypes.c_int, _P, _P, _P, _SZ, _P]),
+    "dsa_index_topk_attn_ex": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
+                                              _F, _P, ctypes.c_int, _P, _P, _P, _SZ, ctypes.c_uint, _P, _P]),
     "dsa_check_error": (ctypes.c_int, [_P, _P]),
     "dsa_check_error_noalloc": (ctypes.c_int, [_P]),
     "dsa_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
@@ -342,7 +347,12 @@ def dsa_sparse_mla_fwd_noalloc(seqs: Seqs, q, kv, idx, scale: float, out=None, l
 
 
 def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: float, out=None, lse=None,
-                        idx_out=None, want_lse=True, ws=None, out_dtype=torch.bfloat16):
+                        idx_out=None, want_lse=True, ws=None, out_dtype=torch.bfloat16, q_ready=None,
+                        select_in_indexer=False):
+    """The whole path.  q_ready (a torch.cuda.Event, optional): the attention
+    launch waits on it, so q may still be in flight on another stream.
+    select_in_indexer: decode rows that fit are selected inside the indexer
+    kernel (DSA_SELECT_IN_INDEXER)."""
     T, H, _ = q.shape
     out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
@@ -354,12 +364,15 @@ def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: f
         _need(idx_out, "idx_out", _I32T, (T, K), dev)
     ki_dtype = DSA_KI_FP8_E4M3 if kI_scale is not None else DSA_KI_BF16
     c = seqs.c()
-    need = _lib.dsa_workspace_size(DSA_OP_INDEX_TOPK_ATTN, ctypes.byref(c), K, H)
+    op = DSA_OP_INDEX_TOPK_ATTN_FUSED if select_in_indexer else DSA_OP_INDEX_TOPK_ATTN
+    need = _lib.dsa_workspace_size(op, ctypes.byref(c), K, H)
     ws = ws if ws is not None else workspace(need, q.device, "index_topk_attn")
     _need_ws(ws, dev)
-    _check(_lib.dsa_index_topk_attn(ctypes.byref(c), _ptr(qI), _ptr(w), _ptr(kI), _ptr(kI_scale), ki_dtype, _ptr(q),
-                                    _ptr(kv), K, H, scale, _ptr(out), _out_dtype(out), _ptr(lse), _ptr(idx_out),
-                                    _ptr(ws), ws.numel(), _stream(q.device)), "dsa_index_topk_attn")
+    ev = None if q_ready is None else ctypes.c_void_p(q_ready.cuda_event)
+    _check(_lib.dsa_index_topk_attn_ex(ctypes.byref(c), _ptr(qI), _ptr(w), _ptr(kI), _ptr(kI_scale), ki_dtype, _ptr(q),
+                                       _ptr(kv), K, H, scale, _ptr(out), _out_dtype(out), _ptr(lse), _ptr(idx_out),
+                                       _ptr(ws), ws.numel(), DSA_SELECT_IN_INDEXER if select_in_indexer else 0, ev,
+                                       _stream(q.device)), "dsa_index_topk_attn")
     return out, lse
 
 

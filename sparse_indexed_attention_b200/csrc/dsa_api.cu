@@ -24,9 +24,11 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // the sticky error word.
 struct Layout {
   size_t tok_seq = 0, tok_pos = 0, seq_gstart = 0, groups = 0, items = 0, counts = 0;
-  size_t q_codes = 0, w_scaled = 0, scores = 0, idx = 0, topk = 0, partials = 0;
+  size_t q_codes = 0, w_scaled = 0, scores = 0, idx = 0, topk = 0, partials = 0, tail = 0, cand = 0;
   size_t total = 0;
   int64_t ld = 0;
+  bool fused = false;       // the indexer selects the Top-K itself (no score scratch)
+  int64_t tail_words = 0;
 };
 
 // The indexer's work-list capacity must hold for either index-cache dtype, so
@@ -41,6 +43,8 @@ Layout make_layout(dsa_op_t op, int T, int B, int max_ctx, int K, int H) {
     off = align_up(off + bytes);
     return o;
   };
+  const bool fused_op = op == DSA_OP_INDEX_TOPK_ATTN_FUSED;
+  if (fused_op) op = DSA_OP_INDEX_TOPK_ATTN;  // the same call, its selection inside the indexer when the rows fit
   const bool seq_ops = op == DSA_OP_INDEX_SCORES || op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN;
   const bool indexer = op == DSA_OP_INDEX_SCORES || op == DSA_OP_INDEX_TOPK_ATTN;
   if (seq_ops) {
@@ -58,9 +62,17 @@ Layout make_layout(dsa_op_t op, int T, int B, int max_ctx, int K, int H) {
   }
   if (op == DSA_OP_INDEX_TOPK_ATTN) {
     L.ld = ((int64_t)max_ctx + 3) / 4 * 4;
-    L.scores = take((size_t)T * (size_t)L.ld * sizeof(float));
-    L.idx = take((size_t)T * K * sizeof(int32_t));
-    L.topk = take(topk_scratch_bytes(T, L.ld, K));
+    L.fused = fused_op && indexer_fused_fits(T, B, max_ctx);
+    if (L.fused) {  // decode: selection inside the indexer, its histograms and counts only
+      L.tail_words = fused_topk_words(T, B, max_ctx);
+      L.tail = take((size_t)L.tail_words * sizeof(uint32_t));
+      L.cand = take(fused_topk_cand_bytes(T));
+      L.idx = take((size_t)T * K * sizeof(int32_t));
+    } else {
+      L.scores = take((size_t)T * (size_t)L.ld * sizeof(float));
+      L.idx = take((size_t)T * K * sizeof(int32_t));
+      L.topk = take(topk_scratch_bytes(T, L.ld, K));
+    }
   }
   if (op == DSA_OP_TOPK) L.topk = take(topk_scratch_bytes(T, max_ctx, K));
   if (op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN) L.partials = take(sparse_mla_partials_bytes(T, K, H));
@@ -153,7 +165,7 @@ PlanBufs plan_bufs(void* ws, const Layout& L) {
 dsa_status_t run_indexer(const dsa_seqs_t* seqs, const SeqsDev& sd, const PlanBufs& plan, int tg, const void* qI,
                          const float* w, const void* kI, const float* kI_scale, dsa_ki_dtype_t ki_dtype,
                          float* scores, int64_t ld, void* ws, const Layout& L, uint32_t* hist, uint32_t* zero,
-                         int64_t zero_words, uint32_t* err, cudaStream_t st) {
+                         int64_t zero_words, uint32_t* err, cudaStream_t st, const FusedTopk* fused = nullptr) {
   const bool fp8 = ki_dtype == DSA_KI_FP8_E4M3;
   const void* q_operand = qI;
   const float* w_operand = w;
@@ -165,7 +177,8 @@ dsa_status_t run_indexer(const dsa_seqs_t* seqs, const SeqsDev& sd, const PlanBu
     q_operand = codes;
     w_operand = w_scaled;
   }
-  DSA_CUDA(launch_index_scores(sd, plan, tg, q_operand, w_operand, kI, kI_scale, fp8, scores, ld, hist, err, st));
+  DSA_CUDA(launch_index_scores(sd, plan, tg, q_operand, w_operand, kI, kI_scale, fp8, scores, ld, hist, err, st,
+                               fused));
   return DSA_OK;
 }
 
@@ -177,9 +190,11 @@ size_t dsa_workspace_size(dsa_op_t op, const dsa_seqs_t* seqs, int K, int H) {
   if (!seqs || seqs->num_q_tokens < 1 || seqs->max_ctx < 1) return 0;
   if (op == DSA_OP_QUANTIZE_INDEX_QUERY) return 0;
   if (op == DSA_OP_TOPK) return make_layout(op, seqs->num_q_tokens, 1, seqs->max_ctx, K, 16).total;
-  if (op < 0 || op > DSA_OP_INDEX_TOPK_ATTN) return 0;
+  if (op < 0 || op > DSA_OP_INDEX_TOPK_ATTN_FUSED) return 0;
   if (seqs->batch < 1) return 0;
-  if ((op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN) && (K < 1 || K > kMaxK || !valid_H(H))) return 0;
+  if ((op == DSA_OP_SPARSE_MLA || op == DSA_OP_INDEX_TOPK_ATTN || op == DSA_OP_INDEX_TOPK_ATTN_FUSED) &&
+      (K < 1 || K > kMaxK || !valid_H(H)))
+    return 0;
   return make_layout(op, seqs->num_q_tokens, seqs->batch, seqs->max_ctx, K, H).total;
 }
 
@@ -248,25 +263,42 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const voi
   return DSA_OK;
 }
 
-dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
-                                 const float* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
-                                 int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse,
-                                 int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
+                                    const float* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
+                                    int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse,
+                                    int32_t* idx_out, void* ws, size_t ws_bytes, unsigned flags,
+                                    dsa_event_t q_ready, dsa_stream_t stream) {
   g_launches = 0;
   DSA_TRY(check_indexer_args(seqs, qI, w, kI, kI_scale, ki_dtype));
   DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, out_dtype, lse));
   if (idx_out && !aligned(idx_out, 16)) return DSA_ERR_INVALID_ARG;
-  const Layout L = make_layout(DSA_OP_INDEX_TOPK_ATTN, seqs->num_q_tokens, seqs->batch, seqs->max_ctx, K, H);
+  if (flags & ~(unsigned)DSA_SELECT_IN_INDEXER) return DSA_ERR_INVALID_ARG;
+  const Layout L = make_layout((flags & DSA_SELECT_IN_INDEXER) ? DSA_OP_INDEX_TOPK_ATTN_FUSED : DSA_OP_INDEX_TOPK_ATTN,
+                               seqs->num_q_tokens, seqs->batch, seqs->max_ctx, K, H);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
   cudaStream_t st = (cudaStream_t)stream;
   uint32_t* err = at<uint32_t>(ws, 0);
   const SeqsDev sd = to_dev(seqs);
   const PlanBufs plan = plan_bufs(ws, L);
   TokenMap tm{plan.tok_seq, plan.tok_pos};
-  float* scores = at<float>(ws, L.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
   const int T = seqs->num_q_tokens;
   const int tg = indexer_group_tokens(T, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
+  if (L.fused) {
+    // decode: prep, the indexer with the Top-K selection inside, attention
+    uint32_t* tail = at<uint32_t>(ws, L.tail);
+    const FusedTopk f{tail, reinterpret_cast<int2*>(tail + (size_t)T * kFusedTailWordsPerToken),
+                      at<int2>(ws, L.cand), idx, K};
+    timer_begin(st);
+    DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, nullptr, L.ld, ws, L, nullptr, tail,
+                        L.tail_words, err, st, &f));
+    if (q_ready) DSA_CUDA(cudaStreamWaitEvent(st, (cudaEvent_t)q_ready, 0));
+    DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/true, reinterpret_cast<const __nv_bfloat16*>(q),
+                               reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
+                               out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
+    return DSA_OK;
+  }
+  float* scores = at<float>(ws, L.scores);
   // one token per group: the indexer also builds Top-K's first-digit histogram
   const bool fuse_hist = tg == 1 && topk_uses_hist(T, L.ld);
   uint32_t* hist = fuse_hist ? topk_hist_in_scratch(at<void>(ws, L.topk), T) : nullptr;
@@ -275,10 +307,20 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const f
   DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, L.ld, ws, L, hist, zero,
                       fuse_hist ? topk_zero_words(T) : 0, err, st));
   DSA_CUDA(launch_topk(scores, L.ld, T, nullptr, tm.pos, K, idx, at<void>(ws, L.topk), hist != nullptr, err, st));
+  // the query may still be in flight on another stream: attention is the first step that reads it
+  if (q_ready) DSA_CUDA(cudaStreamWaitEvent(st, (cudaEvent_t)q_ready, 0));
   DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/true, reinterpret_cast<const __nv_bfloat16*>(q),
                              reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
                              out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
   return DSA_OK;
+}
+
+dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
+                                 const float* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
+                                 int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse,
+                                 int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  return dsa_index_topk_attn_ex(seqs, qI, w, kI, kI_scale, ki_dtype, q, kv, K, H, scale, out, out_dtype, lse, idx_out,
+                                ws, ws_bytes, 0u, nullptr, stream);
 }
 
 dsa_status_t dsa_check_error(void* ws, dsa_stream_t stream) {

@@ -174,11 +174,29 @@ cudaError_t launch_prep(const SeqsDev& s, int tg, int ch, const PlanBufs& plan, 
                         uint32_t* err, cudaStream_t st);
 cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w, int T, uint8_t* codes,
                                         float* w_scaled, cudaStream_t st);
+// Fused selection (decode): the indexer also selects the Top-K of every row
+// (no score scratch).  Its grid is one CTA on each of kFusedGrid SMs, all
+// resident; `tail` / `tail_items` (fused_topk_words words) start zeroed.
+constexpr int kFusedGrid = 148;
+constexpr int kFusedTailWordsPerToken = 2 * kTopkHistBins + 1024 + 8;  // 3 histograms, arrival counters
+struct FusedTopk {
+  uint32_t* tail;
+  int2* tail_items;
+  int2* cand;    // fused_topk_cand_bytes, need not be zeroed
+  int32_t* idx;  // [T, K]
+  int K;
+};
+int indexer_fused_capacity();                          // items per CTA
+bool indexer_fused_fits(int T, int B, int max_ctx);    // the geometry fits the fused selection
+int64_t fused_topk_words(int T, int B, int max_ctx);   // its zeroed scratch, in 32-bit words
+size_t fused_topk_cand_bytes(int T);                   // its candidate lists
 // FP8 cache: codes/w_scaled from the quantizer; bf16 cache: qI/w directly.
 // hist (may be null; used for one token per group): Top-K first-digit histogram to accumulate into.
+// fused (may be null): select the Top-K in the same kernel instead of writing scores.
 cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
                                 const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
-                                float* scores, int64_t ld, uint32_t* hist, uint32_t* err, cudaStream_t st);
+                                float* scores, int64_t ld, uint32_t* hist, uint32_t* err, cudaStream_t st,
+                                const FusedTopk* fused = nullptr);
 size_t topk_scratch_bytes(int T, int64_t ld, int K);
 // Several CTAs per row use a region at the head of the scratch that must be
 // zero when they start (row counters + first-digit histogram, topk_zero_words

@@ -21,9 +21,21 @@
 //    weighting and the reduction over heads stay inside one thread; no
 //    [T, H_I, N] value ever leaves the SM.
 // The CTA grid is persistent (one CTA per SM) over the work items of k_plan.
+//
+// Decode (one token per group) can also select the Top-K inside the same
+// kernel, the fused scoring-weighting-selection operator of [P2] section 4(1)
+// and [P4] section 3.1: the epilogue keeps every score of the CTA's items in
+// shared memory as its order-preserving key (no score ever reaches global
+// memory), and once a CTA has scored its items it resolves, together with
+// the other CTAs holding parts of the same rows, the K-th largest key of
+// each row digit by digit (11, 11 and 10 bits) through per-row histograms in
+// global memory, then writes its own selections, ascending, at offsets
+// derived from per-item counts.  Rows meet through arrival counters with
+// bounded waits; the persistent grid (one CTA per SM) is all resident.
 #include <cudaTypedefs.h>
 
 #include "sm100.cuh"
+#include "topk_select.cuh"
 
 namespace dsa {
 
@@ -37,13 +49,40 @@ constexpr int kRecAhead = 6;                 // item records are fetched this ma
 constexpr int kPgAhead = 3;                  // page ids this many items ahead
 constexpr int kIdxThreads = (4 + kEpiWarps) * 32;
 
-template <bool kBf16, int TG>
+constexpr int kTailRuns = 32;                // rows a CTA can hold parts of (fused selection)
+constexpr int kTailItemsMax = 32;            // items a CTA can keep the scores of (fused selection)
+
+// Fast path of the fused selection: a row's candidates (keys whose first
+// digit reaches the row's threshold bin, typically a little over K) go to one
+// list per row that the CTA holding the row's last item resolves alone; it
+// emits the selected positions in order through two bitmaps over the row.
+constexpr int kCandCap = 6144;               // candidates per row
+constexpr int kBitmapWords = 4608;           // rows of up to 147,456 positions
+constexpr int kFastScratch = kCandCap * 8 + 2 * kBitmapWords * 4;  // in the score-key area
+
+// Shared-memory scratch of the fused selection tail.
+struct TailSmem {
+  uint32_t hist[kTopkHistBins];
+  uint32_t buf[33];
+  uint32_t bin, above;
+  int nruns, bad;
+  uint32_t red[8];
+  int4 item_info[kTailItemsMax];  // per item of the CTA: {token, position, tile begin, tile end}
+  int4 runs[kTailRuns];          // {token, first item, end item, position}
+  uint32_t prefix[kTailRuns];    // resolved high digits of the row's K-th key
+  uint32_t need[kTailRuns];      // selections still to find below the resolved digits
+  uint32_t ncand[kTailRuns];     // candidates of the row (first digit at or above its threshold bin)
+  int fast[kTailRuns];           // the row takes the candidate-list path
+};
+
+template <bool kBf16, int TG, bool kFused = false>
 struct IdxCfg {
+  static_assert(!kFused || TG == 1, "the fused selection serves one token per group");
   static constexpr int N = 64 * TG;                        // MMA N: heads x tokens of a group
   static constexpr int A_BYTES = kBf16 ? 32768 : 16384;    // 128 keys x d_I
   static constexpr int B_BYTES = kBf16 ? N * 256 : N * 128;
   static constexpr int KSTEPS = kBf16 ? 8 : 4;             // 32-byte K steps per tile
-  static constexpr int NS = kBf16 ? 3 : (TG == 1 ? 8 : 6);
+  static constexpr int NS = kBf16 ? 3 : (TG == 1 ? (kFused ? 6 : 8) : 6);
   static constexpr int NACC = (512 / N) < 4 ? (512 / N) : 4;
   static constexpr int TMEM_COLS = (NACC * N) <= 256 ? 256 : 512;
   // shared-memory layout (offsets from a 1024-aligned base)
@@ -52,15 +91,22 @@ struct IdxCfg {
   static constexpr int OFF_SC = OFF_B + 2 * B_BYTES;       // NS x 128 fp32 row scales
   static constexpr int OFF_W = OFF_SC + NS * 512;          // 2 x TG x 64 fp32 head weights
   static constexpr int OFF_HIST = OFF_W + 2 * TG * 256;   // TG == 1: per-epilogue-warp Top-K histograms
-  static constexpr int OFF_RING = OFF_HIST + (TG == 1 ? kEpiWarps * kTopkHistBins * 4 : 0);
+  static constexpr int OFF_RING = OFF_HIST + ((TG == 1 && !kFused) ? kEpiWarps * kTopkHistBins * 4 : 0);
   static constexpr int OFF_BAR = OFF_RING + kRingSlots * (32 + 128);  // producer's item records + page ids
   static constexpr int NBARS = 2 * NS + 4 + 2 * NACC + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
-  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int OFF_TAIL = (OFF_MISC + 16 + 15) / 16 * 16;     // fused: selection scratch
+  static constexpr int OFF_KEYS = OFF_TAIL + (kFused ? (int)((sizeof(TailSmem) + 15) / 16 * 16) : 0);
+  // fused: score keys of up to CAP_ITEMS items (1024 keys each) in shared memory
+  static constexpr int CAP_RAW = kFused ? (227 * 1024 - 1024 - OFF_KEYS) / 4096 : 0;
+  static constexpr int CAP_ITEMS = CAP_RAW < kTailItemsMax ? CAP_RAW : kTailItemsMax;
+  static constexpr int BYTES = OFF_KEYS + CAP_ITEMS * 4096;
   static constexpr int SMEM = BYTES + 1024;                // slack for 1024-byte alignment
   static constexpr uint32_t IDESC = make_idesc(kBf16, 128, N);
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(NACC * N <= TMEM_COLS, "TMEM");
+  static_assert(!kFused || CAP_ITEMS >= 8, "fused selection capacity");
+  static_assert(!kFused || CAP_ITEMS * 4096 >= kFastScratch, "fused selection fast-path scratch");
 };
 
 struct IdxArgs {
@@ -73,7 +119,360 @@ struct IdxArgs {
   uint32_t* hist;          // TG == 1 only, may be null: Top-K first-digit histogram [T][2048]
   uint32_t* err;
   uint64_t wait_ns;        // limit of each wait for another role's progress
+  // fused selection (zeroed by the call's prep kernel): per token
+  // [digit-1 hist 2048][digit-2 hist 2048][digit-3 hist 1024][arrivals 4][pad 4],
+  // then per item {keys > tau, keys == tau} of its CTA's run
+  uint32_t* tail;
+  int2* tail_items;
+  int2* cand;              // [T][kCandCap] (position, key) candidates, not zeroed
+  int32_t* idx;            // [T, K] selected positions
+  int K;
 };
+
+constexpr int kTailWords = kFusedTailWordsPerToken;  // per token
+static_assert(kTailWords == 2 * kTopkHistBins + topk::kD3Bins + 8, "fused tail layout");
+constexpr int kTailArrive = 2 * kTopkHistBins + topk::kD3Bins;  // 4 arrival counters
+constexpr int kTailCandCount = kTailArrive + 4;                  // candidates published so far
+
+// Waits (bounded) until the arrival counter at p has reached target.
+__device__ __forceinline__ bool wait_count(const uint32_t* p, uint32_t target, uint32_t* err, uint64_t limit) {
+  uint64_t t0 = 0;
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if (v >= target) return true;
+    const uint64_t now = globaltimer();
+    if (t0 == 0) {
+      t0 = now;
+    } else if (now - t0 > limit) {
+      raise_error(err, kErrTimeout);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
+// Selection of the min(K, pos+1) largest scores of every row this CTA holds
+// part of, from the keys in shared memory (slot (item - it_lo) * 1024 + i =
+// position 128 * tile_begin(item) + i).  All threads of the CTA take part.
+//   1. rows of at most K candidates select every position;
+//   2. the first digit's histogram of each row is summed over its CTAs and
+//      gives the threshold bin b1 (like dsa_topk's first step);
+//   3. fast path (the candidates fit one list per row): every CTA appends its
+//      candidates (first digit >= b1) to the row's list, and the CTA holding
+//      the row's last item resolves the other two digits in shared memory,
+//      marks the selected positions (key > tau; key == tau, the lowest
+//      positions first) in two bitmaps and writes them in ascending order;
+//   4. otherwise every CTA of the row resolves digits two and three through
+//      row histograms as well, then counts, per item, keys above and equal to
+//      tau, and writes its own selections at the offsets those counts give.
+// Rows meet at arrival counters (bounded waits).  A CTA takes its rows' steps
+// in the order 2, 3 (publish), 4, 3 (resolve), so a CTA resolving a row never
+// holds back a step another CTA waits on.
+__device__ void fused_topk_tail(const IdxArgs& a, uint32_t* keys, int it_lo, int it_hi, TailSmem& sm) {
+  using namespace topk;
+  const int tid = threadIdx.x, nthreads = blockDim.x;
+  const int4* recs = a.plan.items;
+  const int K = a.K;
+  const int nitems = it_hi - it_lo;  // <= kTailItemsMax (checked by the caller)
+  if (tid < nitems) {
+    const int4 ga = recs[2 * (it_lo + tid)], gb = recs[2 * (it_lo + tid) + 1];
+    sm.item_info[tid] = make_int4(ga.y, ga.w, gb.x, gb.y);  // {token, position, tile begin, tile end}
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int n = 0;
+    for (int i = 0; i < nitems; ++i) {
+      const int4 in = sm.item_info[i];
+      if (n > 0 && sm.runs[n - 1].x == in.x)
+        sm.runs[n - 1].z = it_lo + i + 1;
+      else if (n < kTailRuns)
+        sm.runs[n++] = make_int4(in.x, it_lo + i, it_lo + i + 1, in.y);
+    }
+    sm.nruns = n;
+    sm.bad = 0;
+  }
+  __syncthreads();
+  const int nruns = sm.nruns;
+  auto info = [&](int item) { return sm.item_info[item - it_lo]; };
+  auto run_s0 = [&](const int4& rn) { return 128 * info(rn.y).z; };  // first position of the run
+  auto items_total = [&](int pos) { return (uint32_t)((((pos >> 7) + 1) + 7) >> 3); };
+  auto holds_last = [&](const int4& rn) { return info(rn.z - 1).w == (rn.w >> 7) + 1; };
+  auto arrive = [&](int token, int counter, uint32_t v) {  // after a __syncthreads
+    if (tid == 0) {
+      __threadfence();
+      atomicAdd(a.tail + (int64_t)token * kTailWords + kTailArrive + counter, v);
+    }
+  };
+  auto wait_row = [&](int token, int counter, int pos) {  // every CTA of the row arrived; ends with a barrier
+    if (tid == 0 && !wait_count(a.tail + (int64_t)token * kTailWords + kTailArrive + counter, items_total(pos), a.err,
+                                a.wait_ns))
+      sm.bad = 1;
+    __syncthreads();
+    return !sm.bad;
+  };
+  auto load_hist = [&](const uint32_t* gh, int bins) {
+    for (int b = tid; b < bins; b += nthreads) sm.hist[b] = __ldcg(gh + b);
+    __syncthreads();
+  };
+  // 1. rows with at most K candidates: every candidate is selected, in order
+  for (int ri = 0; ri < nruns; ++ri) {
+    const int4 rn = sm.runs[ri];
+    const int pos = rn.w, n = pos + 1;
+    if (n > K) continue;
+    int32_t* out = a.idx + (int64_t)rn.x * K;
+    const int s0 = run_s0(rn), L = (rn.z - rn.y) * 1024;
+    for (int i = tid; i < L; i += nthreads)
+      if (s0 + i <= pos) out[s0 + i] = s0 + i;
+    if (holds_last(rn))  // the run holding the row's last tile pads it
+      for (int s = n + tid; s < K; s += nthreads) out[s] = -1;
+  }
+  // 2. first digit: row histograms, then the threshold bin of each row
+  for (int ri = 0; ri < nruns; ++ri) {
+    const int4 rn = sm.runs[ri];
+    if (rn.w + 1 <= K) continue;
+    for (int b = tid; b < kD1Bins; b += nthreads) sm.hist[b] = 0u;
+    __syncthreads();
+    const int s0 = run_s0(rn), L = (rn.z - rn.y) * 1024;
+    const uint32_t* kk = keys + (rn.y - it_lo) * 1024;
+    for (int i = tid; i < L; i += nthreads)
+      if (s0 + i <= rn.w) atomicAdd(&sm.hist[digit1(kk[i])], 1u);
+    __syncthreads();
+    uint32_t* gh = a.tail + (int64_t)rn.x * kTailWords;
+    for (int b = tid; b < kD1Bins; b += nthreads)
+      if (sm.hist[b]) atomicAdd(gh + b, sm.hist[b]);
+    __syncthreads();
+    arrive(rn.x, 0, (uint32_t)(rn.z - rn.y));
+  }
+  for (int ri = 0; ri < nruns; ++ri) {
+    const int4 rn = sm.runs[ri];
+    if (rn.w + 1 <= K) continue;
+    if (!wait_row(rn.x, 0, rn.w)) return;
+    load_hist(a.tail + (int64_t)rn.x * kTailWords, kD1Bins);
+    find_bin<kD1Bins>(sm.hist, (uint32_t)K, &sm.bin, &sm.above);
+    if (tid == 0) {
+      const uint32_t nc = sm.above + sm.hist[sm.bin];
+      sm.prefix[ri] = sm.bin;
+      sm.need[ri] = (uint32_t)K - sm.above;
+      sm.ncand[ri] = nc;
+      sm.fast[ri] = nc <= (uint32_t)kCandCap && rn.w + 1 <= 32 * kBitmapWords;
+    }
+    __syncthreads();
+  }
+  // 3 (publish). fast rows: this CTA's candidates into the row's list
+  for (int ri = 0; ri < nruns; ++ri) {
+    const int4 rn = sm.runs[ri];
+    if (rn.w + 1 <= K || !sm.fast[ri]) continue;
+    const uint32_t b1 = sm.prefix[ri];
+    const int s0 = run_s0(rn), L = (rn.z - rn.y) * 1024;
+    const uint32_t* kk = keys + (rn.y - it_lo) * 1024;
+    uint32_t cnt = 0;
+    for (int i = tid; i < L; i += nthreads) cnt += (s0 + i <= rn.w && digit1(kk[i]) >= b1) ? 1u : 0u;
+    if (tid < 2) sm.red[tid] = 0u;
+    __syncthreads();
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if ((tid & 31) == 0) atomicAdd(&sm.red[0], cnt);
+    __syncthreads();
+    if (tid == 0) sm.red[2] = atomicAdd(a.tail + (int64_t)rn.x * kTailWords + kTailCandCount, sm.red[0]);
+    __syncthreads();
+    const uint32_t base = sm.red[2];
+    int2* cl = a.cand + (int64_t)rn.x * kCandCap;
+    for (int i = tid; i < L; i += nthreads) {
+      const uint32_t key = kk[i];
+      if (s0 + i <= rn.w && digit1(key) >= b1) {
+        const uint32_t slot = base + atomicAdd(&sm.red[1], 1u);
+        if (slot < (uint32_t)kCandCap) cl[slot] = make_int2(s0 + i, (int)key);
+      }
+    }
+    __syncthreads();
+    arrive(rn.x, 1, (uint32_t)(rn.z - rn.y));
+  }
+  // 4. other rows: digits two and three through row histograms, then counts
+  for (int level = 1; level < 3 && !sm.bad; ++level) {
+    const int bins = level < 2 ? kD1Bins : kD3Bins;
+    for (int ri = 0; ri < nruns; ++ri) {
+      const int4 rn = sm.runs[ri];
+      if (rn.w + 1 <= K || sm.fast[ri]) continue;
+      for (int b = tid; b < bins; b += nthreads) sm.hist[b] = 0u;
+      __syncthreads();
+      const uint32_t prefix = sm.prefix[ri];
+      const int s0 = run_s0(rn), L = (rn.z - rn.y) * 1024;
+      const uint32_t* kk = keys + (rn.y - it_lo) * 1024;
+      for (int i = tid; i < L; i += nthreads) {
+        if (s0 + i > rn.w) continue;
+        const uint32_t key = kk[i];
+        if (level == 1 ? digit1(key) == prefix : (key >> 10) == prefix)
+          atomicAdd(&sm.hist[level == 1 ? digit2(key) : digit3(key)], 1u);
+      }
+      __syncthreads();
+      uint32_t* gh = a.tail + (int64_t)rn.x * kTailWords + (level == 1 ? kD1Bins : 2 * kD1Bins);
+      for (int b = tid; b < bins; b += nthreads)
+        if (sm.hist[b]) atomicAdd(gh + b, sm.hist[b]);
+      __syncthreads();
+      arrive(rn.x, level, (uint32_t)(rn.z - rn.y));
+    }
+    for (int ri = 0; ri < nruns; ++ri) {
+      const int4 rn = sm.runs[ri];
+      if (rn.w + 1 <= K || sm.fast[ri]) continue;
+      if (!wait_row(rn.x, level, rn.w)) return;
+      load_hist(a.tail + (int64_t)rn.x * kTailWords + (level == 1 ? kD1Bins : 2 * kD1Bins), bins);
+      if (level < 2)
+        find_bin<kD1Bins>(sm.hist, sm.need[ri], &sm.bin, &sm.above);
+      else
+        find_bin<kD3Bins>(sm.hist, sm.need[ri], &sm.bin, &sm.above);
+      if (tid == 0) {
+        sm.prefix[ri] = (sm.prefix[ri] << (level < 2 ? 11 : 10)) | sm.bin;
+        sm.need[ri] -= sm.above;
+      }
+      __syncthreads();
+    }
+  }
+  if (sm.bad) return;
+  // tau = the row's K-th largest key; need = how many tau-valued keys are taken
+  // (the lowest positions).  Per run: keys above tau and equal to it.
+  for (int ri = 0; ri < nruns; ++ri) {
+    const int4 rn = sm.runs[ri];
+    if (rn.w + 1 <= K || sm.fast[ri]) continue;
+    const uint32_t tau = sm.prefix[ri];
+    const int s0 = run_s0(rn), L = (rn.z - rn.y) * 1024;
+    const uint32_t* kk = keys + (rn.y - it_lo) * 1024;
+    uint32_t gt = 0, eq = 0;
+    for (int i = tid; i < L; i += nthreads) {
+      if (s0 + i > rn.w) continue;
+      const uint32_t key = kk[i];
+      gt += key > tau ? 1u : 0u;
+      eq += key == tau ? 1u : 0u;
+    }
+    if (tid < 2) sm.red[tid] = 0u;
+    __syncthreads();
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    eq = __reduce_add_sync(0xffffffffu, eq);
+    if ((tid & 31) == 0) {
+      atomicAdd(&sm.red[0], gt);
+      atomicAdd(&sm.red[1], eq);
+    }
+    __syncthreads();
+    if (tid == 0) a.tail_items[rn.y] = make_int2((int)sm.red[0], (int)sm.red[1]);
+    __syncthreads();
+    arrive(rn.x, 3, (uint32_t)(rn.z - rn.y));
+  }
+  for (int ri = 0; ri < nruns; ++ri) {
+    const int4 rn = sm.runs[ri];
+    if (rn.w + 1 <= K || sm.fast[ri]) continue;
+    if (tid < 2) sm.red[2 + tid] = 0u;
+    if (!wait_row(rn.x, 3, rn.w)) return;
+    // the row's selections in earlier items: counts of the runs before this one
+    const int first = rn.y - (info(rn.y).z >> 3);  // the row's first item
+    uint32_t bgt = 0, beq = 0;
+    for (int k = first + tid; k < rn.y; k += nthreads) {
+      const int2 c = __ldcg(a.tail_items + k);
+      bgt += (uint32_t)c.x;
+      beq += (uint32_t)c.y;
+    }
+    bgt = __reduce_add_sync(0xffffffffu, bgt);
+    beq = __reduce_add_sync(0xffffffffu, beq);
+    if ((tid & 31) == 0) {
+      atomicAdd(&sm.red[2], bgt);
+      atomicAdd(&sm.red[3], beq);
+    }
+    __syncthreads();
+    const uint32_t tau = sm.prefix[ri], r = sm.need[ri];
+    const uint32_t taken_eq = min(sm.red[3], r);
+    const uint32_t off = sm.red[2] + taken_eq;
+    const int s0 = run_s0(rn), L = (rn.z - rn.y) * 1024, pos = rn.w;
+    const uint32_t* kk = keys + (rn.y - it_lo) * 1024;
+    emit_selected(
+        L, tau, r - taken_eq, K - (int)off,
+        [&](int i) { return make_int2(s0 + i, s0 + i <= pos ? (int)kk[i] : 0); },
+        a.idx + (int64_t)rn.x * K + off, sm.buf);
+    __syncthreads();
+  }
+  // 3 (resolve). fast rows whose last item is here: the rest of the
+  // selection from the row's candidate list, in shared memory (the score keys
+  // are no longer needed: every step above that reads them is done)
+  int2* cands = reinterpret_cast<int2*>(keys);
+  uint32_t* gt_bits = reinterpret_cast<uint32_t*>(keys + 2 * kCandCap);
+  uint32_t* eq_bits = gt_bits + kBitmapWords;
+  for (int ri = 0; ri < nruns; ++ri) {
+    const int4 rn = sm.runs[ri];
+    if (rn.w + 1 <= K || !sm.fast[ri] || !holds_last(rn)) continue;
+    if (!wait_row(rn.x, 1, rn.w)) return;
+    const int nc = (int)sm.ncand[ri];
+    const int2* cl = a.cand + (int64_t)rn.x * kCandCap;
+    for (int i = tid; i < nc; i += nthreads) cands[i] = __ldcg(cl + i);
+    const int nw = (rn.w + 32) >> 5;  // bitmap words of the row
+    for (int w = tid; w < nw; w += nthreads) {
+      gt_bits[w] = 0u;
+      eq_bits[w] = 0u;
+    }
+    uint32_t prefix = sm.prefix[ri], need = sm.need[ri];
+    for (int level = 1; level < 3; ++level) {  // digits two and three, over the candidates only
+      const int bins = level < 2 ? kD1Bins : kD3Bins;
+      for (int b = tid; b < bins; b += nthreads) sm.hist[b] = 0u;
+      __syncthreads();
+      for (int i = tid; i < nc; i += nthreads) {
+        const uint32_t key = (uint32_t)cands[i].y;
+        if (level == 1 ? digit1(key) == prefix : (key >> 10) == prefix)
+          atomicAdd(&sm.hist[level == 1 ? digit2(key) : digit3(key)], 1u);
+      }
+      __syncthreads();
+      if (level < 2)
+        find_bin<kD1Bins>(sm.hist, need, &sm.bin, &sm.above);
+      else
+        find_bin<kD3Bins>(sm.hist, need, &sm.bin, &sm.above);
+      prefix = (prefix << (level < 2 ? 11 : 10)) | sm.bin;
+      need -= sm.above;
+      __syncthreads();  // every thread has read bin / above
+    }
+    const uint32_t tau = prefix, r = need;  // r: tau-valued keys taken, the lowest positions first
+    for (int i = tid; i < nc; i += nthreads) {
+      const int2 c = cands[i];
+      if ((uint32_t)c.y > tau)
+        atomicOr(&gt_bits[c.x >> 5], 1u << (c.x & 31));
+      else if ((uint32_t)c.y == tau)
+        atomicOr(&eq_bits[c.x >> 5], 1u << (c.x & 31));
+    }
+    __syncthreads();
+    // ascending emission: each thread takes a run of consecutive words
+    const int per = (nw + nthreads - 1) / nthreads;
+    const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
+    uint32_t my_gt = 0, my_eq = 0;
+    for (int w = w0; w < w1; ++w) {
+      my_gt += (uint32_t)__popc(gt_bits[w]);
+      my_eq += (uint32_t)__popc(eq_bits[w]);
+    }
+    uint32_t tot;
+    uint32_t gt_before = block_scan(my_gt, sm.buf, &tot);
+    uint32_t eq_before = block_scan(my_eq, sm.buf, &tot);
+    int32_t* out = a.idx + (int64_t)rn.x * K;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t g = gt_bits[w], e = eq_bits[w];
+      // eq bits of this word that are among the first r overall
+      const uint32_t e_cnt = (uint32_t)__popc(e);
+      if (eq_before >= r) {
+        e = 0u;
+      } else if (eq_before + e_cnt > r) {
+        uint32_t keep = r - eq_before, m = 0u, x = e;
+        while (keep--) {
+          const uint32_t low = x & (~x + 1u);
+          m |= low;
+          x ^= low;
+        }
+        e = m;
+      }
+      eq_before += e_cnt;
+      uint32_t sel = g | e;
+      while (sel) {
+        const int bit = __ffs(sel) - 1;
+        sel &= sel - 1u;
+        const uint32_t slot = gt_before + min(eq_before - e_cnt, r) + (uint32_t)__popc((g | e) & ((1u << bit) - 1u));
+        if (slot < (uint32_t)K) out[slot] = (w << 5) + bit;
+      }
+      gt_before += (uint32_t)__popc(g);
+    }
+    __syncthreads();
+  }
+}
 
 // Adds one epilogue warp's histogram of the current token to the global one
 // and clears it (warp-private, so only the warp synchronises).
@@ -89,11 +488,11 @@ __device__ __forceinline__ void flush_hist(uint32_t* sh, uint32_t* gh, int t, in
   __syncwarp();
 }
 
-template <bool kBf16, int TG>
+template <bool kBf16, int TG, bool kFused>
 __global__ void __launch_bounds__(kIdxThreads, 1)
 k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                   const IdxArgs a) {
-  using C = IdxCfg<kBf16, TG>;
+  using C = IdxCfg<kBf16, TG, kFused>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -321,7 +720,8 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
     int stage = 0, sphase = 0, acc = 0, aphase = 0, prev_g = -1, gcount = 0, slot = 0, prev_t = -1, ti = 0;
     float wreg[64];
     uint32_t* sh_hist = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST) + (warp - 4) * kTopkHistBins;
-    const bool do_hist = TG == 1 && a.hist != nullptr;
+    const bool do_hist = TG == 1 && !kFused && a.hist != nullptr;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem + C::OFF_KEYS);
     if (do_hist) {
       for (int i = lane; i < kTopkHistBins; i += 32) sh_hist[i] = 0u;
       __syncwarp();
@@ -389,8 +789,14 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
             }
             const float score = ((p0 + p1) + (p2 + p3)) * sk;
             const bool valid = k < grp.z && s <= grp.w + k;
-            if (valid) a.scores[(int64_t)(grp.y + k) * a.ld + s] = score;
-            if (do_hist) hist_add(sh_hist, order_key(score) >> kTopkLowBits, valid);
+            if constexpr (kFused) {
+              // the host sizes the grid so that a CTA's items fit; the guard keeps
+              // an oversized share from writing past the buffer all the same
+              if (it - it_lo < C::CAP_ITEMS) keys[(it - it_lo) * 1024 + (tile - item.y) * 128 + r] = order_key(score);
+            } else {
+              if (valid) a.scores[(int64_t)(grp.y + k) * a.ld + s] = score;
+              if (do_hist) hist_add(sh_hist, order_key(score) >> kTopkLowBits, valid);
+            }
           }
         }
         if (++stage == C::NS) { stage = 0; sphase ^= 1; }
@@ -405,6 +811,13 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if constexpr (kFused) {
+    // the selection, once every score of this CTA is in shared memory (the
+    // barrier above); a CTA that gave up on a wait leaves its rows to time out
+    if (!*abort_flag && it_hi - it_lo <= C::CAP_ITEMS)
+      fused_topk_tail(a, reinterpret_cast<uint32_t*>(smem + C::OFF_KEYS), it_lo, it_hi,
+                      *reinterpret_cast<TailSmem*>(smem + C::OFF_TAIL));
   }
 }
 
@@ -443,42 +856,80 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <bool kBf16, int TG>
-cudaError_t launch_tc(const CUtensorMap& mk, const CUtensorMap& mq, const IdxArgs& a, cudaStream_t st) {
-  using C = IdxCfg<kBf16, TG>;
+template <bool kBf16, int TG, bool kFused>
+cudaError_t launch_tc(const CUtensorMap& mk, const CUtensorMap& mq, const IdxArgs& a, int grid, cudaStream_t st) {
+  using C = IdxCfg<kBf16, TG, kFused>;
   static thread_local int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(k_index_scores_tc<kBf16, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(k_index_scores_tc<kBf16, TG, kFused>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  cudaError_t e = launch_pdl("index_scores", k_index_scores_tc<kBf16, TG>, dim3(sm_count()), dim3(kIdxThreads), (size_t)C::SMEM, st, mk,
-                             mq, a);
+  cudaError_t e = launch_pdl("index_scores", k_index_scores_tc<kBf16, TG, kFused>, dim3(grid), dim3(kIdxThreads),
+                             (size_t)C::SMEM, st, mk, mq, a);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }
 
 }  // namespace
 
+int indexer_fused_capacity() {
+  const int a = IdxCfg<false, 1, true>::CAP_ITEMS, b = IdxCfg<true, 1, true>::CAP_ITEMS;
+  return a < b ? a : b;
+}
+
+bool indexer_fused_fits(int T, int B, int max_ctx) {
+  if (T != B) return false;  // one query token per sequence
+  const int64_t items = plan_max_items(T, B, max_ctx, 1);
+  return (items + kFusedGrid - 1) / kFusedGrid <= indexer_fused_capacity();
+}
+
+int64_t fused_topk_words(int T, int B, int max_ctx) {
+  return (int64_t)T * kTailWords + 2 * plan_max_items(T, B, max_ctx, 1);
+}
+
+size_t fused_topk_cand_bytes(int T) { return (size_t)T * kCandCap * sizeof(int2); }
+
 cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
                                 const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
-                                float* scores, int64_t ld, uint32_t* hist, uint32_t* err, cudaStream_t st) {
+                                float* scores, int64_t ld, uint32_t* hist, uint32_t* err, cudaStream_t st,
+                                const FusedTopk* fused) {
   const bool bf16 = !fp8;
   const uint64_t R = (uint64_t)s.num_phys_pages * kPage;
   const uint64_t qrows = (uint64_t)s.num_tokens * kHI;
   CUtensorMap mk, mq;
   if (!make_map(&mk, kI, bf16, kDI, R, bf16 ? 64 : 128, 64)) return cudaErrorInvalidValue;
   if (!make_map(&mq, q_operand, bf16, kDI, qrows, bf16 ? 64 : 128, 64 * tg)) return cudaErrorInvalidValue;
-  IdxArgs a{s, plan, w_operand, kI_scale, scores, ld, tg == 1 ? hist : nullptr, err, wait_limit_ns()};
+  IdxArgs a{s,
+            plan,
+            w_operand,
+            kI_scale,
+            scores,
+            ld,
+            tg == 1 ? hist : nullptr,
+            err,
+            wait_limit_ns(),
+            fused ? fused->tail : nullptr,
+            fused ? fused->tail_items : nullptr,
+            fused ? fused->cand : nullptr,
+            fused ? fused->idx : nullptr,
+            fused ? fused->K : 0};
+  const int grid = sm_count();
+  if (fused) {
+    // the rows' CTAs wait on one another: every CTA must be resident (one per
+    // SM) and hold at most the capacity the workspace was sized for
+    if (tg != 1 || grid < kFusedGrid) return cudaErrorInvalidConfiguration;
+    return fp8 ? launch_tc<false, 1, true>(mk, mq, a, kFusedGrid, st) : launch_tc<true, 1, true>(mk, mq, a, kFusedGrid, st);
+  }
   if (fp8) {
-    if (tg == 1) return launch_tc<false, 1>(mk, mq, a, st);
-    if (tg == 4) return launch_tc<false, 4>(mk, mq, a, st);
+    if (tg == 1) return launch_tc<false, 1, false>(mk, mq, a, grid, st);
+    if (tg == 4) return launch_tc<false, 4, false>(mk, mq, a, grid, st);
   } else {
-    if (tg == 1) return launch_tc<true, 1>(mk, mq, a, st);
-    if (tg == 2) return launch_tc<true, 2>(mk, mq, a, st);
+    if (tg == 1) return launch_tc<true, 1, false>(mk, mq, a, grid, st);
+    if (tg == 2) return launch_tc<true, 2, false>(mk, mq, a, grid, st);
   }
   return cudaErrorInvalidValue;
 }

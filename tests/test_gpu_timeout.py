@@ -58,6 +58,12 @@ def test_fused_wait_runs_out_then_next_call_is_clean(lib):
 
     _short_limit(lib, call)
     assert lib.dsa_check_error(ws) == lib.DSA_ERR_TIMEOUT
+    # the selection inside the indexer waits across CTAs too: let those waits run out
+    ws_f = torch.zeros(lib.dsa_workspace_size(lib.DSA_OP_INDEX_TOPK_ATTN_FUSED, d.seqs, K, H), dtype=torch.uint8,
+                       device="cuda")
+    _short_limit(lib, lambda: lib.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale,
+                                                      ws=ws_f, select_in_indexer=True))
+    assert lib.dsa_check_error(ws_f) == lib.DSA_ERR_TIMEOUT
     out, lse = call(out_dtype=torch.float32)
     assert lib.dsa_check_error(ws) == lib.DSA_OK
     tokens = np.arange(wl.T)
