@@ -36,7 +36,11 @@ Readings taken where the pages are silent (each repeated at its function):
   * a row with fewer than K candidates takes all of them, index list padded
     with -1, and the selected indices are emitted in ascending order;
   * the FP8 index cache is OCP E4M3 with one fp32 scale per token row; the bf16
-    index query is quantized per (token, head) with a power-of-two scale.
+    index query is quantized per (token, head) with a power-of-two scale;
+  * MXFP8 (the pages' index format: one shared scale per group of 32) is read
+    as the OCP Microscaling format: E4M3 elements sharing an E8M0 power-of-two
+    scale per block of 32, the scale 2^(floor(log2 amax) - 8), elements of the
+    block's top binade above 448 saturating.  Cache and query both take it.
 
 Every function here is pinned by a test in ``tests/test_oracle_*.py`` against
 something other than itself (library routines, brute force, closed forms,
@@ -148,6 +152,68 @@ def quantize_index_query(qI_bits):
 
 
 # ----------------------------------------------------------------------------
+# MXFP8 ([P2] §5 table, "Indexer Q/K": MXFP8 dynamic quantization, per group of
+# 32 elements sharing one scale factor; [P3] §4 "Layered Quantization"; [P4]
+# §4.2 "Per-Group Dynamic Quantization")
+# ----------------------------------------------------------------------------
+
+MX_BLOCK = 32        # elements sharing one scale
+E8M0_BIAS = 127
+E4M3_EMAX = 8        # exponent of E4M3's top binade: 448 = 1.75 * 2^8
+
+
+def e8m0_decode(codes) -> np.ndarray:
+    """Exact value of E8M0 scale codes: 2^(code - 127), code 255 is NaN.  E8M0
+    (8 exponent bits, no sign, no mantissa) is the shared-scale format of the
+    OCP Microscaling formats, of which MXFP8 is the E4M3 member."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    v = np.ldexp(1.0, c - E8M0_BIAS)
+    return np.where(c == 255, np.nan, v)
+
+
+def mx_shared_exponent(amax: float) -> int:
+    """Exponent e of one block's scale 2^e: floor(log2(amax)) - 8, so that the
+    block's largest magnitude lands in E4M3's top binade [256, 512); clamped to
+    E8M0's range [-127, 127].  An all-zero block takes e = 0 (reading: the
+    format leaves it open, and any scale encodes zeros)."""
+    amax = float(amax)
+    if amax == 0.0:
+        return 0
+    _, ex = math.frexp(amax)           # amax = m * 2^ex, 0.5 <= m < 1: floor(log2 amax) = ex - 1
+    return int(min(127, max(-127, ex - 1 - E4M3_EMAX)))
+
+
+def mxfp8_quantize(x):
+    """Real values [..., n] (n a multiple of 32) -> (E4M3 codes [..., n],
+    E8M0 scale codes [..., n/32]).  Block i covers elements 32i .. 32i+31 of
+    the last axis; codes = E4M3(x / 2^e) rounded to nearest-even and saturated
+    at +-448 (``e4m3_encode``), e = ``mx_shared_exponent(max |block|)``."""
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[-1]
+    if n % MX_BLOCK:
+        raise ValueError("the last axis must be a multiple of 32")
+    blocks = x.reshape(*x.shape[:-1], n // MX_BLOCK, MX_BLOCK)
+    amax = np.abs(blocks).max(axis=-1)
+    e = np.vectorize(mx_shared_exponent, otypes=[np.int64])(amax)
+    codes = e4m3_encode(blocks / np.ldexp(1.0, e)[..., None])
+    return codes.reshape(x.shape), (e + E8M0_BIAS).astype(np.uint8)
+
+
+def mxfp8_dequantize(codes, scales) -> np.ndarray:
+    """Exact value of MXFP8 data: E4M3(codes) * 2^(scale - 127) per block of 32."""
+    c = np.asarray(codes, dtype=np.uint8)
+    n = c.shape[-1]
+    v = e4m3_decode_fast(c).reshape(*c.shape[:-1], n // MX_BLOCK, MX_BLOCK)
+    return (v * e8m0_decode(scales)[..., None]).reshape(c.shape)
+
+
+def is_mx_scale(kI_scale) -> bool:
+    """An MXFP8 index cache carries E8M0 codes [R, 4] (uint8); an E4M3 cache one
+    fp32 scale per row."""
+    return kI_scale is not None and np.asarray(kI_scale).dtype == np.uint8
+
+
+# ----------------------------------------------------------------------------
 # Sequences and the paged caches
 # ([P2] §2 item 2: the indexer reads the paged K cache directly;
 #  [P5] "Operator Fusion and Memory Access Optimization for Sparse Attention
@@ -209,13 +275,20 @@ def index_scores(seqs: Seqs, qI_bits, w, kI, kI_scale=None, tokens=None):
     qI is replaced by its quantized form E4M3(q^)[t,h] * sq[t,h]
     (``quantize_index_query``); since sq, kI_scale > 0 the ReLU commutes with
     them, so the score is  kI_scale[s] * sum_h w[t,h] sq[t,h] ReLU(q^ . k^).
+    MXFP8 index cache (kI_scale = E8M0 codes [R, 4], ``is_mx_scale``): kI[s] =
+    ``mxfp8_dequantize(codes[s], kI_scale[s])`` and each (token, head) row of
+    qI is replaced by ``mxfp8_dequantize(*mxfp8_quantize(row))``; the scores
+    are the formula above on those values.
 
     Returns a list with one float64 array of length pos(t)+1 per token
     (in the order of ``tokens``; all tokens when None).
     """
     w = np.asarray(w, dtype=np.float64)
-    fp8 = kI_scale is not None
-    if fp8:
+    mx = is_mx_scale(kI_scale)
+    fp8 = kI_scale is not None and not mx
+    if mx:
+        qvals = mxfp8_dequantize(*mxfp8_quantize(bf16_to_f64(qI_bits)))
+    elif fp8:
         qhat, sq = quantize_index_query(qI_bits)
         qvals = e4m3_decode_fast(qhat)
     else:
@@ -224,7 +297,10 @@ def index_scores(seqs: Seqs, qI_bits, w, kI, kI_scale=None, tokens=None):
     for t in _token_list(seqs, tokens):
         b, pos = seqs.token_seq_pos(t)
         rows = seqs.rows(b, np.arange(pos + 1))
-        if fp8:
+        if mx:
+            kmat = mxfp8_dequantize(np.asarray(kI)[rows], np.asarray(kI_scale)[rows])
+            wt = w[t]
+        elif fp8:
             kmat = e4m3_decode_fast(np.asarray(kI)[rows])
             wt = w[t] * sq[t]
         else:

@@ -17,6 +17,7 @@ ORACLE = os.path.join(ROOT, "oracle", "dsa_oracle.py")
 
 CODEC, QUANT, INDEXER = "test_oracle_codec.py", "test_oracle_quant.py", "test_oracle_indexer.py"
 TOPK, ATTN, PIPE = "test_oracle_topk.py", "test_oracle_attention.py", "test_oracle_pipeline.py"
+MX = "test_oracle_mx.py"
 
 # name: (text in the oracle, replacement, pin files that must fail)
 MUTANTS = {
@@ -52,6 +53,17 @@ MUTANTS = {
     "dense_mask_one_short": ("logit[: pos + 1] = scale * (full[: pos + 1] @ qh)",
                              "logit[: pos] = scale * (full[: pos] @ qh)", [ATTN]),
     "path_rows_to_wrong_tokens": ("full_idx[t] = idx_rows[i]", "full_idx[i] = idx_rows[i]", [PIPE]),
+    "mx_exponent_off_by_one": ("ex - 1 - E4M3_EMAX", "ex - E4M3_EMAX", [MX]),
+    "mx_no_clamp": ("return int(min(127, max(-127, ex - 1 - E4M3_EMAX)))", "return int(ex - 1 - E4M3_EMAX)", [MX]),
+    "mx_block_16": ("MX_BLOCK = 32        # elements sharing one scale", "MX_BLOCK = 16        # elements sharing one scale",
+                    [MX]),
+    "mx_e8m0_bias": ("v = np.ldexp(1.0, c - E8M0_BIAS)", "v = np.ldexp(1.0, c - E8M0_BIAS + 1)", [MX]),
+    "mx_query_not_quantized": ("qvals = mxfp8_dequantize(*mxfp8_quantize(bf16_to_f64(qI_bits)))",
+                               "qvals = bf16_to_f64(qI_bits)", [MX]),
+    "mx_key_scale_dropped": ("kmat = mxfp8_dequantize(np.asarray(kI)[rows], np.asarray(kI_scale)[rows])",
+                             "kmat = e4m3_decode_fast(np.asarray(kI)[rows])", [MX]),
+    "mx_key_scale_wrong_row": ("kmat = mxfp8_dequantize(np.asarray(kI)[rows], np.asarray(kI_scale)[rows])",
+                               "kmat = mxfp8_dequantize(np.asarray(kI)[rows], np.asarray(kI_scale)[rows[::-1]])", [MX]),
 }
 
 
