@@ -74,6 +74,8 @@ def parse():
                     help="override the workload's context length (profiling a smaller case of the same kernels)")
     ap.add_argument("--all-configs", action="store_true",
                     help="one JSON line per workload: fused-call time and the binding roofline of each stage")
+    ap.add_argument("--ki", choices=["workload", "mxfp8"], default="workload",
+                    help="index-cache format: the workload's own (E4M3 + row scale for the headline) or MXFP8")
     ap.add_argument("--select-in-indexer", action="store_true",
                     help="decode: select the Top-K inside the indexer kernel (DSA_SELECT_IN_INDEXER)")
     ap.add_argument("--only", choices=["index_scores", "topk", "sparse_mla", "fused"], default=None,
@@ -245,14 +247,26 @@ def workload_config(spec, wl, world: int) -> dict:
     return {"workload": spec.name, "batch_per_gpu": spec.batch, "global_batch": wl.T * world,
             "ctx": int(wl.ctx_len[0]), "topk": spec.topk, "heads": spec.heads, "index_heads": spec.index_heads,
             "index_dim": spec.index_dim, "page_size": spec.page_size, "pool_tokens": wl.num_phys_pages * 64,
-            "index_cache": "fp8_e4m3" if spec.ki_fp8 else "bf16", "parallelism": f"dp{world}",
+            "index_cache": "mxfp8" if spec.ki_mx else ("fp8_e4m3" if spec.ki_fp8 else "bf16"),
+            "parallelism": f"dp{world}",
             "l2": "256 MiB buffer written before every timed GPU step"}
+
+
+def bench_spec(args):
+    """The workload both arms measure: the named config, with the index-cache
+    format and context length the flags ask for."""
+    spec = CONFIGS[args.config]
+    if args.ki == "mxfp8":
+        spec = spec.scaled(ki_mx=True)
+    if args.ctx > 0:
+        spec = spec.scaled(ctx=(args.ctx, args.ctx))
+    return spec
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    spec = CONFIGS[args.config]
+    spec = bench_spec(args)
     wl = make_workload(spec)
     n_tok = wl.T                                   # one step = the whole batch, as in our arm
     for _ in range(args.warmup):
@@ -351,7 +365,7 @@ def run_all_configs(args, dsa, dev, stream, flush):
     from dsa_workloads import to_device
     hbm, hbm_src = hbm_peak()
     for name in CONFIGS:
-        spec = CONFIGS[name]
+        spec = CONFIGS[name].scaled(ki_mx=True) if args.ki == "mxfp8" else CONFIGS[name]
         wl = make_workload(spec)
         d = to_device(wl)
         T, H, K = wl.T, spec.heads, spec.topk
@@ -432,10 +446,7 @@ def run_ours(args, world, rank, local):
         run_all_configs(args, dsa, dev, torch.cuda.current_stream(dev),
                         torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev))
         return
-    spec = CONFIGS[args.config]
-    if args.ctx > 0:
-        spec = spec.scaled(ctx=(args.ctx, args.ctx))
-    spec = rank_spec(spec, rank)                         # each rank serves its own batch
+    spec = rank_spec(bench_spec(args), rank)                         # each rank serves its own batch
     wl = make_workload(spec)
     d = to_device(wl)
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -572,7 +583,8 @@ def run_ours(args, world, rank, local):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 index / bf16 attention / fp32 accum",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": ("mxfp8" if spec.ki_mx else "fp8-e4m3") + " index / bf16 attention / fp32 accum",
             "data": "synthetic (seeded, 64 planted keys per sequence)",
             "config": workload_config(spec, wl, world),
             "launch": launch_mode,

@@ -24,9 +24,12 @@ the order written below):
      u = sum_h max(w[h], 0) qI[h] of the sequence's query; latent row :=
      3*sqrt(576) * g/|g| with g the mean over heads of the query q.  Their
      purpose is a known, clearly separated relevant set;
-  6. storage: latent KV as bf16; index keys as bf16 (bf16 cache) or as FP8 E4M3
+  6. storage: latent KV as bf16; index keys as bf16 (bf16 cache), as FP8 E4M3
      codes with one fp32 scale per row, scale = max|row| / 448 (1 for a zero
-     row), codes = E4M3(row / scale) by torch's round-to-nearest cast.
+     row), codes = E4M3(row / scale) by torch's round-to-nearest cast, or as
+     MXFP8: E4M3 codes with one E8M0 scale byte per 32 elements, scale
+     2^(floor(log2 max|block|) - 8) (2^0 for a zero block), codes =
+     E4M3(block / scale) clamped to +-448, by the same cast.
 """
 from __future__ import annotations
 
@@ -48,6 +51,7 @@ class Spec:
     prefix: tuple = (0, 0)          # chunked: cached prefix length range
     chunk: tuple = (0, 0)           # chunked: new chunk length range
     ki_fp8: bool = True             # FP8 E4M3 index cache with per-row scale
+    ki_mx: bool = False             # MXFP8 index cache (E4M3 + E8M0 per 32 elements); overrides ki_fp8
     heads: int = 128                # attention query heads
     topk: int = 2048
     planted: int = 0
@@ -88,7 +92,7 @@ class Workload:
     qI: torch.Tensor               # bf16 [T, H_I, d_I]
     w: torch.Tensor                # fp32 [T, H_I]
     kI: torch.Tensor               # uint8 FP8 codes or bf16 [R, d_I]
-    kI_scale: torch.Tensor | None  # fp32 [R] (FP8 cache) or None
+    kI_scale: torch.Tensor | None  # fp32 [R] (FP8 cache), uint8 E8M0 [R, 4] (MXFP8) or None
     q: torch.Tensor                # bf16 [T, H, d_qk]
     kv: torch.Tensor               # bf16 [R, d_qk]
     planted: list                  # per sequence: np.ndarray of planted positions
@@ -141,6 +145,19 @@ def fp8_rows(x: torch.Tensor):
     scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
     codes = (x / scale[:, None]).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
     return codes, scale.to(torch.float32)
+
+
+def mx_rows(x: torch.Tensor):
+    """Store fp32 rows as MXFP8 (cache format): E4M3 codes [R, d] and one E8M0
+    scale byte per 32 elements [R, d/32]."""
+    R, d = x.shape
+    blocks = x.reshape(R, d // 32, 32)
+    amax = blocks.abs().amax(dim=2)
+    _, ex = torch.frexp(amax)                      # amax = m * 2^ex, 0.5 <= m < 1
+    e = torch.where(amax > 0, (ex - 9).clamp(-127, 127), torch.zeros_like(ex))
+    codes = (blocks * torch.exp2(-e.to(torch.float32))[..., None]).clamp_(-448.0, 448.0)
+    codes = codes.to(torch.float8_e4m3fn).view(torch.uint8).reshape(R, d)
+    return codes, (e + 127).to(torch.uint8)
 
 
 def make_workload(spec: Spec) -> Workload:
@@ -220,7 +237,13 @@ def make_workload(spec: Spec) -> Workload:
     kv = torch.zeros((R, spec.d_qk), dtype=torch.bfloat16)
     kv[phys_rows] = kv_vals.to(torch.bfloat16)
     del kv_vals
-    if spec.ki_fp8:
+    if spec.ki_mx:
+        codes, sc = mx_rows(ki_vals)
+        kI = torch.zeros((R, d_I), dtype=torch.uint8)
+        kI[phys_rows] = codes
+        kI_scale = torch.full((R, d_I // 32), 127, dtype=torch.uint8)
+        kI_scale[phys_rows] = sc
+    elif spec.ki_fp8:
         codes, sc = fp8_rows(ki_vals)
         kI = torch.zeros((R, d_I), dtype=torch.uint8)
         kI[phys_rows] = codes

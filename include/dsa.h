@@ -37,8 +37,10 @@
  *   (q_len = 1), prefill (q_len = ctx) and chunked prefill share one form.
  * Paged pools.  Logical position s of sequence b lives in physical row
  *   page_table[b*max_pages + s/64]*64 + s%64 of each pool (page size 64).
- *   Pools: index keys kI [R, 128] (bf16, or FP8 E4M3 codes with one fp32 scale
- *   per row in kI_scale [R]) and latent KV [R, 576] bf16, R = num_phys_pages*64.
+ *   Pools: index keys kI [R, 128] (bf16; FP8 E4M3 codes with one fp32 scale
+ *   per row in kI_scale [R]; or MXFP8: E4M3 codes with one E8M0 scale byte
+ *   per 32 elements in kI_scale [R, 4]) and latent KV [R, 576] bf16,
+ *   R = num_phys_pages*64.
  * Fixed sizes.  Index heads H_I = 64, index dim d_I = 128, latent dims
  *   576 (keys) / 512 (values), page size 64.  Attention heads H in {16, 32,
  *   64, 128}.  1 <= K <= 2048.  Anything else returns DSA_ERR_UNSUPPORTED.
@@ -92,7 +94,11 @@ typedef enum {
 
 typedef enum {
   DSA_KI_BF16 = 0,     /* kI pool is bf16 [R,128]; kI_scale must be NULL         */
-  DSA_KI_FP8_E4M3 = 1  /* kI pool is OCP E4M3 codes [R,128] + fp32 kI_scale [R] */
+  DSA_KI_FP8_E4M3 = 1, /* kI pool is OCP E4M3 codes [R,128] + fp32 kI_scale [R] */
+  DSA_KI_MXFP8 = 2     /* kI pool is OCP E4M3 codes [R,128] + E8M0 kI_scale
+                          uint8 [R,4]: byte g scales elements 32g..32g+31 by
+                          2^(byte - 127) ([P2] section 5 table, "Indexer Q/K":
+                          MXFP8, one shared scale per group of 32; [P4] 4.2) */
 } dsa_ki_dtype_t;
 
 typedef enum {
@@ -162,19 +168,33 @@ dsa_status_t dsa_quantize_index_query(const void *qI, const float *w, int T,
                                       uint8_t *codes, float *w_scaled,
                                       dsa_stream_t stream);
 
+/* MXFP8 index-query quantization (the query side of DSA_KI_MXFP8; format:
+ * [P2] section 5 table, "Indexer Q/K", one shared scale per group of 32;
+ * [P4] section 4.2 per-group dynamic quantization).  For every group of 32
+ * elements g of row (t,h): e = floor(log2(max |group|)) - 8 clamped to
+ * [-127, 127] (e = 0 for an all-zero group); scales[t,h,g] = e + 127 (E8M0);
+ * codes = E4M3(group / 2^e) rounded to nearest-even with saturation at 448.
+ *   qI bf16 [T,64,128]; codes uint8 E4M3 [T,64,128] (out); scales uint8
+ *   [T,64,4] (out).  No workspace.  Errors: DSA_ERR_INVALID_ARG / DSA_ERR_CUDA. */
+dsa_status_t dsa_quantize_index_query_mx(const void *qI, int T, uint8_t *codes,
+                                         uint8_t *scales, dsa_stream_t stream);
+
 /* Lightweight-indexer scores ([P2] section 2 item 2 and section 4(1); [P3]
  * sections 1 and 3 `fused_lightning_indexer`; [P4] section 3.1): for every
  * query token t and candidate s = 0..pos(t),
  *   scores[t*ld + s] = sum_h w[t,h] * ReLU(qI[t,h,:] . kI[s,:]).
  * FP8 cache: kI[s] = E4M3(codes[s]) * kI_scale[s] and qI is first quantized as
  * in dsa_quantize_index_query (the scores are those of the quantized qI).
+ * MXFP8 cache: kI[s,32g..32g+31] = E4M3(codes) * 2^(kI_scale[s,g] - 127) and qI
+ * is first quantized as in dsa_quantize_index_query_mx; the group scales are
+ * applied by the tensor core's block-scaled MMA.
  * Entries s > pos(t) of a row are left untouched.  ld >= max_ctx.
  * The reduction over heads happens in the kernel; no [T,H_I,N] tensor exists.
- *   qI bf16 [T,64,128]; w fp32 [T,64]; kI pool; kI_scale fp32 [R] or NULL;
- *   scores fp32 [T,ld] (out). */
+ *   qI bf16 [T,64,128]; w fp32 [T,64]; kI pool; kI_scale fp32 [R], uint8
+ *   [R,4] (MXFP8) or NULL (bf16); scores fp32 [T,ld] (out). */
 dsa_status_t dsa_index_scores(const dsa_seqs_t *seqs, const void *qI,
                               const float *w, const void *kI,
-                              const float *kI_scale, dsa_ki_dtype_t ki_dtype,
+                              const void *kI_scale, dsa_ki_dtype_t ki_dtype,
                               float *scores, int64_t ld, void *ws,
                               size_t ws_bytes, dsa_stream_t stream);
 
@@ -253,7 +273,7 @@ dsa_status_t dsa_check_error_noalloc(dsa_stream_t stream);
  * receives the selected positions [T,K] as dsa_topk returns them. */
 dsa_status_t dsa_index_topk_attn(const dsa_seqs_t *seqs, const void *qI,
                                  const float *w, const void *kI,
-                                 const float *kI_scale, dsa_ki_dtype_t ki_dtype,
+                                 const void *kI_scale, dsa_ki_dtype_t ki_dtype,
                                  const void *q, const void *kv, int K, int H,
                                  float scale, void *out,
                                  dsa_out_dtype_t out_dtype, float *lse,
@@ -271,7 +291,7 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t *seqs, const void *qI,
  * before the call. */
 dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t *seqs, const void *qI,
                                     const float *w, const void *kI,
-                                    const float *kI_scale, dsa_ki_dtype_t ki_dtype,
+                                    const void *kI_scale, dsa_ki_dtype_t ki_dtype,
                                     const void *q, const void *kv, int K, int H,
                                     float scale, void *out,
                                     dsa_out_dtype_t out_dtype, float *lse,

@@ -30,7 +30,7 @@ LIB_PATH = _build.LIB
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_BAD_INDEX, \
     DSA_ERR_TIMEOUT = range(7)
-DSA_KI_BF16, DSA_KI_FP8_E4M3 = 0, 1
+DSA_KI_BF16, DSA_KI_FP8_E4M3, DSA_KI_MXFP8 = 0, 1, 2
 DSA_OUT_BF16, DSA_OUT_F32 = 0, 1
 DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_INDEX_TOPK_ATTN, \
@@ -38,7 +38,8 @@ DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA
 DSA_SELECT_IN_INDEXER = 1
 
 # Names the C header declares (checked against include/dsa.h by the tests).
-EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_index_scores", "dsa_topk",
+EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_quantize_index_query_mx", "dsa_index_scores",
+           "dsa_topk",
            "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_noalloc", "dsa_check_error_noalloc", "dsa_index_topk_attn",
            "dsa_index_topk_attn_ex",
            "dsa_check_error", "dsa_set_wait_limit_ns", "dsa_launches_in_last_call", "dsa_launch_timing",
@@ -57,6 +58,7 @@ _SEQ = ctypes.POINTER(DsaSeqsC)
 _sig = {
     "dsa_workspace_size": (_SZ, [ctypes.c_int, _SEQ, ctypes.c_int, ctypes.c_int]),
     "dsa_quantize_index_query": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, _P]),
+    "dsa_quantize_index_query_mx": (ctypes.c_int, [_P, ctypes.c_int, _P, _P, _P]),
     "dsa_index_scores": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _I64, _P, _SZ, _P]),
     "dsa_topk": (ctypes.c_int, [_P, _I64, ctypes.c_int, _P, ctypes.c_int, _P, _P, _SZ, _P]),
     "dsa_sparse_mla_fwd": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, ctypes.c_int, _F, _P, ctypes.c_int, _P, _P,
@@ -168,9 +170,22 @@ def _need_index_inputs(seqs: "Seqs", qI, w, kI, kI_scale, check_seqs: bool = Tru
     _need(qI, "qI", _BF16T, (T, 64, 128), dev)
     _need(w, "w", _F32T, (T, 64), dev)
     _need(kI, "kI", _FP8T if kI_scale is not None else _BF16T, (None, 128), dev, rows)
-    if kI_scale is not None:
+    if _is_mx(kI_scale):
+        _need(kI_scale, "kI_scale", (torch.uint8,), (None, 4), dev, rows)
+    elif kI_scale is not None:
         _need(kI_scale, "kI_scale", _F32T, (None,), dev, rows)
     return dev
+
+
+def _is_mx(kI_scale) -> bool:
+    """An MXFP8 index cache carries E8M0 group scales (uint8 [R, 4])."""
+    return kI_scale is not None and kI_scale.dtype == torch.uint8
+
+
+def _ki_dtype(kI_scale) -> int:
+    if kI_scale is None:
+        return DSA_KI_BF16
+    return DSA_KI_MXFP8 if _is_mx(kI_scale) else DSA_KI_FP8_E4M3
 
 
 def _need_attn_inputs(seqs: "Seqs", q, kv, out, lse) -> torch.device:
@@ -259,6 +274,19 @@ def dsa_quantize_index_query(qI: torch.Tensor, w: torch.Tensor, codes=None, w_sc
     return codes, w_scaled
 
 
+def dsa_quantize_index_query_mx(qI: torch.Tensor, codes=None, scales=None):
+    dev = _cuda_device(qI, "qI")
+    T = qI.shape[0]
+    codes = codes if codes is not None else torch.empty((T, 64, 128), dtype=torch.uint8, device=qI.device)
+    scales = scales if scales is not None else torch.empty((T, 64, 4), dtype=torch.uint8, device=qI.device)
+    _need(qI, "qI", _BF16T, (T, 64, 128), dev)
+    _need(codes, "codes", _FP8T, (T, 64, 128), dev)
+    _need(scales, "scales", (torch.uint8,), (T, 64, 4), dev)
+    _check(_lib.dsa_quantize_index_query_mx(_ptr(qI), T, _ptr(codes), _ptr(scales), _stream(qI.device)),
+           "dsa_quantize_index_query_mx")
+    return codes, scales
+
+
 def dsa_index_scores(seqs: Seqs, qI, w, kI, kI_scale=None, scores=None, ld=None, ws=None):
     """Scores into `scores` [T, ld] fp32 (allocated zeroed when None).  When
     `scores` is given, ld defaults to its row stride and must equal it."""
@@ -272,7 +300,7 @@ def dsa_index_scores(seqs: Seqs, qI, w, kI, kI_scale=None, scores=None, ld=None,
         if ld is not None and ld != scores.stride(0):
             raise ValueError(f"ld={ld} differs from the row stride {scores.stride(0)} of scores")
         ld = scores.stride(0)
-    ki_dtype = DSA_KI_FP8_E4M3 if kI_scale is not None else DSA_KI_BF16
+    ki_dtype = _ki_dtype(kI_scale)
     c = seqs.c()
     need = _lib.dsa_workspace_size(DSA_OP_INDEX_SCORES, ctypes.byref(c), 1, 16)
     ws = ws if ws is not None else workspace(need, qI.device, "index_scores")
@@ -362,7 +390,7 @@ def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: f
         raise ValueError("qI and q are on different devices")
     if idx_out is not None:
         _need(idx_out, "idx_out", _I32T, (T, K), dev)
-    ki_dtype = DSA_KI_FP8_E4M3 if kI_scale is not None else DSA_KI_BF16
+    ki_dtype = _ki_dtype(kI_scale)
     c = seqs.c()
     op = DSA_OP_INDEX_TOPK_ATTN_FUSED if select_in_indexer else DSA_OP_INDEX_TOPK_ATTN
     need = _lib.dsa_workspace_size(op, ctypes.byref(c), K, H)

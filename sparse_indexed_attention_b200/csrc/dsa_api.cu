@@ -24,7 +24,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // the sticky error word.
 struct Layout {
   size_t tok_seq = 0, tok_pos = 0, seq_gstart = 0, groups = 0, items = 0, counts = 0;
-  size_t q_codes = 0, w_scaled = 0, scores = 0, idx = 0, topk = 0, partials = 0, tail = 0, cand = 0;
+  size_t q_codes = 0, w_scaled = 0, q_sf = 0, scores = 0, idx = 0, topk = 0, partials = 0, tail = 0, cand = 0;
   size_t total = 0;
   int64_t ld = 0;
   bool fused = false;       // the indexer selects the Top-K itself (no score scratch)
@@ -59,6 +59,7 @@ Layout make_layout(dsa_op_t op, int T, int B, int max_ctx, int K, int H) {
     L.items = take((size_t)plan_max_items(T, B, max_ctx, tg) * 2 * sizeof(int4));
     L.q_codes = take((size_t)T * kHI * kDI);
     L.w_scaled = take((size_t)T * kHI * sizeof(float));
+    L.q_sf = take((size_t)T * kHI * 4);  // MXFP8 query group scales (E8M0)
   }
   if (op == DSA_OP_INDEX_TOPK_ATTN) {
     L.ld = ((int64_t)max_ctx + 3) / 4 * 4;
@@ -125,11 +126,11 @@ dsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA
 #define DSA_CUDA(x) DSA_TRY(cuda_status(x))
 
 dsa_status_t check_indexer_args(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
-                                const float* kI_scale, dsa_ki_dtype_t ki_dtype) {
+                                const void* kI_scale, dsa_ki_dtype_t ki_dtype) {
   DSA_TRY(check_seqs(seqs));
   if (!qI || !w || !kI) return DSA_ERR_INVALID_ARG;
-  if (ki_dtype != DSA_KI_BF16 && ki_dtype != DSA_KI_FP8_E4M3) return DSA_ERR_UNSUPPORTED;
-  if ((ki_dtype == DSA_KI_FP8_E4M3) != (kI_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  if (ki_dtype != DSA_KI_BF16 && ki_dtype != DSA_KI_FP8_E4M3 && ki_dtype != DSA_KI_MXFP8) return DSA_ERR_UNSUPPORTED;
+  if ((ki_dtype != DSA_KI_BF16) != (kI_scale != nullptr)) return DSA_ERR_INVALID_ARG;
   if (!aligned(qI, 16) || !aligned(w, 16) || !aligned(kI, 128) || (kI_scale && !aligned(kI_scale, 16)))
     return DSA_ERR_INVALID_ARG;
   return DSA_OK;
@@ -158,26 +159,37 @@ PlanBufs plan_bufs(void* ws, const Layout& L) {
   return p;
 }
 
+// Tokens per indexer group for a call: one for decode, else two (bf16 and
+// MXFP8 caches) or four (E4M3 cache).
+int group_tokens(const dsa_seqs_t* seqs, dsa_ki_dtype_t ki_dtype) {
+  return indexer_group_tokens(seqs->num_q_tokens, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
+}
+
 // Indexer launch sequence shared by dsa_index_scores and the fused call: one
-// prep launch (plan, FP8 query quantization, zeroing of `zero`) and the
-// indexer, which also accumulates Top-K's first-digit histogram into `hist`
-// when that is given (one token per group).
+// prep launch (plan, FP8 / MXFP8 query quantization, zeroing of `zero`) and
+// the indexer, which also accumulates Top-K's first-digit histogram into
+// `hist` when that is given (one token per group).
 dsa_status_t run_indexer(const dsa_seqs_t* seqs, const SeqsDev& sd, const PlanBufs& plan, int tg, const void* qI,
-                         const float* w, const void* kI, const float* kI_scale, dsa_ki_dtype_t ki_dtype,
+                         const float* w, const void* kI, const void* kI_scale, dsa_ki_dtype_t ki_dtype,
                          float* scores, int64_t ld, void* ws, const Layout& L, uint32_t* hist, uint32_t* zero,
                          int64_t zero_words, uint32_t* err, cudaStream_t st, const FusedTopk* fused = nullptr) {
-  const bool fp8 = ki_dtype == DSA_KI_FP8_E4M3;
+  const bool fp8 = ki_dtype == DSA_KI_FP8_E4M3, mx = ki_dtype == DSA_KI_MXFP8;
   const void* q_operand = qI;
   const float* w_operand = w;
-  uint8_t* codes = fp8 ? at<uint8_t>(ws, L.q_codes) : nullptr;
+  uint8_t* codes = (fp8 || mx) ? at<uint8_t>(ws, L.q_codes) : nullptr;
   float* w_scaled = fp8 ? at<float>(ws, L.w_scaled) : nullptr;
-  DSA_CUDA(launch_prep(sd, tg, indexer_item_tiles(tg), plan, fp8 ? reinterpret_cast<const __nv_bfloat16*>(qI) : nullptr,
-                       w, codes, w_scaled, zero, zero_words, err, st));
+  uint8_t* q_sf = mx ? at<uint8_t>(ws, L.q_sf) : nullptr;
+  DSA_CUDA(launch_prep(sd, tg, indexer_item_tiles(tg), plan,
+                       (fp8 || mx) ? reinterpret_cast<const __nv_bfloat16*>(qI) : nullptr, w, codes, w_scaled, q_sf,
+                       zero, zero_words, err, st));
   if (fp8) {
     q_operand = codes;
     w_operand = w_scaled;
+  } else if (mx) {
+    q_operand = codes;  // the head weights stay as given: the group scales ride in the MMA
   }
-  DSA_CUDA(launch_index_scores(sd, plan, tg, q_operand, w_operand, kI, kI_scale, fp8, scores, ld, hist, err, st,
+  const IdxFmt fmt = mx ? IdxFmt::kMx : (fp8 ? IdxFmt::kE4M3 : IdxFmt::kBf16);
+  DSA_CUDA(launch_index_scores(sd, plan, tg, q_operand, w_operand, q_sf, kI, kI_scale, fmt, scores, ld, hist, err, st,
                                fused));
   return DSA_OK;
 }
@@ -209,8 +221,18 @@ dsa_status_t dsa_quantize_index_query(const void* qI, const float* w, int T, uin
                                                  (cudaStream_t)stream));
 }
 
+dsa_status_t dsa_quantize_index_query_mx(const void* qI, int T, uint8_t* codes, uint8_t* scales,
+                                         dsa_stream_t stream) {
+  g_launches = 0;
+  if (!qI || !codes || !scales || T < 1) return DSA_ERR_INVALID_ARG;
+  if (!aligned(qI, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return DSA_ERR_INVALID_ARG;
+  timer_begin((cudaStream_t)stream);
+  return cuda_status(launch_quantize_index_query_mx(reinterpret_cast<const __nv_bfloat16*>(qI), T, codes, scales,
+                                                    (cudaStream_t)stream));
+}
+
 dsa_status_t dsa_index_scores(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
-                              const float* kI_scale, dsa_ki_dtype_t ki_dtype, float* scores, int64_t ld, void* ws,
+                              const void* kI_scale, dsa_ki_dtype_t ki_dtype, float* scores, int64_t ld, void* ws,
                               size_t ws_bytes, dsa_stream_t stream) {
   g_launches = 0;
   DSA_TRY(check_indexer_args(seqs, qI, w, kI, kI_scale, ki_dtype));
@@ -221,7 +243,7 @@ dsa_status_t dsa_index_scores(const dsa_seqs_t* seqs, const void* qI, const floa
   uint32_t* err = at<uint32_t>(ws, 0);
   const SeqsDev sd = to_dev(seqs);
   const PlanBufs plan = plan_bufs(ws, L);
-  const int tg = indexer_group_tokens(seqs->num_q_tokens, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
+  const int tg = group_tokens(seqs, ki_dtype);
   timer_begin(st);
   return run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, scores, ld, ws, L, nullptr, nullptr, 0, err,
                      st);
@@ -264,7 +286,7 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const voi
 }
 
 dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
-                                    const float* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
+                                    const void* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
                                     int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse,
                                     int32_t* idx_out, void* ws, size_t ws_bytes, unsigned flags,
                                     dsa_event_t q_ready, dsa_stream_t stream) {
@@ -283,7 +305,7 @@ dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t* seqs, const void* qI, cons
   TokenMap tm{plan.tok_seq, plan.tok_pos};
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
   const int T = seqs->num_q_tokens;
-  const int tg = indexer_group_tokens(T, seqs->batch, ki_dtype == DSA_KI_FP8_E4M3);
+  const int tg = group_tokens(seqs, ki_dtype);
   if (L.fused) {
     // decode: prep, the indexer with the Top-K selection inside, attention
     uint32_t* tail = at<uint32_t>(ws, L.tail);
@@ -316,7 +338,7 @@ dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t* seqs, const void* qI, cons
 }
 
 dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
-                                 const float* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
+                                 const void* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
                                  int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse,
                                  int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
   return dsa_index_topk_attn_ex(seqs, qI, w, kI, kI_scale, ki_dtype, q, kv, K, H, scale, out, out_dtype, lse, idx_out,

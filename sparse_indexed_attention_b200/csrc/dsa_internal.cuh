@@ -168,12 +168,16 @@ inline int64_t plan_max_items(int T, int B, int max_ctx, int tg) {
 
 // ---- launchers (each returns cudaGetLastError() of its launch) ----
 cudaError_t launch_plan(const SeqsDev& s, int tg, int ch, const PlanBufs& p, uint32_t* err, cudaStream_t st);
-// Plan + (FP8 cache: qI quantization) + zeroing of `zero_words` words, one launch.
+// Plan + (FP8 / MXFP8 cache: qI quantization) + zeroing of `zero_words` words,
+// one launch.  q_sf non-null selects MXFP8: the E8M0 group scales go to
+// q_sf [T*64, 4].
 cudaError_t launch_prep(const SeqsDev& s, int tg, int ch, const PlanBufs& plan, const __nv_bfloat16* qI,
-                        const float* w, uint8_t* codes, float* w_scaled, uint32_t* zero, int64_t zero_words,
-                        uint32_t* err, cudaStream_t st);
+                        const float* w, uint8_t* codes, float* w_scaled, uint8_t* q_sf, uint32_t* zero,
+                        int64_t zero_words, uint32_t* err, cudaStream_t st);
 cudaError_t launch_quantize_index_query(const __nv_bfloat16* qI, const float* w, int T, uint8_t* codes,
                                         float* w_scaled, cudaStream_t st);
+cudaError_t launch_quantize_index_query_mx(const __nv_bfloat16* qI, int T, uint8_t* codes, uint8_t* scales,
+                                           cudaStream_t st);
 // Fused selection (decode): the indexer also selects the Top-K of every row
 // (no score scratch).  Its grid is one CTA on each of kFusedGrid SMs, all
 // resident; `tail` / `tail_items` (fused_topk_words words) start zeroed.
@@ -190,13 +194,17 @@ int indexer_fused_capacity();                          // items per CTA
 bool indexer_fused_fits(int T, int B, int max_ctx);    // the geometry fits the fused selection
 int64_t fused_topk_words(int T, int B, int max_ctx);   // its zeroed scratch, in 32-bit words
 size_t fused_topk_cand_bytes(int T);                   // its candidate lists
-// FP8 cache: codes/w_scaled from the quantizer; bf16 cache: qI/w directly.
+// Index-cache formats of the indexer kernel.
+enum class IdxFmt { kBf16, kE4M3, kMx };
+// E4M3 cache: codes/w_scaled from the quantizer, kI_scale fp32 [R];
+// MXFP8 cache: codes and q_sf (E8M0 group scales) from the quantizer, w
+// directly, kI_scale E8M0 bytes [R, 4]; bf16 cache: qI/w directly.
 // hist (may be null; used for one token per group): Top-K first-digit histogram to accumulate into.
 // fused (may be null): select the Top-K in the same kernel instead of writing scores.
 cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
-                                const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
-                                float* scores, int64_t ld, uint32_t* hist, uint32_t* err, cudaStream_t st,
-                                const FusedTopk* fused = nullptr);
+                                const float* w_operand, const uint8_t* q_sf, const void* kI, const void* kI_scale,
+                                IdxFmt fmt, float* scores, int64_t ld, uint32_t* hist, uint32_t* err,
+                                cudaStream_t st, const FusedTopk* fused = nullptr);
 size_t topk_scratch_bytes(int T, int64_t ld, int K);
 // Several CTAs per row use a region at the head of the scratch that must be
 // zero when they start (row counters + first-digit histogram, topk_zero_words

@@ -15,6 +15,16 @@
 //  * warp 1, one lane: issues tcgen05.mma (kind::f8f6f4 E4M3, or kind::f16
 //    bf16) into a ring of TMEM accumulators; tcgen05.commit frees the stage
 //    and publishes the accumulator.
+//  * MXFP8 cache ([P2] section 5 table, "Indexer Q/K": one shared scale per
+//    group of 32; [P4] section 4.2): keys and the quantized query carry one
+//    E8M0 scale per 32 of the 128 dims, applied by the tensor core itself
+//    (kind::mxf8f6f4.block_scale, one MMA per 32-wide K block).  The
+//    producer warp's 32 lanes copy a tile's key scales (4-byte cp.async) into
+//    shared memory in the scale-factor layout -- key r in row r % 32, 32-bit
+//    column r / 32, byte = K block -- and a group's query scales likewise;
+//    the MMA lane moves them into TMEM with tcgen05.cp (32 rows x 128 bits,
+//    written to every lane quarter) ahead of the tile's MMAs.  The epilogue
+//    is that of the E4M3 cache without the key scale.
 //  * warp 2: allocates and frees TMEM.
 //  * warps 4-11: epilogue, two warpgroups taking alternate tiles.  Thread r
 //    of a warpgroup owns TMEM lane r = key row r, so the ReLU, the head
@@ -75,22 +85,34 @@ struct TailSmem {
   int fast[kTailRuns];           // the row takes the candidate-list path
 };
 
-template <bool kBf16, int TG, bool kFused = false>
+template <bool kBf16, int TG, bool kFused = false, bool kMx = false>
 struct IdxCfg {
   static_assert(!kFused || TG == 1, "the fused selection serves one token per group");
+  static_assert(!kMx || (!kBf16 && TG <= 2), "MXFP8: E4M3 codes, at most two tokens per group");
   static constexpr int N = 64 * TG;                        // MMA N: heads x tokens of a group
   static constexpr int A_BYTES = kBf16 ? 32768 : 16384;    // 128 keys x d_I
   static constexpr int B_BYTES = kBf16 ? N * 256 : N * 128;
   static constexpr int KSTEPS = kBf16 ? 8 : 4;             // 32-byte K steps per tile
   static constexpr int NS = kBf16 ? 3 : (TG == 1 ? (kFused ? 6 : 8) : 6);
-  static constexpr int NACC = (512 / N) < 4 ? (512 / N) : 4;
-  static constexpr int TMEM_COLS = (NACC * N) <= 256 ? 256 : 512;
+  // Accumulator ring.  NACC is even: the two epilogue warpgroups take
+  // alternate tiles, so each accumulator (and its barriers) belongs to one
+  // warpgroup and is waited on one phase at a time.  MXFP8 also keeps scale
+  // columns in TMEM: 4 per stage (128 keys), 4 per group slot and 128 query rows.
+  static constexpr int NACC = kMx ? (N == 64 ? 4 : 2) : ((512 / N) < 4 ? (512 / N) : 4);
+  static constexpr int SFB_COPIES = kMx ? (N + 127) / 128 : 0;   // 32x128b copies per group
+  static constexpr int SFB_BYTES = SFB_COPIES * 512;
+  static constexpr int SFA0 = NACC * N;                    // TMEM column of stage 0's key scales
+  static constexpr int SFB0 = SFA0 + 4 * NS;               // TMEM column of slot 0's query scales
+  static constexpr int SFB_COLS = 4 * SFB_COPIES;
+  static constexpr int TMEM_COLS = kMx ? 512 : ((NACC * N) <= 256 ? 256 : 512);
   // shared-memory layout (offsets from a 1024-aligned base)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + NS * A_BYTES;
   static constexpr int OFF_SC = OFF_B + 2 * B_BYTES;       // NS x 128 fp32 row scales
   static constexpr int OFF_W = OFF_SC + NS * 512;          // 2 x TG x 64 fp32 head weights
-  static constexpr int OFF_HIST = OFF_W + 2 * TG * 256;   // TG == 1: per-epilogue-warp Top-K histograms
+  // (MXFP8: the OFF_SC area holds each stage's key scales in the scale-factor layout, 512 B)
+  static constexpr int OFF_SFB = OFF_W + 2 * TG * 256;    // MXFP8: 2 x the group's query scales
+  static constexpr int OFF_HIST = OFF_SFB + 2 * SFB_BYTES;  // TG == 1: per-epilogue-warp Top-K histograms
   static constexpr int OFF_RING = OFF_HIST + ((TG == 1 && !kFused) ? kEpiWarps * kTopkHistBins * 4 : 0);
   static constexpr int OFF_BAR = OFF_RING + kRingSlots * (32 + 128);  // producer's item records + page ids
   static constexpr int NBARS = 2 * NS + 4 + 2 * NACC + 1;
@@ -104,7 +126,9 @@ struct IdxCfg {
   static constexpr int SMEM = BYTES + 1024;                // slack for 1024-byte alignment
   static constexpr uint32_t IDESC = make_idesc(kBf16, 128, N);
   static_assert(SMEM <= 227 * 1024, "shared memory");
-  static_assert(NACC * N <= TMEM_COLS, "TMEM");
+  static_assert(NACC * N <= TMEM_COLS && NACC % 2 == 0, "TMEM accumulators (an even number)");
+  static_assert(!kMx || SFB0 + 2 * SFB_COLS <= TMEM_COLS, "TMEM scale columns");
+  static_assert(OFF_SFB % 512 == 0, "scale-factor sources need 16-byte alignment");
   static_assert(!kFused || CAP_ITEMS >= 8, "fused selection capacity");
   static_assert(!kFused || CAP_ITEMS * 4096 >= kFastScratch, "fused selection fast-path scratch");
 };
@@ -114,6 +138,8 @@ struct IdxArgs {
   PlanBufs plan;
   const float* w_operand;  // [T, 64] head weights (scaled by 2^e for FP8)
   const float* kI_scale;   // [R] (FP8) or null
+  const uint8_t* kI_sf;    // MXFP8: key group scales [R, 4] (E8M0)
+  const uint8_t* q_sf;     // MXFP8: query group scales [T * 64, 4] (E8M0)
   float* scores;
   int64_t ld;
   uint32_t* hist;          // TG == 1 only, may be null: Top-K first-digit histogram [T][2048]
@@ -488,11 +514,11 @@ __device__ __forceinline__ void flush_hist(uint32_t* sh, uint32_t* gh, int t, in
   __syncwarp();
 }
 
-template <bool kBf16, int TG, bool kFused>
+template <bool kBf16, int TG, bool kFused, bool kMx>
 __global__ void __launch_bounds__(kIdxThreads, 1)
 k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                   const IdxArgs a) {
-  using C = IdxCfg<kBf16, TG, kFused>;
+  using C = IdxCfg<kBf16, TG, kFused, kMx>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -510,12 +536,13 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    // MXFP8: the producer's 32 lanes also arrive, once their scale copies land
     for (int i = 0; i < C::NS; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], kMx ? 1 + 32 : 1);
       mbar_init(&empty[i], 1 + 4);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&b_full[i], 1);
+      mbar_init(&b_full[i], kMx ? 1 + 32 : 1);
       mbar_init(&b_empty[i], 1 + kEpiWarps);
     }
     for (int i = 0; i < C::NACC; ++i) {
@@ -592,11 +619,13 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
       const int pages = ring_pg[(it % kRingSlots) * 32 + lane];  // lanes past the item's pages are unused
       const int4 grp = ca;  // {b, t0, cnt, pos0}
       if (cb.z != prev_g) {
+        const int slot = gcount & 1, use = gcount >> 1;
+        int b_ok = 0;
         if (lane == 0) {
-          const int slot = gcount & 1, use = gcount >> 1;
           if (!mbar_wait(&b_empty[slot], (use & 1) ^ 1, a.err, a.wait_ns)) {
             *abort_flag = 1;
           } else {
+            b_ok = 1;
             const uint32_t wbytes = (uint32_t)grp.z * 256u;
             mbar_arrive_expect_tx(&b_full[slot], (uint32_t)C::B_BYTES + wbytes);
             uint8_t* bdst = smem + C::OFF_B + slot * C::B_BYTES;
@@ -610,6 +639,21 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
             ++b_issued;
           }
         }
+        if constexpr (kMx) {
+          // the group's query scales: query row n = 64 k + h (token k, head h)
+          // goes to row n % 32, column n / 32 of the scale-factor layout
+          if (__shfl_sync(0xffffffffu, b_ok, 0)) {
+            uint8_t* sfb = smem + C::OFF_SFB + slot * C::SFB_BYTES;
+            for (int k = 0; k < grp.z; ++k)
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                const int col = 2 * k + c;
+                cp_async_4(sfb + (col >> 2) * 512 + lane * 16 + (col & 3) * 4,
+                           a.q_sf + ((int64_t)(grp.y + k) * 64 + 32 * c + lane) * 4);
+              }
+            cp_async_mbar_arrive(&b_full[slot]);  // once this lane's copies land
+          }
+        }
         prev_g = cb.z;
         ++gcount;
       }
@@ -617,11 +661,13 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
         const int j = tile - cb.x;
         const int pg0 = __shfl_sync(0xffffffffu, pages, 2 * j);
         const int pg1 = __shfl_sync(0xffffffffu, pages, 2 * j + 1);
+        const int last = grp.w + grp.z - 1;
+        int t_ok = 0;
         if (lane == 0 && !*abort_flag) {
           if (!mbar_wait(&empty[stage], sphase ^ 1, a.err, a.wait_ns)) {
             *abort_flag = 1;
           } else {
-            const int last = grp.w + grp.z - 1;
+            t_ok = 1;
             int rows[2];
             const int pg[2] = {pg0, pg1};
             uint32_t bytes = 0;
@@ -631,7 +677,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
               if ((tile * 2 + h) * kPage <= last) {
                 if (pg[h] >= 0 && pg[h] < a.s.num_phys_pages) {
                   rows[h] = pg[h] * kPage;
-                  bytes += (uint32_t)(C::A_BYTES / 2) + (kBf16 ? 0u : 256u);
+                  bytes += (uint32_t)(C::A_BYTES / 2) + ((kBf16 || kMx) ? 0u : 256u);
                 } else {
                   raise_error(a.err, kErrBadIndex);
                 }
@@ -648,9 +694,25 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
                 tma_load_2d(adst + 16384 + h * 8192, &tmap_k, &full[stage], 64, rows[h]);
               } else {
                 tma_load_2d(adst + h * 8192, &tmap_k, &full[stage], 0, rows[h]);
-                bulk_load(smem + C::OFF_SC + stage * 512 + h * 256, a.kI_scale + rows[h], 256, &full[stage]);
+                if constexpr (!kMx)
+                  bulk_load(smem + C::OFF_SC + stage * 512 + h * 256, a.kI_scale + rows[h], 256, &full[stage]);
               }
             }
+          }
+        }
+        if constexpr (kMx) {
+          // the tile's key scales: key 32 c + l (page c / 2, row 32 (c % 2) + l)
+          // goes to row l, column c; every lane arrives once its copies land
+          if (__shfl_sync(0xffffffffu, t_ok, 0)) {
+            uint8_t* sfa = smem + C::OFF_SC + stage * 512;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int h = c >> 1;
+              const int pgh = h ? pg1 : pg0;
+              if ((tile * 2 + h) * kPage <= last && pgh >= 0 && pgh < a.s.num_phys_pages)
+                cp_async_4(sfa + lane * 16 + c * 4, a.kI_sf + ((int64_t)pgh * kPage + 32 * (c & 1) + lane) * 4);
+            }
+            cp_async_mbar_arrive(&full[stage]);
           }
         }
         if (++stage == C::NS) { stage = 0; sphase ^= 1; }
@@ -680,6 +742,14 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
           if (prev_g >= 0) mma_commit(&b_empty[slot]);  // previous group's operands free once its MMAs finish
           slot = gcount & 1;
           if (!mbar_wait(&b_full[slot], (gcount >> 1) & 1, a.err, a.wait_ns)) { *abort_flag = 1; break; }
+          if constexpr (kMx) {  // the group's query scales into TMEM (in order before its MMAs)
+            fence_proxy_async_smem();  // written by cp.async (generic proxy)
+            tc_fence_after();
+#pragma unroll
+            for (int cp = 0; cp < C::SFB_COPIES; ++cp)
+              tmem_cp_32x128b_x4(tmem + C::SFB0 + slot * C::SFB_COLS + 4 * cp,
+                                 rows16_desc(smem_u32(smem + C::OFF_SFB + slot * C::SFB_BYTES + cp * 512)));
+          }
           prev_g = item.x;
           ++gcount;
         }
@@ -689,13 +759,25 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
           if (!mbar_wait(&acc_empty[acc], aphase ^ 1, a.err, a.wait_ns)) { *abort_flag = 1; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + C::OFF_A + stage * C::A_BYTES);
+          if constexpr (kMx) {
+            // the tile's key scales into TMEM, then one block-scaled MMA per
+            // 32-wide K block (byte k of each scale column)
+            fence_proxy_async_smem();  // written by cp.async (generic proxy)
+            tmem_cp_32x128b_x4(tmem + C::SFA0 + 4 * stage, rows16_desc(smem_u32(smem + C::OFF_SC + stage * 512)));
 #pragma unroll
-          for (int k = 0; k < C::KSTEPS; ++k) {
-            // K step k: 32 bytes inside a 128-byte swizzle row; bf16 rows span two 128-byte blocks
-            const uint32_t a_off = kBf16 ? (k >> 2) * 16384 + (k & 3) * 32 : k * 32;
-            const uint32_t b_off = kBf16 ? (k >> 2) * (C::N * 128) + (k & 3) * 32 : k * 32;
-            mma_ss<kBf16>(tmem + acc * C::N, sw128_kmajor_desc(a_base + a_off), sw128_kmajor_desc(b_base + b_off),
-                          C::IDESC, k > 0);
+            for (int k = 0; k < 4; ++k)
+              mma_mx(tmem + acc * C::N, sw128_kmajor_desc(a_base + k * 32), sw128_kmajor_desc(b_base + k * 32),
+                     make_idesc_mx(128, C::N, k), (tmem + C::SFA0 + 4 * stage) | ((uint32_t)k << 30),
+                     (tmem + C::SFB0 + slot * C::SFB_COLS) | ((uint32_t)k << 30), k > 0);
+          } else {
+#pragma unroll
+            for (int k = 0; k < C::KSTEPS; ++k) {
+              // K step k: 32 bytes inside a 128-byte swizzle row; bf16 rows span two 128-byte blocks
+              const uint32_t a_off = kBf16 ? (k >> 2) * 16384 + (k & 3) * 32 : k * 32;
+              const uint32_t b_off = kBf16 ? (k >> 2) * (C::N * 128) + (k & 3) * 32 : k * 32;
+              mma_ss<kBf16>(tmem + acc * C::N, sw128_kmajor_desc(a_base + a_off), sw128_kmajor_desc(b_base + b_off),
+                            C::IDESC, k > 0);
+            }
           }
           mma_commit(&empty[stage]);
           mma_commit(&acc_full[acc]);
@@ -758,7 +840,7 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
           if (!kBf16) okw = okw && mbar_wait(&full[stage], sphase, a.err, a.wait_ns);
           if (!__all_sync(0xffffffffu, okw)) { *abort_flag = 1; break; }
           tc_fence_after();
-          const float sk = kBf16 ? 1.f : sc_smem[stage * 128 + r];
+          const float sk = (kBf16 || kMx) ? 1.f : sc_smem[stage * 128 + r];
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[stage]);
           const int s = tile * 128 + r;
@@ -795,7 +877,8 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
               if (it - it_lo < C::CAP_ITEMS) keys[(it - it_lo) * 1024 + (tile - item.y) * 128 + r] = order_key(score);
             } else {
               if (valid) a.scores[(int64_t)(grp.y + k) * a.ld + s] = score;
-              if (do_hist) hist_add(sh_hist, order_key(score) >> kTopkLowBits, valid);
+              // scores fall in random bins: a plain shared-memory add beats aggregating equal bins
+              if (do_hist && valid) atomicAdd(&sh_hist[order_key(score) >> kTopkLowBits], 1u);
             }
           }
         }
@@ -803,7 +886,6 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
         if (++acc == C::NACC) { acc = 0; aphase ^= 1; }
       }
     }
-    if (do_hist && prev_t >= 0) flush_hist(sh_hist, a.hist, prev_t, lane);
     __syncwarp();
   }
   tc_fence_before();
@@ -811,6 +893,18 @@ k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_const
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (TG == 1 && !kFused && a.hist != nullptr && !*abort_flag && it_hi > it_lo) {
+    // the last token's histogram: the eight warps' copies summed here and
+    // added once per CTA (earlier tokens were flushed per warp as they ended)
+    const int t_last = recs[2 * (it_hi - 1)].y;
+    const uint32_t* hb = reinterpret_cast<const uint32_t*>(smem + C::OFF_HIST);
+    for (int i = threadIdx.x; i < kTopkHistBins; i += blockDim.x) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int w = 0; w < kEpiWarps; ++w) v += hb[w * kTopkHistBins + i];
+      if (v) atomicAdd(a.hist + (int64_t)t_last * kTopkHistBins + i, v);
+    }
   }
   if constexpr (kFused) {
     // the selection, once every score of this CTA is in shared memory (the
@@ -856,19 +950,19 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <bool kBf16, int TG, bool kFused>
+template <bool kBf16, int TG, bool kFused, bool kMx = false>
 cudaError_t launch_tc(const CUtensorMap& mk, const CUtensorMap& mq, const IdxArgs& a, int grid, cudaStream_t st) {
-  using C = IdxCfg<kBf16, TG, kFused>;
+  using C = IdxCfg<kBf16, TG, kFused, kMx>;
   static thread_local int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(k_index_scores_tc<kBf16, TG, kFused>,
+    cudaError_t e = cudaFuncSetAttribute(k_index_scores_tc<kBf16, TG, kFused, kMx>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  cudaError_t e = launch_pdl("index_scores", k_index_scores_tc<kBf16, TG, kFused>, dim3(grid), dim3(kIdxThreads),
+  cudaError_t e = launch_pdl("index_scores", k_index_scores_tc<kBf16, TG, kFused, kMx>, dim3(grid), dim3(kIdxThreads),
                              (size_t)C::SMEM, st, mk, mq, a);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
@@ -878,7 +972,9 @@ cudaError_t launch_tc(const CUtensorMap& mk, const CUtensorMap& mq, const IdxArg
 
 int indexer_fused_capacity() {
   const int a = IdxCfg<false, 1, true>::CAP_ITEMS, b = IdxCfg<true, 1, true>::CAP_ITEMS;
-  return a < b ? a : b;
+  const int c = IdxCfg<false, 1, true, true>::CAP_ITEMS;
+  const int ab = a < b ? a : b;
+  return ab < c ? ab : c;
 }
 
 bool indexer_fused_fits(int T, int B, int max_ctx) {
@@ -894,10 +990,10 @@ int64_t fused_topk_words(int T, int B, int max_ctx) {
 size_t fused_topk_cand_bytes(int T) { return (size_t)T * kCandCap * sizeof(int2); }
 
 cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, const void* q_operand,
-                                const float* w_operand, const void* kI, const float* kI_scale, bool fp8,
-                                float* scores, int64_t ld, uint32_t* hist, uint32_t* err, cudaStream_t st,
-                                const FusedTopk* fused) {
-  const bool bf16 = !fp8;
+                                const float* w_operand, const uint8_t* q_sf, const void* kI, const void* kI_scale,
+                                IdxFmt fmt, float* scores, int64_t ld, uint32_t* hist, uint32_t* err,
+                                cudaStream_t st, const FusedTopk* fused) {
+  const bool bf16 = fmt == IdxFmt::kBf16, mx = fmt == IdxFmt::kMx;
   const uint64_t R = (uint64_t)s.num_phys_pages * kPage;
   const uint64_t qrows = (uint64_t)s.num_tokens * kHI;
   CUtensorMap mk, mq;
@@ -906,7 +1002,9 @@ cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, 
   IdxArgs a{s,
             plan,
             w_operand,
-            kI_scale,
+            fmt == IdxFmt::kE4M3 ? static_cast<const float*>(kI_scale) : nullptr,
+            mx ? static_cast<const uint8_t*>(kI_scale) : nullptr,
+            mx ? q_sf : nullptr,
             scores,
             ld,
             tg == 1 ? hist : nullptr,
@@ -922,9 +1020,13 @@ cudaError_t launch_index_scores(const SeqsDev& s, const PlanBufs& plan, int tg, 
     // the rows' CTAs wait on one another: every CTA must be resident (one per
     // SM) and hold at most the capacity the workspace was sized for
     if (tg != 1 || grid < kFusedGrid) return cudaErrorInvalidConfiguration;
-    return fp8 ? launch_tc<false, 1, true>(mk, mq, a, kFusedGrid, st) : launch_tc<true, 1, true>(mk, mq, a, kFusedGrid, st);
+    if (mx) return launch_tc<false, 1, true, true>(mk, mq, a, kFusedGrid, st);
+    return bf16 ? launch_tc<true, 1, true>(mk, mq, a, kFusedGrid, st) : launch_tc<false, 1, true>(mk, mq, a, kFusedGrid, st);
   }
-  if (fp8) {
+  if (mx) {
+    if (tg == 1) return launch_tc<false, 1, false, true>(mk, mq, a, grid, st);
+    if (tg == 2) return launch_tc<false, 2, false, true>(mk, mq, a, grid, st);
+  } else if (!bf16) {
     if (tg == 1) return launch_tc<false, 1, false>(mk, mq, a, grid, st);
     if (tg == 4) return launch_tc<false, 4, false>(mk, mq, a, grid, st);
   } else {

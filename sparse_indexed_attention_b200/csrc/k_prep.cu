@@ -7,8 +7,11 @@
 // quantize_index_query: the "Q quantization" input-preparation step of the
 //   indexer ([P2] "Hybrid Attention LLM Inference Acceleration...", section
 //   4(2); [P3] "Inference Acceleration for a New Domestic LLM Architecture...",
-//   section 3 `q_quantize`).  One power-of-two scale per (token, head) row,
-//   folded into the head weight.
+//   section 3 `q_quantize`).  For the E4M3 cache: one power-of-two scale per
+//   (token, head) row, folded into the head weight.  For the MXFP8 cache
+//   ([P2] section 5 table, "Indexer Q/K"; [P4] section 4.2): one E8M0 scale
+//   per group of 32 elements, 2^(floor(log2 amax) - 8), kept as bytes
+//   [T, 64, 4] for the indexer's block-scaled MMA.
 #include <cuda_fp8.h>
 
 #include "dsa_internal.cuh"
@@ -308,6 +311,44 @@ __device__ __forceinline__ void quant_row(const __nv_bfloat16* __restrict__ qI, 
   if (lane == 0) w_scaled[row] = ldexpf(__ldg(w + row), e);
 }
 
+// MXFP8: one warp per (token, head) row of 128 bf16; lane l holds elements
+// 4l..4l+3, so lanes 8g..8g+7 hold group g.  The group's shared exponent is
+// floor(log2 amax) - 8 (from frexpf, exact for any finite float), clamped to
+// [-127, 127]; an all-zero group takes 0.  Elements divided by 2^e (exact)
+// round to E4M3 with saturation; the scale goes out as its E8M0 byte e + 127.
+__device__ __forceinline__ void quant_row_mx(const __nv_bfloat16* __restrict__ qI, int row, uint8_t* __restrict__ codes,
+                                             uint8_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qI + (int64_t)row * kDI) + lane);
+  __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+  __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+  float x[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
+  float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));  // within the 8-lane group
+  int e = 0;
+  if (amax > 0.f) {
+    int ex;
+    frexpf(amax, &ex);  // amax = m * 2^ex, 0.5 <= m < 1
+    e = min(127, max(-127, ex - 9));
+  }
+  float y[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) y[i] = ldexpf(x[i], -e);
+  __nv_fp8x2_storage_t c01 = __nv_cvt_float2_to_fp8x2(make_float2(y[0], y[1]), __NV_SATFINITE, __NV_E4M3);
+  __nv_fp8x2_storage_t c23 = __nv_cvt_float2_to_fp8x2(make_float2(y[2], y[3]), __NV_SATFINITE, __NV_E4M3);
+  reinterpret_cast<uint32_t*>(codes + (int64_t)row * kDI)[lane] = (uint32_t)c01 | ((uint32_t)c23 << 16);
+  if ((lane & 7) == 0) scales[(int64_t)row * 4 + (lane >> 3)] = (uint8_t)(e + 127);
+}
+
+__global__ void k_quantize_index_query_mx(const __nv_bfloat16* __restrict__ qI, int rows, uint8_t* __restrict__ codes,
+                                          uint8_t* __restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (row < rows) quant_row_mx(qI, row, codes, scales);
+}
+
 __global__ void k_quantize_index_query(const __nv_bfloat16* __restrict__ qI, const float* __restrict__ w,
                                        int rows, uint8_t* __restrict__ codes, float* __restrict__ w_scaled) {
   pdl_wait();
@@ -318,7 +359,8 @@ __global__ void k_quantize_index_query(const __nv_bfloat16* __restrict__ qI, con
 
 // Everything the indexer needs before it starts, in one launch: block 0 builds
 // the plan; the other blocks quantize the index query (32 rows per block, FP8
-// cache only) and zero a scratch range (Top-K's first-digit histogram).
+// and MXFP8 caches only) and zero a scratch range (Top-K's first-digit
+// histogram).
 struct PrepArgs {
   SeqsDev s;
   int tg, ch;
@@ -328,6 +370,7 @@ struct PrepArgs {
   const float* w;
   uint8_t* codes;
   float* w_scaled;
+  uint8_t* q_sf;  // MXFP8: E8M0 group scales [rows, 4] (w_scaled unused)
   int quant_rows;
   uint32_t* zero;
   int64_t zero_words;
@@ -343,7 +386,12 @@ __global__ void __launch_bounds__(1024) k_prep(const PrepArgs a) {
   const int b = blockIdx.x - 1, nb = gridDim.x - 1;
   if (a.qI) {
     const int row = b * 32 + (threadIdx.x >> 5);
-    if (row < a.quant_rows) quant_row(a.qI, a.w, row, a.codes, a.w_scaled);
+    if (row < a.quant_rows) {
+      if (a.q_sf)
+        quant_row_mx(a.qI, row, a.codes, a.q_sf);
+      else
+        quant_row(a.qI, a.w, row, a.codes, a.w_scaled);
+    }
   }
   if (a.zero) {
     const int64_t per = (a.zero_words + nb - 1) / nb;
@@ -353,13 +401,24 @@ __global__ void __launch_bounds__(1024) k_prep(const PrepArgs a) {
 }
 
 cudaError_t launch_prep(const SeqsDev& s, int tg, int ch, const PlanBufs& plan, const __nv_bfloat16* qI,
-                        const float* w, uint8_t* codes, float* w_scaled, uint32_t* zero, int64_t zero_words,
-                        uint32_t* err, cudaStream_t st) {
-  PrepArgs a{s, tg, ch, plan, err, qI, w, codes, w_scaled, qI ? s.num_tokens * kHI : 0, zero, zero ? zero_words : 0};
+                        const float* w, uint8_t* codes, float* w_scaled, uint8_t* q_sf, uint32_t* zero,
+                        int64_t zero_words, uint32_t* err, cudaStream_t st) {
+  PrepArgs a{s,     tg,   ch, plan, err, qI, w, codes, w_scaled, q_sf, qI ? s.num_tokens * kHI : 0,
+             zero, zero ? zero_words : 0};
   const int64_t nq = qI ? ((int64_t)s.num_tokens * kHI + 31) / 32 : 0;
   const int64_t nz = zero ? (zero_words + 4095) / 4096 : 0;
   const int64_t extra = nq > nz ? nq : nz;
   cudaError_t e = launch_pdl("prep", k_prep, dim3((unsigned)(1 + extra)), dim3(1024), 0, st, a);
+  if (e != cudaSuccess) return e;
+  return counted(cudaGetLastError());
+}
+
+cudaError_t launch_quantize_index_query_mx(const __nv_bfloat16* qI, int T, uint8_t* codes, uint8_t* scales,
+                                           cudaStream_t st) {
+  const int rows = T * kHI, threads = 256;
+  const int blocks = (rows * 32 + threads - 1) / threads;
+  cudaError_t e = launch_pdl("quantize_index_query_mx", k_quantize_index_query_mx, dim3(blocks), dim3(threads), 0, st,
+                             qI, rows, codes, scales);
   if (e != cudaSuccess) return e;
   return counted(cudaGetLastError());
 }

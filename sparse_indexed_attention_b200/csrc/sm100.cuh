@@ -351,5 +351,43 @@ __host__ __device__ constexpr uint32_t make_idesc_major(bool bf16, int M, int N,
   return make_idesc(bf16, M, N) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
 }
 
+// ---------------------------------------------------------------- block-scaled MMA (MXFP8)
+// Instruction descriptor of kind::mxf8f6f4.block_scale: A and B E4M3 and
+// K-major, E8M0 scale factors, D f32 (implied), M x N, K = 32 per instruction.
+// sf_id (bits 4-5 for B, 29-30 for A) picks the byte of each 32-bit scale
+// column: the instruction's 32-wide K block inside a 128-wide K tile.
+__host__ __device__ constexpr uint32_t make_idesc_mx(int M, int N, int sf_id) {
+  return ((uint32_t)sf_id << 4)              // B scale-factor byte
+         | ((uint32_t)(N >> 3) << 17)        // N / 8
+         | (1u << 23)                        // scale format E8M0
+         | ((uint32_t)(M >> 4) << 24)        // M / 16
+         | ((uint32_t)sf_id << 29);          // A scale-factor byte
+}
+
+// D (+)= (A * 2^sfa) (B * 2^sfb)^T per 32-wide K block.  sfa / sfb are TMEM
+// addresses of the scale columns with the byte index in bits 30-31.  Scale
+// layout (M = 128 rows of A, and likewise the N rows of B): row r has its
+// scale in lane r % 32 of every lane quarter (the same 32 lanes written four
+// times), column r / 32, byte = K block.
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t sfa, uint32_t sfb, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
+// 32 rows x 128 bits from shared memory into TMEM columns [taddr, taddr + 4),
+// the same 32 rows written to lanes 0-31 of each of the four lane quarters
+// (the scale-factor layout above).  Executes in order with this thread's MMAs.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of 32 rows of 16 bytes stored back to back, no
+// swizzle: 8-row core matrices 128 bytes apart (the source of tmem_cp_32x128b_x4).
+__device__ __forceinline__ uint64_t rows16_desc(uint32_t saddr) { return smem_desc(saddr, 128, 128, 0); }
+
 }  // namespace sm100
 }  // namespace dsa

@@ -56,3 +56,23 @@ def test_entry_points_want_cuda_tensors():
         dsa.dsa_sparse_mla_fwd_noalloc(seqs, q, kv, idx, 0.1)
     with pytest.raises(TypeError, match="CUDA"):
         dsa.dsa_index_topk_attn(seqs, qI, w, kI, None, q, kv, K, 0.1)
+
+
+def test_index_cache_format_follows_the_scale_dtype(monkeypatch):
+    """No scale: bf16 cache; fp32 [R]: E4M3 with a row scale; uint8 [R, 4]:
+    MXFP8 with E8M0 group scales.  Each form is checked against its own shape."""
+    assert dsa._ki_dtype(None) == dsa.DSA_KI_BF16
+    assert dsa._ki_dtype(torch.ones(128)) == dsa.DSA_KI_FP8_E4M3
+    assert dsa._ki_dtype(torch.full((128, 4), 127, dtype=torch.uint8)) == dsa.DSA_KI_MXFP8
+    seqs = dsa.Seqs(torch.tensor([0, 1], dtype=torch.int32), torch.tensor([5], dtype=torch.int32),
+                    torch.zeros(1, 1, dtype=torch.int32), 1, 5, 1)
+    qI, w = torch.zeros(1, 64, 128, dtype=torch.bfloat16), torch.zeros(1, 64)
+    kI = torch.zeros(64, 128, dtype=torch.uint8)
+    with pytest.raises(TypeError, match="CUDA"):
+        dsa.dsa_quantize_index_query_mx(qI)
+    monkeypatch.setattr(dsa, "_cuda_device", lambda t, name: t.device)  # the shape rules, on CPU tensors
+    dsa._need_index_inputs(seqs, qI, w, kI, torch.full((64, 4), 127, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="shape"):
+        dsa._need_index_inputs(seqs, qI, w, kI, torch.full((64, 2), 127, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="at least 64"):
+        dsa._need_index_inputs(seqs, qI, w, kI, torch.full((63, 4), 127, dtype=torch.uint8))

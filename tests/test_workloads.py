@@ -46,3 +46,18 @@ def test_modes():
     assert np.all(c.q_len <= c.ctx_len) and np.all(c.q_len >= 10)
     p = make_workload(SMALL["pool"])
     assert p.num_phys_pages == 100
+
+
+def test_mx_cache_rows_are_mxfp8_encodings():
+    """Every MXFP8 cache row is a fixed point of the format: its decoded values
+    quantize back to the same codes and scales (each block's largest code lies
+    in E4M3's top binade, as the shared-exponent rule puts it)."""
+    from oracle import dsa_oracle as O
+    spec = CONFIGS["decode_b64_8k_32k"].scaled(batch=2, ctx=(300, 700), ki_mx=True, planted=8)
+    wl = make_workload(spec)
+    codes, sc = wl.kI.numpy(), wl.kI_scale.numpy()
+    assert codes.dtype == np.uint8 and sc.shape == (codes.shape[0], 4)
+    c2, s2 = O.mxfp8_quantize(O.mxfp8_dequantize(codes, sc))
+    assert np.array_equal(c2, codes) and np.array_equal(s2, sc)
+    used = np.abs(O.mxfp8_dequantize(codes, sc)).reshape(-1, 4, 32).max(-1) > 0
+    assert used.mean() > 0.5
