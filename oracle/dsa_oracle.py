@@ -40,7 +40,11 @@ Readings taken where the pages are silent (each repeated at its function):
   * MXFP8 (the pages' index format: one shared scale per group of 32) is read
     as the OCP Microscaling format: E4M3 elements sharing an E8M0 power-of-two
     scale per block of 32, the scale 2^(floor(log2 amax) - 8), elements of the
-    block's top binade above 448 saturating.  Cache and query both take it.
+    block's top binade above 448 saturating.  Cache and query both take it;
+  * the FP8 latent KV cache (the pages: FP8, per token-head tile of 128) cuts
+    each 576-value latent row into tiles of 128 (the last, the 64 rope dims,
+    of 64) with one power-of-two scale per tile, the tightest that needs no
+    saturation (so every dequantized value is an exact bf16 number).
 
 Every function here is pinned by a test in ``tests/test_oracle_*.py`` against
 something other than itself (library routines, brute force, closed forms,
@@ -207,6 +211,58 @@ def mxfp8_dequantize(codes, scales) -> np.ndarray:
     return (v * e8m0_decode(scales)[..., None]).reshape(c.shape)
 
 
+# ----------------------------------------------------------------------------
+# FP8 latent KV cache ([P2] §5 table, "Main attention KV cache": FP8, per
+# token-head tile, tile size 128; [P3] §4 "Layered Quantization")
+# ----------------------------------------------------------------------------
+
+KV_TILE = 128        # elements per scale along the latent row
+KV_SCALE_COLS = 8    # scale bytes stored per row: one per tile (5 used), zero padding
+
+
+def kv_fp8_quantize(kv):
+    """Real latent rows [R, 576] -> (E4M3 codes [R, 576], scale bytes [R, 8]).
+
+    Tile j holds elements 128j .. 128j+127 of the row (tile 4: the 64 rope
+    dims 512..575).  Its scale is 2^e with e = ``pow2_exponent(max |tile|)``,
+    the smallest power of two for which nothing saturates; codes = E4M3(x / 2^e)
+    rounded to nearest-even; byte j of the row's scales holds e + 127, bytes
+    5..7 are 0.  Reading: the pages fix the granularity, not the scale format;
+    a power-of-two scale keeps every dequantized value an exact bf16 number."""
+    x = np.asarray(kv, dtype=np.float64)
+    R, D = x.shape
+    ntiles = (D + KV_TILE - 1) // KV_TILE
+    codes = np.zeros((R, D), dtype=np.uint8)
+    scales = np.zeros((R, KV_SCALE_COLS), dtype=np.uint8)
+    for j in range(ntiles):
+        lo, hi = j * KV_TILE, min(D, (j + 1) * KV_TILE)
+        amax = np.abs(x[:, lo:hi]).max(axis=1)
+        e = np.vectorize(pow2_exponent, otypes=[np.int64])(amax)
+        codes[:, lo:hi] = e4m3_encode(x[:, lo:hi] / np.ldexp(1.0, e)[:, None])
+        scales[:, j] = (e + E8M0_BIAS).astype(np.uint8)
+    return codes, scales
+
+
+def kv_fp8_dequantize(codes, scales) -> np.ndarray:
+    """Exact values of FP8 latent rows: E4M3(codes) * 2^(scale byte - 127) per tile."""
+    c = np.asarray(codes, dtype=np.uint8)
+    sc = np.asarray(scales, dtype=np.uint8)
+    v = e4m3_decode_fast(c).copy()
+    for j in range((c.shape[-1] + KV_TILE - 1) // KV_TILE):
+        lo, hi = j * KV_TILE, min(c.shape[-1], (j + 1) * KV_TILE)
+        v[..., lo:hi] *= e8m0_decode(sc[..., j])[..., None]
+    return v
+
+
+def kv_rows(kv, rows) -> np.ndarray:
+    """Exact values of latent-pool rows `rows`: the pool is bf16 bit patterns
+    [R, 576] (uint16), or an FP8 cache given as (codes [R, 576], scales [R, 8])."""
+    if isinstance(kv, tuple):
+        codes, scales = kv
+        return kv_fp8_dequantize(np.asarray(codes)[rows], np.asarray(scales)[rows])
+    return bf16_to_f64(np.asarray(kv)[rows])
+
+
 def is_mx_scale(kI_scale) -> bool:
     """An MXFP8 index cache carries E8M0 codes [R, 4] (uint8); an E4M3 cache one
     fp32 scale per row."""
@@ -359,6 +415,7 @@ def sparse_mla(seqs: Seqs, q_bits, kv_bits, idx, scale: float, d_v: int = 512, t
     Keys are the whole latent row (latent + rope, 576 values); values are its
     first d_v = 512 (the latent).  All heads share the KV rows.  idx[t] holds
     logical positions with -1 padding; the order of idx does not matter.
+    kv_bits: the bf16 pool, or an FP8 cache (codes, scales) (``kv_rows``).
     Returns (out [n_tok, H, d_v], lse [n_tok, H]) in float64.
     """
     idx = np.asarray(idx)
@@ -371,7 +428,7 @@ def sparse_mla(seqs: Seqs, q_bits, kv_bits, idx, scale: float, d_v: int = 512, t
         sel = idx[t][idx[t] >= 0].astype(np.int64)
         if sel.size == 0 or sel.max() > pos or np.unique(sel).size != sel.size:
             raise ValueError(f"token {t}: invalid selection")
-        kmat = bf16_to_f64(np.asarray(kv_bits)[seqs.rows(b, sel)])    # [k, 576]
+        kmat = kv_rows(kv_bits, seqs.rows(b, sel))                    # [k, 576]
         qt = bf16_to_f64(np.asarray(q_bits)[t])                       # [H, 576]
         logits = scale * (qt @ kmat.T)                                # [H, k]
         m = logits.max(axis=1, keepdims=True)

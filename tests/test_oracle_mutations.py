@@ -17,7 +17,7 @@ ORACLE = os.path.join(ROOT, "oracle", "dsa_oracle.py")
 
 CODEC, QUANT, INDEXER = "test_oracle_codec.py", "test_oracle_quant.py", "test_oracle_indexer.py"
 TOPK, ATTN, PIPE = "test_oracle_topk.py", "test_oracle_attention.py", "test_oracle_pipeline.py"
-MX = "test_oracle_mx.py"
+MX, KV8 = "test_oracle_mx.py", "test_oracle_kv8.py"
 
 # name: (text in the oracle, replacement, pin files that must fail)
 MUTANTS = {
@@ -64,6 +64,14 @@ MUTANTS = {
                              "kmat = e4m3_decode_fast(np.asarray(kI)[rows])", [MX]),
     "mx_key_scale_wrong_row": ("kmat = mxfp8_dequantize(np.asarray(kI)[rows], np.asarray(kI_scale)[rows])",
                                "kmat = mxfp8_dequantize(np.asarray(kI)[rows], np.asarray(kI_scale)[rows[::-1]])", [MX]),
+    "kv8_tile_64": ("KV_TILE = 128        # elements per scale", "KV_TILE = 64         # elements per scale", [KV8]),
+    "kv8_scale_dropped": ("v[..., lo:hi] *= e8m0_decode(sc[..., j])[..., None]", "v[..., lo:hi] *= 1.0", [KV8]),
+    "kv8_scale_of_first_tile": ("v[..., lo:hi] *= e8m0_decode(sc[..., j])[..., None]",
+                                "v[..., lo:hi] *= e8m0_decode(sc[..., 0])[..., None]", [KV8]),
+    "kv8_rope_tile_unscaled": ("for j in range((c.shape[-1] + KV_TILE - 1) // KV_TILE):",
+                               "for j in range(c.shape[-1] // KV_TILE):", [KV8]),
+    "kv8_attention_reads_raw_codes": ("return kv_fp8_dequantize(np.asarray(codes)[rows], np.asarray(scales)[rows])",
+                                      "return e4m3_decode_fast(np.asarray(codes)[rows])", [KV8]),
 }
 
 
