@@ -76,6 +76,8 @@ def parse():
                     help="one JSON line per workload: fused-call time and the binding roofline of each stage")
     ap.add_argument("--ki", choices=["workload", "mxfp8"], default="workload",
                     help="index-cache format: the workload's own (E4M3 + row scale for the headline) or MXFP8")
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
+                    help="latent KV cache: bf16, or FP8 E4M3 with a power-of-two scale per 128-element tile")
     ap.add_argument("--select-in-indexer", action="store_true",
                     help="decode: select the Top-K inside the indexer kernel (DSA_SELECT_IN_INDEXER)")
     ap.add_argument("--only", choices=["index_scores", "topk", "sparse_mla", "fused"], default=None,
@@ -229,7 +231,8 @@ def cpu_baseline(wl, n_tokens: int):
         kI, sc = bits16(wl.kI), None
     else:
         kI, sc = wl.kI.numpy(), wl.kI_scale.numpy()
-    qI, w, q, kv = bits16(wl.qI), wl.w.numpy(), bits16(wl.q), bits16(wl.kv)
+    qI, w, q = bits16(wl.qI), wl.w.numpy(), bits16(wl.q)
+    kv = bits16(wl.kv) if wl.kv_scale is None else (wl.kv.numpy(), wl.kv_scale.numpy())
     toks = list(range(n_tokens))
     t0 = time.perf_counter()
     O.index_topk_attn(seqs, qI, w, kI, sc, q, kv, wl.spec.topk, wl.scale, tokens=toks)
@@ -248,6 +251,7 @@ def workload_config(spec, wl, world: int) -> dict:
             "ctx": int(wl.ctx_len[0]), "topk": spec.topk, "heads": spec.heads, "index_heads": spec.index_heads,
             "index_dim": spec.index_dim, "page_size": spec.page_size, "pool_tokens": wl.num_phys_pages * 64,
             "index_cache": "mxfp8" if spec.ki_mx else ("fp8_e4m3" if spec.ki_fp8 else "bf16"),
+            "latent_cache": "fp8_e4m3_tile128" if spec.kv_fp8 else "bf16",
             "parallelism": f"dp{world}",
             "l2": "256 MiB buffer written before every timed GPU step"}
 
@@ -258,6 +262,8 @@ def bench_spec(args):
     spec = CONFIGS[args.config]
     if args.ki == "mxfp8":
         spec = spec.scaled(ki_mx=True)
+    if args.kv == "fp8":
+        spec = spec.scaled(kv_fp8=True)
     if args.ctx > 0:
         spec = spec.scaled(ctx=(args.ctx, args.ctx))
     return spec
@@ -350,7 +356,8 @@ def run_only(args, dsa, wl, d, dev, stream, flush, world, fused=None):
     fns = {
         "index_scores": lambda: dsa.dsa_index_scores(d.seqs, d.qI, d.w, d.kI, d.kI_scale, scores=scores),
         "topk": lambda: dsa.dsa_topk(scores, row_len, K, idx=idx),
-        "sparse_mla": lambda: dsa.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out=out, lse=lse),
+        "sparse_mla": lambda: dsa.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out=out, lse=lse,
+                                                     kv_scale=d.kv_scale),
         "fused": fused,
     }
     times = time_device(fns[args.only], args.steps, args.warmup, stream, flush)
@@ -365,7 +372,7 @@ def run_all_configs(args, dsa, dev, stream, flush):
     from dsa_workloads import to_device
     hbm, hbm_src = hbm_peak()
     for name in CONFIGS:
-        spec = CONFIGS[name].scaled(ki_mx=True) if args.ki == "mxfp8" else CONFIGS[name]
+        spec = CONFIGS[name].scaled(ki_mx=args.ki == "mxfp8", kv_fp8=args.kv == "fp8")
         wl = make_workload(spec)
         d = to_device(wl)
         T, H, K = wl.T, spec.heads, spec.topk
@@ -376,7 +383,7 @@ def run_all_configs(args, dsa, dev, stream, flush):
 
         def step():
             dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse,
-                                    ws=ws, select_in_indexer=args.select_in_indexer)
+                                    ws=ws, select_in_indexer=args.select_in_indexer, kv_scale=d.kv_scale)
 
         for _ in range(2):
             step()
@@ -419,7 +426,7 @@ def run_all_configs(args, dsa, dev, stream, flush):
         if attn_us:
             t_s = attn_us * 1e-6
             if decode:
-                b = sel * 1152
+                b = sel * (584 if spec.kv_fp8 else 1152)
                 stages["sparse_mla"] = {"bound": "hbm", "us": attn_us, "achieved": b / t_s / 1e9, "peak": hbm,
                                         "unit": "GB/s", "frac": b / t_s / 1e9 / hbm}
             else:
@@ -461,7 +468,7 @@ def run_ours(args, world, rank, local):
 
     def step():
         dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse, ws=ws,
-                                select_in_indexer=sel)
+                                select_in_indexer=sel, kv_scale=d.kv_scale)
 
     if args.only:
         run_only(args, dsa, wl, d, dev, stream, flush, world, fused=step)
@@ -516,12 +523,13 @@ def run_ours(args, world, rank, local):
     t_idx = time_device(lambda: dsa.dsa_index_scores(d.seqs, d.qI, d.w, d.kI, d.kI_scale, scores=scores, ws=ws_i),
                         reps, 3, stream, flush)
     t_topk = time_device(lambda: dsa.dsa_topk(scores, row_len, K, idx=idx, ws=ws_t), reps, 3, stream, flush)
-    t_attn = time_device(lambda: dsa.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out=out, lse=lse, ws=ws_a),
+    t_attn = time_device(lambda: dsa.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out=out, lse=lse, ws=ws_a,
+                                                        kv_scale=d.kv_scale),
                          reps, 3, stream, flush)
     n_keys = int((wl.token_pos() + 1).sum())
     n_sel = int(np.minimum(wl.token_pos() + 1, K).sum())
     idx_bytes = n_keys * (132 if spec.ki_fp8 else 256)          # index-cache bytes read
-    attn_bytes = n_sel * 1152                                    # gathered latent rows
+    attn_bytes = n_sel * (584 if spec.kv_fp8 else 1152)           # gathered latent rows (FP8: codes + 8 scale bytes)
     peak, peak_kind = hbm_peak()
     ms_idx = statistics.mean(t_idx)
     score_bytes = n_keys * 4 + T * K * 4                          # Top-K: score rows read, indices written
@@ -557,7 +565,7 @@ def run_ours(args, world, rank, local):
             d.q.copy_(h_q, non_blocking=True)
             q_ready.record(side)
         dsa.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale, out=out, lse=lse, ws=ws,
-                                q_ready=q_ready, select_in_indexer=sel)
+                                q_ready=q_ready, select_in_indexer=sel, kv_scale=d.kv_scale)
         h_out.copy_(out, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
 
@@ -604,7 +612,8 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": ("mxfp8" if spec.ki_mx else "fp8-e4m3") + " index / bf16 attention / fp32 accum",
+            "dtype": ("mxfp8" if spec.ki_mx else "fp8-e4m3") + " index / "
+                     + ("fp8-e4m3 latent, " if spec.kv_fp8 else "") + "bf16 attention / fp32 accum",
             "data": "synthetic (seeded, 64 planted keys per sequence)",
             "config": workload_config(spec, wl, world),
             "launch": launch_mode,

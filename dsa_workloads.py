@@ -29,7 +29,11 @@ the order written below):
      row), codes = E4M3(row / scale) by torch's round-to-nearest cast, or as
      MXFP8: E4M3 codes with one E8M0 scale byte per 32 elements, scale
      2^(floor(log2 max|block|) - 8) (2^0 for a zero block), codes =
-     E4M3(block / scale) clamped to +-448, by the same cast.
+     E4M3(block / scale) clamped to +-448, by the same cast; latent KV as bf16
+     or as the FP8 cache: per row, tiles of 128 values (the last of 64), each
+     with scale 2^e, e the smallest integer with max|tile| <= 448 * 2^e (2^0
+     for a zero tile), codes = E4M3(tile / 2^e), scale bytes e + 127 in [R, 8]
+     (bytes 5..7 zero).
 """
 from __future__ import annotations
 
@@ -52,6 +56,7 @@ class Spec:
     chunk: tuple = (0, 0)           # chunked: new chunk length range
     ki_fp8: bool = True             # FP8 E4M3 index cache with per-row scale
     ki_mx: bool = False             # MXFP8 index cache (E4M3 + E8M0 per 32 elements); overrides ki_fp8
+    kv_fp8: bool = False            # FP8 latent KV cache (E4M3, power-of-two scale per 128-element tile)
     heads: int = 128                # attention query heads
     topk: int = 2048
     planted: int = 0
@@ -94,8 +99,9 @@ class Workload:
     kI: torch.Tensor               # uint8 FP8 codes or bf16 [R, d_I]
     kI_scale: torch.Tensor | None  # fp32 [R] (FP8 cache), uint8 E8M0 [R, 4] (MXFP8) or None
     q: torch.Tensor                # bf16 [T, H, d_qk]
-    kv: torch.Tensor               # bf16 [R, d_qk]
+    kv: torch.Tensor               # bf16 [R, d_qk], or uint8 E4M3 codes [R, d_qk] (FP8 cache)
     planted: list                  # per sequence: np.ndarray of planted positions
+    kv_scale: torch.Tensor | None = None  # FP8 latent cache: uint8 [R, 8] tile-scale bytes
 
     @property
     def T(self) -> int:
@@ -145,6 +151,25 @@ def fp8_rows(x: torch.Tensor):
     scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
     codes = (x / scale[:, None]).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
     return codes, scale.to(torch.float32)
+
+
+def kv8_rows(x: torch.Tensor):
+    """Store fp32 latent rows as the FP8 cache: E4M3 codes [R, d] and the tiles'
+    scale bytes [R, 8] (tile j = elements 128j .. 128j+127)."""
+    R, d = x.shape
+    codes = torch.zeros((R, d), dtype=torch.uint8)
+    scales = torch.zeros((R, 8), dtype=torch.uint8)
+    for j in range((d + 127) // 128):
+        lo, hi = 128 * j, min(d, 128 * (j + 1))
+        a = x[:, lo:hi].abs().amax(dim=1).double()
+        e = torch.where(a > 0, torch.ceil(torch.log2(a / 448.0)), torch.zeros_like(a))
+        for _ in range(2):  # the estimate, made exact by comparisons (448 * 2^e is exact in fp64)
+            e = torch.where(a > 448.0 * torch.exp2(e), e + 1, e)
+            e = torch.where((a > 0) & (a <= 448.0 * torch.exp2(e - 1)), e - 1, e)
+        t = (x[:, lo:hi].double() * torch.exp2(-e)[:, None]).clamp_(-448.0, 448.0).float()
+        codes[:, lo:hi] = t.to(torch.float8_e4m3fn).view(torch.uint8)
+        scales[:, j] = (e + 127).to(torch.uint8)
+    return codes, scales
 
 
 def mx_rows(x: torch.Tensor):
@@ -234,8 +259,17 @@ def make_workload(spec: Spec) -> Workload:
     phys_rows = torch.from_numpy((slot_page[:, None] * ps + np.arange(ps)[None, :]).reshape(-1))
 
     R = num_phys * ps
-    kv = torch.zeros((R, spec.d_qk), dtype=torch.bfloat16)
-    kv[phys_rows] = kv_vals.to(torch.bfloat16)
+    kv_scale = None
+    if spec.kv_fp8:
+        codes, sc = kv8_rows(kv_vals)
+        kv = torch.zeros((R, spec.d_qk), dtype=torch.uint8)
+        kv[phys_rows] = codes
+        kv_scale = torch.zeros((R, 8), dtype=torch.uint8)
+        kv_scale[:, :5] = 127
+        kv_scale[phys_rows] = sc
+    else:
+        kv = torch.zeros((R, spec.d_qk), dtype=torch.bfloat16)
+        kv[phys_rows] = kv_vals.to(torch.bfloat16)
     del kv_vals
     if spec.ki_mx:
         codes, sc = mx_rows(ki_vals)
@@ -257,7 +291,7 @@ def make_workload(spec: Spec) -> Workload:
     return Workload(spec=spec, ctx_len=ctx.astype(np.int32), q_len=q_len.astype(np.int32),
                     q_seq_start=q_seq_start.astype(np.int32), page_table=page_table,
                     num_phys_pages=num_phys, qI=qI, w=w, kI=kI, kI_scale=kI_scale, q=q, kv=kv,
-                    planted=planted)
+                    planted=planted, kv_scale=kv_scale)
 
 
 def bits16(x: torch.Tensor) -> np.ndarray:
@@ -276,6 +310,7 @@ class DeviceWorkload:
     kI_scale: torch.Tensor | None
     q: torch.Tensor
     kv: torch.Tensor
+    kv_scale: torch.Tensor | None = None
 
     @property
     def K(self) -> int:
@@ -295,4 +330,5 @@ def to_device(wl: Workload, device="cuda") -> DeviceWorkload:
     from sparse_indexed_attention_b200 import Seqs
     seqs = Seqs.from_host(wl.q_seq_start, wl.ctx_len, wl.page_table, wl.num_phys_pages, device=device)
     dev = lambda x: None if x is None else x.contiguous().to(device)  # noqa: E731
-    return DeviceWorkload(wl, seqs, dev(wl.qI), dev(wl.w), dev(wl.kI), dev(wl.kI_scale), dev(wl.q), dev(wl.kv))
+    return DeviceWorkload(wl, seqs, dev(wl.qI), dev(wl.w), dev(wl.kI), dev(wl.kI_scale), dev(wl.q), dev(wl.kv),
+                          dev(wl.kv_scale))

@@ -102,6 +102,16 @@ typedef enum {
 } dsa_ki_dtype_t;
 
 typedef enum {
+  DSA_KV_BF16 = 0,     /* latent KV pool is bf16 [R,576]; kv_scale must be NULL   */
+  DSA_KV_FP8_E4M3 = 1  /* latent KV pool is OCP E4M3 codes [R,576] + kv_scale uint8
+                          [R,8]: byte j (j = 0..4) scales elements 128j..128j+127
+                          (the last tile: the 64 rope dims) by 2^(byte - 127),
+                          bytes 5..7 unused.  Bytes 1..254 are valid.  ([P2]
+                          section 5 table, "Main attention KV cache": FP8, per
+                          token-head tile of 128.)                              */
+} dsa_kv_dtype_t;
+
+typedef enum {
   DSA_OUT_BF16 = 0,    /* attention output stored as bf16 (rounded to nearest even) */
   DSA_OUT_F32 = 1      /* attention output stored as fp32 (no output rounding)      */
 } dsa_out_dtype_t;
@@ -226,6 +236,20 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t *seqs, const void *q,
                                 dsa_out_dtype_t out_dtype, float *lse,
                                 void *ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* dsa_sparse_mla_fwd with the latent pool's format: kv_dtype DSA_KV_BF16
+ * (kv_scale NULL) is dsa_sparse_mla_fwd; DSA_KV_FP8_E4M3 reads E4M3 codes kv
+ * [R,576] and tile-scale bytes kv_scale [R,8] (16-byte aligned) and attends
+ * over the dequantized rows KV[s,d] = E4M3(kv[s,d]) * 2^(kv_scale[s,d/128] - 127),
+ * which are exact bf16 values, so the arithmetic is that of a bf16 pool
+ * holding them.  Same workspace as dsa_sparse_mla_fwd. */
+dsa_status_t dsa_sparse_mla_fwd_ex(const dsa_seqs_t *seqs, const void *q,
+                                   const void *kv, const void *kv_scale,
+                                   dsa_kv_dtype_t kv_dtype, const int32_t *idx,
+                                   int K, int H, float scale, void *out,
+                                   dsa_out_dtype_t out_dtype, float *lse,
+                                   void *ws, size_t ws_bytes,
+                                   dsa_stream_t stream);
+
 /* Size of the scratch array dsa_sparse_mla_fwd_noalloc uses (32 MiB). */
 #define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
 
@@ -280,7 +304,8 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t *seqs, const void *qI,
                                  int32_t *idx_out, void *ws, size_t ws_bytes,
                                  dsa_stream_t stream);
 
-/* dsa_index_topk_attn with options.  `flags`: 0 or DSA_SELECT_IN_INDEXER.
+/* dsa_index_topk_attn with options.  `kv_scale` / `kv_dtype`: the latent
+ * pool's format, as in dsa_sparse_mla_fwd_ex.  `flags`: 0 or DSA_SELECT_IN_INDEXER.
  * `q_ready`: for a caller whose attention query q is still being
  * produced or copied on another stream when the call is made ([P2] section
  * 4(2): the indexer's inputs are prepared apart from the attention's, so the
@@ -292,8 +317,9 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t *seqs, const void *qI,
 dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t *seqs, const void *qI,
                                     const float *w, const void *kI,
                                     const void *kI_scale, dsa_ki_dtype_t ki_dtype,
-                                    const void *q, const void *kv, int K, int H,
-                                    float scale, void *out,
+                                    const void *q, const void *kv,
+                                    const void *kv_scale, dsa_kv_dtype_t kv_dtype,
+                                    int K, int H, float scale, void *out,
                                     dsa_out_dtype_t out_dtype, float *lse,
                                     int32_t *idx_out, void *ws, size_t ws_bytes,
                                     unsigned flags, dsa_event_t q_ready,

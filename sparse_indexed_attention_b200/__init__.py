@@ -31,6 +31,7 @@ LIB_PATH = _build.LIB
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_BAD_INDEX, \
     DSA_ERR_TIMEOUT = range(7)
 DSA_KI_BF16, DSA_KI_FP8_E4M3, DSA_KI_MXFP8 = 0, 1, 2
+DSA_KV_BF16, DSA_KV_FP8_E4M3 = 0, 1
 DSA_OUT_BF16, DSA_OUT_F32 = 0, 1
 DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_INDEX_TOPK_ATTN, \
@@ -40,7 +41,7 @@ DSA_SELECT_IN_INDEXER = 1
 # Names the C header declares (checked against include/dsa.h by the tests).
 EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_quantize_index_query_mx", "dsa_index_scores",
            "dsa_topk",
-           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_noalloc", "dsa_check_error_noalloc", "dsa_index_topk_attn",
+           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_ex", "dsa_sparse_mla_fwd_noalloc", "dsa_check_error_noalloc", "dsa_index_topk_attn",
            "dsa_index_topk_attn_ex",
            "dsa_check_error", "dsa_set_wait_limit_ns", "dsa_launches_in_last_call", "dsa_launch_timing",
            "dsa_last_launch_times", "dsa_status_string")
@@ -63,12 +64,15 @@ _sig = {
     "dsa_topk": (ctypes.c_int, [_P, _I64, ctypes.c_int, _P, ctypes.c_int, _P, _P, _SZ, _P]),
     "dsa_sparse_mla_fwd": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, ctypes.c_int, _F, _P, ctypes.c_int, _P, _P,
                                           _SZ, _P]),
+    "dsa_sparse_mla_fwd_ex": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, ctypes.c_int, _F, _P,
+                                             ctypes.c_int, _P, _P, _SZ, _P]),
     "dsa_sparse_mla_fwd_noalloc": (ctypes.c_int, [_SEQ, _P, _P, _P, ctypes.c_int, ctypes.c_int, _F, _P, ctypes.c_int,
                                                   _P, _P]),
     "dsa_index_topk_attn": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
                                            _F, _P, ctypes.c_int, _P, _P, _P, _SZ, _P]),
-    "dsa_index_topk_attn_ex": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, ctypes.c_int,
-                                              _F, _P, ctypes.c_int, _P, _P, _P, _SZ, ctypes.c_uint, _P, _P]),
+    "dsa_index_topk_attn_ex": (ctypes.c_int, [_SEQ, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, _F, _P, ctypes.c_int, _P, _P, _P, _SZ,
+                                              ctypes.c_uint, _P, _P]),
     "dsa_check_error": (ctypes.c_int, [_P, _P]),
     "dsa_check_error_noalloc": (ctypes.c_int, [_P]),
     "dsa_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
@@ -188,12 +192,17 @@ def _ki_dtype(kI_scale) -> int:
     return DSA_KI_MXFP8 if _is_mx(kI_scale) else DSA_KI_FP8_E4M3
 
 
-def _need_attn_inputs(seqs: "Seqs", q, kv, out, lse) -> torch.device:
+def _need_attn_inputs(seqs: "Seqs", q, kv, out, lse, kv_scale=None) -> torch.device:
     dev = _cuda_device(q, "q")
     _need_seqs(seqs, dev)
     _need(q, "q", _BF16T, (seqs.num_q_tokens, None, 576), dev)
     T, H = q.shape[0], q.shape[1]
-    _need(kv, "kv", _BF16T, (None, 576), dev, seqs.num_phys_pages * 64)
+    rows = seqs.num_phys_pages * 64
+    if kv_scale is None:
+        _need(kv, "kv", _BF16T, (None, 576), dev, rows)
+    else:  # FP8 latent cache: E4M3 codes and per-row tile-scale bytes
+        _need(kv, "kv", _FP8T, (None, 576), dev, rows)
+        _need(kv_scale, "kv_scale", (torch.uint8,), (None, 8), dev, rows)
     _need(out, "out", (torch.bfloat16, torch.float32), (T, H, 512), dev)
     if lse is not None:
         _need(lse, "lse", _F32T, (T, H), dev)
@@ -337,21 +346,24 @@ def _out_dtype(out: torch.Tensor) -> int:
 
 
 def dsa_sparse_mla_fwd(seqs: Seqs, q, kv, idx, scale: float, out=None, lse=None, want_lse=True, ws=None,
-                       out_dtype=torch.bfloat16):
+                       out_dtype=torch.bfloat16, kv_scale=None):
+    """Sparse MLA over the selected rows.  kv_scale (uint8 [R, 8]) marks an FP8
+    latent cache: kv then holds E4M3 codes [R, 576] (dsa_sparse_mla_fwd_ex)."""
     T, H, _ = q.shape
     K = idx.shape[1]
     out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
-    dev = _need_attn_inputs(seqs, q, kv, out, lse)
+    dev = _need_attn_inputs(seqs, q, kv, out, lse, kv_scale)
     _need(idx, "idx", _I32T, (T, K), dev)
     c = seqs.c()
     need = _lib.dsa_workspace_size(DSA_OP_SPARSE_MLA, ctypes.byref(c), K, H)
     ws = ws if ws is not None else workspace(need, q.device, "sparse_mla")
     _need_ws(ws, dev)
-    _check(_lib.dsa_sparse_mla_fwd(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(idx), K, H, scale, _ptr(out),
-                                   _out_dtype(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device)),
-           "dsa_sparse_mla_fwd")
+    kv_dtype = DSA_KV_BF16 if kv_scale is None else DSA_KV_FP8_E4M3
+    _check(_lib.dsa_sparse_mla_fwd_ex(ctypes.byref(c), _ptr(q), _ptr(kv), _ptr(kv_scale), kv_dtype, _ptr(idx), K, H,
+                                      scale, _ptr(out), _out_dtype(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                      _stream(q.device)), "dsa_sparse_mla_fwd")
     return out, lse
 
 
@@ -376,16 +388,17 @@ def dsa_sparse_mla_fwd_noalloc(seqs: Seqs, q, kv, idx, scale: float, out=None, l
 
 def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: float, out=None, lse=None,
                         idx_out=None, want_lse=True, ws=None, out_dtype=torch.bfloat16, q_ready=None,
-                        select_in_indexer=False):
+                        select_in_indexer=False, kv_scale=None):
     """The whole path.  q_ready (a torch.cuda.Event, optional): the attention
     launch waits on it, so q may still be in flight on another stream.
     select_in_indexer: decode rows that fit are selected inside the indexer
-    kernel (DSA_SELECT_IN_INDEXER)."""
+    kernel (DSA_SELECT_IN_INDEXER).  kv_scale (uint8 [R, 8]) marks an FP8
+    latent cache (kv = E4M3 codes [R, 576])."""
     T, H, _ = q.shape
     out = out if out is not None else torch.empty((T, H, 512), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
-    dev = _need_attn_inputs(seqs, q, kv, out, lse)
+    dev = _need_attn_inputs(seqs, q, kv, out, lse, kv_scale)
     if _need_index_inputs(seqs, qI, w, kI, kI_scale, check_seqs=False) != dev:
         raise ValueError("qI and q are on different devices")
     if idx_out is not None:
@@ -397,10 +410,12 @@ def dsa_index_topk_attn(seqs: Seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: f
     ws = ws if ws is not None else workspace(need, q.device, "index_topk_attn")
     _need_ws(ws, dev)
     ev = None if q_ready is None else ctypes.c_void_p(q_ready.cuda_event)
+    kv_dtype = DSA_KV_BF16 if kv_scale is None else DSA_KV_FP8_E4M3
     _check(_lib.dsa_index_topk_attn_ex(ctypes.byref(c), _ptr(qI), _ptr(w), _ptr(kI), _ptr(kI_scale), ki_dtype, _ptr(q),
-                                       _ptr(kv), K, H, scale, _ptr(out), _out_dtype(out), _ptr(lse), _ptr(idx_out),
-                                       _ptr(ws), ws.numel(), DSA_SELECT_IN_INDEXER if select_in_indexer else 0, ev,
-                                       _stream(q.device)), "dsa_index_topk_attn")
+                                       _ptr(kv), _ptr(kv_scale), kv_dtype, K, H, scale, _ptr(out), _out_dtype(out),
+                                       _ptr(lse), _ptr(idx_out), _ptr(ws), ws.numel(),
+                                       DSA_SELECT_IN_INDEXER if select_in_indexer else 0, ev, _stream(q.device)),
+           "dsa_index_topk_attn")
     return out, lse
 
 

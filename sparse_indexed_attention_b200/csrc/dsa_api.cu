@@ -136,6 +136,13 @@ dsa_status_t check_indexer_args(const dsa_seqs_t* seqs, const void* qI, const fl
   return DSA_OK;
 }
 
+dsa_status_t check_kv_args(const void* kv_scale, dsa_kv_dtype_t kv_dtype) {
+  if (kv_dtype != DSA_KV_BF16 && kv_dtype != DSA_KV_FP8_E4M3) return DSA_ERR_UNSUPPORTED;
+  if ((kv_dtype == DSA_KV_FP8_E4M3) != (kv_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  if (kv_scale && !aligned(kv_scale, 16)) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
 dsa_status_t check_attn_args(const dsa_seqs_t* seqs, const void* q, const void* kv, int K, int H, float scale,
                              const void* out, dsa_out_dtype_t out_dtype, const float* lse) {
   DSA_TRY(check_seqs(seqs));
@@ -264,11 +271,13 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, int T, const int32_t* row
                   (cudaStream_t)stream));
 }
 
-dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const void* kv, const int32_t* idx, int K,
-                                int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse, void* ws,
-                                size_t ws_bytes, dsa_stream_t stream) {
+dsa_status_t dsa_sparse_mla_fwd_ex(const dsa_seqs_t* seqs, const void* q, const void* kv, const void* kv_scale,
+                                   dsa_kv_dtype_t kv_dtype, const int32_t* idx, int K, int H, float scale, void* out,
+                                   dsa_out_dtype_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                                   dsa_stream_t stream) {
   g_launches = 0;
   DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, out_dtype, lse));
+  DSA_TRY(check_kv_args(kv_scale, kv_dtype));
   if (!idx || !aligned(idx, 16)) return DSA_ERR_INVALID_ARG;
   const Layout L = make_layout(DSA_OP_SPARSE_MLA, seqs->num_q_tokens, seqs->batch, seqs->max_ctx, K, H);
   DSA_TRY(check_ws(ws, ws_bytes, L.total));
@@ -279,20 +288,29 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const voi
   TokenMap tm{plan.tok_seq, plan.tok_pos};
   timer_begin(st);
   DSA_CUDA(launch_plan(sd, 1, 0, plan, err, st));  // token geometry only
-  DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/false, reinterpret_cast<const __nv_bfloat16*>(q),
-                             reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
-                             out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
+  DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/false, reinterpret_cast<const __nv_bfloat16*>(q), kv,
+                             static_cast<const uint8_t*>(kv_scale), idx, K, H, scale, out,
+                             out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
   return DSA_OK;
 }
 
+dsa_status_t dsa_sparse_mla_fwd(const dsa_seqs_t* seqs, const void* q, const void* kv, const int32_t* idx, int K,
+                                int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse, void* ws,
+                                size_t ws_bytes, dsa_stream_t stream) {
+  return dsa_sparse_mla_fwd_ex(seqs, q, kv, nullptr, DSA_KV_BF16, idx, K, H, scale, out, out_dtype, lse, ws, ws_bytes,
+                               stream);
+}
+
 dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t* seqs, const void* qI, const float* w, const void* kI,
-                                    const void* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
+                                    const void* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv,
+                                    const void* kv_scale, dsa_kv_dtype_t kv_dtype, int K,
                                     int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse,
                                     int32_t* idx_out, void* ws, size_t ws_bytes, unsigned flags,
                                     dsa_event_t q_ready, dsa_stream_t stream) {
   g_launches = 0;
   DSA_TRY(check_indexer_args(seqs, qI, w, kI, kI_scale, ki_dtype));
   DSA_TRY(check_attn_args(seqs, q, kv, K, H, scale, out, out_dtype, lse));
+  DSA_TRY(check_kv_args(kv_scale, kv_dtype));
   if (idx_out && !aligned(idx_out, 16)) return DSA_ERR_INVALID_ARG;
   if (flags & ~(unsigned)DSA_SELECT_IN_INDEXER) return DSA_ERR_INVALID_ARG;
   const Layout L = make_layout((flags & DSA_SELECT_IN_INDEXER) ? DSA_OP_INDEX_TOPK_ATTN_FUSED : DSA_OP_INDEX_TOPK_ATTN,
@@ -315,8 +333,8 @@ dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t* seqs, const void* qI, cons
     DSA_TRY(run_indexer(seqs, sd, plan, tg, qI, w, kI, kI_scale, ki_dtype, nullptr, L.ld, ws, L, nullptr, tail,
                         L.tail_words, err, st, &f));
     if (q_ready) DSA_CUDA(cudaStreamWaitEvent(st, (cudaEvent_t)q_ready, 0));
-    DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/true, reinterpret_cast<const __nv_bfloat16*>(q),
-                               reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
+    DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/true, reinterpret_cast<const __nv_bfloat16*>(q), kv,
+                               static_cast<const uint8_t*>(kv_scale), idx, K, H, scale,
                                out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
     return DSA_OK;
   }
@@ -331,8 +349,8 @@ dsa_status_t dsa_index_topk_attn_ex(const dsa_seqs_t* seqs, const void* qI, cons
   DSA_CUDA(launch_topk(scores, L.ld, T, nullptr, tm.pos, K, idx, at<void>(ws, L.topk), hist != nullptr, err, st));
   // the query may still be in flight on another stream: attention is the first step that reads it
   if (q_ready) DSA_CUDA(cudaStreamWaitEvent(st, (cudaEvent_t)q_ready, 0));
-  DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/true, reinterpret_cast<const __nv_bfloat16*>(q),
-                             reinterpret_cast<const __nv_bfloat16*>(kv), idx, K, H, scale,
+  DSA_CUDA(launch_sparse_mla(sd, tm, /*tm_early=*/true, reinterpret_cast<const __nv_bfloat16*>(q), kv,
+                             static_cast<const uint8_t*>(kv_scale), idx, K, H, scale,
                              out, out_dtype == DSA_OUT_F32, lse, at<void>(ws, L.partials), err, st));
   return DSA_OK;
 }
@@ -341,8 +359,8 @@ dsa_status_t dsa_index_topk_attn(const dsa_seqs_t* seqs, const void* qI, const f
                                  const void* kI_scale, dsa_ki_dtype_t ki_dtype, const void* q, const void* kv, int K,
                                  int H, float scale, void* out, dsa_out_dtype_t out_dtype, float* lse,
                                  int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
-  return dsa_index_topk_attn_ex(seqs, qI, w, kI, kI_scale, ki_dtype, q, kv, K, H, scale, out, out_dtype, lse, idx_out,
-                                ws, ws_bytes, 0u, nullptr, stream);
+  return dsa_index_topk_attn_ex(seqs, qI, w, kI, kI_scale, ki_dtype, q, kv, nullptr, DSA_KV_BF16, K, H, scale, out,
+                                out_dtype, lse, idx_out, ws, ws_bytes, 0u, nullptr, stream);
 }
 
 dsa_status_t dsa_check_error(void* ws, dsa_stream_t stream) {

@@ -215,9 +215,10 @@ uint32_t* topk_hist_in_scratch(void* scratch, int T);
 cudaError_t launch_topk(const float* scores, int64_t ld, int T, const int32_t* row_len, const int32_t* tok_pos,
                         int K, int32_t* idx, void* scratch, bool hist_ready, uint32_t* err, cudaStream_t st);
 size_t sparse_mla_partials_bytes(int T, int K, int H);
-cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, const __nv_bfloat16* q,
-                              const __nv_bfloat16* kv,
-                              const int32_t* idx, int K, int H, float scale, void* out, bool out_f32,
-                              float* lse, void* partials, uint32_t* err, cudaStream_t st);
+// kv: the bf16 pool, or (kv8_scale non-null) the FP8 cache's E4M3 codes with
+// their tile-scale bytes [rows, 8].
+cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, const __nv_bfloat16* q, const void* kv,
+                              const uint8_t* kv8_scale, const int32_t* idx, int K, int H, float scale, void* out,
+                              bool out_f32, float* lse, void* partials, uint32_t* err, cudaStream_t st);
 
 }  // namespace dsa

@@ -44,7 +44,18 @@
 //     leave through shared memory with one bulk copy per head row.
 // Decode batches split the index list over several CTAs per (token, head
 // group); k_combine merges their partials (log-sum-exp weights).
+//
+// FP8 latent KV cache ([P2] section 5 table, "Main attention KV cache": FP8,
+// per token-head tile of 128): rows of 576 E4M3 codes with one power-of-two
+// scale per 128-element tile (the last tile, the rope dims, of 64).  The
+// loaders then read each row's codes (8 bytes per piece, all of a block's
+// loads issued before any is used) and its scale bytes, convert to bf16 --
+// exactly: an E4M3 value times a power of two has at most 4 significant bits --
+// and store the same 16-byte pieces the bf16 gather would have copied; the
+// MMAs, softmax and epilogue are the bf16 path's.
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "sm100.cuh"
 
@@ -114,6 +125,35 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   return y;
 }
 
+// 8 bytes from global memory through the read-only path.
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+// 2^(byte - 127) for a tile-scale byte, exact (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float tile_scale(uint32_t byte) {
+  return byte == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(byte << 23);
+}
+
+// Eight E4M3 codes (little-endian: element k in byte k) times a power-of-two
+// scale, as eight bf16 (element 2i in the low half of word i).  Exact: an
+// E4M3 value is an fp16 value, and times 2^e it has at most 4 significant bits.
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 codes, float sc) {
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w = i < 2 ? codes.x : codes.y;
+    const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w >> (16 * (i & 1))) & 0xFFFFu);
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+    o[i] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 __device__ __forceinline__ void store_out(void* out, bool f32, int64_t i, float v) {
   if (f32)
     reinterpret_cast<float*>(out)[i] = v;
@@ -135,6 +175,8 @@ struct AttnArgs {
   SeqsDev s;
   TokenMap tm;
   const __nv_bfloat16* kv;  // latent pool [rows, 576]
+  const uint8_t* kv8;       // FP8 cache: E4M3 codes [rows, 576] (kv unused)
+  const uint8_t* kv8_scale; // FP8 cache: per row 8 bytes, byte j = exponent + 127 of tile j (0..4)
   const int32_t* idx;
   int K, H, G, ks, splits;  // G head groups of 64; ks selected slots per split
   bool tm_early;            // the token map was written two or more launches back
@@ -172,7 +214,7 @@ __device__ __forceinline__ void query_to_tmem(const uint8_t* qs, bool valid, int
   }
 }
 
-template <int BK, int NS>
+template <int BK, int NS, bool kKv8>
 __global__ void __launch_bounds__(kThreads, 1)
 k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
   using C = AttnCfg<BK, NS>;
@@ -308,7 +350,40 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
       bool ok = mbar_wait(&kv_empty[stage], ((j / kStages) & 1) ^ 1, a.err, a.wait_ns);
       // the last stage first holds the query tile
       if (j == NS - 1) ok = ok && mbar_wait(q_full, 0, a.err, a.wait_ns);
-      if (ok) {
+      if (ok && kKv8) {
+        // FP8 cache: this thread's pieces of the block (4 rows x 9 atoms of 8
+        // codes) are all loaded before any is converted, so their latencies overlap
+        static_assert(BK / 4 == 16, "four row quads per loader warp");
+        uint2 raw[4][kNAtoms], scl[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = 4 * (lw + 4 * u) + rsub;
+          const int row = ring_rows[j * kBK + r];
+          if (row >= 0) {
+            const uint8_t* src = a.kv8 + (int64_t)row * kDQK + 8 * piece;
+#pragma unroll
+            for (int at = 0; at < kNAtoms; ++at) raw[u][at] = ld_nc_v2(src + 64 * at);
+            scl[u] = ld_nc_v2(a.kv8_scale + (int64_t)row * 8);
+          } else {  // masked row: zeros, as the bf16 gather's zero fill
+#pragma unroll
+            for (int at = 0; at < kNAtoms; ++at) raw[u][at] = make_uint2(0u, 0u);
+            scl[u] = make_uint2(0x7F7F7F7Fu, 0x7Fu);
+          }
+        }
+        uint8_t* dst0 = smem + OFF_KV + stage * kStageBytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = 4 * (lw + 4 * u) + rsub;
+          uint8_t* drow = dst0 + r * 128 + ((((uint32_t)piece) ^ ((uint32_t)r & 7u)) << 4);
+#pragma unroll
+          for (int at = 0; at < kNAtoms; ++at) {
+            const int tile = at >> 1;  // atom at holds dims 64 at .. 64 at + 63
+            const uint32_t byte = (tile < 4 ? (scl[u].x >> (8 * tile)) : scl[u].y) & 0xFFu;
+            *reinterpret_cast<uint4*>(drow + at * kAtom) = e4m3x8_to_bf16x8(raw[u][at], tile_scale(byte));
+          }
+        }
+        fence_proxy_async_smem();  // the MMAs read these stores through the async proxy
+      } else if (ok) {
         // one row per (warp, quad): its pool row is looked up once, then the
         // nine 128-byte pieces (one per atom) go out back to back; a warp's
         // 32 copies of one atom fill 512 contiguous bytes (no bank conflict)
@@ -324,7 +399,10 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
           for (int at = 0; at < kNAtoms; ++at) cp_async_16_zfill(dst + at * kAtom, src + 128 * at, v ? 16u : 0u);
         }
       }
-      cp_async_mbar_arrive(&kv_full[stage]);     // counts once this thread's copies land
+      if constexpr (kKv8)
+        mbar_arrive(&kv_full[stage]);            // the stores above are done
+      else
+        cp_async_mbar_arrive(&kv_full[stage]);   // counts once this thread's copies land
       if (li == 0) mbar_arrive(&kv_full[stage]);  // releases the masks read by the softmax warps
       failed = bar_red_or(kLoaderBarrier, kLoaders, !ok || *abort_flag != 0);
       if (failed) *abort_flag = 1;
@@ -696,20 +774,20 @@ int keys_per_split(int K, int splits, int bk) {
   return (ks + bk - 1) / bk * bk;
 }
 
-template <int BK, int NS>
+template <int BK, int NS, bool kKv8>
 cudaError_t launch_attn(const CUtensorMap& tq, const AttnArgs& a, int64_t ctas, cudaStream_t st) {
   using C = AttnCfg<BK, NS>;
   static thread_local int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_sparse_mla_tc<BK, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(k_sparse_mla_tc<BK, NS, kKv8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  return launch_pdl("sparse_mla", k_sparse_mla_tc<BK, NS>, dim3((unsigned)ctas), dim3(kThreads), (size_t)C::SMEM, st,
-                    tq, a);
+  return launch_pdl("sparse_mla", k_sparse_mla_tc<BK, NS, kKv8>, dim3((unsigned)ctas), dim3(kThreads),
+                    (size_t)C::SMEM, st, tq, a);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -745,8 +823,8 @@ size_t sparse_mla_partials_bytes(int T, int K, int H) {
   return (size_t)T * splits * H * (kDV * sizeof(float) + sizeof(float2));
 }
 
-cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, const __nv_bfloat16* q,
-                              const __nv_bfloat16* kv, const int32_t* idx, int K, int H, float scale, void* out,
+cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, const __nv_bfloat16* q, const void* kv,
+                              const uint8_t* kv8_scale, const int32_t* idx, int K, int H, float scale, void* out,
                               bool out_f32, float* lse, void* partials, uint32_t* err, cudaStream_t st) {
   const int T = s.num_tokens;
   const int G = head_groups(H);
@@ -757,11 +835,18 @@ cudaError_t launch_sparse_mla(const SeqsDev& s, TokenMap tm, bool tm_early, cons
   float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)T * splits * H * kDV);
   CUtensorMap tq;
   if (!make_map_576(&tq, q, (uint64_t)T * H)) return cudaErrorInvalidValue;
-  AttnArgs a{s, tm, kv, idx, K, H, G, ks, splits, tm_early, scale * kLog2e, out, out_f32, lse, part_o, part_ml,
-             err, wait_limit_ns()};
+  const bool kv8 = kv8_scale != nullptr;
+  AttnArgs a{s,
+             tm,
+             kv8 ? nullptr : static_cast<const __nv_bfloat16*>(kv),
+             kv8 ? static_cast<const uint8_t*>(kv) : nullptr,
+             kv8_scale,
+             idx,
+             K, H, G, ks, splits, tm_early, scale * kLog2e, out, out_f32, lse, part_o, part_ml, err, wait_limit_ns()};
   const int64_t ctas = (int64_t)T * G * splits;
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
-  cudaError_t e = launch_attn<Cfg::BK, Cfg::NS>(tq, a, ctas, st);
+  cudaError_t e = kv8 ? launch_attn<Cfg::BK, Cfg::NS, true>(tq, a, ctas, st)
+                      : launch_attn<Cfg::BK, Cfg::NS, false>(tq, a, ctas, st);
   if (e == cudaSuccess) e = counted(cudaGetLastError());
   if (e != cudaSuccess || splits == 1) return e;
   e = launch_pdl("sparse_mla_combine", k_combine, dim3(T, H), dim3(128), 0, st, H, splits, (const float*)part_o,

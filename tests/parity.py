@@ -39,6 +39,14 @@ def kI_host(wl: Workload):
     return wl.kI.numpy(), wl.kI_scale.numpy()
 
 
+def kv_host(wl: Workload):
+    """The latent pool as the oracle takes it: bf16 bit patterns, or the FP8
+    cache's (codes, scale bytes)."""
+    if wl.kv_scale is None:
+        return bits16(wl.kv)
+    return wl.kv.numpy(), wl.kv_scale.numpy()
+
+
 def oracle_scores(wl: Workload, tokens=None):
     kI, sc = kI_host(wl)
     return O.index_scores(oracle_seqs(wl), bits16(wl.qI), wl.w.numpy(), kI, sc, tokens=tokens)

@@ -18,7 +18,8 @@ def _fused_check(lib, wl, tokens, min_agree=0.9, out_dtype=torch.bfloat16, selec
     K = wl.spec.topk
     idx_out = torch.empty((wl.T, K), dtype=torch.int32, device="cuda")
     out, lse = lib.dsa_index_topk_attn(d.seqs, d.qI, d.w, d.kI, d.kI_scale, d.q, d.kv, K, wl.scale,
-                                       idx_out=idx_out, out_dtype=out_dtype, select_in_indexer=select_in_indexer)
+                                       idx_out=idx_out, out_dtype=out_dtype, select_in_indexer=select_in_indexer,
+                                       kv_scale=d.kv_scale)
     assert lib.dsa_check_error(lib.workspace(0, "cuda", "index_topk_attn")) == lib.DSA_OK
     gidx = idx_out.cpu().numpy()
     ref_rows = P.oracle_scores(wl, tokens)
@@ -32,7 +33,7 @@ def _fused_check(lib, wl, tokens, min_agree=0.9, out_dtype=torch.bfloat16, selec
             agree.append(t)
     assert len(agree) >= min_agree * len(tokens), f"{len(agree)}/{len(tokens)} rows with identical sets"
     ref_idx = P.topk_idx_for(wl, [ref_rows[list(tokens).index(t)] for t in agree], agree)
-    ref_out, ref_lse = O.sparse_mla(P.oracle_seqs(wl), bits16(wl.q), bits16(wl.kv), ref_idx, wl.scale,
+    ref_out, ref_lse = O.sparse_mla(P.oracle_seqs(wl), bits16(wl.q), P.kv_host(wl), ref_idx, wl.scale,
                                     tokens=agree)
     sel = torch.from_numpy(np.asarray(agree)).cuda()
     P.assert_attention_close(out[sel], lse[sel], ref_out, ref_lse)

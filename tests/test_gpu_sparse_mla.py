@@ -14,11 +14,11 @@ pytestmark = pytest.mark.gpu
 def _check(lib, wl, idx_np, tokens):
     d = to_device(wl)
     idx = torch.from_numpy(idx_np).cuda()
-    ref_out, ref_lse = O.sparse_mla(P.oracle_seqs(wl), bits16(wl.q), bits16(wl.kv), idx_np, wl.scale,
+    ref_out, ref_lse = O.sparse_mla(P.oracle_seqs(wl), bits16(wl.q), P.kv_host(wl), idx_np, wl.scale,
                                     tokens=tokens)
     sel = torch.from_numpy(np.asarray(tokens)).cuda()
     for dt in (torch.float32, torch.bfloat16):
-        out, lse = lib.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out_dtype=dt)
+        out, lse = lib.dsa_sparse_mla_fwd(d.seqs, d.q, d.kv, idx, wl.scale, out_dtype=dt, kv_scale=d.kv_scale)
         P.assert_attention_close(out[sel], lse[sel], ref_out, ref_lse)
     assert lib.dsa_check_error(lib.workspace(0, "cuda", "sparse_mla")) == lib.DSA_OK
 

@@ -35,7 +35,8 @@ def _inputs(spec):
     seqs = dsa.Seqs(*(_aligned(torch.from_numpy(x)) for x in (wl.q_seq_start, wl.ctx_len, wl.page_table)),
                     wl.num_phys_pages, int(wl.ctx_len.max()), wl.T)
     ks = None if wl.kI_scale is None else _aligned(wl.kI_scale)
-    return wl, seqs, _aligned(wl.qI), _aligned(wl.w), _aligned(wl.kI), ks, _aligned(wl.q), _aligned(wl.kv)
+    vs = None if wl.kv_scale is None else _aligned(wl.kv_scale)
+    return wl, seqs, _aligned(wl.qI), _aligned(wl.w), _aligned(wl.kI), ks, _aligned(wl.q), _aligned(wl.kv), vs
 
 
 SPECS = {
@@ -44,12 +45,13 @@ SPECS = {
     "mx_prefill": CONFIGS["long_prefill_32k"].scaled(ctx=(2048, 2048), ki_mx=True),
     "fp8_decode": CONFIGS["decode_b64_8k_32k"].scaled(batch=3),
     "mx_decode": CONFIGS["decode_b64_8k_32k"].scaled(batch=3, ki_mx=True),
+    "kv8_decode": CONFIGS["decode_b64_8k_32k"].scaled(batch=3, kv_fp8=True),
 }
 
 
 @pytest.mark.parametrize("name", list(SPECS))
 def test_entry_points_return_without_a_gpu(host_binding, name):
-    wl, seqs, qI, w, kI, ks, q, kv = _inputs(SPECS[name])
+    wl, seqs, qI, w, kI, ks, q, kv, vs = _inputs(SPECS[name])
     K = wl.spec.topk
     scores = _aligned(torch.zeros((wl.T, (wl.max_ctx + 3) // 4 * 4), dtype=torch.float32))
     out = _aligned(torch.zeros((wl.T, wl.spec.heads, 512), dtype=torch.bfloat16))
@@ -57,10 +59,10 @@ def test_entry_points_return_without_a_gpu(host_binding, name):
     idx = _aligned(torch.zeros((wl.T, K), dtype=torch.int32))
     calls = [
         lambda: dsa.dsa_index_scores(seqs, qI, w, kI, ks, scores=scores),
-        lambda: dsa.dsa_sparse_mla_fwd(seqs, q, kv, idx, wl.scale, out=out, lse=lse),
-        lambda: dsa.dsa_index_topk_attn(seqs, qI, w, kI, ks, q, kv, K, wl.scale, out=out, lse=lse),
+        lambda: dsa.dsa_sparse_mla_fwd(seqs, q, kv, idx, wl.scale, out=out, lse=lse, kv_scale=vs),
+        lambda: dsa.dsa_index_topk_attn(seqs, qI, w, kI, ks, q, kv, K, wl.scale, out=out, lse=lse, kv_scale=vs),
         lambda: dsa.dsa_index_topk_attn(seqs, qI, w, kI, ks, q, kv, K, wl.scale, out=out, lse=lse,
-                                        select_in_indexer=True),
+                                        select_in_indexer=True, kv_scale=vs),
     ]
     for call in calls:
         with pytest.raises(dsa.DsaError, match="DSA_ERR_CUDA"):

@@ -61,3 +61,23 @@ def test_mx_cache_rows_are_mxfp8_encodings():
     assert np.array_equal(c2, codes) and np.array_equal(s2, sc)
     used = np.abs(O.mxfp8_dequantize(codes, sc)).reshape(-1, 4, 32).max(-1) > 0
     assert used.mean() > 0.5
+
+
+def test_fp8_kv_cache_rows_follow_the_tile_scale_rule():
+    """Each tile of the FP8 latent cache is stored with the tightest
+    power-of-two scale: its largest code magnitude lies in [224, 448] (amax in
+    (224, 448] x 2^e before rounding); zero tiles carry scale byte 127, the
+    padding bytes are zero, unused pool rows decode to zero."""
+    from oracle import dsa_oracle as O
+    spec = CONFIGS["decode_b64_8k_32k"].scaled(batch=2, ctx=(300, 700), kv_fp8=True, planted=8)
+    wl = make_workload(spec)
+    codes, sc = wl.kv.numpy(), wl.kv_scale.numpy()
+    assert codes.dtype == np.uint8 and sc.shape == (codes.shape[0], 8) and np.all(sc[:, 5:] == 0)
+    mag = np.abs(O.e4m3_decode_fast(codes))
+    for j, (lo, hi) in enumerate([(0, 128), (128, 256), (256, 384), (384, 512), (512, 576)]):
+        top = mag[:, lo:hi].max(axis=1)
+        nz = top > 0
+        assert np.all((top[nz] >= 224.0) & (top[nz] <= 448.0))
+        assert np.all(sc[~nz, j] == 127)
+    used = np.abs(O.kv_fp8_dequantize(codes, sc)).max(axis=1) > 0
+    assert 0.5 < used.mean() <= 1.0
