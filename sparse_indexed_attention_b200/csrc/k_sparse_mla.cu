@@ -344,6 +344,32 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
     const int rsub = lane >> 3, piece = lane & 7;  // a warp copies 4 rows x 128 bytes of one atom at a time
     constexpr int kQuads = BK / 4;  // row quads per block
     bool failed = bar_red_or(kLoaderBarrier, kLoaders, false);
+    // FP8 cache: this thread's pieces of a block (4 rows x 9 atoms of 8 codes)
+    // and its rows' scale words, loaded one block ahead: the next block's loads
+    // are issued as soon as this block's pieces are stored, so their latency
+    // overlaps the wait for the next free stage
+    static_assert(!kKv8 || BK / 4 == 16, "four row quads per loader warp");
+    uint2 raw[4][kNAtoms], scl[4];
+    auto load_block = [&](int jb) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = 4 * (lw + 4 * u) + rsub;
+        const int row = ring_rows[jb * kBK + r];
+        if (row >= 0) {
+          const uint8_t* src = a.kv8 + (int64_t)row * kDQK + 8 * piece;
+#pragma unroll
+          for (int at = 0; at < kNAtoms; ++at) raw[u][at] = ld_nc_v2(src + 64 * at);
+          scl[u] = ld_nc_v2(a.kv8_scale + (int64_t)row * 8);
+        } else {  // masked row: zeros, as the bf16 gather's zero fill
+#pragma unroll
+          for (int at = 0; at < kNAtoms; ++at) raw[u][at] = make_uint2(0u, 0u);
+          scl[u] = make_uint2(0x7F7F7F7Fu, 0x7Fu);
+        }
+      }
+    };
+    if constexpr (kKv8) {
+      if (!failed) load_block(0);
+    }
     for (int j = 0; j < nblk && !failed; ++j) {
       const int stage = j % kStages;
       // the PV of the stage's previous block has completed
@@ -351,25 +377,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
       // the last stage first holds the query tile
       if (j == NS - 1) ok = ok && mbar_wait(q_full, 0, a.err, a.wait_ns);
       if (ok && kKv8) {
-        // FP8 cache: this thread's pieces of the block (4 rows x 9 atoms of 8
-        // codes) are all loaded before any is converted, so their latencies overlap
-        static_assert(BK / 4 == 16, "four row quads per loader warp");
-        uint2 raw[4][kNAtoms], scl[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int r = 4 * (lw + 4 * u) + rsub;
-          const int row = ring_rows[j * kBK + r];
-          if (row >= 0) {
-            const uint8_t* src = a.kv8 + (int64_t)row * kDQK + 8 * piece;
-#pragma unroll
-            for (int at = 0; at < kNAtoms; ++at) raw[u][at] = ld_nc_v2(src + 64 * at);
-            scl[u] = ld_nc_v2(a.kv8_scale + (int64_t)row * 8);
-          } else {  // masked row: zeros, as the bf16 gather's zero fill
-#pragma unroll
-            for (int at = 0; at < kNAtoms; ++at) raw[u][at] = make_uint2(0u, 0u);
-            scl[u] = make_uint2(0x7F7F7F7Fu, 0x7Fu);
-          }
-        }
+        // FP8 cache: convert the block loaded ahead and store its pieces
         uint8_t* dst0 = smem + OFF_KV + stage * kStageBytes;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -383,6 +391,7 @@ k_sparse_mla_tc(const __grid_constant__ CUtensorMap tq, const AttnArgs a) {
           }
         }
         fence_proxy_async_smem();  // the MMAs read these stores through the async proxy
+        if (j + 1 < nblk) load_block(j + 1);
       } else if (ok) {
         // one row per (warp, quad): its pool row is looked up once, then the
         // nine 128-byte pieces (one per atom) go out back to back; a warp's
