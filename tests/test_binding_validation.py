@@ -76,3 +76,22 @@ def test_index_cache_format_follows_the_scale_dtype(monkeypatch):
         dsa._need_index_inputs(seqs, qI, w, kI, torch.full((64, 2), 127, dtype=torch.uint8))
     with pytest.raises(ValueError, match="at least 64"):
         dsa._need_index_inputs(seqs, qI, w, kI, torch.full((63, 4), 127, dtype=torch.uint8))
+
+
+def test_latent_cache_format_follows_kv_scale(monkeypatch):
+    """kv_scale absent: a bf16 pool [R, 576]; present: E4M3 codes [R, 576] with
+    uint8 scale bytes [R, 8], each checked for shape and pool size."""
+    monkeypatch.setattr(dsa, "_cuda_device", lambda t, name: t.device)
+    seqs = dsa.Seqs(torch.tensor([0, 1], dtype=torch.int32), torch.tensor([5], dtype=torch.int32),
+                    torch.zeros(1, 1, dtype=torch.int32), 1, 5, 1)
+    q = torch.zeros(1, 16, 576, dtype=torch.bfloat16)
+    out = torch.zeros(1, 16, 512, dtype=torch.bfloat16)
+    codes, scales = torch.zeros(64, 576, dtype=torch.uint8), torch.full((64, 8), 127, dtype=torch.uint8)
+    dsa._need_attn_inputs(seqs, q, torch.zeros(64, 576, dtype=torch.bfloat16), out, None)
+    dsa._need_attn_inputs(seqs, q, codes, out, None, scales)
+    with pytest.raises(TypeError, match="dtype"):
+        dsa._need_attn_inputs(seqs, q, codes, out, None)              # codes without their scales
+    with pytest.raises(ValueError, match="shape"):
+        dsa._need_attn_inputs(seqs, q, codes, out, None, scales[:, :5].contiguous())
+    with pytest.raises(ValueError, match="at least 64"):
+        dsa._need_attn_inputs(seqs, q, codes, out, None, scales[:63])
