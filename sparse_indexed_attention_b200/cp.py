@@ -9,7 +9,7 @@ position, so pairing an early segment with a late one gives every rank the
 same causal work.
 
 Each rank holds the index keys (FP8 codes + scales, or bf16) and latent rows
-of its own two segments, segment r first.  One all-gather per pool (NCCL over
+(bf16, or FP8 codes + tile-scale bytes) of its own two segments, segment r first.  One all-gather per pool (NCCL over
 NVLink, into each rank's own memory) gives every rank the pools of the whole
 sequence laid out rank by rank: rank q's rows sit at [2 seg q, 2 seg (q+1)).
 Nothing is copied back into sequence order: a page table maps the sequence's
@@ -95,20 +95,22 @@ def _all_gather(x: torch.Tensor, group) -> torch.Tensor:
     return out.view(R, *x.shape)
 
 
-def _fused_call(seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: float):
+def _fused_call(seqs, qI, w, kI, kI_scale, q, kv, K: int, scale: float, kv_scale=None):
     import sparse_indexed_attention_b200 as dsa
-    return dsa.dsa_index_topk_attn(seqs, qI, w, kI, kI_scale, q, kv, K, scale)
+    return dsa.dsa_index_topk_attn(seqs, qI, w, kI, kI_scale, q, kv, K, scale, kv_scale=kv_scale)
 
 
 def cp_prefill(plan: ZigzagPlan, group, qI, w, q, kI_local, kI_scale_local, kv_local, K: int, scale: float,
-               attend=None, gather_output: bool = True):
+               attend=None, gather_output: bool = True, kv_scale_local=None):
     """One zigzag-parallel prefill step on this rank.
 
     qI [2 seg, 64, 128], w [2 seg, 64], q [2 seg, H, 576]: this rank's query
-    tokens in local order; kI_local [2 seg, 128] (+ kI_scale_local [2 seg] or
-    None) and kv_local [2 seg, 576]: its rows of the pools, same order.
-    `attend(seqs, qI, w, kI, kI_scale, q, kv, K, scale) -> (out, lse)` runs the
-    hot path (default: dsa_index_topk_attn).  Returns (out, lse) of the whole
+    tokens in local order; kI_local [2 seg, 128] (+ kI_scale_local [2 seg],
+    [2 seg, 4] for MXFP8, or None) and kv_local [2 seg, 576] (+ kv_scale_local
+    [2 seg, 8] for the FP8 latent cache, or None): its rows of the pools, same
+    order.  `attend(seqs, qI, w, kI, kI_scale, q, kv, K, scale[, kv_scale=])`
+    -> (out, lse) runs the hot path (default: dsa_index_topk_attn; kv_scale is
+    passed only for the FP8 latent cache).  Returns (out, lse) of the whole
     sequence in order when gather_output, else this rank's rows (local order).
     """
     import torch.distributed as dist
@@ -123,12 +125,15 @@ def cp_prefill(plan: ZigzagPlan, group, qI, w, q, kI_local, kI_scale_local, kv_l
     kI = _all_gather(kI_local, group).reshape(plan.R * n, *kI_local.shape[1:])
     kI_scale = None
     if kI_scale_local is not None:
-        kI_scale = _all_gather(kI_scale_local, group).reshape(plan.R * n)
+        kI_scale = _all_gather(kI_scale_local, group).reshape(plan.R * n, *kI_scale_local.shape[1:])
     kv = _all_gather(kv_local, group).reshape(plan.R * n, *kv_local.shape[1:])
+    kv_extra = {}
+    if kv_scale_local is not None:
+        kv_extra["kv_scale"] = _all_gather(kv_scale_local, group).reshape(plan.R * n, *kv_scale_local.shape[1:])
     qs, cl, pt = plan.rank_batch(r)
     from sparse_indexed_attention_b200 import Seqs
     seqs = Seqs.from_host(qs, cl, pt, plan.T // PAGE, device=q.device)
-    out, lse = (attend or _fused_call)(seqs, qI, w, kI, kI_scale, q, kv, K, scale)
+    out, lse = (attend or _fused_call)(seqs, qI, w, kI, kI_scale, q, kv, K, scale, **kv_extra)
     if not gather_output:
         return out, lse
     return plan.restore(_all_gather(out, group)), plan.restore(_all_gather(lse, group))

@@ -53,18 +53,24 @@ def test_zigzag_plan_rejects_ragged_lengths():
         ZigzagPlan.make(512, 0)
 
 
-def _spec():
+def _spec(kv_fp8=False):
     from dsa_workloads import CONFIGS
-    return CONFIGS["long_prefill_32k"].scaled(name="cp_prefill_512", ctx=(512, 512), heads=16, topk=64)
+    return CONFIGS["long_prefill_32k"].scaled(name="cp_prefill_512", ctx=(512, 512), heads=16, topk=64,
+                                              kv_fp8=kv_fp8)
 
 
-def _oracle_attend(seqs, qI, w, kI, kI_scale, q, kv, K, scale):
+def _kv_arg(kv, kv_scale):
+    from dsa_workloads import bits16
+    return bits16(kv) if kv_scale is None else (kv.numpy(), kv_scale.numpy())
+
+
+def _oracle_attend(seqs, qI, w, kI, kI_scale, q, kv, K, scale, kv_scale=None):
     from dsa_workloads import bits16
     from oracle import dsa_oracle as O
     os_ = O.Seqs(seqs.ctx_len.numpy().astype(np.int64), seqs.q_seq_start.numpy().astype(np.int64),
                  seqs.page_table.numpy(), PAGE)
     _, _, out, lse = O.index_topk_attn(os_, bits16(qI), w.numpy(), kI.numpy(), kI_scale.numpy(), bits16(q),
-                                       bits16(kv), K, scale)
+                                       _kv_arg(kv, kv_scale), K, scale)
     return torch.from_numpy(out), torch.from_numpy(lse)
 
 
@@ -73,10 +79,11 @@ def _shard(wl, plan, r):
     rows = wl.page_table[0][pos // PAGE].astype(np.int64) * PAGE + pos % PAGE
     t = torch.from_numpy(pos)
     rw = torch.from_numpy(rows)
-    return wl.qI[t], wl.w[t], wl.q[t], wl.kI[rw], wl.kI_scale[rw], wl.kv[rw]
+    kvs = None if wl.kv_scale is None else wl.kv_scale[rw]
+    return wl.qI[t], wl.w[t], wl.q[t], wl.kI[rw], wl.kI_scale[rw], wl.kv[rw], kvs
 
 
-def _rank_main(rank, world, port, q):
+def _rank_main(rank, world, port, q, kv_fp8):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -85,10 +92,11 @@ def _rank_main(rank, world, port, q):
     from sparse_indexed_attention_b200.cp import ZigzagPlan, cp_prefill
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        wl = make_workload(_spec())
+        wl = make_workload(_spec(kv_fp8))
         plan = ZigzagPlan.make(wl.T, world)
-        qI, w, qq, kI, ks, kv = _shard(wl, plan, rank)
-        out, lse = cp_prefill(plan, None, qI, w, qq, kI, ks, kv, wl.spec.topk, wl.scale, attend=_oracle_attend)
+        qI, w, qq, kI, ks, kv, kvs = _shard(wl, plan, rank)
+        out, lse = cp_prefill(plan, None, qI, w, qq, kI, ks, kv, wl.spec.topk, wl.scale, attend=_oracle_attend,
+                              kv_scale_local=kvs)
         if rank == 0:
             q.put((out.numpy(), lse.numpy()))
     finally:
@@ -101,11 +109,12 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def test_two_gloo_ranks_zigzag_prefill_equals_one_rank():
+@pytest.mark.parametrize("kv_fp8", [False, True])
+def test_two_gloo_ranks_zigzag_prefill_equals_one_rank(kv_fp8):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q, kv_fp8)) for r in range(2)]
     for p in procs:
         p.start()
     got = None
@@ -125,9 +134,9 @@ def test_two_gloo_ranks_zigzag_prefill_equals_one_rank():
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     from dsa_workloads import bits16, make_workload
     from oracle import dsa_oracle as O
-    wl = make_workload(_spec())
+    wl = make_workload(_spec(kv_fp8))
     seqs = O.Seqs(wl.ctx_len.astype(np.int64), wl.q_seq_start.astype(np.int64), wl.page_table, PAGE)
     _, _, ref_out, ref_lse = O.index_topk_attn(seqs, bits16(wl.qI), wl.w.numpy(), wl.kI.numpy(),
-                                               wl.kI_scale.numpy(), bits16(wl.q), bits16(wl.kv), wl.spec.topk,
-                                               wl.scale)
+                                               wl.kI_scale.numpy(), bits16(wl.q), _kv_arg(wl.kv, wl.kv_scale),
+                                               wl.spec.topk, wl.scale)
     assert np.array_equal(out, ref_out) and np.array_equal(lse, ref_lse)
