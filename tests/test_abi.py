@@ -104,3 +104,52 @@ def test_host_validation_rejects_before_launch():
     # quantizer
     assert lib.dsa_quantize_index_query(good, good, 0, good, good, None) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_check_error(None, None) == dsa.DSA_ERR_WORKSPACE
+
+
+def test_host_validation_of_cache_formats_and_options():
+    """The index-cache and latent-cache formats, the flags and the MXFP8
+    quantizer are checked on the host, before any launch."""
+    lib = dsa.raw()
+    P = ctypes.c_void_p
+    good = P(0x10000)
+    s = _fake_seqs()
+    f = ctypes.c_float(0.04)
+    B16, MX, E4 = dsa.DSA_OUT_BF16, dsa.DSA_KI_MXFP8, dsa.DSA_KI_FP8_E4M3
+    KB, K8 = dsa.DSA_KV_BF16, dsa.DSA_KV_FP8_E4M3
+    # MXFP8 index cache: scales required; an unknown cache kind is unsupported
+    assert lib.dsa_index_scores(ctypes.byref(s), good, good, good, None, MX, good, 128, good, 1 << 20,
+                                None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_index_scores(ctypes.byref(s), good, good, good, good, 7, good, 128, good, 1 << 20,
+                                None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_index_scores(ctypes.byref(s), good, good, good, P(0x10008), MX, good, 128, good, 1 << 20,
+                                None) == dsa.DSA_ERR_INVALID_ARG               # scales not 16-B aligned
+
+    def attn_ex(kv_scale, kv_dtype, flags=0, kI_scale=good, ki=E4):
+        return lib.dsa_index_topk_attn_ex(ctypes.byref(s), good, good, good, kI_scale, ki, good, good, kv_scale,
+                                          kv_dtype, 16, 128, f, good, B16, None, None, good, 1 << 30, flags, None,
+                                          None)
+    assert attn_ex(None, K8) == dsa.DSA_ERR_INVALID_ARG                        # FP8 latent cache without scales
+    assert attn_ex(good, KB) == dsa.DSA_ERR_INVALID_ARG                        # bf16 pool with scales
+    assert attn_ex(None, 5) == dsa.DSA_ERR_UNSUPPORTED                         # unknown latent format
+    assert attn_ex(P(0x10008), K8) == dsa.DSA_ERR_INVALID_ARG                  # scales not 16-B aligned
+    assert attn_ex(None, KB, flags=2) == dsa.DSA_ERR_INVALID_ARG               # unknown flag
+    assert attn_ex(None, KB, kI_scale=None, ki=MX) == dsa.DSA_ERR_INVALID_ARG
+    # attention alone
+    assert lib.dsa_sparse_mla_fwd_ex(ctypes.byref(s), good, good, None, K8, good, 16, 128, f, good, B16, None,
+                                     good, 1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_sparse_mla_fwd_ex(ctypes.byref(s), good, good, good, 9, good, 16, 128, f, good, B16, None,
+                                     good, 1 << 20, None) == dsa.DSA_ERR_UNSUPPORTED
+    # MXFP8 quantizer
+    assert lib.dsa_quantize_index_query_mx(good, 0, good, good, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_quantize_index_query_mx(good, 4, good, P(0x10002), None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_in_indexer_selection_workspace_has_no_score_scratch():
+    """With the selection inside the indexer the decode workspace drops the
+    [T, ld] fp32 scores and Top-K's scratch (row histograms and candidate
+    lists take their place)."""
+    lib = dsa.raw()
+    s = _fake_seqs(T=8, B=8, max_ctx=131072, max_pages=2048, phys=32768)
+    plain = lib.dsa_workspace_size(dsa.DSA_OP_INDEX_TOPK_ATTN, ctypes.byref(s), 2048, 128)
+    fused = lib.dsa_workspace_size(dsa.DSA_OP_INDEX_TOPK_ATTN_FUSED, ctypes.byref(s), 2048, 128)
+    assert 0 < fused and plain - fused >= 8 * 131072 * 4
