@@ -39,8 +39,9 @@
  *   page_table[b*max_pages + s/64]*64 + s%64 of each pool (page size 64).
  *   Pools: index keys kI [R, 128] (bf16; FP8 E4M3 codes with one fp32 scale
  *   per row in kI_scale [R]; or MXFP8: E4M3 codes with one E8M0 scale byte
- *   per 32 elements in kI_scale [R, 4]) and latent KV [R, 576] bf16,
- *   R = num_phys_pages*64.
+ *   per 32 elements in kI_scale [R, 4]) and latent KV [R, 576] (bf16; or
+ *   E4M3 codes with five power-of-two tile-scale bytes per row in
+ *   kv_scale [R, 8], see dsa_kv_dtype_t), R = num_phys_pages*64.
  * Fixed sizes.  Index heads H_I = 64, index dim d_I = 128, latent dims
  *   576 (keys) / 512 (values), page size 64.  Attention heads H in {16, 32,
  *   64, 128}.  1 <= K <= 2048.  Anything else returns DSA_ERR_UNSUPPORTED.

@@ -66,7 +66,8 @@ import numpy as np
 def bf16_to_f64(bits) -> np.ndarray:
     """Exact value of bfloat16 bit patterns (the top half of an IEEE binary32)."""
     b = np.asarray(bits, dtype=np.uint16)
-    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # NaN patterns widen to NaN
+        return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
 
 
 def e4m3_decode(codes) -> np.ndarray:
