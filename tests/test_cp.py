@@ -53,10 +53,10 @@ def test_zigzag_plan_rejects_ragged_lengths():
         ZigzagPlan.make(512, 0)
 
 
-def _spec(kv_fp8=False):
+def _spec(kv_fp8=False, ki_mx=False):
     from dsa_workloads import CONFIGS
     return CONFIGS["long_prefill_32k"].scaled(name="cp_prefill_512", ctx=(512, 512), heads=16, topk=64,
-                                              kv_fp8=kv_fp8)
+                                              kv_fp8=kv_fp8, ki_mx=ki_mx)
 
 
 def _kv_arg(kv, kv_scale):
@@ -83,7 +83,7 @@ def _shard(wl, plan, r):
     return wl.qI[t], wl.w[t], wl.q[t], wl.kI[rw], wl.kI_scale[rw], wl.kv[rw], kvs
 
 
-def _rank_main(rank, world, port, q, kv_fp8):
+def _rank_main(rank, world, port, q, kv_fp8, ki_mx):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -92,7 +92,7 @@ def _rank_main(rank, world, port, q, kv_fp8):
     from sparse_indexed_attention_b200.cp import ZigzagPlan, cp_prefill
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        wl = make_workload(_spec(kv_fp8))
+        wl = make_workload(_spec(kv_fp8, ki_mx))
         plan = ZigzagPlan.make(wl.T, world)
         qI, w, qq, kI, ks, kv, kvs = _shard(wl, plan, rank)
         out, lse = cp_prefill(plan, None, qI, w, qq, kI, ks, kv, wl.spec.topk, wl.scale, attend=_oracle_attend,
@@ -109,12 +109,13 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("kv_fp8", [False, True])
-def test_two_gloo_ranks_zigzag_prefill_equals_one_rank(kv_fp8):
+@pytest.mark.parametrize("kv_fp8,ki_mx", [(False, False), (True, False), (False, True)],
+                         ids=["bf16_latent", "fp8_latent", "mxfp8_index"])
+def test_two_gloo_ranks_zigzag_prefill_equals_one_rank(kv_fp8, ki_mx):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q, kv_fp8)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q, kv_fp8, ki_mx)) for r in range(2)]
     for p in procs:
         p.start()
     got = None
@@ -134,7 +135,8 @@ def test_two_gloo_ranks_zigzag_prefill_equals_one_rank(kv_fp8):
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     from dsa_workloads import bits16, make_workload
     from oracle import dsa_oracle as O
-    wl = make_workload(_spec(kv_fp8))
+    wl = make_workload(_spec(kv_fp8, ki_mx))
+    assert (wl.kI_scale.dim() == 2) == ki_mx      # MXFP8: E8M0 bytes [R, 4]
     seqs = O.Seqs(wl.ctx_len.astype(np.int64), wl.q_seq_start.astype(np.int64), wl.page_table, PAGE)
     _, _, ref_out, ref_lse = O.index_topk_attn(seqs, bits16(wl.qI), wl.w.numpy(), wl.kI.numpy(),
                                                wl.kI_scale.numpy(), bits16(wl.q), _kv_arg(wl.kv, wl.kv_scale),
