@@ -57,13 +57,22 @@ def test_entry_points_return_without_a_gpu(host_binding, name):
     out = _aligned(torch.zeros((wl.T, wl.spec.heads, 512), dtype=torch.bfloat16))
     lse = _aligned(torch.zeros((wl.T, wl.spec.heads), dtype=torch.float32))
     idx = _aligned(torch.zeros((wl.T, K), dtype=torch.int32))
+    codes = _aligned(torch.zeros((wl.T, 64, 128), dtype=torch.float8_e4m3fn))
+    w_scaled = _aligned(torch.zeros((wl.T, 64), dtype=torch.float32))
+    q_sf = _aligned(torch.zeros((wl.T, 64, 4), dtype=torch.uint8))
+    row_len = _aligned(torch.full((wl.T,), scores.shape[1], dtype=torch.int32))
     calls = [
         lambda: dsa.dsa_index_scores(seqs, qI, w, kI, ks, scores=scores),
         lambda: dsa.dsa_sparse_mla_fwd(seqs, q, kv, idx, wl.scale, out=out, lse=lse, kv_scale=vs),
         lambda: dsa.dsa_index_topk_attn(seqs, qI, w, kI, ks, q, kv, K, wl.scale, out=out, lse=lse, kv_scale=vs),
         lambda: dsa.dsa_index_topk_attn(seqs, qI, w, kI, ks, q, kv, K, wl.scale, out=out, lse=lse,
                                         select_in_indexer=True, kv_scale=vs),
+        lambda: dsa.dsa_quantize_index_query(qI, w, codes=codes, w_scaled=w_scaled),
+        lambda: dsa.dsa_quantize_index_query_mx(qI, codes=codes, scales=q_sf),
+        lambda: dsa.dsa_topk(scores, row_len, K, idx=idx),
     ]
+    if vs is None:  # the allocation-free attention reads the bf16 latent pool only
+        calls.append(lambda: dsa.dsa_sparse_mla_fwd_noalloc(seqs, q, kv, idx, wl.scale, out=out, lse=lse))
     for call in calls:
         with pytest.raises(dsa.DsaError, match="DSA_ERR_CUDA"):
             call()
