@@ -7,7 +7,8 @@ raises.
 
 Functions carry the C names (``dsa_index_scores`` ...).  Outputs not passed in
 are allocated with torch on the inputs' device; workspaces are allocated
-zeroed and cached per (device, op, size), unless one is passed in.
+zeroed and cached per (device, op), unless one is passed in (concurrent
+calls on different streams pass their own).
 """
 from __future__ import annotations
 
@@ -39,12 +40,13 @@ DSA_OP_QUANTIZE_INDEX_QUERY, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_MLA
 DSA_SELECT_IN_INDEXER = 1
 
 # Names the C header declares (checked against include/dsa.h by the tests).
-EXPORTS = ("dsa_workspace_size", "dsa_quantize_index_query", "dsa_quantize_index_query_mx", "dsa_index_scores",
-           "dsa_topk",
-           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_ex", "dsa_sparse_mla_fwd_noalloc", "dsa_check_error_noalloc", "dsa_index_topk_attn",
-           "dsa_index_topk_attn_ex",
-           "dsa_check_error", "dsa_set_wait_limit_ns", "dsa_launches_in_last_call", "dsa_launch_timing",
-           "dsa_last_launch_times", "dsa_status_string")
+EXPORTS = ("dsa_workspace_size",
+           "dsa_quantize_index_query", "dsa_quantize_index_query_mx",
+           "dsa_index_scores", "dsa_topk",
+           "dsa_sparse_mla_fwd", "dsa_sparse_mla_fwd_ex", "dsa_sparse_mla_fwd_noalloc",
+           "dsa_index_topk_attn", "dsa_index_topk_attn_ex",
+           "dsa_check_error", "dsa_check_error_noalloc", "dsa_set_wait_limit_ns",
+           "dsa_launches_in_last_call", "dsa_launch_timing", "dsa_last_launch_times", "dsa_status_string")
 
 
 class DsaSeqsC(ctypes.Structure):
@@ -252,7 +254,12 @@ _ws_cache: dict = {}
 
 
 def workspace(nbytes: int, device, key=None) -> torch.Tensor:
-    """A zeroed device workspace of at least nbytes (cached by key)."""
+    """A zeroed device workspace of at least nbytes, cached per (device, key).
+
+    Every call that is not given `ws` uses this cached buffer, whatever its
+    stream.  Calls that may run at the same time on different streams must
+    each pass a workspace of their own: the library requires that concurrent
+    calls do not share one (its first word is the sticky error flag)."""
     device = torch.device(device)
     if device.type == "cuda" and device.index is None:
         device = torch.device("cuda", torch.cuda.current_device())
