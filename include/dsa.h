@@ -142,7 +142,8 @@ enum {
  *   num_q_tokens   T = q_seq_start[B] >= 1 (host copy of the last entry)
  *   page_size      must be 64
  *   max_pages      columns of page_table, >= ceil(max_ctx / 64)
- *   num_phys_pages pages in each pool (R = 64 * num_phys_pages rows)
+ *   num_phys_pages pages in each pool (R = 64 * num_phys_pages rows);
+ *                  R above 2^31 - 1 returns DSA_ERR_UNSUPPORTED
  *   max_ctx        host-known upper bound of ctx_len[b]; sizes grids and
  *                  workspace.  A ctx_len above it is a device error.
  *   q_seq_start    int32 [B+1], non-decreasing, q_seq_start[0] = 0

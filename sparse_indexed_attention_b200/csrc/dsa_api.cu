@@ -94,7 +94,8 @@ dsa_status_t check_seqs(const dsa_seqs_t* s) {
     return DSA_ERR_INVALID_ARG;
   if (s->page_size != kPage) return DSA_ERR_UNSUPPORTED;
   if ((int64_t)s->max_pages * kPage < (int64_t)s->max_ctx) return DSA_ERR_INVALID_ARG;
-  if ((int64_t)s->num_phys_pages * kPage > (int64_t)INT32_MAX * kPage) return DSA_ERR_UNSUPPORTED;
+  // pool rows are 32-bit in the kernels (TMA coordinates, gathered row ids)
+  if ((int64_t)s->num_phys_pages * kPage > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
 }
 

@@ -84,6 +84,11 @@ def test_host_validation_rejects_before_launch():
     bad_ps = _fake_seqs(page_size=32)
     assert lib.dsa_sparse_mla_fwd(ctypes.byref(bad_ps), good, good, good, 16, 128, f, good, B16, None, good,
                                   1 << 20, None) == dsa.DSA_ERR_UNSUPPORTED
+    for phys, want in (((1 << 25) - 1, dsa.DSA_OK), (1 << 25, dsa.DSA_ERR_UNSUPPORTED)):  # 2^31 pool rows
+        big = _fake_seqs(phys=phys)
+        got = lib.dsa_sparse_mla_fwd(ctypes.byref(big), good, good, good, 16, 128, f, good, B16, None, good, 16,
+                                     None)
+        assert got == (dsa.DSA_ERR_WORKSPACE if want == dsa.DSA_OK else want)  # past the pool check: workspace
     small_pt = _fake_seqs(max_ctx=200, max_pages=2)
     assert lib.dsa_sparse_mla_fwd(ctypes.byref(small_pt), good, good, good, 16, 128, f, good, B16, None, good,
                                   1 << 20, None) == dsa.DSA_ERR_INVALID_ARG
