@@ -4,7 +4,7 @@
 A step is one dsa_index_topk_attn call (indexer -> Top-K -> sparse MLA) over
 one batch of the long-context decode workload (8 sequences x 131072 cached
 tokens, one query token each, K = 2048, 128 heads, FP8 paged index cache in a
-2 Mi-token pool).  Inputs are synthetic and seeded (workloads.py).
+2 Mi-token pool).  Inputs are synthetic and seeded (dsa_workloads.py).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,30 +36,53 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
-# DRAM bytes (read + write) per launch from one ncu capture on this workload,
-# valid only while the kernel's sources hash to what was captured: any edit
-# turns the figure back into null.  (Re-keyed after the FP8 latent cache was
-# added: that change left the captured kernels -- the indexer, k_topk_filter
-# and the bf16 instantiation of the attention kernel -- as they were.)
-NCU_TRAFFIC = {
-    "index_scores": (145.60e6, ("k_indexer.cu",), "e0e0692b453fdc25"),
-    "topk_filter": (4.35e6, ("k_topk.cu",), "e4402930e3a60776"),
-    "sparse_mla": (20.25e6, ("k_sparse_mla.cu",), "ddd016a86f793cee"),
-}
+# DRAM bytes (read + write) per launch from ncu captures of the 128K decode
+# workload, each valid only for the cache formats it was captured with and
+# while the kernel's sources hash to what was captured: any edit turns the
+# figure back into null.
+NCU_CAPTURES = (
+    # kernel, config keys that must match, bytes per launch, sources, digest
+    ("index_scores", {"index_cache": "fp8_e4m3"}, 145.60e6, ("k_indexer.cu",), "e0e0692b453fdc25"),
+    ("index_scores", {"index_cache": "mxfp8"}, 144.81e6, ("k_indexer.cu",), "e0e0692b453fdc25"),
+    ("topk_filter", {}, 4.35e6, ("k_topk.cu",), "e4402930e3a60776"),
+    ("sparse_mla", {"latent_cache": "bf16"}, 20.25e6, ("k_sparse_mla.cu",), "ddd016a86f793cee"),
+)
+NCU_WORKLOAD = {"workload": "decode_b8_128k", "ctx": 131072}
 CSRC = os.path.join(ROOT, "sparse_indexed_attention_b200", "csrc")
 
 
-def ncu_traffic(kernel: str, config: str):
-    """Captured DRAM traffic of `kernel` per launch, or None if stale / not captured."""
-    if config != "decode_b8_128k" or kernel not in NCU_TRAFFIC:
-        return None
+def source_digest(files) -> str:
     import hashlib
-    nbytes, files, digest = NCU_TRAFFIC[kernel]
     m = hashlib.sha256()
     for f in (*files, "dsa_internal.cuh", "sm100.cuh"):
         with open(os.path.join(CSRC, f), "rb") as fh:
             m.update(fh.read())
-    return nbytes if m.hexdigest()[:16] == digest else None
+    return m.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, config: dict):
+    """Captured DRAM traffic of `kernel` per launch for this `config` (the JSON
+    line's config object), or None if not captured for it or stale."""
+    for name, keys, nbytes, files, digest in NCU_CAPTURES:
+        want = {**NCU_WORKLOAD, **keys}
+        if name == kernel and all(config.get(k) == v for k, v in want.items()):
+            return nbytes if source_digest(files) == digest else None
+    return None
+
+
+def index_cache(spec) -> str:
+    """The index cache's format; MXFP8 overrides the per-row E4M3 flag."""
+    return "mxfp8" if spec.ki_mx else ("fp8_e4m3" if spec.ki_fp8 else "bf16")
+
+
+def data_desc(spec) -> str:
+    return "synthetic (seeded" + (f", {spec.planted} planted keys per sequence)" if spec.planted else ")")
+
+
+def index_row_bytes(spec) -> int:
+    """Index-cache bytes per key: 128 codes + 4 scale bytes (one fp32, or four
+    E8M0 bytes), or 128 bf16 values."""
+    return 256 if index_cache(spec) == "bf16" else 132
 
 
 def parse():
@@ -252,7 +275,7 @@ def workload_config(spec, wl, world: int) -> dict:
     return {"workload": spec.name, "batch_per_gpu": spec.batch, "global_batch": wl.T * world,
             "ctx": int(wl.ctx_len[0]), "topk": spec.topk, "heads": spec.heads, "index_heads": spec.index_heads,
             "index_dim": spec.index_dim, "page_size": spec.page_size, "pool_tokens": wl.num_phys_pages * 64,
-            "index_cache": "mxfp8" if spec.ki_mx else ("fp8_e4m3" if spec.ki_fp8 else "bf16"),
+            "index_cache": index_cache(spec),
             "latent_cache": "fp8_e4m3_tile128" if spec.kv_fp8 else "bf16",
             "parallelism": f"dp{world}",
             "l2": "256 MiB buffer written before every timed GPU step"}
@@ -289,7 +312,7 @@ def run_reference(args, world, rank):
               f"(ctx {int(wl.ctx_len[0])}) per step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": data_desc(spec),
             "config": workload_config(spec, wl, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
@@ -336,7 +359,7 @@ def kernel_times(dsa, step, steps, stream, flush):
     return per
 
 
-def roofline_entry(name, per, algorithmic_bytes, peak, peak_kind, config):
+def roofline_entry(name, per, algorithmic_bytes, peak, peak_kind, config: dict):
     ms = statistics.mean(per[name])
     achieved = algorithmic_bytes / (ms / 1e3) / 1e9
     return {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -408,15 +431,16 @@ def run_all_configs(args, dsa, dev, stream, flush):
         if "index_scores" in us:
             t_s = us["index_scores"] * 1e-6
             if decode:
-                b = pairs * (132 if spec.ki_fp8 else 256)
+                b = pairs * index_row_bytes(spec)
                 stages["index_scores"] = {"bound": "hbm", "us": us["index_scores"], "achieved": b / t_s / 1e9,
                                           "peak": hbm, "unit": "GB/s", "frac": b / t_s / 1e9 / hbm}
             else:
-                pk, src = tensor_peak("fp8" if spec.ki_fp8 else "bf16")
+                eight_bit = index_cache(spec) != "bf16"
+                pk, src = tensor_peak("fp8" if eight_bit else "bf16")
                 f = pairs * 16384
                 stages["index_scores"] = {"bound": "tensor", "us": us["index_scores"], "achieved": f / t_s / 1e12,
                                           "peak": pk, "unit": "TFLOP/s", "frac": f / t_s / 1e12 / pk,
-                                          "dtype": "fp8" if spec.ki_fp8 else "bf16"}
+                                          "dtype": "fp8" if eight_bit else "bf16"}
         topk_us = sum(v for k, v in us.items() if k.startswith("topk"))
         b = pairs * 4 + T * K * 4
         if topk_us > 0:
@@ -530,7 +554,7 @@ def run_ours(args, world, rank, local):
                          reps, 3, stream, flush)
     n_keys = int((wl.token_pos() + 1).sum())
     n_sel = int(np.minimum(wl.token_pos() + 1, K).sum())
-    idx_bytes = n_keys * (132 if spec.ki_fp8 else 256)          # index-cache bytes read
+    idx_bytes = n_keys * index_row_bytes(spec)                   # index-cache bytes read
     attn_bytes = n_sel * (584 if spec.kv_fp8 else 1152)           # gathered latent rows (FP8: codes + 8 scale bytes)
     peak, peak_kind = hbm_peak()
     ms_idx = statistics.mean(t_idx)
@@ -539,7 +563,7 @@ def run_ours(args, world, rank, local):
     for name, nbytes in (("index_scores", idx_bytes), ("topk_filter", score_bytes),
                          ("sparse_mla", attn_bytes)):
         if name in kern:
-            roofs[name] = roofline_entry(name, kern, nbytes, peak, peak_kind, spec.name)
+            roofs[name] = roofline_entry(name, kern, nbytes, peak, peak_kind, workload_config(spec, wl, world))
     dominant = max(roofs.values(), key=lambda r: r["launch_us"])
 
     # ---- end to end through the C ABI with host buffers ----
@@ -614,9 +638,9 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": ("mxfp8" if spec.ki_mx else "fp8-e4m3") + " index / "
+            "dtype": {"mxfp8": "mxfp8", "fp8_e4m3": "fp8-e4m3", "bf16": "bf16"}[index_cache(spec)] + " index / "
                      + ("fp8-e4m3 latent, " if spec.kv_fp8 else "") + "bf16 attention / fp32 accum",
-            "data": "synthetic (seeded, 64 planted keys per sequence)",
+            "data": data_desc(spec),
             "config": workload_config(spec, wl, world),
             "launch": launch_mode,
             "stages_us": {"index_scores": ms_idx * 1e3, "topk": statistics.mean(t_topk) * 1e3,
