@@ -61,3 +61,12 @@ def test_captured_traffic_only_for_the_captured_formats(fresh_sources):
 def test_captured_traffic_goes_stale_with_the_source(monkeypatch):
     monkeypatch.setattr(bench, "source_digest", lambda files: "0" * 16)
     assert bench.ncu_traffic("index_scores", _config(CONFIGS["decode_b8_128k"])) is None
+
+
+def test_roofline_entry(fresh_sources):
+    cfg = _config(CONFIGS["decode_b8_128k"])
+    r = bench.roofline_entry("index_scores", {"index_scores": [0.040, 0.044]}, 138_412_032, 6552.3, "measured", cfg)
+    assert r["launch_us"] == pytest.approx(42.0)
+    assert r["achieved"] == pytest.approx(138_412_032 / 42.0e-6 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6552.3)
+    assert (r["bound"], r["unit"], r["traffic"]) == ("hbm", "GB/s", 145.60e6)
