@@ -99,6 +99,8 @@ def parse():
                     help="override the workload's context length (profiling a smaller case of the same kernels)")
     ap.add_argument("--all-configs", action="store_true",
                     help="one JSON line per workload: fused-call time and the binding roofline of each stage")
+    ap.add_argument("--no-all-configs", action="store_true",
+                    help="leave out the per-workload summary that a 1-GPU headline line carries")
     ap.add_argument("--ki", choices=["workload", "mxfp8"], default="workload",
                     help="index-cache format: the workload's own (E4M3 + row scale for the headline) or MXFP8")
     ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
@@ -392,6 +394,27 @@ def run_only(args, dsa, wl, d, dev, stream, flush, world, fused=None):
 
 
 def run_all_configs(args, dsa, dev, stream, flush):
+    for line in all_config_lines(args, dsa, dev, stream, flush):
+        print(json.dumps(line), flush=True)
+
+
+def all_configs_summary(args, dsa, dev, stream, flush) -> dict:
+    """The per-workload lines condensed for the headline line: time per call,
+    tokens/s, launches and each stage's binding roofline fraction.  A failure
+    is recorded in the summary; the headline line is printed regardless."""
+    out = {}
+    try:
+        for ln in all_config_lines(args, dsa, dev, stream, flush):
+            out[ln["config"]] = {
+                "us_per_call": ln["us_per_call"], "tokens_per_s": ln["tokens_per_s"], "launches": ln["launches"],
+                "stages": {k: {f: v[f] for f in ("bound", "us", "frac", "unit", "dtype") if f in v}
+                           for k, v in ln["stages"].items()}}
+    except Exception as exc:  # noqa: BLE001
+        out["error"] = f"{type(exc).__name__}: {str(exc)[:160]}"
+    return out
+
+
+def all_config_lines(args, dsa, dev, stream, flush):
     """Every workload once: the fused call (graph replay, L2 flushed before each
     step) and per-kernel device times, each stage against its binding roofline."""
     from dsa_workloads import to_device
@@ -465,9 +488,9 @@ def run_all_configs(args, dsa, dev, stream, flush):
                 "select_in_indexer": args.select_in_indexer,
                 "peak_source": hbm_src, "timing": "graph replay, 256 MiB L2 flush before each step; "
                 "kernels_us from events around each launch (serialised)"}
-        print(json.dumps(line), flush=True)
         del d, ws, out, lse
         torch.cuda.empty_cache()
+        yield line
 
 
 def run_ours(args, world, rank, local):
@@ -633,6 +656,11 @@ def run_ours(args, world, rank, local):
     launch_mode = "cuda graph replay" if graph is not None else "eager"
     if graph is not None:
         del graph
+    # every workload once more, untimed for the headline: each one's call time
+    # and stage rooflines, recorded beside the headline number (1 GPU only)
+    all_cfg = None
+    if rank == 0 and world == 1 and not args.no_all_configs:
+        all_cfg = all_configs_summary(args, dsa, dev, stream, flush)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -655,6 +683,8 @@ def run_ours(args, world, rank, local):
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }
+        if all_cfg is not None:
+            line["all_configs"] = all_cfg
         print(json.dumps(line), flush=True)
 
 

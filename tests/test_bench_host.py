@@ -70,3 +70,99 @@ def test_roofline_entry(fresh_sources):
     assert r["achieved"] == pytest.approx(138_412_032 / 42.0e-6 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / 6552.3)
     assert (r["bound"], r["unit"], r["traffic"]) == ("hbm", "GB/s", 145.60e6)
+
+
+class _FakeGraph:
+    def replay(self):
+        pass
+
+
+class _FakeCapture:
+    def __init__(self, graph):
+        pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def _fake_library(calls, launches):
+    from types import SimpleNamespace as NS
+    return NS(DSA_OK=0, DSA_OP_INDEX_TOPK_ATTN=4, DSA_OP_INDEX_TOPK_ATTN_FUSED=5,
+              dsa_workspace_size=lambda op, seqs, K, H: 256,
+              dsa_index_topk_attn=lambda *a, **k: calls.append(k),
+              dsa_check_error=lambda ws: 0,
+              dsa_launches_in_last_call=lambda: len(launches),
+              dsa_launch_timing=lambda on: None,
+              dsa_last_launch_times=lambda: list(launches))
+
+
+@pytest.fixture
+def host_only_bench(monkeypatch):
+    """all_config_lines on CPU: small workloads, a fake library and fake CUDA
+    timing, so only the bench's own bookkeeping runs."""
+    import torch
+    import dsa_workloads
+    from types import SimpleNamespace as NS
+    small = {
+        "tiny_prefill_1k": CONFIGS["tiny_prefill_1k"].scaled(ctx=(256, 256)),
+        "decode_b64_8k_32k": CONFIGS["decode_b64_8k_32k"].scaled(batch=3, ctx=(300, 900)),
+    }
+    monkeypatch.setattr(bench, "CONFIGS", small)
+    monkeypatch.setattr(dsa_workloads, "to_device", lambda wl: NS(seqs=None, qI=wl.qI, w=wl.w, kI=wl.kI,
+                                                                  kI_scale=wl.kI_scale, q=wl.q, kv=wl.kv,
+                                                                  kv_scale=wl.kv_scale))
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: None)
+    monkeypatch.setattr(torch.cuda, "CUDAGraph", _FakeGraph)
+    monkeypatch.setattr(torch.cuda, "graph", _FakeCapture)
+    monkeypatch.setattr(torch.cuda, "empty_cache", lambda: None)
+    monkeypatch.setattr(bench, "time_device", lambda fn, steps, warmup, stream, flush: (fn(), [0.25, 0.25])[1])
+    monkeypatch.setattr(bench, "hbm_peak", lambda: (6552.3, "measured"))
+    monkeypatch.setattr(bench, "tensor_peak", lambda kind: (1640.5 * (2 if kind == "fp8" else 1), "measured"))
+    args = NS(ki="workload", kv="bf16", select_in_indexer=False)
+    return args, small
+
+
+def test_all_config_lines_bookkeeping(host_only_bench):
+    import torch
+    args, small = host_only_bench
+    calls = []
+    launches = [("prep", 0.01), ("index_scores", 0.04), ("topk_row", 0.02), ("sparse_mla", 0.1)]
+    lines = list(bench.all_config_lines(args, _fake_library(calls, launches), torch.device("cpu"), None,
+                                        torch.empty(64, dtype=torch.uint8)))
+    assert [ln["config"] for ln in lines] == list(small)
+    tiny, dec = lines
+    assert tiny["us_per_call"] == pytest.approx(250.0) and dec["launches"] == 4
+    assert tiny["kernels_us"]["index_scores"] == pytest.approx(40.0)
+    # bf16 prefill indexer: tensor bound against the bf16 peak, 16,384 flop per causal pair
+    pairs = 256 * 257 // 2
+    s = tiny["stages"]["index_scores"]
+    assert (s["bound"], s["dtype"]) == ("tensor", "bf16")
+    assert s["frac"] == pytest.approx(pairs * 16384 / 40e-6 / 1e12 / 1640.5)
+    # decode indexer: HBM bound, 132 B per key of the FP8 cache
+    wl = bench.make_workload(small["decode_b64_8k_32k"])
+    keys = int((wl.token_pos() + 1).sum())
+    s = dec["stages"]["index_scores"]
+    assert s["bound"] == "hbm" and s["frac"] == pytest.approx(keys * 132 / 40e-6 / 1e9 / 6552.3)
+    assert dec["stages"]["sparse_mla"]["bound"] == "hbm"
+    assert all(not k.get("select_in_indexer") for k in calls)
+
+
+def test_all_configs_summary_condenses_and_survives_failures(host_only_bench, monkeypatch):
+    import torch
+    args, small = host_only_bench
+    launches = [("prep", 0.01), ("index_scores", 0.04), ("topk_row", 0.02), ("sparse_mla", 0.1)]
+    flush = torch.empty(64, dtype=torch.uint8)
+    summ = bench.all_configs_summary(args, _fake_library([], launches), torch.device("cpu"), None, flush)
+    assert set(summ) == set(small)
+    assert set(summ["tiny_prefill_1k"]) == {"us_per_call", "tokens_per_s", "launches", "stages"}
+    assert summ["tiny_prefill_1k"]["stages"]["index_scores"]["bound"] == "tensor"
+
+    def broken(*a):
+        yield {"config": "first", "us_per_call": 1.0, "tokens_per_s": 1.0, "launches": 1, "stages": {}}
+        raise RuntimeError("device error flag set on second")
+    monkeypatch.setattr(bench, "all_config_lines", broken)
+    summ = bench.all_configs_summary(args, None, None, None, None)
+    assert "first" in summ and summ["error"].startswith("RuntimeError: device error flag")
