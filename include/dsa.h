@@ -146,7 +146,10 @@ enum {
  *                  R above 2^31 - 1 returns DSA_ERR_UNSUPPORTED
  *   max_ctx        host-known upper bound of ctx_len[b]; sizes grids and
  *                  workspace.  A ctx_len above it is a device error.
- *   q_seq_start    int32 [B+1], non-decreasing, q_seq_start[0] = 0
+ *   q_seq_start    int32 [B+1], non-decreasing, q_seq_start[0] = 0.  A
+ *                  sequence whose rows leave 0..T-1 is skipped, and rows that
+ *                  overlap (a decreasing entry) leave the indexer no work;
+ *                  both are device errors (DSA_ERR_BAD_INDEX)
  *   ctx_len        int32 [B], q_len[b] <= ctx_len[b] <= max_ctx
  *   page_table     int32 [B, max_pages]; entries past ceil(ctx_len/64) unread
  */

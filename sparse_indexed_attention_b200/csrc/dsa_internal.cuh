@@ -155,7 +155,7 @@ struct PlanBufs {
 // Tokens per indexer group and key tiles per work item for a geometry.
 inline int indexer_group_tokens(int T, int B, bool fp8) { return T == B ? 1 : (fp8 ? 4 : 2); }
 inline int indexer_item_tiles(int tg) { return tg == 1 ? 8 : 16; }
-inline int64_t plan_max_groups(int T, int B, int tg) {
+__host__ __device__ inline int64_t plan_max_groups(int T, int B, int tg) {
   const int64_t g = (int64_t)T / tg + B;
   return g < T ? g : T;
 }

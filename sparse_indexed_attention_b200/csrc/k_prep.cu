@@ -71,7 +71,9 @@ __device__ __forceinline__ bool seq_ok(const SeqsDev& s, const int* qs, const in
   const int ctx = cl[b];
   *q_len_out = q_len;
   *ctx_out = ctx;
-  return q_len >= 0 && ctx >= 1 && ctx <= s.max_ctx && q_len <= ctx && (ctx + kPage - 1) / kPage <= s.max_pages;
+  // the sequence's query rows lie inside the T rows of every per-token tensor
+  return q_len >= 0 && qs[b] >= 0 && qs[b + 1] <= s.num_tokens && ctx >= 1 && ctx <= s.max_ctx && q_len <= ctx &&
+         (ctx + kPage - 1) / kPage <= s.max_pages;
 }
 
 }  // namespace
@@ -179,6 +181,18 @@ __device__ __forceinline__ void plan_impl(const SeqsDev& s, int tg, int ch, cons
     __syncthreads();
   }
   const int G = running;
+  // Sequences whose query rows do not overlap give at most plan_max_groups
+  // groups, the capacity the workspace holds.  Only a q_seq_start that
+  // decreases somewhere (overlapping rows) gives more: no work is planned and
+  // the error is raised.
+  if (G > plan_max_groups(s.num_tokens, s.batch, tg)) {
+    if (tid == 0) {
+      raise_error(err, kErrBadIndex);
+      p.counts[0] = 0;
+      p.counts[1] = 0;
+    }
+    return;
+  }
   int* s_istart = sm.istart;
   int* s_tiles = sm.tiles;
   int4* s_gd = sm.gd;
