@@ -33,6 +33,19 @@ def test_library_exports_every_declared_symbol():
         assert getattr(lib, name) is not None
 
 
+def test_binding_constants_match_the_header():
+    """Every enumerator and #define value of include/dsa.h has the same value
+    in the binding (the binding restates them for ctypes)."""
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    consts = {n: int(v) for n, v in re.findall(r"^\s*(DSA_[A-Z0-9_]+)\s*=\s*(\d+)", src, flags=re.M)}
+    for n, a, b in re.findall(r"^#define\s+(DSA_[A-Z0-9_]+)\s+\((\d+)u\s*<<\s*(\d+)\)", src, flags=re.M):
+        consts[n] = int(a) << int(b)
+    assert len(consts) >= 20 and "DSA_NOALLOC_SCRATCH_BYTES" in consts
+    for name, value in consts.items():
+        assert getattr(dsa, name) == value, name
+
+
 def test_status_strings():
     for code, name in enumerate(["DSA_OK", "DSA_ERR_INVALID_ARG", "DSA_ERR_UNSUPPORTED", "DSA_ERR_WORKSPACE",
                                  "DSA_ERR_CUDA", "DSA_ERR_BAD_INDEX", "DSA_ERR_TIMEOUT"]):
