@@ -46,6 +46,42 @@ def test_binding_constants_match_the_header():
         assert getattr(dsa, name) == value, name
 
 
+def _ctype_of(param: str):
+    """The ctypes class a C parameter (or return) declaration marshals as."""
+    p = " ".join(param.replace("const", " ").split())
+    if "*" in p or p.split()[0] in ("dsa_stream_t", "dsa_event_t"):
+        return "pointer"
+    base = p.split()[0]
+    return {"int": ctypes.c_int, "int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "size_t": ctypes.c_size_t,
+            "float": ctypes.c_float, "unsigned": ctypes.c_uint, "uint64_t": ctypes.c_uint64,
+            "dsa_status_t": ctypes.c_int, "dsa_op_t": ctypes.c_int, "dsa_ki_dtype_t": ctypes.c_int,
+            "dsa_kv_dtype_t": ctypes.c_int, "dsa_out_dtype_t": ctypes.c_int}[base]
+
+
+def test_binding_signatures_match_the_header():
+    """Each ctypes prototype has the header's parameter count and, parameter by
+    parameter, a type of the same width (pointers as pointers)."""
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    protos = re.findall(r"^([A-Za-z_][\w \*]*?)\b(dsa_\w+)\s*\(([^;{]*?)\)\s*;", src, flags=re.M | re.S)
+    assert {n for _, n, _ in protos} == set(dsa.EXPORTS)
+    for ret, name, params in protos:
+        res, args = dsa._sig[name]
+        params = [] if params.strip() in ("", "void") else [x.strip() for x in params.split(",")]
+        assert len(args) == len(params), name
+        for i, (decl, got) in enumerate(zip(params, args)):
+            want = _ctype_of(decl)
+            if want == "pointer":
+                assert got in (ctypes.c_void_p, ctypes.c_char_p) or issubclass(got, ctypes._Pointer), (name, i, decl)
+            else:
+                assert ctypes.sizeof(got) == ctypes.sizeof(want), (name, i, decl, got)
+        want = _ctype_of(ret.strip())
+        if want == "pointer":
+            assert res in (ctypes.c_void_p, ctypes.c_char_p), name
+        else:
+            assert ctypes.sizeof(res) == ctypes.sizeof(want), (name, "return")
+
+
 def test_status_strings():
     for code, name in enumerate(["DSA_OK", "DSA_ERR_INVALID_ARG", "DSA_ERR_UNSUPPORTED", "DSA_ERR_WORKSPACE",
                                  "DSA_ERR_CUDA", "DSA_ERR_BAD_INDEX", "DSA_ERR_TIMEOUT"]):
