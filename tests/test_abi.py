@@ -82,6 +82,23 @@ def test_binding_signatures_match_the_header():
             assert ctypes.sizeof(res) == ctypes.sizeof(want), (name, "return")
 
 
+def test_seqs_struct_layout_matches_the_header(tmp_path):
+    """dsa_seqs_t as a C compiler lays it out (size, field offsets, enum size)
+    equals the binding's ctypes structure."""
+    fields = [f for f, _ in dsa.DsaSeqsC._fields_]
+    prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "dsa.h"', "int main(void) {",
+            '  printf("%zu %zu\\n", sizeof(dsa_seqs_t), sizeof(dsa_ki_dtype_t));']
+    prog += [f'  printf("%zu\\n", offsetof(dsa_seqs_t, {f}));' for f in fields]
+    prog += ["  return 0;", "}"]
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-x", "c", "-",
+                    "-o", str(exe)], input="\n".join(prog), text=True, check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    size, enum_size, *offsets = map(int, out)
+    assert size == ctypes.sizeof(dsa.DsaSeqsC) and enum_size == ctypes.sizeof(ctypes.c_int)
+    assert offsets == [getattr(dsa.DsaSeqsC, f).offset for f in fields]
+
+
 def test_status_strings():
     for code, name in enumerate(["DSA_OK", "DSA_ERR_INVALID_ARG", "DSA_ERR_UNSUPPORTED", "DSA_ERR_WORKSPACE",
                                  "DSA_ERR_CUDA", "DSA_ERR_BAD_INDEX", "DSA_ERR_TIMEOUT"]):
