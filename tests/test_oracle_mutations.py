@@ -70,6 +70,13 @@ MUTANTS = {
                                 "v[..., lo:hi] *= e8m0_decode(sc[..., 0])[..., None]", [KV8]),
     "kv8_rope_tile_unscaled": ("for j in range((c.shape[-1] + KV_TILE - 1) // KV_TILE):",
                                "for j in range(c.shape[-1] // KV_TILE):", [KV8]),
+    "index_weight_of_first_token": ("wt = w[t] * sq[t]", "wt = w[0] * sq[t]", [INDEXER]),
+    "page_offset_reversed": ("return pages * self.page_size + s % self.page_size",
+                             "return pages * self.page_size + (self.page_size - 1 - s % self.page_size)",
+                             [INDEXER, ATTN, PIPE]),
+    "attn_lse_base_2": ("lse[i] = (m + np.log(l))[:, 0]", "lse[i] = (m + np.log2(l))[:, 0]", [ATTN]),
+    "kv8_scale_byte_bias": ("scales[:, j] = (e + E8M0_BIAS).astype(np.uint8)",
+                            "scales[:, j] = (e + E8M0_BIAS + 1).astype(np.uint8)", [KV8]),
     "kv8_attention_reads_raw_codes": ("return kv_fp8_dequantize(np.asarray(codes)[rows], np.asarray(scales)[rows])",
                                       "return e4m3_decode_fast(np.asarray(codes)[rows])", [KV8]),
 }
