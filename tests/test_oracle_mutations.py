@@ -64,6 +64,11 @@ MUTANTS = {
                              "kmat = e4m3_decode_fast(np.asarray(kI)[rows])", [MX]),
     "mx_key_scale_wrong_row": ("kmat = mxfp8_dequantize(np.asarray(kI)[rows], np.asarray(kI_scale)[rows])",
                                "kmat = mxfp8_dequantize(np.asarray(kI)[rows], np.asarray(kI_scale)[rows[::-1]])", [MX]),
+    "mx_blocks_strided": ("blocks = x.reshape(*x.shape[:-1], n // MX_BLOCK, MX_BLOCK)",
+                          "blocks = x.reshape(*x.shape[:-1], MX_BLOCK, n // MX_BLOCK).swapaxes(-1, -2)", [MX]),
+    "mx_dequantize_strided": ("v = e4m3_decode_fast(c).reshape(*c.shape[:-1], n // MX_BLOCK, MX_BLOCK)",
+                              "v = e4m3_decode_fast(c).reshape(*c.shape[:-1], MX_BLOCK, n // MX_BLOCK)"
+                              ".swapaxes(-1, -2)", [MX]),
     "kv8_tile_64": ("KV_TILE = 128        # elements per scale", "KV_TILE = 64         # elements per scale", [KV8]),
     "kv8_scale_dropped": ("v[..., lo:hi] *= e8m0_decode(sc[..., j])[..., None]", "v[..., lo:hi] *= 1.0", [KV8]),
     "kv8_scale_of_first_tile": ("v[..., lo:hi] *= e8m0_decode(sc[..., j])[..., None]",
