@@ -9,9 +9,10 @@ position, so pairing an early segment with a late one gives every rank the
 same causal work.
 
 Each rank holds the index keys (FP8 codes + scales, or bf16) and latent rows
-(bf16, or FP8 codes + tile-scale bytes) of its own two segments, segment r first.  One all-gather per pool (NCCL over
-NVLink, into each rank's own memory) gives every rank the pools of the whole
-sequence laid out rank by rank: rank q's rows sit at [2 seg q, 2 seg (q+1)).
+(bf16, or FP8 codes + tile-scale bytes) of its own two segments, segment r
+first.  One all-gather per pool (NCCL over NVLink, into each rank's own
+memory) gives every rank the pools of the whole sequence laid out rank by
+rank: rank q's rows sit at [2 seg q, 2 seg (q+1)).
 Nothing is copied back into sequence order: a page table maps the sequence's
 logical pages onto that layout (segments are whole pages).  Each rank then runs
 the unchanged hot path (dsa_index_topk_attn) on its two segments as a batch
