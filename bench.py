@@ -42,10 +42,10 @@ L2_FLUSH_BYTES = 256 << 20
 # figure back into null.
 NCU_CAPTURES = (
     # kernel, config keys that must match, bytes per launch, sources, digest
-    ("index_scores", {"index_cache": "fp8_e4m3"}, 145.60e6, ("k_indexer.cu",), "e0e0692b453fdc25"),
-    ("index_scores", {"index_cache": "mxfp8"}, 144.81e6, ("k_indexer.cu",), "e0e0692b453fdc25"),
-    ("topk_filter", {}, 4.35e6, ("k_topk.cu",), "e4402930e3a60776"),
-    ("sparse_mla", {"latent_cache": "bf16"}, 20.25e6, ("k_sparse_mla.cu",), "ddd016a86f793cee"),
+    ("index_scores", {"index_cache": "fp8_e4m3"}, 145.60e6, ("k_indexer.cu",), "6a6254d29a2242f3"),
+    ("index_scores", {"index_cache": "mxfp8"}, 144.81e6, ("k_indexer.cu",), "6a6254d29a2242f3"),
+    ("topk_filter", {}, 4.35e6, ("k_topk.cu",), "507b32e02ae94d9e"),
+    ("sparse_mla", {"latent_cache": "bf16"}, 20.25e6, ("k_sparse_mla.cu",), "412a2a7f29ba3946"),
 )
 NCU_WORKLOAD = {"workload": "decode_b8_128k", "ctx": 131072}
 CSRC = os.path.join(ROOT, "sparse_indexed_attention_b200", "csrc")
